@@ -1,0 +1,382 @@
+#!/usr/bin/env python
+"""Benchmark of one MLA decode step over a paged latent + RoPE cache on B200.
+
+A step is the whole hot path on one batch: cache append of the new rows, query
+absorption through W_UK, decode attention (tcgen05), split-KV combine and the W_UV
+output projection, all in libmla.so kernels. The metric is cache bytes read per
+second (every visible cached row of 1,152 bytes counted once per step), with the
+step's FLOPs and the decode kernel's roofline fraction beside it.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
+
+N > 1 runs under torchrun, one process per GPU; every rank decodes its own batch
+of the workload (sequences are independent: no collective on the data path) and
+rank 0 prints the JSON line, timed as the max over ranks.
+`--impl reference` times the fp64 CPU oracle (the only other implementation of
+this computation) on the host cores on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import re
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "MLA decode: cache GB/s and TFLOP/s, fraction of B200 roofline"
+DEFAULT_WORKLOAD = "deepseek_h128_b128_ragged"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+L2_FLUSH_BYTES = 512 << 20
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return {k: float(d[k]) for k in FALLBACK_PEAKS}, "measured"
+    except Exception:
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def traffic_record(workload):
+    """DRAM bytes per launch of the decode kernel from a committed ncu summary, valid
+    only while the kernel source is unchanged (its sha256 is recorded there)."""
+    src = os.path.join(ROOT, "mla_latent_kv_46_b200", "csrc", "decode_tc.cuh")
+    sha = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+    path = os.path.join(ROOT, "profiles", f"ncu_decode_attn_{workload}.md")
+    if not os.path.exists(path):
+        return None, sha
+    text = open(path).read()
+    m_sha = re.search(r"decode_tc\.cuh sha256\[:16\]:\s*([0-9a-f]{16})", text)
+    m_tr = re.search(r"traffic per full launch \(bytes\):\s*([0-9]+)", text)
+    if not m_sha or not m_tr or m_sha.group(1) != sha:
+        return None, sha
+    return int(m_tr.group(1)), sha
+
+
+# ----------------------------------------------------------------------------- clocks (NVML poller)
+
+class ClockSampler:
+    """Polls SM clock and throttle reasons of one GPU every few ms while running."""
+
+    REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+               0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
+               0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting"}
+
+    def __init__(self, device_index: int):
+        self.samples = []
+        self.ok = False
+        self._stop = threading.Event()
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            import torch
+            uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+            h = None
+            for i in range(pynvml.nvmlDeviceGetCount()):
+                hh = pynvml.nvmlDeviceGetHandleByIndex(i)
+                u = pynvml.nvmlDeviceGetUUID(hh)
+                u = u.decode() if isinstance(u, bytes) else u
+                if uuid in u:
+                    h = hh
+            if h is None:
+                h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.nv, self.h = pynvml, h
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception as e:  # noqa: BLE001
+            self.err = repr(e)
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                mhz = self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM)
+                rs = self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                self.samples.append((mhz, rs))
+            except Exception:  # noqa: BLE001
+                pass
+            time.sleep(0.002)
+
+    def __enter__(self):
+        if self.ok:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self.ok:
+            self._stop.set()
+            self.t.join()
+
+    def summary(self):
+        if not self.ok:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0, "note": "nvml unavailable"}
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0}
+        mhz = [s[0] for s in self.samples]
+        bits = 0
+        for s in self.samples:
+            bits |= s[1]
+        reasons = sorted(name for b, name in self.REASONS.items() if bits & b and name != "gpu_idle")
+        return {"sm_mhz": statistics.median(mhz), "sm_max_mhz": self.max_mhz, "reasons": reasons,
+                "samples": len(mhz), "sm_mhz_min": min(mhz)}
+
+
+# ----------------------------------------------------------------------------- reference arm (oracle, CPU)
+
+def cpu_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except Exception:  # noqa: BLE001
+        pass
+    return len(os.sched_getaffinity(0))
+
+
+def oracle_sample(spec, w, budget_s=20.0, max_seqs=None):
+    """Time the oracle (non-absorbed fp64 definition) on whole sequences of the
+    workload, shortest first, until about budget_s of CPU work. Returns (bytes, seconds, desc)."""
+    from oracle import mla_oracle as orc
+    lens = w["seq_lens"]
+    order = np.argsort(lens, kind="stable")
+    done_bytes, spent, seqs = 0, 0.0, []
+    for b in order:
+        b = int(b)
+        t0 = time.perf_counter()
+        sl = slice(b * spec.q_len, (b + 1) * spec.q_len)
+        orc.decode_nonabsorbed(w["q_nope"][sl], w["q_rope"][sl], w["kv_cache"], w["block_table"][b:b + 1],
+                               w["seq_lens"][b:b + 1], w["W_UK"], w["W_UV"], w["scale"], q_len=spec.q_len,
+                               page_size=spec.page_size)
+        spent += time.perf_counter() - t0
+        seqs.append(b)
+        done_bytes += int(lens[b]) * spec.row * (2 if spec.dtype == "bf16" else 4)
+        if spent >= budget_s or (max_seqs and len(seqs) >= max_seqs):
+            break
+    desc = (f"oracle (fp64 numpy, non-absorbed) on {len(seqs)} of {len(lens)} sequences "
+            f"(shortest first, {int(sum(int(lens[b]) for b in seqs))} tokens, all {spec.H} heads)")
+    return done_bytes, spent, desc
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    from mla_latent_kv_46_b200 import workloads as wl
+    spec = wl.WORKLOADS[args.workload]
+    w = wl.make(spec, seed=0)
+    per_step_budget = 4.0
+    for _ in range(args.warmup):
+        oracle_sample(spec, w, budget_s=per_step_budget, max_seqs=1)
+    tot_b, tot_t, desc = 0, 0.0, ""
+    for _ in range(args.steps):
+        b, t, desc = oracle_sample(spec, w, budget_s=per_step_budget, max_seqs=1)
+        tot_b += b
+        tot_t += t
+    value = tot_b / tot_t / 1e9
+    cores = cpu_threads()
+    line = {"metric": METRIC, "value": value, "unit": "GB/s", "impl": "reference", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * tot_t / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": workload_config(spec, w, args),
+            "cpu_baseline": {"value": value, "unit": "GB/s", "cores": cores, "kind": "oracle",
+                             "sample": f"per step: {desc}"},
+            "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ----------------------------------------------------------------------------- GPU arm
+
+def workload_config(spec, w, args):
+    lens = w["seq_lens"]
+    return {"workload": spec.name, "B": int(len(lens)), "H": spec.H, "kv_lora_rank": spec.R, "rope_dim": spec.Dr,
+            "D_nope": spec.Dn, "D_v": spec.Dv, "q_len": spec.q_len, "page_size": spec.page_size,
+            "seq_lens": (f"uniform in [{spec.ragged[0]},{spec.ragged[1]}], seed 0" if spec.ragged
+                         else f"{spec.seq_len} each"),
+            "cached_tokens": int(np.sum(lens, dtype=np.int64)),
+            "l2": f"flushed between timed steps ({L2_FLUSH_BYTES >> 20} MiB write); cache also larger than L2",
+            "parallelism": f"replicas x{args.gpus} (independent sequences per GPU)"}
+
+
+def run_gpu(args):
+    import torch
+    import torch.distributed as dist
+
+    from mla_latent_kv_46_b200 import build as mbuild
+    mbuild.build()
+    import mla_latent_kv_46_b200 as mla
+    from mla_latent_kv_46_b200 import decoder as dec
+    from mla_latent_kv_46_b200 import workloads as wl
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    dev = torch.device("cuda", torch.cuda.current_device())
+    spec = wl.WORKLOADS[args.workload]
+    w = wl.make(spec, seed=rank)
+    step = dec.DecodeStep(w, device=dev)
+    mla.mla_set_policy(mla.MLA_POLICY_AUTO)
+    stream = torch.cuda.current_stream()
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    # ---------------------------------------------------------------- device-resident timing
+    names = ["append", "absorb", "attend", "combine", "project"]
+    for _ in range(args.warmup):
+        step.run()
+    torch.cuda.synchronize()
+    mla.mla_check_status()
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(len(names) + 1)] for _ in range(args.steps)]
+    barrier()
+    with ClockSampler(dev.index) as clk:
+        for k in range(args.steps):
+            flush.fill_(k & 0xFF)          # evict the cache from L2 (outside the timed events)
+            e = ev[k]
+            e[0].record(stream)
+            step.append()
+            e[1].record(stream)
+            step.absorb()
+            e[2].record(stream)
+            step.attend()
+            e[3].record(stream)
+            step.combine()
+            e[4].record(stream)
+            step.project()
+            e[5].record(stream)
+        barrier()
+    mla.mla_check_status()
+    per_kernel = {n: 0.0 for n in names}
+    step_ms = []
+    for e in ev:
+        for i, n in enumerate(names):
+            per_kernel[n] += e[i].elapsed_time(e[i + 1])
+        step_ms.append(e[0].elapsed_time(e[-1]))
+    total_ms = float(sum(step_ms))
+    total_ms_max = total_ms
+    if world > 1:
+        t = torch.tensor([total_ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms_max = float(t.item())
+
+    cache_bytes = wl.cache_bytes(spec, w["seq_lens"])
+    flops = wl.attention_flops(spec, w["seq_lens"])
+    ms_per_step = total_ms_max / args.steps
+    value = world * cache_bytes * args.steps / (total_ms_max / 1e3) / 1e9
+
+    # ---------------------------------------------------------------- roofline of the decode kernel
+    peaks, peak_src = load_peaks()
+    attn_ms = per_kernel["attend"] / args.steps
+    t_hbm = cache_bytes / (peaks["hbm_gbs"] * 1e9)
+    t_tc = flops / (peaks["bf16_tflops"] * 1e12)
+    bound = "hbm" if t_hbm >= t_tc else "tensor"
+    traffic, sha = traffic_record(spec.name)
+    if bound == "hbm":
+        roof = {"bound": "hbm", "achieved": cache_bytes / (attn_ms / 1e3) / 1e9, "peak": peaks["hbm_gbs"],
+                "unit": "GB/s"}
+    else:
+        roof = {"bound": "tensor", "achieved": flops / (attn_ms / 1e3) / 1e12, "peak": peaks["bf16_tflops"],
+                "unit": "TFLOP/s"}
+    roof["frac"] = roof["achieved"] / roof["peak"]
+    roof["traffic"] = traffic
+    roof["peak_source"] = f"{peak_src} (MEASURED_PEAKS.json)" if peak_src == "measured" else "fallback"
+    roof["kernel"] = "mla_decode_attn (tcgen05 decode_kernel)"
+    roof["algorithmic_bytes_per_launch"] = cache_bytes
+    roof["algorithmic_flops_per_launch"] = flops
+    roof["roofline_ms"] = 1e3 * max(t_hbm, t_tc)
+    roof["frac_of_roofline_time"] = 1e3 * max(t_hbm, t_tc) / attn_ms
+    roof["tflops"] = flops / (attn_ms / 1e3) / 1e12
+    roof["decode_tc_sha256_16"] = sha
+
+    # ---------------------------------------------------------------- end to end through the public API
+    hostin = dec.HostInputs(step, w)
+    for _ in range(max(3, args.warmup)):
+        dec.run_e2e(step, hostin, stream)
+    torch.cuda.synchronize()
+    e2e_steps = args.steps
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e2e_ms = 0.0
+    barrier()
+    for k in range(e2e_steps):
+        flush.fill_(k & 0xFF)
+        e0.record(stream)
+        dec.run_e2e(step, hostin, stream)
+        e1.record(stream)
+        e1.synchronize()          # the step's result is on the host
+        e2e_ms += e0.elapsed_time(e1)
+    barrier()
+    mla.mla_check_status()
+    if world > 1:
+        t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    e2e = {"value": world * cache_bytes * e2e_steps / (e2e_ms / 1e3) / 1e9, "unit": "GB/s",
+           "h2d_bytes_per_step": hostin.h2d_bytes(step), "d2h_bytes_per_step": hostin.d2h_bytes(),
+           "ms_per_step": e2e_ms / e2e_steps}
+
+    line = None
+    if rank == 0:
+        cpu = None
+        if world == 1 and not args.no_cpu_baseline:
+            b, t, desc = oracle_sample(spec, w, budget_s=args.cpu_budget)
+            cpu = {"value": b / t / 1e9, "unit": "GB/s", "cores": cpu_threads(), "kind": "oracle",
+                   "sample": desc, "seconds": t}
+        line = {"metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+                "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+                "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+                "config": workload_config(spec, w, argparse.Namespace(gpus=world)),
+                "tflops": world * flops * args.steps / (total_ms_max / 1e3) / 1e12,
+                "per_kernel_ms": {n: per_kernel[n] / args.steps for n in names},
+                "roofline": roof, "cpu_baseline": cpu, "e2e": e2e,
+                "gpu_launches": step.launches_per_step() * args.steps,
+                "clocks": clk.summary()}
+        print(json.dumps(line), flush=True)
+    del flush
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--cpu-budget", type=float, default=15.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_gpu(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

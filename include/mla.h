@@ -1,0 +1,189 @@
+/*
+ * mla.h -- C ABI of the B200 (sm_100a) MLA decode library (libmla.so).
+ *
+ * Multi-head Latent Attention decode over a paged cache whose rows hold only a
+ * latent c_t (kv_lora_rank R, 512) and one decoupled-RoPE key k_t (Dr, 64) shared
+ * by every head: 576 elements, 1,152 bytes in bf16, per token per layer
+ * (modeldna.ai "learn/mla", section "Under the hood" and its cache-size table).
+ * Each head's content query is absorbed through W_UK into latent space, scored
+ * against c_t, its rope query against k_t; the softmax scale is 1/sqrt(Dn + Dr)
+ * (kimi-k3 docs "GatedMLA", section "Observe logits, then compute causal
+ * attention"); the probabilities weight c_t itself and the R-wide result is
+ * up-projected per head through W_UV, so per-head K/V are never materialised.
+ *
+ * One decode step on one CUDA stream:
+ *   mla_cache_append   write the newest q_len rows of every sequence into its pages
+ *   mla_absorb_q       q_lat = q_nope @ W_UK[h]                       (per head)
+ *   mla_plan_splits    host: cut the work into balanced (sequence, page range) units
+ *   mla_decode_attn    scores, online softmax and latent value sum per unit
+ *   mla_combine        log-sum-exp merge of units that share a query
+ *   mla_out_proj       out = W_UV[h] @ o_lat                          (per head)
+ *
+ * Conventions for every call:
+ *  - Tensor pointers are DEVICE pointers unless the name ends in _host; all
+ *    tensors are row-major and contiguous with the shapes given; the caller owns
+ *    every buffer. The library never allocates device memory and never
+ *    synchronises the stream (except mla_check_status, which says so).
+ *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
+ *    Calls are asynchronous on it.
+ *  - Arguments are validated before any launch. On error the call returns a
+ *    negative mla_status, launches nothing, and mla_last_error() describes why.
+ *  - dtype MLA_BF16: q_nope, q_rope, W_UK, W_UV, kv_cache, new_ckr, q_lat, o_lat and
+ *    out are bf16 (RN-even conversions); accumulation is fp32. MLA_F32: all fp32.
+ *    Partial outputs and log-sum-exp values are always fp32.
+ *  - A cache row is [c (R) ; k_rope (Dr)]; k_rope is stored already rotated.
+ *    seq_lens[b] counts cached tokens of sequence b INCLUDING its q_len new ones.
+ *    Query i (0 <= i < q_len) of sequence b sits at position seq_lens[b]-q_len+i
+ *    and sees tokens t <= that position (causal within the chunk). A query that
+ *    sees no token yields o_lat = 0, out = 0 and lse = -inf.
+ *  - Token t of sequence b is row t % page_size of page block_table[b*max_pages +
+ *    t / page_size] of kv_cache[num_pages][page_size][R+Dr].
+ *  - Kernels bound every wait; a wait that runs out sets a device status word
+ *    that mla_check_status() reports as MLA_ERR_TIMEOUT. A page id outside
+ *    [0, num_pages) is skipped and reported as MLA_ERR_INVALID the same way.
+ */
+#ifndef MLA_H_
+#define MLA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define MLA_ABI_VERSION 1
+
+typedef enum {
+  MLA_OK = 0,
+  MLA_ERR_INVALID = -1,      /* bad argument (null pointer, size, layout, plan) */
+  MLA_ERR_UNSUPPORTED = -2,  /* dims or policy this build has no kernel for */
+  MLA_ERR_WORKSPACE = -3,    /* workspace / plan buffer too small */
+  MLA_ERR_CUDA = -4,         /* a CUDA runtime or driver call failed */
+  MLA_ERR_TIMEOUT = -5       /* a kernel wait ran out (reported by mla_check_status) */
+} mla_status;
+
+typedef enum { MLA_BF16 = 0, MLA_F32 = 1 } mla_dtype;
+
+/* Geometry of one MLA layer. Validated like a KV-state ledger config (every
+ * field a positive integer; datawhalechina "ARCH-MLA", section "Step 4"). */
+typedef struct {
+  int32_t H;          /* query heads */
+  int32_t Dn;         /* per-head content query width (W_UK rows) */
+  int32_t Dr;         /* shared rope key width */
+  int32_t Dv;         /* per-head value width (W_UV rows) */
+  int32_t R;          /* latent width, kv_lora_rank */
+  int32_t page_size;  /* tokens per cache page */
+  int32_t dtype;      /* mla_dtype */
+} mla_dims;
+
+/* Kernel selection for mla_decode_attn / mla_absorb_q / mla_out_proj.
+ * AUTO: tensor-core (tcgen05) kernels where the dims allow (bf16, R=512, Dr=64,
+ * page_size=64, H a multiple of 64, Dn=Dv=128), else the SIMT CUDA kernels.
+ * SIMT: always the SIMT CUDA kernels. TCGEN05: tensor-core kernels or
+ * MLA_ERR_UNSUPPORTED. There is no CPU path. */
+typedef enum { MLA_POLICY_AUTO = 0, MLA_POLICY_SIMT = 1, MLA_POLICY_TCGEN05 = 2 } mla_policy;
+
+/* Summary of a split plan (filled by mla_plan_splits). */
+typedef struct {
+  int32_t num_items;    /* B * q_len query tokens */
+  int32_t num_units;    /* (query token, page range) work units */
+  int32_t num_slots;    /* page-balanced groups of units; one CTA per slot and head group */
+  int32_t num_parts;    /* units whose result is partial and needs mla_combine */
+  int32_t head_groups;  /* heads are processed in groups of H / head_groups */
+  int32_t plan_words;   /* int32 words of the plan buffer in use */
+} mla_plan_info;
+
+int32_t mla_abi_version(void);
+
+/* Thread-local description of the last error of this thread ("" if none). */
+const char* mla_last_error(void);
+
+/* Select the kernel policy for later calls (process-wide). */
+mla_status mla_set_policy(int32_t policy);
+
+/* Bound, in nanoseconds, on every wait inside a kernel (default 2e9). */
+mla_status mla_set_wait_timeout_ns(uint64_t ns);
+
+/* Synchronises `stream`, then reads and clears the device status word of the
+ * current device: MLA_OK, MLA_ERR_TIMEOUT (a bounded wait ran out) or
+ * MLA_ERR_INVALID (a page id outside the pool was skipped). */
+mla_status mla_check_status(void* stream);
+
+/* ---------------------------------------------------------------- a2: cache append
+ * Writes new_ckr[b*q_len + i] to position seq_lens[b] - q_len + i of sequence b
+ * ("MLA + KV cache (Tier 3 #5)" ticket, "Description" item 1: project only the
+ * new token and keep earlier ones cached). Positions < 0 are skipped.
+ *   kv_cache    [num_pages][page_size][R+Dr]   dtype, written
+ *   block_table [B][max_pages] int32, seq_lens [B] int32 (device)
+ *   new_ckr     [B*q_len][R+Dr]                dtype                              */
+mla_status mla_cache_append(void* kv_cache, const int32_t* block_table, const int32_t* seq_lens,
+                            const void* new_ckr, int32_t B, int32_t q_len, int32_t max_pages,
+                            int32_t num_pages, mla_dims d, void* stream);
+
+/* ---------------------------------------------------------------- a1: absorb the query
+ * q_lat[t][h][:] = q_nope[t][h][:] @ W_UK[h]  (modeldna "learn/mla", "Under the
+ * hood": the key up-projection folds into the query; W_UK[h] is head h's slice
+ * of the GatedMLA KV up-projection, "Projection geometry and stored weights").
+ *   q_nope [T][H][Dn], W_UK [H][Dn][R]  ->  q_lat [T][H][R]          all dtype      */
+mla_status mla_absorb_q(const void* q_nope, const void* W_UK, void* q_lat, int32_t T, mla_dims d,
+                        void* stream);
+
+/* ---------------------------------------------------------------- split planning (host)
+ * Upper bound, in int32 words, of the plan buffer for these sizes. */
+size_t mla_plan_capacity(int32_t B, int32_t q_len, int32_t num_sms);
+
+/* Cuts the decode work into units of whole pages and groups them into slots
+ * of nearly equal page counts (num_sms / head_groups slots), so that one CTA per
+ * slot and head group covers the GPU evenly; a query whose pages span several
+ * units gets one partial output per unit, merged by mla_combine.
+ *   seq_lens_host [B] int32 HOST; plan_host: HOST int32 buffer of `capacity`
+ *   words, written; copy its first info->plan_words words to the device and pass
+ *   that copy to mla_decode_attn and mla_combine. `info` (host) is written.     */
+mla_status mla_plan_splits(const int32_t* seq_lens_host, int32_t B, int32_t q_len, int32_t max_pages,
+                           mla_dims d, int32_t num_sms, int32_t* plan_host, size_t capacity,
+                           mla_plan_info* info);
+
+/* Bytes of workspace mla_decode_attn / mla_combine need for this plan: fp32
+ * partials [num_parts][H][R] followed by fp32 lse [num_parts][H]. */
+size_t mla_workspace_size(const mla_plan_info* info, mla_dims d);
+
+/* ---------------------------------------------------------------- a3-a5: decode attention
+ * For every query token (b, i) and head h, over the visible tokens t:
+ *   s_t = scale * ([q_lat ; q_rope] . [c_t ; k_t])     one (R+Dr)-long dot product
+ *   p   = softmax_t(s),  o_lat = sum_t p_t c_t  (R wide),  lse = log sum_t exp(s_t)
+ * (the absorbed form of the GatedMLA attention; scale = 1/sqrt(Dn+Dr) there).
+ *   q_lat [B*q_len][H][R], q_rope [B*q_len][H][Dr], kv_cache as above (dtype)
+ *   plan_dev: device copy of the mla_plan_splits buffer; info: its host summary
+ *   o_lat [B*q_len][H][R] dtype and lse [B*q_len][H] fp32 (lse may be NULL):
+ *   written for queries whose work is one unit; others go to the workspace.
+ *   workspace: >= mla_workspace_size bytes, 256-byte aligned (may be NULL when
+ *   the plan has no parts).                                                       */
+mla_status mla_decode_attn(const void* q_lat, const void* q_rope, const void* kv_cache,
+                           const int32_t* block_table, const int32_t* seq_lens, int32_t B,
+                           int32_t q_len, int32_t max_pages, int32_t num_pages, float scale,
+                           const int32_t* plan_dev, const mla_plan_info* info, void* o_lat,
+                           float* lse, void* workspace, size_t workspace_bytes, mla_dims d,
+                           void* stream);
+
+/* ---------------------------------------------------------------- a6: split-KV combine
+ * For each query whose work was split: m = max_s lse_s, w_s = exp(lse_s - m),
+ * o_lat = sum_s w_s o_s / sum_s w_s, lse = m + log sum_s w_s (parts with
+ * lse = -inf weigh 0). Writes o_lat (dtype) and lse (fp32, may be NULL) of those
+ * queries only. A no-op launch-free call when info->num_parts == 0.              */
+mla_status mla_combine(const int32_t* plan_dev, const mla_plan_info* info, const void* workspace,
+                       size_t workspace_bytes, void* o_lat, float* lse, mla_dims d, void* stream);
+
+/* ---------------------------------------------------------------- a7: output up-projection
+ * out[t][h][:] = W_UV[h] @ o_lat[t][h][:]  (the value up-projection folded into
+ * the output side; GatedMLA "Output projection and optional gate" applies Wo and
+ * the gate after this, outside this library).
+ *   o_lat [T][H][R], W_UV [H][Dv][R]  ->  out [T][H][Dv]             all dtype      */
+mla_status mla_out_proj(const void* o_lat, const void* W_UV, void* out, int32_t T, mla_dims d,
+                        void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MLA_H_ */

@@ -1,0 +1,496 @@
+// mla_lib.cu -- host side of libmla.so: the C ABI declared in include/mla.h.
+// Validates arguments, plans the split-KV work, builds TMA descriptors and
+// launches the kernels of simt_kernels.cuh and decode_tc.cuh. It allocates no
+// device memory and never synchronises a stream except in mla_check_status.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cmath>
+#include <atomic>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <string>
+#include <vector>
+
+#include "mla.h"
+#include "common.cuh"
+#include "ptx.cuh"
+#include "simt_kernels.cuh"
+#include "decode_tc.cuh"
+
+namespace {
+
+thread_local std::string g_last_error;
+std::atomic<int32_t> g_policy{MLA_POLICY_AUTO};
+std::atomic<uint64_t> g_timeout_ns{2000000000ull};
+
+mla_status fail(mla_status s, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return s;
+}
+
+mla_status ok() {
+  g_last_error.clear();
+  return MLA_OK;
+}
+
+#define MLA_CUDA_TRY(expr)                                                               \
+  do {                                                                                   \
+    cudaError_t e_ = (expr);                                                             \
+    if (e_ != cudaSuccess)                                                               \
+      return fail(MLA_ERR_CUDA, "%s failed: %s", #expr, cudaGetErrorString(e_));          \
+  } while (0)
+
+mla_status check_dims(const mla_dims& d) {
+  const int32_t v[] = {d.H, d.Dn, d.Dr, d.Dv, d.R, d.page_size};
+  const char* names[] = {"H", "Dn", "Dr", "Dv", "R", "page_size"};
+  for (int i = 0; i < 6; ++i)
+    if (v[i] <= 0) return fail(MLA_ERR_INVALID, "dims.%s must be positive, got %d", names[i], v[i]);
+  if (d.dtype != MLA_BF16 && d.dtype != MLA_F32)
+    return fail(MLA_ERR_INVALID, "dims.dtype must be MLA_BF16 or MLA_F32, got %d", d.dtype);
+  if (d.R + d.Dr > 16384) return fail(MLA_ERR_UNSUPPORTED, "R + Dr = %d is too wide", d.R + d.Dr);
+  return MLA_OK;
+}
+
+size_t elem_size(const mla_dims& d) { return d.dtype == MLA_BF16 ? 2 : 4; }
+
+// Geometry the tensor-core decode kernel is written for.
+bool decode_tc_ok(const mla_dims& d) {
+  return d.dtype == MLA_BF16 && d.R == mla::tc::kR && d.Dr == mla::tc::kDr &&
+         d.page_size == mla::tc::kPage && d.H % mla::tc::kHeads == 0;
+}
+
+bool use_tc_decode(const mla_dims& d) {
+  const int32_t pol = g_policy.load();
+  return pol != MLA_POLICY_SIMT && decode_tc_ok(d);
+}
+
+cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
+
+mla_status launch_check(const char* what) {
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return fail(MLA_ERR_CUDA, "launch of %s failed: %s", what, cudaGetErrorString(e));
+  return ok();
+}
+
+// ---------------------------------------------------------------- TMA descriptors
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*,
+                                  CUtensorMapInterleave, CUtensorMapSwizzle, CUtensorMapL2promotion,
+                                  CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// 2D bf16 tensor [rows][cols] (row pitch `pitch_bytes`), box = 64 rows x 64 cols,
+// 128-byte swizzle, zero fill out of bounds.
+mla_status make_map_2d(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows, uint64_t pitch_bytes) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return fail(MLA_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+  if (reinterpret_cast<uintptr_t>(base) % 16 != 0)
+    return fail(MLA_ERR_INVALID, "tensor base %p is not 16-byte aligned", base);
+  const cuuint64_t dims[2] = {cols, rows};
+  const cuuint64_t strides[1] = {pitch_bytes};
+  const cuuint32_t box[2] = {64, 64};
+  const cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(MLA_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+  return MLA_OK;
+}
+
+// Per-device one-time kernel attributes (large dynamic shared memory).
+mla_status ensure_smem_attr(const void* kernel, int bytes) {
+  static std::mutex mu;
+  static std::vector<std::pair<const void*, int>> done;  // (kernel, device)
+  int dev = 0;
+  MLA_CUDA_TRY(cudaGetDevice(&dev));
+  std::lock_guard<std::mutex> lk(mu);
+  for (auto& e : done)
+    if (e.first == kernel && e.second == dev) return MLA_OK;
+  MLA_CUDA_TRY(cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes));
+  done.emplace_back(kernel, dev);
+  return MLA_OK;
+}
+
+int32_t head_groups_for(const mla_dims& d) {
+  return decode_tc_ok(d) ? d.H / mla::tc::kHeads : 1;
+}
+
+}  // namespace
+
+// =============================================================================== C ABI
+extern "C" {
+
+int32_t mla_abi_version(void) { return MLA_ABI_VERSION; }
+
+const char* mla_last_error(void) { return g_last_error.c_str(); }
+
+mla_status mla_set_policy(int32_t policy) {
+  if (policy < MLA_POLICY_AUTO || policy > MLA_POLICY_TCGEN05)
+    return fail(MLA_ERR_INVALID, "unknown policy %d", policy);
+  g_policy.store(policy);
+  return ok();
+}
+
+mla_status mla_set_wait_timeout_ns(uint64_t ns) {
+  if (ns == 0) return fail(MLA_ERR_INVALID, "timeout must be positive");
+  g_timeout_ns.store(ns);
+  return ok();
+}
+
+mla_status mla_check_status(void* stream) {
+  MLA_CUDA_TRY(cudaStreamSynchronize(as_stream(stream)));
+  unsigned int v = 0, zero = 0;
+  MLA_CUDA_TRY(cudaMemcpyFromSymbol(&v, mla::g_status, sizeof(v)));
+  MLA_CUDA_TRY(cudaMemcpyToSymbol(mla::g_status, &zero, sizeof(zero)));
+  if (v & mla::kStatusTimeout) return fail(MLA_ERR_TIMEOUT, "a kernel wait ran out (status 0x%x)", v);
+  if (v & mla::kStatusBadPage)
+    return fail(MLA_ERR_INVALID, "a block_table entry was outside [0, num_pages) (status 0x%x)", v);
+  return ok();
+}
+
+// ------------------------------------------------------------------------------- append
+mla_status mla_cache_append(void* kv_cache, const int32_t* block_table, const int32_t* seq_lens,
+                            const void* new_ckr, int32_t B, int32_t q_len, int32_t max_pages,
+                            int32_t num_pages, mla_dims d, void* stream) {
+  if (mla_status s = check_dims(d)) return s;
+  if (B < 0 || q_len <= 0 || max_pages <= 0 || num_pages <= 0)
+    return fail(MLA_ERR_INVALID, "bad sizes B=%d q_len=%d max_pages=%d num_pages=%d", B, q_len, max_pages,
+                num_pages);
+  if (B == 0) return ok();
+  if (!kv_cache || !block_table || !seq_lens || !new_ckr) return fail(MLA_ERR_INVALID, "null pointer");
+  const int32_t row = d.R + d.Dr;
+  const dim3 grid(B * q_len);
+  if (d.dtype == MLA_BF16)
+    mla::simt::cache_append_kernel<__nv_bfloat16><<<grid, 128, 0, as_stream(stream)>>>(
+        static_cast<__nv_bfloat16*>(kv_cache), block_table, seq_lens,
+        static_cast<const __nv_bfloat16*>(new_ckr), q_len, max_pages, num_pages, row, d.page_size);
+  else
+    mla::simt::cache_append_kernel<float><<<grid, 128, 0, as_stream(stream)>>>(
+        static_cast<float*>(kv_cache), block_table, seq_lens, static_cast<const float*>(new_ckr), q_len,
+        max_pages, num_pages, row, d.page_size);
+  return launch_check("cache_append");
+}
+
+// ------------------------------------------------------------------------------- absorb
+mla_status mla_absorb_q(const void* q_nope, const void* W_UK, void* q_lat, int32_t T, mla_dims d,
+                        void* stream) {
+  if (mla_status s = check_dims(d)) return s;
+  if (T < 0) return fail(MLA_ERR_INVALID, "T=%d", T);
+  if (T == 0) return ok();
+  if (!q_nope || !W_UK || !q_lat) return fail(MLA_ERR_INVALID, "null pointer");
+  if (g_policy.load() == MLA_POLICY_TCGEN05)
+    return fail(MLA_ERR_UNSUPPORTED, "no tensor-core absorb kernel in this build");
+  const dim3 grid((d.R + 127) / 128, d.H, (T + mla::simt::kTT - 1) / mla::simt::kTT);
+  const size_t smem = sizeof(float) * mla::simt::kTT * d.Dn;
+  if (smem > 48 * 1024) return fail(MLA_ERR_UNSUPPORTED, "Dn=%d too large", d.Dn);
+  if (d.dtype == MLA_BF16)
+    mla::simt::absorb_kernel<__nv_bfloat16><<<grid, 128, smem, as_stream(stream)>>>(
+        static_cast<const __nv_bfloat16*>(q_nope), static_cast<const __nv_bfloat16*>(W_UK),
+        static_cast<__nv_bfloat16*>(q_lat), T, d.H, d.Dn, d.R);
+  else
+    mla::simt::absorb_kernel<float><<<grid, 128, smem, as_stream(stream)>>>(
+        static_cast<const float*>(q_nope), static_cast<const float*>(W_UK), static_cast<float*>(q_lat), T,
+        d.H, d.Dn, d.R);
+  return launch_check("absorb_q");
+}
+
+// ------------------------------------------------------------------------------- out proj
+mla_status mla_out_proj(const void* o_lat, const void* W_UV, void* out, int32_t T, mla_dims d,
+                        void* stream) {
+  if (mla_status s = check_dims(d)) return s;
+  if (T < 0) return fail(MLA_ERR_INVALID, "T=%d", T);
+  if (T == 0) return ok();
+  if (!o_lat || !W_UV || !out) return fail(MLA_ERR_INVALID, "null pointer");
+  if (g_policy.load() == MLA_POLICY_TCGEN05)
+    return fail(MLA_ERR_UNSUPPORTED, "no tensor-core output-projection kernel in this build");
+  const dim3 grid(d.H, (T + mla::simt::kTT - 1) / mla::simt::kTT);
+  const size_t smem = sizeof(float) * mla::simt::kTT * d.R;
+  if (smem > 48 * 1024) return fail(MLA_ERR_UNSUPPORTED, "R=%d too large", d.R);
+  if (d.dtype == MLA_BF16)
+    mla::simt::outproj_kernel<__nv_bfloat16><<<grid, 256, smem, as_stream(stream)>>>(
+        static_cast<const __nv_bfloat16*>(o_lat), static_cast<const __nv_bfloat16*>(W_UV),
+        static_cast<__nv_bfloat16*>(out), T, d.H, d.Dv, d.R);
+  else
+    mla::simt::outproj_kernel<float><<<grid, 256, smem, as_stream(stream)>>>(
+        static_cast<const float*>(o_lat), static_cast<const float*>(W_UV), static_cast<float*>(out), T, d.H,
+        d.Dv, d.R);
+  return launch_check("out_proj");
+}
+
+// ------------------------------------------------------------------------------- planning
+size_t mla_plan_capacity(int32_t B, int32_t q_len, int32_t num_sms) {
+  if (B < 0 || q_len <= 0 || num_sms <= 0) return 0;
+  const size_t items = (size_t)B * q_len;
+  const size_t slots = (size_t)num_sms;
+  const size_t units = items + slots + 1;
+  return mla::kPlanHeader + mla::kUnitWords * units + (slots + 1) + 2 * items;
+}
+
+mla_status mla_plan_splits(const int32_t* seq_lens_host, int32_t B, int32_t q_len, int32_t max_pages,
+                           mla_dims d, int32_t num_sms, int32_t* plan_host, size_t capacity,
+                           mla_plan_info* info) {
+  if (mla_status s = check_dims(d)) return s;
+  if (B < 0 || q_len <= 0 || max_pages <= 0 || num_sms <= 0)
+    return fail(MLA_ERR_INVALID, "bad sizes B=%d q_len=%d max_pages=%d num_sms=%d", B, q_len, max_pages,
+                num_sms);
+  if ((B > 0 && !seq_lens_host) || !plan_host || !info) return fail(MLA_ERR_INVALID, "null pointer");
+  if (capacity < mla_plan_capacity(B, q_len, num_sms))
+    return fail(MLA_ERR_WORKSPACE, "plan capacity %zu < %zu words", capacity,
+                mla_plan_capacity(B, q_len, num_sms));
+  const int32_t ps = d.page_size;
+  const int32_t G = head_groups_for(d);
+  const int32_t slots_max = std::max(1, num_sms / G);
+  const int32_t items = B * q_len;
+  std::vector<int32_t> pages(items);
+  int64_t total = 0;
+  for (int32_t b = 0; b < B; ++b) {
+    const int32_t L = seq_lens_host[b];
+    if (L < 0 || (int64_t)L > (int64_t)max_pages * ps)
+      return fail(MLA_ERR_INVALID, "seq_lens[%d]=%d outside [0, max_pages*page_size=%lld]", b, L,
+                  (long long)max_pages * ps);
+    for (int32_t i = 0; i < q_len; ++i) {
+      const int32_t n = mla::visible_tokens(L, q_len, i);
+      pages[b * q_len + i] = (n + ps - 1) / ps;
+      total += pages[b * q_len + i];
+    }
+  }
+  // Slot s covers flattened pages [s*total/S, (s+1)*total/S): page counts differ by at most one.
+  const int64_t S = std::max<int64_t>(1, std::min<int64_t>(slots_max, total));
+  auto bound = [&](int64_t s) { return s * total / S; };
+  struct U { int32_t item, b, pb, pe, slot; };
+  std::vector<U> units;
+  units.reserve(items + S);
+  int32_t slot = 0;
+  int64_t flat = 0;  // flattened index of the next page
+  for (int32_t it = 0; it < items; ++it) {
+    const int32_t b = it / q_len;
+    int32_t left = pages[it], pb = 0;
+    if (left == 0) {
+      units.push_back({it, b, 0, 0, slot});
+      continue;
+    }
+    while (left > 0) {
+      while (slot + 1 < S && flat >= bound(slot + 1)) ++slot;
+      const int64_t room = (slot + 1 < S) ? bound(slot + 1) - flat : left;
+      const int32_t take = (int32_t)std::min<int64_t>(left, room);
+      units.push_back({it, b, pb, pb + take, slot});
+      pb += take;
+      left -= take;
+      flat += take;
+    }
+  }
+  const int32_t num_slots = units.empty() ? 0 : units.back().slot + 1;
+  // parts: items with more than one unit
+  std::vector<int32_t> count(items, 0);
+  for (const U& u : units) count[u.item]++;
+  std::vector<int32_t> first(items, -1);
+  int32_t parts = 0;
+  for (int32_t it = 0; it < items; ++it)
+    if (count[it] > 1) {
+      first[it] = parts;
+      parts += count[it];
+    }
+  const size_t words = mla::kPlanHeader + mla::kUnitWords * units.size() + (num_slots + 1) + 2 * (size_t)items;
+  if (words > capacity) return fail(MLA_ERR_WORKSPACE, "plan needs %zu words", words);
+  std::memset(plan_host, 0, words * sizeof(int32_t));
+  plan_host[0] = mla::kPlanMagic;
+  plan_host[1] = B;
+  plan_host[2] = q_len;
+  plan_host[3] = (int32_t)units.size();
+  plan_host[4] = num_slots;
+  plan_host[5] = parts;
+  plan_host[6] = G;
+  plan_host[7] = d.H;
+  plan_host[8] = ps;
+  int32_t* uw = plan_host + mla::kPlanHeader;
+  std::vector<int32_t> next(items, 0);
+  for (size_t k = 0; k < units.size(); ++k) {
+    const U& u = units[k];
+    int32_t part = -1;
+    if (count[u.item] > 1) part = first[u.item] + next[u.item]++;
+    int32_t* w = uw + mla::kUnitWords * k;
+    w[0] = u.item;
+    w[1] = u.b;
+    w[2] = u.pb;
+    w[3] = u.pe;
+    w[4] = part;
+    w[5] = u.slot;
+  }
+  int32_t* sb = uw + mla::kUnitWords * units.size();
+  {
+    size_t k = 0;  // units are ordered by slot: sb[s] = first unit of slot s
+    for (int32_t s = 0; s <= num_slots; ++s) {
+      while (k < units.size() && units[k].slot < s) ++k;
+      sb[s] = (int32_t)k;
+    }
+  }
+  int32_t* ip = sb + num_slots + 1;
+  for (int32_t it = 0; it < items; ++it) {
+    ip[2 * it] = count[it] > 1 ? first[it] : -1;
+    ip[2 * it + 1] = count[it] > 1 ? count[it] : 0;
+  }
+  info->num_items = items;
+  info->num_units = (int32_t)units.size();
+  info->num_slots = num_slots;
+  info->num_parts = parts;
+  info->head_groups = G;
+  info->plan_words = (int32_t)words;
+  return ok();
+}
+
+size_t mla_workspace_size(const mla_plan_info* info, mla_dims d) {
+  if (!info || check_dims(d) != MLA_OK) return 0;
+  const size_t parts = (size_t)std::max(0, info->num_parts);
+  size_t o = parts * d.H * d.R * sizeof(float);
+  o = (o + 255) / 256 * 256;
+  return o + parts * d.H * sizeof(float);
+}
+
+static mla_status split_workspace(const mla_plan_info* info, const mla_dims& d, void* ws, size_t bytes,
+                                  float** o_part, float** lse_part) {
+  *o_part = nullptr;
+  *lse_part = nullptr;
+  if (info->num_parts == 0) return MLA_OK;
+  const size_t need = mla_workspace_size(info, d);
+  if (!ws || bytes < need) return fail(MLA_ERR_WORKSPACE, "workspace %zu bytes < %zu needed", bytes, need);
+  if (reinterpret_cast<uintptr_t>(ws) % 256 != 0) return fail(MLA_ERR_INVALID, "workspace not 256-byte aligned");
+  size_t o = (size_t)info->num_parts * d.H * d.R * sizeof(float);
+  o = (o + 255) / 256 * 256;
+  *o_part = static_cast<float*>(ws);
+  *lse_part = reinterpret_cast<float*>(static_cast<char*>(ws) + o);
+  return MLA_OK;
+}
+
+static mla_status check_info(const mla_plan_info* info, int32_t B, int32_t q_len, const mla_dims& d) {
+  if (!info) return fail(MLA_ERR_INVALID, "null plan info");
+  if (info->num_items != B * q_len)
+    return fail(MLA_ERR_INVALID, "plan covers %d query tokens, call has %d", info->num_items, B * q_len);
+  if (info->head_groups != head_groups_for(d))
+    return fail(MLA_ERR_INVALID, "plan was made for %d head groups, dims need %d", info->head_groups,
+                head_groups_for(d));
+  return MLA_OK;
+}
+
+// ------------------------------------------------------------------------------- decode
+mla_status mla_decode_attn(const void* q_lat, const void* q_rope, const void* kv_cache,
+                           const int32_t* block_table, const int32_t* seq_lens, int32_t B,
+                           int32_t q_len, int32_t max_pages, int32_t num_pages, float scale,
+                           const int32_t* plan_dev, const mla_plan_info* info, void* o_lat,
+                           float* lse, void* workspace, size_t workspace_bytes, mla_dims d,
+                           void* stream) {
+  if (mla_status s = check_dims(d)) return s;
+  if (B < 0 || q_len <= 0 || max_pages <= 0 || num_pages <= 0)
+    return fail(MLA_ERR_INVALID, "bad sizes B=%d q_len=%d max_pages=%d num_pages=%d", B, q_len, max_pages,
+                num_pages);
+  if (!(scale > 0.f) || !std::isfinite(scale)) return fail(MLA_ERR_INVALID, "scale must be positive");
+  if (mla_status s = check_info(info, B, q_len, d)) return s;
+  if (B == 0 || info->num_units == 0) return ok();
+  if (!q_lat || !q_rope || !kv_cache || !block_table || !seq_lens || !plan_dev || !o_lat)
+    return fail(MLA_ERR_INVALID, "null pointer");
+  float *o_part, *lse_part;
+  if (mla_status s = split_workspace(info, d, workspace, workspace_bytes, &o_part, &lse_part)) return s;
+  const int32_t pol = g_policy.load();
+  if (pol == MLA_POLICY_TCGEN05 && !decode_tc_ok(d))
+    return fail(MLA_ERR_UNSUPPORTED, "tensor-core decode needs bf16, R=512, Dr=64, page_size=64, H%%64==0");
+  cudaStream_t st = as_stream(stream);
+  if (use_tc_decode(d)) {
+    const int64_t T = (int64_t)B * q_len;
+    CUtensorMap tq, tr, tk;
+    if (mla_status s = make_map_2d(&tq, q_lat, d.R, (uint64_t)T * d.H, (uint64_t)d.R * 2)) return s;
+    if (mla_status s = make_map_2d(&tr, q_rope, d.Dr, (uint64_t)T * d.H, (uint64_t)d.Dr * 2)) return s;
+    if (mla_status s = make_map_2d(&tk, kv_cache, d.R + d.Dr, (uint64_t)num_pages * d.page_size,
+                                   (uint64_t)(d.R + d.Dr) * 2))
+      return s;
+    if (mla_status s = ensure_smem_attr((const void*)mla::tc::decode_kernel, mla::tc::kSmemBytes)) return s;
+    mla::tc::Params p;
+    p.plan = plan_dev;
+    p.block_table = block_table;
+    p.seq_lens = seq_lens;
+    p.max_pages = max_pages;
+    p.num_pages = num_pages;
+    p.H = d.H;
+    p.scale_log2 = scale * 1.4426950408889634f;
+    p.o_lat = static_cast<__nv_bfloat16*>(o_lat);
+    p.lse = lse;
+    p.o_part = o_part;
+    p.lse_part = lse_part;
+    p.timeout_ns = g_timeout_ns.load();
+    const dim3 grid(info->num_slots * info->head_groups);
+    mla::tc::decode_kernel<<<grid, 256, mla::tc::kSmemBytes, st>>>(tq, tr, tk, p);
+    return launch_check("decode_attn (tcgen05)");
+  }
+  mla::simt::DecodeSimtArgs a;
+  a.plan = plan_dev;
+  a.block_table = block_table;
+  a.seq_lens = seq_lens;
+  a.max_pages = max_pages;
+  a.num_pages = num_pages;
+  a.H = d.H;
+  a.R = d.R;
+  a.Dr = d.Dr;
+  a.page_size = d.page_size;
+  a.scale = scale;
+  a.o_lat = o_lat;
+  a.lse = lse;
+  a.o_part = o_part;
+  a.lse_part = lse_part;
+  const size_t smem = sizeof(float) * ((size_t)(d.R + d.Dr) + 4 * (size_t)d.R + 8);
+  if (smem > 200 * 1024) return fail(MLA_ERR_UNSUPPORTED, "R=%d too large for the SIMT decode", d.R);
+  const dim3 grid(info->num_units, d.H);
+  if (d.dtype == MLA_BF16) {
+    if (mla_status s = ensure_smem_attr((const void*)mla::simt::decode_kernel<__nv_bfloat16>, (int)smem)) return s;
+    mla::simt::decode_kernel<__nv_bfloat16><<<grid, 128, smem, st>>>(
+        static_cast<const __nv_bfloat16*>(q_lat), static_cast<const __nv_bfloat16*>(q_rope),
+        static_cast<const __nv_bfloat16*>(kv_cache), a);
+  } else {
+    if (mla_status s = ensure_smem_attr((const void*)mla::simt::decode_kernel<float>, (int)smem)) return s;
+    mla::simt::decode_kernel<float><<<grid, 128, smem, st>>>(static_cast<const float*>(q_lat),
+                                                             static_cast<const float*>(q_rope),
+                                                             static_cast<const float*>(kv_cache), a);
+  }
+  return launch_check("decode_attn (SIMT)");
+}
+
+// ------------------------------------------------------------------------------- combine
+mla_status mla_combine(const int32_t* plan_dev, const mla_plan_info* info, const void* workspace,
+                       size_t workspace_bytes, void* o_lat, float* lse, mla_dims d, void* stream) {
+  if (mla_status s = check_dims(d)) return s;
+  if (!info) return fail(MLA_ERR_INVALID, "null plan info");
+  if (info->num_parts == 0) return ok();
+  if (!plan_dev || !o_lat) return fail(MLA_ERR_INVALID, "null pointer");
+  float *o_part, *lse_part;
+  if (mla_status s = split_workspace(info, d, const_cast<void*>(workspace), workspace_bytes, &o_part, &lse_part))
+    return s;
+  const dim3 grid(info->num_items, d.H);
+  if (d.dtype == MLA_BF16)
+    mla::simt::combine_kernel<__nv_bfloat16><<<grid, 128, 0, as_stream(stream)>>>(
+        plan_dev, o_part, lse_part, static_cast<__nv_bfloat16*>(o_lat), lse, d.H, d.R);
+  else
+    mla::simt::combine_kernel<float><<<grid, 128, 0, as_stream(stream)>>>(plan_dev, o_part, lse_part,
+                                                                           static_cast<float*>(o_lat), lse,
+                                                                           d.H, d.R);
+  return launch_check("combine");
+}
+
+}  // extern "C"

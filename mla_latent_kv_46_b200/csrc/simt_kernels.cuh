@@ -1,0 +1,224 @@
+// simt_kernels.cuh -- CUDA-core kernels of every step, for any geometry and for
+// fp32 as well as bf16 storage. The tensor-core kernels replace some of them
+// where the geometry allows (see decode_tc.cuh, gemm_tc.cuh).
+#pragma once
+
+#include "common.cuh"
+
+namespace mla {
+namespace simt {
+
+// ------------------------------------------------------------------ a2: cache append
+// One block per new row: kv[page][pos % ps][:] = new_ckr[b*q_len + i][:].
+template <typename T>
+__global__ void cache_append_kernel(T* __restrict__ kv, const int32_t* __restrict__ block_table,
+                                    const int32_t* __restrict__ seq_lens,
+                                    const T* __restrict__ new_ckr, int32_t q_len, int32_t max_pages,
+                                    int32_t num_pages, int32_t row, int32_t page_size) {
+  const int32_t item = blockIdx.x;
+  const int32_t b = item / q_len, i = item % q_len;
+  const int32_t pos = seq_lens[b] - q_len + i;
+  if (pos < 0) return;
+  const int32_t pidx = pos / page_size;
+  if (pidx >= max_pages) {
+    if (threadIdx.x == 0) raise_status(kStatusBadPage);
+    return;
+  }
+  const int32_t page = block_table[(int64_t)b * max_pages + pidx];
+  if (page < 0 || page >= num_pages) {
+    if (threadIdx.x == 0) raise_status(kStatusBadPage);
+    return;
+  }
+  T* dst = kv + ((int64_t)page * page_size + pos % page_size) * row;
+  const T* src = new_ckr + (int64_t)item * row;
+  for (int32_t e = threadIdx.x; e < row; e += blockDim.x) dst[e] = src[e];
+}
+
+// ------------------------------------------------------------------ a1: absorb
+// q_lat[t][h][r] = sum_n q_nope[t][h][n] * W_UK[h][n][r]
+// grid (ceil(R/128), H, ceil(T/kTT)), block 128: thread = one r, kTT tokens.
+constexpr int kTT = 8;
+template <typename T>
+__global__ void absorb_kernel(const T* __restrict__ qn, const T* __restrict__ w, T* __restrict__ ql,
+                              int32_t T_, int32_t H, int32_t Dn, int32_t R) {
+  extern __shared__ float sq[];  // [kTT][Dn]
+  const int32_t h = blockIdx.y, t0 = blockIdx.z * kTT;
+  const int32_t r = blockIdx.x * blockDim.x + threadIdx.x;
+  for (int32_t e = threadIdx.x; e < kTT * Dn; e += blockDim.x) {
+    const int32_t t = t0 + e / Dn, n = e % Dn;
+    sq[e] = t < T_ ? to_f32(qn[((int64_t)t * H + h) * Dn + n]) : 0.f;
+  }
+  __syncthreads();
+  if (r >= R) return;
+  float acc[kTT];
+#pragma unroll
+  for (int k = 0; k < kTT; ++k) acc[k] = 0.f;
+  const T* wp = w + (int64_t)h * Dn * R + r;
+  for (int32_t n = 0; n < Dn; ++n) {
+    const float wv = to_f32(wp[(int64_t)n * R]);
+#pragma unroll
+    for (int k = 0; k < kTT; ++k) acc[k] = fmaf(sq[k * Dn + n], wv, acc[k]);
+  }
+#pragma unroll
+  for (int k = 0; k < kTT; ++k)
+    if (t0 + k < T_) ql[((int64_t)(t0 + k) * H + h) * R + r] = from_f32<T>(acc[k]);
+}
+
+// ------------------------------------------------------------------ a7: output projection
+// out[t][h][v] = sum_r W_UV[h][v][r] * o_lat[t][h][r]
+// grid (H, ceil(T/kTT)), block 256: the kTT latent rows in shared memory, one warp per v.
+template <typename T>
+__global__ void outproj_kernel(const T* __restrict__ ol, const T* __restrict__ w, T* __restrict__ out,
+                               int32_t T_, int32_t H, int32_t Dv, int32_t R) {
+  extern __shared__ float so[];  // [kTT][R]
+  const int32_t h = blockIdx.x, t0 = blockIdx.y * kTT;
+  for (int32_t e = threadIdx.x; e < kTT * R; e += blockDim.x) {
+    const int32_t t = t0 + e / R, r = e % R;
+    so[e] = t < T_ ? to_f32(ol[((int64_t)t * H + h) * R + r]) : 0.f;
+  }
+  __syncthreads();
+  const int32_t warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nwarp = blockDim.x >> 5;
+  for (int32_t v = warp; v < Dv; v += nwarp) {
+    const T* wp = w + ((int64_t)h * Dv + v) * R;
+    float acc[kTT];
+#pragma unroll
+    for (int k = 0; k < kTT; ++k) acc[k] = 0.f;
+    for (int32_t r = lane; r < R; r += 32) {
+      const float wv = to_f32(wp[r]);
+#pragma unroll
+      for (int k = 0; k < kTT; ++k) acc[k] = fmaf(wv, so[k * R + r], acc[k]);
+    }
+#pragma unroll
+    for (int k = 0; k < kTT; ++k) {
+      const float s = warp_sum(acc[k]);
+      if (lane == 0 && t0 + k < T_) out[((int64_t)(t0 + k) * H + h) * Dv + v] = from_f32<T>(s);
+    }
+  }
+}
+
+// ------------------------------------------------------------------ a3-a5: decode attention
+// grid (num_units, H), block 128. Each warp runs an online softmax over every
+// 4th visible token of the unit; the four warp states are merged at the end.
+struct DecodeSimtArgs {
+  const int32_t* plan;
+  const int32_t* block_table;
+  const int32_t* seq_lens;
+  int32_t max_pages, num_pages, H, R, Dr, page_size;
+  float scale;
+  void* o_lat;
+  float* lse;
+  float* o_part;
+  float* lse_part;
+};
+
+template <typename T>
+__global__ void decode_kernel(const T* __restrict__ q_lat, const T* __restrict__ q_rope,
+                              const T* __restrict__ kv, DecodeSimtArgs a) {
+  extern __shared__ float smem[];
+  const int32_t row = a.R + a.Dr;
+  float* qs = smem;                   // [row]
+  float* os = qs + row;               // [4][R]
+  float* ms = os + 4 * a.R;           // [4]
+  float* ls = ms + 4;                 // [4]
+  const PlanView plan{a.plan};
+  const Unit u = plan.units()[blockIdx.x];
+  const int32_t h = blockIdx.y;
+  const int32_t q_len = plan.q_len();
+  const int32_t L = a.seq_lens[u.b];
+  const int32_t n = visible_tokens(L, q_len, u.item % q_len);
+  const int32_t tb = u.page_begin * a.page_size;
+  const int32_t te = min(u.page_end * a.page_size, n);
+  const int32_t warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  for (int32_t e = threadIdx.x; e < row; e += blockDim.x)
+    qs[e] = e < a.R ? to_f32(q_lat[((int64_t)u.item * a.H + h) * a.R + e])
+                    : to_f32(q_rope[((int64_t)u.item * a.H + h) * a.Dr + (e - a.R)]);
+  float* ow = os + warp * a.R;
+  for (int32_t e = lane; e < a.R; e += 32) ow[e] = 0.f;
+  __syncthreads();
+
+  float m = -CUDART_INF_F, l = 0.f;
+  for (int32_t t = tb + warp; t < te; t += 4) {
+    const int32_t page = a.block_table[(int64_t)u.b * a.max_pages + t / a.page_size];
+    if (page < 0 || page >= a.num_pages) {
+      if (lane == 0) raise_status(kStatusBadPage);
+      continue;
+    }
+    const T* rp = kv + ((int64_t)page * a.page_size + t % a.page_size) * row;
+    float part = 0.f;
+    for (int32_t e = lane; e < row; e += 32) part = fmaf(qs[e], to_f32(rp[e]), part);
+    const float x = warp_sum(part) * a.scale;
+    const float m_new = fmaxf(m, x);
+    const float corr = expf(m - m_new);  // 0 on the first token (m = -inf)
+    const float p = expf(x - m_new);
+    l = l * corr + p;
+    for (int32_t e = lane; e < a.R; e += 32) ow[e] = fmaf(p, to_f32(rp[e]), ow[e] * corr);
+    m = m_new;
+  }
+  if (lane == 0) {
+    ms[warp] = m;
+    ls[warp] = l;
+  }
+  __syncthreads();
+  float M = fmaxf(fmaxf(ms[0], ms[1]), fmaxf(ms[2], ms[3]));
+  float wgt[4], tot = 0.f;
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    wgt[k] = (M == -CUDART_INF_F) ? 0.f : expf(ms[k] - M);
+    tot += wgt[k] * ls[k];
+  }
+  const float inv = tot > 0.f ? 1.f / tot : 0.f;
+  const float lse_v = tot > 0.f ? M + logf(tot) : -CUDART_INF_F;
+  if (u.part < 0) {
+    T* dst = reinterpret_cast<T*>(a.o_lat) + ((int64_t)u.item * a.H + h) * a.R;
+    for (int32_t e = threadIdx.x; e < a.R; e += blockDim.x) {
+      float s = 0.f;
+#pragma unroll
+      for (int k = 0; k < 4; ++k) s = fmaf(wgt[k], os[k * a.R + e], s);
+      dst[e] = from_f32<T>(s * inv);
+    }
+    if (threadIdx.x == 0 && a.lse) a.lse[(int64_t)u.item * a.H + h] = lse_v;
+  } else {
+    float* dst = a.o_part + ((int64_t)u.part * a.H + h) * a.R;
+    for (int32_t e = threadIdx.x; e < a.R; e += blockDim.x) {
+      float s = 0.f;
+#pragma unroll
+      for (int k = 0; k < 4; ++k) s = fmaf(wgt[k], os[k * a.R + e], s);
+      dst[e] = s * inv;
+    }
+    if (threadIdx.x == 0) a.lse_part[(int64_t)u.part * a.H + h] = lse_v;
+  }
+}
+
+// ------------------------------------------------------------------ a6: split-KV combine
+// grid (num_items, H), block 128. Items computed by a single unit are skipped.
+template <typename T>
+__global__ void combine_kernel(const int32_t* __restrict__ plan_w, const float* __restrict__ o_part,
+                               const float* __restrict__ lse_part, T* __restrict__ o_lat,
+                               float* __restrict__ lse, int32_t H, int32_t R) {
+  const PlanView plan{plan_w};
+  const int32_t item = blockIdx.x, h = blockIdx.y;
+  const int32_t first = plan.item_parts()[2 * item], np = plan.item_parts()[2 * item + 1];
+  if (np == 0) return;
+  float M = -CUDART_INF_F;
+  for (int32_t s = 0; s < np; ++s) M = fmaxf(M, lse_part[(int64_t)(first + s) * H + h]);
+  float tot = 0.f;
+  for (int32_t s = 0; s < np; ++s) {
+    const float z = lse_part[(int64_t)(first + s) * H + h];
+    tot += (M == -CUDART_INF_F) ? 0.f : expf(z - M);
+  }
+  const float inv = tot > 0.f ? 1.f / tot : 0.f;
+  for (int32_t e = threadIdx.x; e < R; e += blockDim.x) {
+    float acc = 0.f;
+    for (int32_t s = 0; s < np; ++s) {
+      const float z = lse_part[(int64_t)(first + s) * H + h];
+      const float wgt = (M == -CUDART_INF_F) ? 0.f : expf(z - M);
+      if (wgt > 0.f) acc = fmaf(wgt, o_part[((int64_t)(first + s) * H + h) * R + e], acc);
+    }
+    o_lat[((int64_t)item * H + h) * R + e] = from_f32<T>(acc * inv);
+  }
+  if (threadIdx.x == 0 && lse) lse[(int64_t)item * H + h] = tot > 0.f ? M + logf(tot) : -CUDART_INF_F;
+}
+
+}  // namespace simt
+}  // namespace mla

@@ -239,3 +239,17 @@ def attention_flops(spec: WorkloadSpec, seq_lens: np.ndarray) -> int:
     """2*H*((R+Dr) + R) FLOP per (query, token) pair: scores over the 576-wide row,
     then the latent value sum over R."""
     return attention_pairs(spec, seq_lens) * 2 * spec.H * (spec.row + spec.R)
+
+
+def latent_queries(spec: WorkloadSpec, T: int, seed: int = 0) -> np.ndarray:
+    """Seeded stand-in for an absorbed query, [T, H, R] in storage dtype: entries
+    N(0, 0.5^2), the spread W_UK^T q_nope has with q_nope ~ N(0,1), W_UK std 1/sqrt(R)
+    and Dn = R/4 (the kernel-level decode tests feed it directly)."""
+    g = _rng(seed, 6)
+    return _store(spec, g.standard_normal((T, spec.H, spec.R), dtype=np.float32) * np.float32(0.5))
+
+
+def latent_outputs(spec: WorkloadSpec, T: int, seed: int = 0) -> np.ndarray:
+    """Seeded stand-in for a latent attention output, [T, H, R]: entries N(0, 0.1^2)."""
+    g = _rng(seed, 7)
+    return _store(spec, g.standard_normal((T, spec.H, spec.R), dtype=np.float32) * np.float32(0.1))

@@ -1,0 +1,164 @@
+"""Host-side checks of the C ABI (CPU only): symbols, planning, validation.
+
+Nothing here launches a kernel: every call below either is host-only
+(mla_plan_*, mla_workspace_size) or must fail validation before any launch.
+"""
+import ctypes
+import math
+import os
+import re
+
+import numpy as np
+import pytest
+
+import mla_latent_kv_46_b200 as mla
+from mla_latent_kv_46_b200 import workloads as wl
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "mla.h")
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(mla_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_library_exports_every_declared_symbol():
+    lib = ctypes.CDLL(mla.LIB_PATH)
+    names = declared_functions()
+    assert len(names) >= 13
+    for n in names:
+        assert hasattr(lib, n), n
+    assert sorted(mla.EXPORTS) == names
+
+
+def test_abi_version_and_error_text():
+    assert mla.mla_abi_version() == 1
+    with pytest.raises(mla.MlaError) as e:
+        mla.mla_set_policy(7)
+    assert e.value.status == mla._binding.MLA_ERR_INVALID
+    assert "policy" in mla.mla_last_error()
+
+
+def parse_plan(plan):
+    B, q_len, nu, ns, nparts, G, H, ps = (int(x) for x in plan[1:9])
+    assert plan[0] == 0x4D4C4131
+    units = plan[16:16 + 8 * nu].reshape(nu, 8)
+    sb = plan[16 + 8 * nu:16 + 8 * nu + ns + 1]
+    ip = plan[16 + 8 * nu + ns + 1:].reshape(-1, 2)
+    return dict(B=B, q_len=q_len, units=units, slot_begin=sb, item_parts=ip, num_parts=nparts, G=G, H=H, ps=ps)
+
+
+def dims(H=64, R=512, Dr=64, ps=64, dtype=mla.MLA_BF16):
+    return mla.Dims(H, 128, Dr, 128, R, ps, dtype)
+
+
+@pytest.mark.parametrize("q_len", [1, 3])
+@pytest.mark.parametrize("sms", [1, 7, 148])
+@pytest.mark.parametrize("H", [64, 128, 16])
+def test_plan_covers_every_visible_page_once(q_len, sms, H):
+    rng = np.random.default_rng(q_len * 1000 + sms + H)
+    lens = rng.integers(0, 700, size=9).astype(np.int32)
+    lens[0] = 0
+    lens[1] = max(lens[1], q_len)
+    max_pages = 12
+    d = dims(H=H)
+    plan, info = mla.mla_plan_splits(lens, len(lens), q_len, max_pages, d, sms)
+    p = parse_plan(plan)
+    G = H // 64 if H % 64 == 0 else 1
+    assert p["G"] == info.head_groups == G
+    assert info.num_slots <= max(1, sms // G)
+    cover = {}
+    for (item, b, pb, pe, part, slot, _, _) in p["units"]:
+        assert item // q_len == b
+        cover.setdefault(item, []).append((pb, pe, part, slot))
+    slots = p["units"][:, 5]
+    assert np.all(np.diff(slots) >= 0)
+    for s in range(info.num_slots):
+        assert np.all(slots[p["slot_begin"][s]:p["slot_begin"][s + 1]] == s)
+    parts_seen = set()
+    for item in range(len(lens) * q_len):
+        b, i = divmod(item, q_len)
+        n = max(0, int(lens[b]) - q_len + i + 1)
+        npg = math.ceil(n / 64)
+        segs = sorted(cover[item])
+        got = []
+        for pb, pe, part, slot in segs:
+            got.extend(range(pb, pe))
+        assert got == list(range(npg)), (item, segs)
+        first, cnt = p["item_parts"][item]
+        if len(segs) > 1:
+            assert cnt == len(segs)
+            assert sorted(s[2] for s in segs) == list(range(first, first + cnt))
+            parts_seen.update(s[2] for s in segs)
+        else:
+            assert cnt == 0 and segs[0][2] == -1
+    assert parts_seen == set(range(info.num_parts))
+
+
+def test_plan_balances_pages_over_slots():
+    lens = np.full(64, 4096, np.int32)
+    plan, info = mla.mla_plan_splits(lens, 64, 1, 64, dims(), 148)
+    p = parse_plan(plan)
+    per = np.zeros(info.num_slots, np.int64)
+    for u in p["units"]:
+        per[u[5]] += u[3] - u[2]
+    assert per.sum() == 64 * 64
+    assert per.max() <= math.ceil(4096 / 148)
+    assert info.num_slots == 148
+
+
+def test_plan_rejects_too_long_sequences_and_small_buffers():
+    with pytest.raises(mla.MlaError) as e:
+        mla.mla_plan_splits(np.array([65], np.int32), 1, 1, 1, dims(), 148)
+    assert e.value.status == mla._binding.MLA_ERR_INVALID
+    info = mla.PlanInfo()
+    buf = np.zeros(4, np.int32)
+    st = mla._binding._lib.mla_plan_splits(np.array([5], np.int32).ctypes.data, 1, 1, 1, dims(), 148,
+                                           buf.ctypes.data, 4, ctypes.byref(info))
+    assert st == mla._binding.MLA_ERR_WORKSPACE
+
+
+def test_workspace_size_formula():
+    info = mla.PlanInfo(num_items=4, num_units=6, num_slots=3, num_parts=5, head_groups=1, plan_words=0)
+    d = dims(H=16, R=32)
+    o = 5 * 16 * 32 * 4
+    assert mla.mla_workspace_size(info, d) == (o + 255) // 256 * 256 + 5 * 16 * 4
+
+
+@pytest.mark.parametrize("call", ["absorb", "out_proj", "append", "decode", "combine", "dims"])
+def test_invalid_arguments_fail_before_launch(call):
+    d = dims()
+    info = mla.PlanInfo(num_items=1, num_units=1, num_slots=1, num_parts=1, head_groups=1, plan_words=30)
+    with pytest.raises(mla.MlaError) as e:
+        if call == "absorb":
+            mla.mla_absorb_q(None, None, None, 4, d, stream=0)
+        elif call == "out_proj":
+            mla.mla_out_proj(None, 16, 16, 4, d, stream=0)
+        elif call == "append":
+            mla.mla_cache_append(16, 16, None, 16, 1, 1, 1, 1, d, stream=0)
+        elif call == "decode":   # plan made for 2 query tokens, call has 1
+            info.num_items = 2
+            mla.mla_decode_attn(16, 16, 16, 16, 16, 1, 1, 1, 1, 0.1, 16, info, 16, None, None, 0, d, stream=0)
+        elif call == "combine":  # parts but no workspace
+            mla.mla_combine(16, info, None, 0, 16, None, d, stream=0)
+        else:
+            mla.mla_absorb_q(16, 16, 16, 4, mla.Dims(64, 0, 64, 128, 512, 64, 0), stream=0)
+    assert e.value.status in (mla._binding.MLA_ERR_INVALID, mla._binding.MLA_ERR_WORKSPACE)
+
+
+def test_generator_streams_are_independent_of_batch_subset():
+    spec = wl.WORKLOADS["deepseek_h128_b128_ragged"]
+    lens = wl.seq_lens_of(spec)
+    assert lens.min() >= 512 and lens.max() <= 16384 and len(lens) == 128
+    a = wl.sequence_rows(wl.spec_with("kimi_h64_b64_l4096"), 5, 100)
+    b = wl.sequence_rows(wl.spec_with("kimi_h64_b64_l4096"), 5, 100)
+    assert np.array_equal(a, b) and a.dtype == np.uint16
+
+
+def test_bf16_rounding_is_nearest_even():
+    x = np.array([1.0, 1.0 + 2 ** -8, 1.0 + 3 * 2 ** -8, -2.5, 3.1415926], np.float32)
+    got = wl.bf16_bits_to_f32(wl.f32_to_bf16_bits(x))
+    assert got[0] == 1.0 and got[1] == 1.0 and got[2] == 1.0 + 2 ** -6 and got[3] == -2.5
+    assert abs(got[4] - 3.140625) < 1e-7

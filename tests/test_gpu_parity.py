@@ -1,0 +1,288 @@
+"""GPU parity: every libmla.so kernel against the fp64 oracle on the same seeded inputs.
+
+Tolerances (from the arithmetic, as the benchmark spec of this path sets them):
+bf16 storage with fp32 accumulation: |got - ref| <= 2e-3 + 1e-2 |ref| elementwise;
+fp32 storage: |got - ref| <= 1e-5. Cache append is bit-exact.
+
+Small cases span several pages and a ragged tail and include empty sequences; both
+kernel policies (SIMT CUDA cores, tcgen05 tensor cores) run where the geometry allows.
+The full-size workloads run in the launch configuration the benchmark times and are
+checked on sampled (query, head) outputs the oracle computes one by one.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import mla_latent_kv_46_b200 as mla
+from mla_latent_kv_46_b200 import decoder as dec
+from mla_latent_kv_46_b200 import workloads as wl
+from oracle import mla_oracle as orc
+
+pytestmark = pytest.mark.gpu
+
+POLICIES = {"simt": mla.MLA_POLICY_SIMT, "tcgen05": mla.MLA_POLICY_TCGEN05}
+
+
+@pytest.fixture(autouse=True)
+def _policy_reset():
+    yield
+    mla.mla_set_policy(mla.MLA_POLICY_AUTO)
+
+
+def host(t: torch.Tensor) -> np.ndarray:
+    return t.detach().float().cpu().numpy().astype(np.float64)
+
+
+def assert_close(got, ref, fp32, what=""):
+    got = np.asarray(got, np.float64)
+    ref = np.asarray(ref, np.float64)
+    assert got.shape == ref.shape, (what, got.shape, ref.shape)
+    ninf_r, ninf_g = np.isneginf(ref), np.isneginf(got)
+    assert np.array_equal(ninf_r, ninf_g), f"{what}: -inf pattern differs"
+    m = ~ninf_r
+    err = np.abs(got[m] - ref[m])
+    bound = 1e-5 if fp32 else 2e-3 + 1e-2 * np.abs(ref[m])
+    bad = err > bound
+    assert not np.any(np.isnan(got[m])), f"{what}: NaN in output"
+    assert not np.any(bad), (f"{what}: {bad.sum()} of {bad.size} outside tolerance; max err "
+                             f"{err.max():.3e}, worst ratio {(err / bound).max():.2f}")
+
+
+def small_spec(H=64, q_len=1, R=512, Dr=64, Dn=128, Dv=128, dtype="bf16", page=64, noise=0.0):
+    return wl.WorkloadSpec(name=f"small_h{H}_q{q_len}", B=0, H=H, R=R, Dr=Dr, Dn=Dn, Dv=Dv, q_len=q_len,
+                           dtype=dtype, seq_len=None, w_std=1.0 / math.sqrt(R), page_size=page,
+                           logit_noise_std=noise)
+
+
+# lengths: single token, one short of a page, exact page, one over, several pages
+# with a ragged tail, and an empty sequence
+SMALL_LENS = [1, 63, 64, 65, 333, 0]
+
+
+def make_case(spec, lens, seed=11, sms=None):
+    w = wl.make(spec, seed=seed, seq_lens=lens)
+    step = dec.DecodeStep(w, sms=sms)
+    return w, step
+
+
+def run_policy(policy):
+    mla.mla_set_policy(POLICIES[policy])
+
+
+# ----------------------------------------------------------------------------- a2: cache append
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_cache_append_bit_exact(dtype):
+    spec = small_spec(H=64, q_len=3, dtype=dtype) if dtype == "bf16" else \
+        small_spec(H=4, q_len=3, R=32, Dr=16, Dn=16, Dv=16, dtype="f32")
+    lens = [3, 70, 130, 64]
+    full = wl.make(spec, seed=5, seq_lens=lens)
+    empty = wl.make(spec, seed=5, seq_lens=lens, new_rows_in_cache=False)
+    step = dec.DecodeStep(empty)
+    step.append()
+    torch.cuda.synchronize()
+    mla.mla_check_status()
+    got = step.kv.view(torch.int16).cpu().numpy().view(np.uint16) if dtype == "bf16" else step.kv.cpu().numpy()
+    want = orc.cache_append(empty["kv_cache"], empty["block_table"], empty["seq_lens"], empty["new_ckr"],
+                            spec.q_len, spec.page_size)
+    assert np.array_equal(got, want)
+    assert np.array_equal(want, full["kv_cache"])
+
+
+# ----------------------------------------------------------------------------- a1 / a7
+
+@pytest.mark.parametrize("case", ["bf16_h64", "bf16_h128", "f32_tiny"])
+def test_absorb_q_matches_oracle(case):
+    if case == "f32_tiny":
+        w = wl.make("tiny_fp32")
+    else:
+        w = wl.make(small_spec(H=64 if case == "bf16_h64" else 128), seed=3, seq_lens=[5] * 37)
+    step = dec.DecodeStep(w)
+    step.absorb()
+    torch.cuda.synchronize()
+    ref = orc.absorb_q(w["q_nope"], w["W_UK"])
+    assert_close(host(step.q_lat), ref, w["spec"].dtype == "f32", "q_lat")
+
+
+@pytest.mark.parametrize("case", ["bf16_h64", "bf16_h128", "f32_tiny"])
+def test_out_proj_matches_oracle(case):
+    if case == "f32_tiny":
+        w = wl.make("tiny_fp32")
+    else:
+        w = wl.make(small_spec(H=64 if case == "bf16_h64" else 128), seed=4, seq_lens=[5] * 37)
+    spec = w["spec"]
+    step = dec.DecodeStep(w)
+    ol = wl.latent_outputs(spec, step.T, seed=4)
+    step.o_lat.copy_(dec.to_torch(ol, step.device))
+    step.project()
+    torch.cuda.synchronize()
+    ref = orc.out_proj(ol, w["W_UV"])
+    assert_close(host(step.out), ref, spec.dtype == "f32", "out")
+
+
+# ----------------------------------------------------------------------------- a3-a6: attention (+ combine)
+
+def attention_case(policy, H, q_len, lens, sms, noise=0.0):
+    run_policy(policy)
+    spec = small_spec(H=H, q_len=q_len, noise=noise)
+    w, step = make_case(spec, lens, sms=sms)
+    ql = wl.latent_queries(spec, step.T, seed=9)
+    step.q_lat.copy_(dec.to_torch(ql, step.device))
+    step.attend()
+    step.combine()
+    torch.cuda.synchronize()
+    mla.mla_check_status()
+    ref = orc.attend_latent(ql, w["q_rope"], w["kv_cache"], w["block_table"], w["seq_lens"], w["scale"],
+                            q_len=q_len, page_size=spec.page_size)
+    assert_close(host(step.o_lat), ref["o_lat"], False, "o_lat")
+    assert_close(host(step.lse), ref["lse"], False, "lse")
+    return step
+
+
+@pytest.mark.parametrize("policy", ["simt", "tcgen05"])
+@pytest.mark.parametrize("H", [64, 128])
+@pytest.mark.parametrize("sms", [148, 5])
+def test_decode_attention_matches_oracle(policy, H, sms):
+    step = attention_case(policy, H, 1, SMALL_LENS, sms)
+    if sms == 5:
+        assert step.info.num_parts > 0   # the combine ran
+
+
+@pytest.mark.parametrize("policy", ["simt", "tcgen05"])
+def test_causal_chunk_attention_matches_oracle(policy):
+    attention_case(policy, 64, 5, [70, 5, 129], 6)
+
+
+@pytest.mark.parametrize("policy", ["simt", "tcgen05"])
+def test_attention_with_large_logit_offsets(policy):
+    """Per-token logit noise of std 4 (the long-context workload's stress): the
+    reference maximum moves several times inside a unit."""
+    attention_case(policy, 64, 1, [1000, 777], 3, noise=4.0)
+
+
+def test_decode_fp32_tiny_matches_oracle():
+    w = wl.make("tiny_fp32")
+    spec = w["spec"]
+    step = dec.DecodeStep(w)
+    ql = wl.latent_queries(spec, step.T, seed=9)
+    step.q_lat.copy_(dec.to_torch(ql, step.device))
+    step.attend()
+    step.combine()
+    torch.cuda.synchronize()
+    ref = orc.attend_latent(ql, w["q_rope"], w["kv_cache"], w["block_table"], w["seq_lens"], w["scale"])
+    assert_close(host(step.o_lat), ref["o_lat"], True, "o_lat")
+    assert_close(host(step.lse), ref["lse"], True, "lse")
+
+
+def test_tcgen05_policy_rejects_unsupported_dims():
+    mla.mla_set_policy(mla.MLA_POLICY_TCGEN05)
+    w = wl.make(small_spec(H=32), seed=1, seq_lens=[10, 20])
+    step = dec.DecodeStep(w)
+    with pytest.raises(mla.MlaError) as e:
+        step.attend()
+    assert e.value.status == mla._binding.MLA_ERR_UNSUPPORTED
+
+
+# ----------------------------------------------------------------------------- whole step vs the definition
+
+@pytest.mark.parametrize("policy", ["simt", "tcgen05"])
+@pytest.mark.parametrize("H,q_len,lens,sms", [(64, 1, SMALL_LENS, 148), (128, 1, SMALL_LENS, 7),
+                                              (64, 4, [200, 4, 65], 9)])
+def test_whole_step_matches_nonabsorbed_definition(policy, H, q_len, lens, sms):
+    run_policy(policy)
+    spec = small_spec(H=H, q_len=q_len)
+    empty = wl.make(spec, seed=21, seq_lens=lens, new_rows_in_cache=False)
+    full = wl.make(spec, seed=21, seq_lens=lens)
+    step = dec.DecodeStep(empty, sms=sms)
+    step.run(append=True)
+    torch.cuda.synchronize()
+    mla.mla_check_status()
+    ref = orc.decode_nonabsorbed(full["q_nope"], full["q_rope"], full["kv_cache"], full["block_table"],
+                                 full["seq_lens"], full["W_UK"], full["W_UV"], full["scale"], q_len=q_len,
+                                 page_size=spec.page_size)
+    assert_close(host(step.out), ref["out"], False, "out")
+    assert_close(host(step.lse), ref["lse"], False, "lse")
+
+
+def test_whole_step_tiny_fp32_matches_definition():
+    w = wl.make("tiny_fp32")
+    step = dec.DecodeStep(w)
+    step.run()
+    torch.cuda.synchronize()
+    ref = orc.decode_nonabsorbed(w["q_nope"], w["q_rope"], w["kv_cache"], w["block_table"], w["seq_lens"],
+                                 w["W_UK"], w["W_UV"], w["scale"])
+    assert_close(host(step.out), ref["out"], True, "out")
+
+
+def test_incremental_gpu_decode_equals_full_causal_tiny():
+    """Decode at every prefix 1..64 of the tiny fp32 sequence equals the oracle's full
+    causal forward (the ticket's incremental-vs-full acceptance, atol 1e-5)."""
+    s = wl.spec_with("tiny_fp32", all_query_positions=True)
+    rows = wl.sequence_rows(s, 0, 64, seed=0)
+    qn, qr = wl.queries_of(s, 0, 64, seed=0)
+    wuk, wuv = wl.weights_of(s, seed=0)
+    full = orc.full_causal(orc.to_f64(rows[:, :s.R]), orc.to_f64(rows[:, s.R:]), qn, qr, wuk, wuv, s.scale)
+    for n in (1, 2, 17, 63, 64):
+        w = dict(spec=wl.spec_with("tiny_fp32"), kv_cache=np.zeros((1, 64, s.row), np.float32),
+                 block_table=np.zeros((1, 1), np.int32), seq_lens=np.array([n], np.int32), q_nope=qn[n - 1:n],
+                 q_rope=qr[n - 1:n], W_UK=wuk, W_UV=wuv, new_ckr=rows[n - 1:n], num_pages=1, scale=s.scale)
+        w["kv_cache"][0, :n] = rows[:n]
+        step = dec.DecodeStep(w)
+        step.run(append=False)
+        torch.cuda.synchronize()
+        assert_close(host(step.out)[0], full[n - 1], True, f"prefix {n}")
+
+
+# ----------------------------------------------------------------------------- full-size workloads, sampled
+
+FULL = ["kimi_h64_b64_l4096", "deepseek_h128_b128_ragged", "longctx_h64_b4_l131072",
+        "causal_chunk_h64_b8_2048p256"]
+
+
+@pytest.mark.parametrize("name", FULL)
+def test_full_size_workload_sampled(name):
+    spec = wl.WORKLOADS[name]
+    w = wl.make(spec, seed=0, new_rows_in_cache=False)
+    step = dec.DecodeStep(w)
+    step.run(append=True)
+    torch.cuda.synchronize()
+    mla.mla_check_status()
+    out, lse = host(step.out), host(step.lse)
+    rng = np.random.default_rng(123)
+    seqs = sorted(rng.choice(len(w["seq_lens"]), size=min(2, len(w["seq_lens"])), replace=False).tolist())
+    heads = sorted(rng.choice(spec.H, size=2, replace=False).tolist())
+    full = wl.make(spec, seed=0)   # the cache as it must be after the append
+    if spec.all_query_positions:
+        for b in seqs[:1]:
+            L = int(w["seq_lens"][b])
+            rows = orc.to_f64(wl.sequence_rows(spec, b, L, seed=0))
+            qn, qr = full["all_queries"][b]
+            ref = orc.full_causal(rows[:, :spec.R], rows[:, spec.R:], qn, qr, w["W_UK"], w["W_UV"], w["scale"],
+                                  heads=heads)
+            got = out[b * spec.q_len:(b + 1) * spec.q_len]
+            assert_close(got[:, heads], ref[L - spec.q_len:, heads], False, f"{name} b={b}")
+        return
+    ref = orc.decode_nonabsorbed(full["q_nope"], full["q_rope"], full["kv_cache"], full["block_table"],
+                                 full["seq_lens"], full["W_UK"], full["W_UV"], full["scale"], q_len=spec.q_len,
+                                 page_size=spec.page_size, seqs=seqs, heads=heads)
+    for b in seqs:
+        for h in heads:
+            assert_close(out[b, h], ref["out"][b, h], False, f"{name} out b={b} h={h}")
+            assert_close(lse[b, h], ref["lse"][b, h], False, f"{name} lse b={b} h={h}")
+    assert np.all(np.isfinite(out))
+
+
+# ----------------------------------------------------------------------------- failure reporting
+
+def test_bad_page_id_is_reported_not_faulted():
+    w = wl.make(small_spec(H=64), seed=2, seq_lens=[130, 64])
+    w["block_table"][1, 0] = 10_000          # outside the pool
+    step = dec.DecodeStep(w)
+    step.run(append=False)
+    torch.cuda.synchronize()
+    with pytest.raises(mla.MlaError) as e:
+        mla.mla_check_status()
+    assert e.value.status == mla._binding.MLA_ERR_INVALID
+    mla.mla_check_status()                   # cleared
