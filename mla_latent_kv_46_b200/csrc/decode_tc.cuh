@@ -5,9 +5,10 @@
 // through shared memory with TMA and runs, per page:
 //   scores   S[h][t]   = sum_k Q[h][k] * KV[t][k]        k over the 576-wide row
 //            tcgen05.mma M=64 (heads) x N=64 (tokens) x K=576, fp32 in TMEM
-//   softmax  fp32 online softmax per head in registers (4 softmax warps), P in bf16
+//   softmax  fp32 online softmax per head in registers (4 softmax warps); P goes
+//            to the tensor cores as two bf16 terms, P = P_hi + P_lo
 //   values   O^T[d][h] += sum_t C[t][d] * P[h][t]         d over the 512 latent dims
-//            tcgen05.mma M=128 (latent) x N=64 (heads) x K=64 (tokens), 4 tiles
+//            tcgen05.mma M=128 (latent) x N=64 (heads) x K=64 (tokens), 4 tiles, x2
 // The page tile in shared memory is read twice: K-major as the B operand of the
 // score MMA and MN-major (latent contiguous) as the A operand of the value MMA,
 // so every cached byte crosses HBM once per head group. All heads of the group
@@ -25,9 +26,16 @@
 //
 // Online softmax keeps a per-head reference maximum and only moves it (and
 // rescales O and the running sum) when a page's maximum exceeds it by more than
-// 2^8 in linear scale; otherwise the stale reference keeps every P <= 256, which
-// bf16 and the fp32 accumulators hold exactly enough. The result divides by the
-// running sum at the end, so it does not depend on the reference.
+// 2^8 in linear scale; otherwise the stale reference keeps every P <= 256, well
+// inside bf16 and fp32 range. The result divides by the running sum (fp32, of the
+// unrounded P) at the end, so it does not depend on the reference.
+//
+// Why P is split: with P rounded once to bf16 (8 significant bits) the latent
+// output of a query that attends to a few tokens of comparable weight can be off
+// by ~1% of the spread of those tokens' latents, beyond 2e-3 + 1e-2|o|. With
+// P = P_hi + P_lo the rounding error drops by 2^8 for one extra value MMA per
+// K-step. P_lo lives in the page's rope box, idle between the score MMA and the
+// next load into the stage, so shared memory use does not grow.
 #pragma once
 
 #include "common.cuh"
@@ -241,10 +249,12 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_qlat, const __grid_constant
           for (int kk = 0; kk < 4; ++kk) {
             // A = C^T: latent rows 128m.. (boxes 2m, 2m+1), tokens 16kk..16kk+15
             const uint64_t ad = ptx::sdesc_sw128(kv + (2 * m) * kBox + kk * 2048, kBox, 1024);
-            // B = P^T: K-major rows = heads, 16 tokens per step
+            // B = P^T: K-major rows = heads, 16 tokens per step; high part, then remainder
             const uint64_t bd = ptx::sdesc_sw128(sP + kk * 32, 16, 1024);
+            const uint64_t bl = ptx::sdesc_sw128(kv + 8 * kBox + kk * 32, 16, 1024);
             ptx::umma_f16_ss(tbase + kColO + 64 * m, ad, bd, kIdescO,
                              (first_of_unit && kk == 0) ? 0u : 1u);
+            ptx::umma_f16_ss(tbase + kColO + 64 * m, ad, bl, kIdescO, 1u);
           }
         }
         ptx::umma_commit(bar(B_KV_EMPTY + st));
@@ -381,17 +391,25 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_qlat, const __grid_constant
         if (__any_sync(0xffffffffu, need_a || need_b) && lane == 0) need_w[st] = gpg;
         const float za = (mu_a == -CUDART_INF_F) ? 0.f : mu_a;
         const float zb = (mu_b == -CUDART_INF_F) ? 0.f : mu_b;
-        uint32_t pk[16];
+        // P split into a bf16 high part and a bf16 remainder: the value MMA runs on
+        // both, so P enters the sum with ~16 significant bits instead of 8.
+        uint32_t pk[16], pl[16];
         float sa = 0.f, sb = 0.f;
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
-          __nv_bfloat162 pa = __floats2bfloat162_rn(exp2f(v[4 * i] - za), exp2f(v[4 * i + 1] - za));
-          __nv_bfloat162 pb = __floats2bfloat162_rn(exp2f(v[4 * i + 2] - zb), exp2f(v[4 * i + 3] - zb));
-          const float2 fa = __bfloat1622float2(pa), fb = __bfloat1622float2(pb);
-          sa += fa.x + fa.y;
-          sb += fb.x + fb.y;
-          pk[2 * i] = *reinterpret_cast<uint32_t*>(&pa);
-          pk[2 * i + 1] = *reinterpret_cast<uint32_t*>(&pb);
+          const float a0 = exp2f(v[4 * i] - za), a1 = exp2f(v[4 * i + 1] - za);
+          const float b0 = exp2f(v[4 * i + 2] - zb), b1 = exp2f(v[4 * i + 3] - zb);
+          sa += a0 + a1;
+          sb += b0 + b1;
+          __nv_bfloat162 ha2 = __floats2bfloat162_rn(a0, a1);
+          __nv_bfloat162 hb2 = __floats2bfloat162_rn(b0, b1);
+          const float2 fa = __bfloat1622float2(ha2), fb = __bfloat1622float2(hb2);
+          __nv_bfloat162 la2 = __floats2bfloat162_rn(a0 - fa.x, a1 - fa.y);
+          __nv_bfloat162 lb2 = __floats2bfloat162_rn(b0 - fb.x, b1 - fb.y);
+          pk[2 * i] = *reinterpret_cast<uint32_t*>(&ha2);
+          pk[2 * i + 1] = *reinterpret_cast<uint32_t*>(&hb2);
+          pl[2 * i] = *reinterpret_cast<uint32_t*>(&la2);
+          pl[2 * i + 1] = *reinterpret_cast<uint32_t*>(&lb2);
         }
         l_a = l_a * al_a + sa;
         l_b = l_b * al_b + sb;
@@ -422,13 +440,18 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_qlat, const __grid_constant
           }
           ptx::tmem_wait_st();
         }
-        // P[h][t] bf16, K-major rows of 64 tokens with the 128-byte swizzle
+        // P[h][t] bf16, K-major rows of 64 tokens with the 128-byte swizzle. The high
+        // part goes to the P buffer, the remainder to this stage's rope box, which the
+        // score MMA has finished with and the next load into this stage waits for.
+        const uint32_t sPlo = sKV + st * kTileBytes + 8 * kBox;
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
           const uint32_t oa = ha * 128 + (((i ^ (ha & 7)) << 4) | (c2 * 2));
           const uint32_t ob = hb * 128 + (((i ^ (hb & 7)) << 4) | (c2 * 2));
           asm volatile("st.shared.b32 [%0], %1;" ::"r"(sP + oa), "r"(pk[2 * i]) : "memory");
           asm volatile("st.shared.b32 [%0], %1;" ::"r"(sP + ob), "r"(pk[2 * i + 1]) : "memory");
+          asm volatile("st.shared.b32 [%0], %1;" ::"r"(sPlo + oa), "r"(pl[2 * i]) : "memory");
+          asm volatile("st.shared.b32 [%0], %1;" ::"r"(sPlo + ob), "r"(pl[2 * i + 1]) : "memory");
         }
         ptx::fence_proxy_async_smem();
         ptx::tc_fence_before();

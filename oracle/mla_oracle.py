@@ -182,12 +182,29 @@ def out_proj(o_lat, W_UV):
     return np.einsum("hvr,thr->thv", to_f64(W_UV), to_f64(o_lat))
 
 
+def round_bf16(x):
+    """Round to the nearest bf16 value (ties to even), via float32, as a kernel that
+    computes in float32 and stores bf16 does. Returns float64."""
+    f = np.asarray(x, dtype=np.float64).astype(np.float32)
+    u = f.view(np.uint32).astype(np.uint64)
+    u = (u + 0x7FFF + ((u >> 16) & 1)) >> 16
+    return (u.astype(np.uint32) << np.uint32(16)).view(np.float32).astype(np.float64)
+
+
 def decode_absorbed(q_nope, q_rope, kv_cache, block_table, seq_lens, W_UK, W_UV, scale,
-                    q_len=1, page_size=64):
-    """The absorbed pipeline in float64 (cross-check of the reference semantics)."""
-    ql = absorb_q(q_nope, W_UK)
+                    q_len=1, page_size=64, intermediates=None):
+    """The absorbed pipeline in float64 (cross-check of the reference semantics).
+
+    intermediates="bf16" rounds the two tensors a bf16 pipeline stores between its
+    steps, the absorbed query ql and the latent output o_lat, to bf16; everything
+    else stays float64. This is the reference for an end-to-end check of such a
+    pipeline on inputs where those two roundings alone move the result by more than
+    a per-step tolerance (queries that see only a few tokens)."""
+    rnd = round_bf16 if intermediates == "bf16" else (lambda a: a)
+    ql = rnd(absorb_q(q_nope, W_UK))
     a = attend_latent(ql, q_rope, kv_cache, block_table, seq_lens, scale, q_len, page_size)
-    return dict(out=out_proj(a["o_lat"], W_UV), o_lat=a["o_lat"], lse=a["lse"])
+    ol = np.where(np.isnan(a["o_lat"]), np.nan, rnd(np.nan_to_num(a["o_lat"])))
+    return dict(out=out_proj(ol, W_UV), o_lat=ol, lse=a["lse"])
 
 
 # ----------------------------------------------------------------------------- split-KV merge

@@ -143,10 +143,10 @@ def attention_case(policy, H, q_len, lens, sms, noise=0.0):
 
 @pytest.mark.parametrize("policy", ["simt", "tcgen05"])
 @pytest.mark.parametrize("H", [64, 128])
-@pytest.mark.parametrize("sms", [148, 5])
+@pytest.mark.parametrize("sms", [148, 9])
 def test_decode_attention_matches_oracle(policy, H, sms):
     step = attention_case(policy, H, 1, SMALL_LENS, sms)
-    if sms == 5:
+    if sms == 9:
         assert step.info.num_parts > 0   # the combine ran
 
 
@@ -190,20 +190,38 @@ def test_tcgen05_policy_rejects_unsupported_dims():
 @pytest.mark.parametrize("policy", ["simt", "tcgen05"])
 @pytest.mark.parametrize("H,q_len,lens,sms", [(64, 1, SMALL_LENS, 148), (128, 1, SMALL_LENS, 7),
                                               (64, 4, [200, 4, 65], 9)])
-def test_whole_step_matches_nonabsorbed_definition(policy, H, q_len, lens, sms):
-    run_policy(policy)
+def test_whole_step_matches_oracle(policy, H, q_len, lens, sms):
+    """append -> absorb -> attention (policy under test) -> combine -> projection.
+
+    Against the oracle of the same bf16 pipeline (absorbed query and latent output
+    stored in bf16, all else fp64) at the bf16 tolerance everywhere, and against the
+    exact non-absorbed definition on every query that sees at least 64 tokens. (With
+    only a few visible tokens the two bf16 stores alone move `out` by more than the
+    tolerance: the oracle shows it, see test_oracle.py.)"""
     spec = small_spec(H=H, q_len=q_len)
     empty = wl.make(spec, seed=21, seq_lens=lens, new_rows_in_cache=False)
     full = wl.make(spec, seed=21, seq_lens=lens)
     step = dec.DecodeStep(empty, sms=sms)
-    step.run(append=True)
+    step.append()
+    step.absorb()
+    run_policy(policy)
+    step.attend()
+    step.combine()
+    mla.mla_set_policy(mla.MLA_POLICY_AUTO)
+    step.project()
     torch.cuda.synchronize()
     mla.mla_check_status()
-    ref = orc.decode_nonabsorbed(full["q_nope"], full["q_rope"], full["kv_cache"], full["block_table"],
-                                 full["seq_lens"], full["W_UK"], full["W_UV"], full["scale"], q_len=q_len,
-                                 page_size=spec.page_size)
-    assert_close(host(step.out), ref["out"], False, "out")
-    assert_close(host(step.lse), ref["lse"], False, "lse")
+    args = (full["q_nope"], full["q_rope"], full["kv_cache"], full["block_table"], full["seq_lens"],
+            full["W_UK"], full["W_UV"], full["scale"])
+    mixed = orc.decode_absorbed(*args, q_len=q_len, page_size=spec.page_size, intermediates="bf16")
+    out, lse = host(step.out), host(step.lse)
+    assert_close(out, mixed["out"], False, "out vs bf16-pipeline oracle")
+    assert_close(lse, mixed["lse"], False, "lse vs bf16-pipeline oracle")
+    exact = orc.decode_nonabsorbed(*args, q_len=q_len, page_size=spec.page_size)
+    vis = np.array([max(0, L - q_len + i + 1) for L in lens for i in range(q_len)])
+    long_ctx = vis >= 64
+    assert long_ctx.any()
+    assert_close(out[long_ctx], exact["out"][long_ctx], False, "out vs definition")
 
 
 def test_whole_step_tiny_fp32_matches_definition():

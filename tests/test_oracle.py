@@ -415,3 +415,28 @@ def test_planted_mistakes_are_caught(monkeypatch):
                        ("reconstruct_kv", values_from_keys), ("visible_len", off_by_one_visibility)):
         with monkeypatch.context() as m:
             assert _pins_fail(m, name, fake) >= 1, name
+
+
+def test_round_bf16_nearest_even_and_identity_on_bf16_values():
+    x = np.array([1.0, 1.0 + 2 ** -8, 1.0 + 3 * 2 ** -8, 1.0 + 2 ** -8 + 2 ** -20, -2.5, 0.0])
+    got = orc.round_bf16(x)
+    np.testing.assert_array_equal(got, [1.0, 1.0, 1.0 + 2 ** -6, 1.0 + 2 ** -7, -2.5, 0.0])
+    w = small_bf16()
+    v = orc.to_f64(w["kv_cache"])
+    np.testing.assert_array_equal(orc.round_bf16(v), v)
+
+
+def test_bf16_intermediates_variant_stays_near_the_definition():
+    """Rounding ql and o_lat to bf16 perturbs the exact result by at most a few bf16
+    ulps of the output scale on long contexts (no rounding: identical)."""
+    w = small_bf16(lens=(300, 257, 129))
+    s = w["spec"]
+    args = (w["q_nope"], w["q_rope"], w["kv_cache"], w["block_table"], w["seq_lens"], w["W_UK"], w["W_UV"],
+            w["scale"])
+    ref = run_ref(w)
+    exact = orc.decode_absorbed(*args, q_len=s.q_len, page_size=s.page_size)
+    mixed = orc.decode_absorbed(*args, q_len=s.q_len, page_size=s.page_size, intermediates="bf16")
+    np.testing.assert_allclose(exact["out"], ref["out"], rtol=0, atol=1e-10)
+    d = np.abs(mixed["out"] - ref["out"])
+    assert 0 < d.max() < 2e-3 + 1e-2 * np.abs(ref["out"]).max()
+    np.testing.assert_array_equal(mixed["o_lat"], orc.round_bf16(mixed["o_lat"]))
