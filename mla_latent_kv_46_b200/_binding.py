@@ -13,7 +13,8 @@ import os
 import numpy as np
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_PKG, "_lib", "libmla.so")
+# MLA_LIBRARY may point at another build of the same library (e.g. an instrumented one).
+LIB_PATH = os.environ.get("MLA_LIBRARY") or os.path.join(_PKG, "_lib", "libmla.so")
 
 MLA_OK, MLA_ERR_INVALID, MLA_ERR_UNSUPPORTED, MLA_ERR_WORKSPACE, MLA_ERR_CUDA, MLA_ERR_TIMEOUT = 0, -1, -2, -3, -4, -5
 MLA_BF16, MLA_F32 = 0, 1

@@ -104,8 +104,29 @@ struct Params {
   float* lse;                 // [T][H] (nullable)
   float* o_part;              // [parts][H][512]
   float* lse_part;            // [parts][H]
+  const __nv_bfloat16* kv;    // cache base (for L2 prefetch)
+  const __nv_bfloat16* q_lat;
+  const __nv_bfloat16* q_rope;
   uint64_t timeout_ns;
+  unsigned long long* trace;  // per-CTA event clocks, only in builds with MLA_TRACE
 };
+
+// Optional event trace (build with -DMLA_TRACE): per CTA 1024 clock64 values;
+// [0,250) producer load k issued, [256,506) score MMA k issued, [512,762) value
+// MMA k issued, [768,1018) softmax P(k) ready, [1023] kernel start.
+#ifdef MLA_TRACE
+#define MLA_TRACE_AT(slot)                                                       \
+  do {                                                                           \
+    if (p.trace && ((slot) & 255) < 250)                                         \
+      p.trace[(size_t)blockIdx.x * 1024 + (slot)] = (unsigned long long)clock64(); \
+  } while (0)
+#else
+#define MLA_TRACE_AT(slot) \
+  do {                     \
+  } while (0)
+#endif
+
+constexpr int kPrefetchPages = 4;     // pages the producer keeps requested into L2 ahead of its loads
 
 struct UnitInfo {
   int32_t item, b, pb, npg, ntok, part;
@@ -180,6 +201,11 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_qlat, const __grid_constant
   __syncthreads();
   ptx::tc_fence_after();
   const uint32_t tbase = *reinterpret_cast<volatile uint32_t*>(smem + kOffTmem);
+  if (threadIdx.x == 0) {
+#ifdef MLA_TRACE
+    if (p.trace) p.trace[(size_t)blockIdx.x * 1024 + 1023] = (unsigned long long)clock64();
+#endif
+  }
 
   auto fail = [&]() {
     raise_status(kStatusTimeout);
@@ -188,10 +214,39 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_qlat, const __grid_constant
 
   if (warp == 0) {
     // ================================================================ TMA producer
+    // Loads run kStages pages ahead of the MMAs; an L2 prefetch cursor runs a further
+    // kPrefetchPages ahead (across unit boundaries, with the next unit's query rows),
+    // so the loads into shared memory mostly hit L2.
     if (lane == 0) {
       const uint64_t pol_stream = ptx::policy_evict_first();
       uint32_t gpg = 0, nu = 0;
       bool ok = true;
+      // prefetch cursor: unit pf_ui, page pf_k of it (next page to prefetch)
+      int32_t pf_ui = u_begin, pf_k = -1;
+      UnitInfo pf_u = load_unit(p, plan, pf_ui);
+      auto page_ptr = [&](const UnitInfo& u, int32_t k) -> const void* {
+        const int32_t page = p.block_table[(int64_t)u.b * p.max_pages + u.pb + k];
+        if (page < 0 || page >= p.num_pages) return nullptr;
+        return p.kv + (int64_t)page * kPage * kRow;
+      };
+      auto prefetch_next = [&]() {
+        ++pf_k;
+        while (pf_ui < u_end && pf_k >= pf_u.npg) {
+          if (++pf_ui >= u_end) return;
+          pf_u = load_unit(p, plan, pf_ui);
+          pf_k = 0;
+          if (pf_u.npg > 0) {
+            const int64_t qrow = (int64_t)pf_u.item * H + g * kHeads;
+            ptx::prefetch_l2_bulk(p.q_lat + qrow * kR, kHeads * kR * 2);
+            ptx::prefetch_l2_bulk(p.q_rope + qrow * kDr, kHeads * kDr * 2);
+          }
+        }
+        if (pf_ui < u_end) {
+          const void* src = page_ptr(pf_u, pf_k);
+          if (src) ptx::prefetch_l2_bulk(src, kTileBytes);
+        }
+      };
+      for (int i = 0; i < kStages + kPrefetchPages; ++i) prefetch_next();
       for (int32_t ui = u_begin; ui < u_end && ok; ++ui) {
         const UnitInfo u = load_unit(p, plan, ui);
         if (u.npg == 0) continue;
@@ -217,11 +272,13 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_qlat, const __grid_constant
             page = p.num_pages;  // rows past the tensor: TMA fills zeros
           }
           const uint32_t dst = sKV + st * kTileBytes;
+          MLA_TRACE_AT(gpg);
           ptx::mbar_arrive_expect_tx(bar(B_KV_FULL + st), kTileBytes);
 #pragma unroll
           for (int j = 0; j < kBoxes; ++j)
             ptx::tma_load_2d_hint(dst + j * kBox, &tm_kv, bar(B_KV_FULL + st), 64 * j, page * kPage,
                                   pol_stream);
+          prefetch_next();
         }
         ++nu;
       }
@@ -229,6 +286,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_qlat, const __grid_constant
       // (bounded) before the CTA may exit.
       for (uint32_t k = (gpg >= 2 ? gpg - 2 : 0); k < gpg; ++k)
         ptx::mbar_wait_bounded(bar(B_KV_FULL + (k & 1)), (k >> 1) & 1, abort_flag, p.timeout_ns);
+      if (nu > 0) ptx::mbar_wait_bounded(bar(B_Q_FULL), (nu - 1) & 1, abort_flag, p.timeout_ns);
     }
   } else if (warp == 1) {
     // ================================================================ MMA issuer
@@ -241,6 +299,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_qlat, const __grid_constant
             !ptx::mbar_wait_bounded(bar(B_O_FREE), (nu - 1) & 1, abort_flag, p.timeout_ns))
           return false;
         ptx::tc_fence_after();
+        MLA_TRACE_AT(512 + gp);
         const uint32_t st = gp & 1;
         const uint32_t kv = sKV + st * kTileBytes;
 #pragma unroll
@@ -278,6 +337,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_qlat, const __grid_constant
             break;
           }
           ptx::tc_fence_after();
+          MLA_TRACE_AT(256 + gpg);
           const uint32_t kv = sKV + st * kTileBytes;
           const uint32_t d_s = tbase + kColS + 64u * st;
 #pragma unroll
@@ -457,6 +517,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_qlat, const __grid_constant
         ptx::tc_fence_before();
         __syncwarp();
         if (lane == 0) ptx::mbar_arrive(bar(B_P_FULL));
+        if (warp == 4 && lane == 0) MLA_TRACE_AT(768 + gpg);
       }
       if (!ok) break;
 

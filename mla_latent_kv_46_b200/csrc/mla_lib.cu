@@ -26,6 +26,7 @@ namespace {
 thread_local std::string g_last_error;
 std::atomic<int32_t> g_policy{MLA_POLICY_AUTO};
 std::atomic<uint64_t> g_timeout_ns{2000000000ull};
+unsigned long long* g_trace = nullptr;  // event trace buffer (MLA_TRACE builds only)
 
 mla_status fail(mla_status s, const char* fmt, ...) {
   char buf[512];
@@ -60,7 +61,6 @@ mla_status check_dims(const mla_dims& d) {
   return MLA_OK;
 }
 
-size_t elem_size(const mla_dims& d) { return d.dtype == MLA_BF16 ? 2 : 4; }
 
 // Geometry the tensor-core decode kernel is written for.
 bool decode_tc_ok(const mla_dims& d) {
@@ -142,6 +142,11 @@ int32_t head_groups_for(const mla_dims& d) {
 extern "C" {
 
 int32_t mla_abi_version(void) { return MLA_ABI_VERSION; }
+
+#ifdef MLA_TRACE
+// Trace builds only (not declared in mla.h): device buffer of 1024 uint64 per CTA.
+void mla_debug_set_trace(void* dev_buf) { g_trace = static_cast<unsigned long long*>(dev_buf); }
+#endif
 
 const char* mla_last_error(void) { return g_last_error.c_str(); }
 
@@ -435,7 +440,11 @@ mla_status mla_decode_attn(const void* q_lat, const void* q_rope, const void* kv
     p.lse = lse;
     p.o_part = o_part;
     p.lse_part = lse_part;
+    p.kv = static_cast<const __nv_bfloat16*>(kv_cache);
+    p.q_lat = static_cast<const __nv_bfloat16*>(q_lat);
+    p.q_rope = static_cast<const __nv_bfloat16*>(q_rope);
     p.timeout_ns = g_timeout_ns.load();
+    p.trace = g_trace;
     const dim3 grid(info->num_slots * info->head_groups);
     mla::tc::decode_kernel<<<grid, 256, mla::tc::kSmemBytes, st>>>(tq, tr, tk, p);
     return launch_check("decode_attn (tcgen05)");
