@@ -211,164 +211,177 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_qlat, const __grid_constant
     raise_status(kStatusTimeout);
     *abort_flag = 1;
   };
+  // Bounded mbarrier wait whose outcome is the same for every lane of the warp.
+  auto wait_all = [&](uint32_t b, uint32_t parity) -> bool {
+    return __all_sync(0xffffffffu, ptx::mbar_wait_bounded(b, parity, abort_flag, p.timeout_ns));
+  };
 
   if (warp == 0) {
     // ================================================================ TMA producer
+    // The whole warp walks the schedule; one elected lane issues the copies.
     // Loads run kStages pages ahead of the MMAs; an L2 prefetch cursor runs a further
     // kPrefetchPages ahead (across unit boundaries, with the next unit's query rows),
     // so the loads into shared memory mostly hit L2.
-    if (lane == 0) {
-      const uint64_t pol_stream = ptx::policy_evict_first();
-      uint32_t gpg = 0, nu = 0;
-      bool ok = true;
-      // prefetch cursor: unit pf_ui, page pf_k of it (next page to prefetch)
-      int32_t pf_ui = u_begin, pf_k = -1;
-      UnitInfo pf_u = load_unit(p, plan, pf_ui);
-      auto page_ptr = [&](const UnitInfo& u, int32_t k) -> const void* {
-        const int32_t page = p.block_table[(int64_t)u.b * p.max_pages + u.pb + k];
-        if (page < 0 || page >= p.num_pages) return nullptr;
-        return p.kv + (int64_t)page * kPage * kRow;
-      };
-      auto prefetch_next = [&]() {
-        ++pf_k;
-        while (pf_ui < u_end && pf_k >= pf_u.npg) {
-          if (++pf_ui >= u_end) return;
-          pf_u = load_unit(p, plan, pf_ui);
-          pf_k = 0;
-          if (pf_u.npg > 0) {
-            const int64_t qrow = (int64_t)pf_u.item * H + g * kHeads;
-            ptx::prefetch_l2_bulk(p.q_lat + qrow * kR, kHeads * kR * 2);
-            ptx::prefetch_l2_bulk(p.q_rope + qrow * kDr, kHeads * kDr * 2);
-          }
+    const bool leader = ptx::elect_one();
+    const uint64_t pol_stream = ptx::policy_evict_first();
+    uint32_t gpg = 0, nu = 0;
+    bool ok = true;
+    int32_t pf_ui = u_begin, pf_k = -1;   // prefetch cursor: next page to request into L2
+    UnitInfo pf_u = load_unit(p, plan, pf_ui);
+    auto prefetch_next = [&]() {
+      ++pf_k;
+      while (pf_ui < u_end && pf_k >= pf_u.npg) {
+        if (++pf_ui >= u_end) return;
+        pf_u = load_unit(p, plan, pf_ui);
+        pf_k = 0;
+        if (pf_u.npg > 0 && leader) {
+          const int64_t qrow = (int64_t)pf_u.item * H + g * kHeads;
+          ptx::prefetch_l2_bulk(p.q_lat + qrow * kR, kHeads * kR * 2);
+          ptx::prefetch_l2_bulk(p.q_rope + qrow * kDr, kHeads * kDr * 2);
         }
-        if (pf_ui < u_end) {
-          const void* src = page_ptr(pf_u, pf_k);
-          if (src) ptx::prefetch_l2_bulk(src, kTileBytes);
-        }
-      };
-      for (int i = 0; i < kStages + kPrefetchPages; ++i) prefetch_next();
-      for (int32_t ui = u_begin; ui < u_end && ok; ++ui) {
-        const UnitInfo u = load_unit(p, plan, ui);
-        if (u.npg == 0) continue;
-        if (!ptx::mbar_wait_bounded(bar(B_Q_EMPTY), (nu & 1) ^ 1, abort_flag, p.timeout_ns)) {
-          fail();
-          ok = false;
-          break;
-        }
-        const int32_t qrow = u.item * H + g * kHeads;
+      }
+      if (pf_ui < u_end) {
+        const int32_t page = p.block_table[(int64_t)pf_u.b * p.max_pages + pf_u.pb + pf_k];
+        if (page >= 0 && page < p.num_pages && leader)
+          ptx::prefetch_l2_bulk(p.kv + (int64_t)page * kPage * kRow, kTileBytes);
+      }
+    };
+    for (int i = 0; i < kStages + kPrefetchPages; ++i) prefetch_next();
+    for (int32_t ui = u_begin; ui < u_end && ok; ++ui) {
+      const UnitInfo u = load_unit(p, plan, ui);
+      if (u.npg == 0) continue;
+      if (!wait_all(bar(B_Q_EMPTY), (nu & 1) ^ 1)) {
+        if (leader) fail();
+        ok = false;
+        break;
+      }
+      const int32_t qrow = u.item * H + g * kHeads;
+      if (leader) {
         ptx::mbar_arrive_expect_tx(bar(B_Q_FULL), kTileBytes);
         for (int j = 0; j < 8; ++j) ptx::tma_load_2d(sQ + j * kBox, &tm_qlat, bar(B_Q_FULL), 64 * j, qrow);
         ptx::tma_load_2d(sQ + 8 * kBox, &tm_qrope, bar(B_Q_FULL), 0, qrow);
-        for (int32_t k = 0; k < u.npg; ++k, ++gpg) {
-          const uint32_t st = gpg & 1, ph = (gpg >> 1) & 1;
-          if (!ptx::mbar_wait_bounded(bar(B_KV_EMPTY + st), ph ^ 1, abort_flag, p.timeout_ns)) {
-            fail();
-            ok = false;
-            break;
-          }
-          int32_t page = p.block_table[(int64_t)u.b * p.max_pages + u.pb + k];
-          if (page < 0 || page >= p.num_pages) {
-            raise_status(kStatusBadPage);
-            page = p.num_pages;  // rows past the tensor: TMA fills zeros
-          }
-          const uint32_t dst = sKV + st * kTileBytes;
+      }
+      for (int32_t k = 0; k < u.npg; ++k, ++gpg) {
+        const uint32_t st = gpg & 1, ph = (gpg >> 1) & 1;
+        if (!wait_all(bar(B_KV_EMPTY + st), ph ^ 1)) {
+          if (leader) fail();
+          ok = false;
+          break;
+        }
+        int32_t page = p.block_table[(int64_t)u.b * p.max_pages + u.pb + k];
+        if (page < 0 || page >= p.num_pages) {
+          if (leader) raise_status(kStatusBadPage);
+          page = p.num_pages;  // rows past the tensor: TMA fills zeros
+        }
+        const uint32_t dst = sKV + st * kTileBytes;
+        if (leader) {
           MLA_TRACE_AT(gpg);
           ptx::mbar_arrive_expect_tx(bar(B_KV_FULL + st), kTileBytes);
 #pragma unroll
           for (int j = 0; j < kBoxes; ++j)
             ptx::tma_load_2d_hint(dst + j * kBox, &tm_kv, bar(B_KV_FULL + st), 64 * j, page * kPage,
                                   pol_stream);
-          prefetch_next();
         }
-        ++nu;
+        prefetch_next();
       }
-      // Loads still in flight land in this CTA's shared memory: wait for them
-      // (bounded) before the CTA may exit.
-      for (uint32_t k = (gpg >= 2 ? gpg - 2 : 0); k < gpg; ++k)
-        ptx::mbar_wait_bounded(bar(B_KV_FULL + (k & 1)), (k >> 1) & 1, abort_flag, p.timeout_ns);
-      if (nu > 0) ptx::mbar_wait_bounded(bar(B_Q_FULL), (nu - 1) & 1, abort_flag, p.timeout_ns);
+      ++nu;
     }
+    // Loads still in flight land in this CTA's shared memory: wait for them
+    // (bounded) before the CTA may exit.
+    for (uint32_t k = (gpg >= 2 ? gpg - 2 : 0); k < gpg; ++k)
+      wait_all(bar(B_KV_FULL + (k & 1)), (k >> 1) & 1);
+    if (nu > 0) wait_all(bar(B_Q_FULL), (nu - 1) & 1);
   } else if (warp == 1) {
     // ================================================================ MMA issuer
-    if (lane == 0) {
-      uint32_t gpg = 0, nu = 0;
-      bool ok = true;
-      auto gemm_o = [&](uint32_t gp, bool first_of_unit) -> bool {
-        if (!ptx::mbar_wait_bounded(bar(B_P_FULL), gp & 1, abort_flag, p.timeout_ns)) return false;
-        if (first_of_unit && nu > 0 &&
-            !ptx::mbar_wait_bounded(bar(B_O_FREE), (nu - 1) & 1, abort_flag, p.timeout_ns))
-          return false;
-        ptx::tc_fence_after();
+    // The whole warp walks the schedule so the operand descriptors stay warp-uniform;
+    // one elected lane issues the tcgen05 instructions and their commits.
+    const bool leader = ptx::elect_one();
+    // Base descriptors; a K step or box adds (byte offset >> 4) to the start-address field.
+    const uint64_t dQ = ptx::sdesc_sw128(sQ, 16, 1024);
+    const uint64_t dP = ptx::sdesc_sw128(sP, 16, 1024);
+    uint32_t gpg = 0, nu = 0;
+    bool ok = true;
+    auto gemm_o = [&](uint32_t gp, bool first_of_unit) -> bool {
+      if (!wait_all(bar(B_P_FULL), gp & 1)) return false;
+      if (first_of_unit && nu > 0 &&
+          !wait_all(bar(B_O_FREE), (nu - 1) & 1))
+        return false;
+      ptx::tc_fence_after();
+      const uint32_t st = gp & 1;
+      const uint32_t kv = sKV + st * kTileBytes;
+      // A = C^T, MN-major: latent rows 128m.. (boxes 2m, 2m+1), 16 tokens per K step
+      const uint64_t dC = ptx::sdesc_sw128(kv, kBox, 1024);
+      // B = P^T, K-major rows = heads: high part in the P buffer, remainder in the rope box
+      const uint64_t dPlo = ptx::sdesc_sw128(kv + 8 * kBox, 16, 1024);
+      if (leader) {
         MLA_TRACE_AT(512 + gp);
-        const uint32_t st = gp & 1;
-        const uint32_t kv = sKV + st * kTileBytes;
 #pragma unroll
         for (int m = 0; m < 4; ++m) {
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk) {
-            // A = C^T: latent rows 128m.. (boxes 2m, 2m+1), tokens 16kk..16kk+15
-            const uint64_t ad = ptx::sdesc_sw128(kv + (2 * m) * kBox + kk * 2048, kBox, 1024);
-            // B = P^T: K-major rows = heads, 16 tokens per step; high part, then remainder
-            const uint64_t bd = ptx::sdesc_sw128(sP + kk * 32, 16, 1024);
-            const uint64_t bl = ptx::sdesc_sw128(kv + 8 * kBox + kk * 32, 16, 1024);
-            ptx::umma_f16_ss(tbase + kColO + 64 * m, ad, bd, kIdescO,
+            const uint64_t ad = dC + (uint64_t)(((2 * m) * kBox + kk * 2048) >> 4);
+            ptx::umma_f16_ss(tbase + kColO + 64 * m, ad, dP + (uint64_t)((kk * 32) >> 4), kIdescO,
                              (first_of_unit && kk == 0) ? 0u : 1u);
-            ptx::umma_f16_ss(tbase + kColO + 64 * m, ad, bl, kIdescO, 1u);
+            ptx::umma_f16_ss(tbase + kColO + 64 * m, ad, dPlo + (uint64_t)((kk * 32) >> 4), kIdescO, 1u);
           }
         }
         ptx::umma_commit(bar(B_KV_EMPTY + st));
         ptx::umma_commit(bar(B_O_DONE));
-        return true;
-      };
-      for (int32_t ui = u_begin; ui < u_end && ok; ++ui) {
-        const UnitInfo u = load_unit(p, plan, ui);
-        if (u.npg == 0) continue;
-        if (!ptx::mbar_wait_bounded(bar(B_Q_FULL), nu & 1, abort_flag, p.timeout_ns)) {
-          fail();
+      }
+      __syncwarp();
+      return true;
+    };
+    for (int32_t ui = u_begin; ui < u_end && ok; ++ui) {
+      const UnitInfo u = load_unit(p, plan, ui);
+      if (u.npg == 0) continue;
+      if (!wait_all(bar(B_Q_FULL), nu & 1)) {
+        if (leader) fail();
+        ok = false;
+        break;
+      }
+      for (int32_t k = 0; k < u.npg; ++k, ++gpg) {
+        const uint32_t st = gpg & 1, ph = (gpg >> 1) & 1;
+        if (!wait_all(bar(B_KV_FULL + st), ph) ||
+            !wait_all(bar(B_S_EMPTY + st), ph ^ 1)) {
+          if (leader) fail();
           ok = false;
           break;
         }
-        for (int32_t k = 0; k < u.npg; ++k, ++gpg) {
-          const uint32_t st = gpg & 1, ph = (gpg >> 1) & 1;
-          if (!ptx::mbar_wait_bounded(bar(B_KV_FULL + st), ph, abort_flag, p.timeout_ns) ||
-              !ptx::mbar_wait_bounded(bar(B_S_EMPTY + st), ph ^ 1, abort_flag, p.timeout_ns)) {
-            fail();
-            ok = false;
-            break;
-          }
-          ptx::tc_fence_after();
+        ptx::tc_fence_after();
+        const uint64_t dK = ptx::sdesc_sw128(sKV + st * kTileBytes, 16, 1024);
+        const uint32_t d_s = tbase + kColS + 64u * st;
+        if (leader) {
           MLA_TRACE_AT(256 + gpg);
-          const uint32_t kv = sKV + st * kTileBytes;
-          const uint32_t d_s = tbase + kColS + 64u * st;
 #pragma unroll
           for (int j = 0; j < kBoxes; ++j) {
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk) {
-              const uint64_t ad = ptx::sdesc_sw128(sQ + j * kBox + kk * 32, 16, 1024);
-              const uint64_t bd = ptx::sdesc_sw128(kv + j * kBox + kk * 32, 16, 1024);
-              ptx::umma_f16_ss(d_s, ad, bd, kIdescS, (j | kk) ? 1u : 0u);
+              const uint64_t off = (uint64_t)((j * kBox + kk * 32) >> 4);
+              ptx::umma_f16_ss(d_s, dQ + off, dK + off, kIdescS, (j | kk) ? 1u : 0u);
             }
           }
           ptx::umma_commit(bar(B_S_FULL + st));
           if (k == u.npg - 1) ptx::umma_commit(bar(B_Q_EMPTY));
-          if (k > 0 && !gemm_o(gpg - 1, k == 1)) {
-            fail();
-            ok = false;
-            break;
-          }
         }
-        if (!ok) break;
-        if (!gemm_o(gpg - 1, u.npg == 1)) {
-          fail();
+        __syncwarp();
+        if (k > 0 && !gemm_o(gpg - 1, k == 1)) {
+          if (leader) fail();
           ok = false;
           break;
         }
-        ++nu;
       }
-      // Let every MMA issued so far finish before TMEM can be released.
-      ptx::umma_commit(bar(B_DRAIN));
-      ptx::mbar_wait_bounded(bar(B_DRAIN), 0, abort_flag, p.timeout_ns);
+      if (!ok) break;
+      if (!gemm_o(gpg - 1, u.npg == 1)) {
+        if (leader) fail();
+        ok = false;
+        break;
+      }
+      ++nu;
     }
+    // Let every MMA issued so far finish before TMEM can be released.
+    if (leader) ptx::umma_commit(bar(B_DRAIN));
+    __syncwarp();
+    wait_all(bar(B_DRAIN), 0);
   } else if (warp >= 4) {
     // ================================================================ softmax + epilogue
     const int sub = warp & 3;          // TMEM sub-partition
