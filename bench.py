@@ -215,8 +215,8 @@ def run_gpu(args):
     import torch
     import torch.distributed as dist
 
-    from mla_latent_kv_46_b200 import build as mbuild
-    mbuild.build()
+    import __graft_entry__
+    __graft_entry__.build()
     import mla_latent_kv_46_b200 as mla
     from mla_latent_kv_46_b200 import decoder as dec
     from mla_latent_kv_46_b200 import workloads as wl

@@ -51,7 +51,7 @@ class PlanInfo(ctypes.Structure):
 
 def _load():
     if not os.path.exists(LIB_PATH):
-        raise ImportError(f"{LIB_PATH} is not built; run `python -m mla_latent_kv_46_b200.build`")
+        raise ImportError(f"{LIB_PATH} is not built; run `python mla_latent_kv_46_b200/build.py`")
     lib = ctypes.CDLL(LIB_PATH)
     P, I32, U64, SZ, F = ctypes.c_void_p, ctypes.c_int32, ctypes.c_uint64, ctypes.c_size_t, ctypes.c_float
     D, INFO = Dims, ctypes.POINTER(PlanInfo)

@@ -1,6 +1,9 @@
 """Build libmla.so in-tree with nvcc for sm_100a (no GPU needed to compile).
 
-    python -m mla_latent_kv_46_b200.build [--force] [-v]
+    python mla_latent_kv_46_b200/build.py [--force] [-v]
+
+Run it as a file (or load it by path, as __graft_entry__.build() does): importing
+the package loads libmla.so, which is what this script produces.
 """
 from __future__ import annotations
 

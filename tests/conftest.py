@@ -8,3 +8,6 @@ if ROOT not in sys.path:
 
 def pytest_configure(config):
     config.addinivalue_line("markers", "gpu: needs a CUDA device (B200, sm_100a)")
+    # (re)build libmla.so if a source is newer, before any test imports the package
+    import __graft_entry__
+    __graft_entry__._builder().build(force=False)

@@ -162,3 +162,4 @@ def test_bf16_rounding_is_nearest_even():
     got = wl.bf16_bits_to_f32(wl.f32_to_bf16_bits(x))
     assert got[0] == 1.0 and got[1] == 1.0 and got[2] == 1.0 + 2 ** -6 and got[3] == -2.5
     assert abs(got[4] - 3.140625) < 1e-7
+
