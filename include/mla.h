@@ -182,6 +182,33 @@ mla_status mla_combine(const int32_t* plan_dev, const mla_plan_info* info, const
 mla_status mla_out_proj(const void* o_lat, const void* W_UV, void* out, int32_t T, mla_dims d,
                         void* stream);
 
+/* ---------------------------------------------------------------- allocation-free decode
+ * The pages describe no counterpart of this call; it exists for callers that cannot
+ * allocate device memory: code running inside a CUDA-graph capture or another
+ * framework's fixed memory pool, or a host environment with no allocator exposed.
+ * It computes exactly what mla_decode_attn followed by mla_combine computes, final
+ * o_lat and lse for every query, but keeps the partial outputs of split queries in
+ * a scratch array that the library owns: a file-scope device array of 48 MiB
+ * (50,331,648 bytes) that every GPU which loads libmla.so holds until the process
+ * exits. The caller still allocates and passes all inputs, the plan and the
+ * outputs. It calls no cudaMalloc, cudaFree or other allocating routine.
+ *  - A plan whose partials need more than 48 MiB (mla_workspace_size) is rejected
+ *    with MLA_ERR_WORKSPACE before any launch: fewer num_sms or fewer splits, or
+ *    mla_decode_attn with a caller workspace, serve those.
+ *  - The first call on each device looks up the array's device address
+ *    (cudaGetSymbolAddress) with that device current; make that first call before
+ *    any stream capture.
+ *  - Every call on a device shares the one array, which keeps the last call's
+ *    contents. Nothing in it has to start at zero: each partial is written before it
+ *    is read in the same call. Calls that overlap on the GPU (concurrent streams)
+ *    race on it; order them on one stream or with events.
+ * Arguments as for mla_decode_attn, without the workspace. */
+mla_status mla_decode_attn_noalloc(const void* q_lat, const void* q_rope, const void* kv_cache,
+                                   const int32_t* block_table, const int32_t* seq_lens, int32_t B,
+                                   int32_t q_len, int32_t max_pages, int32_t num_pages, float scale,
+                                   const int32_t* plan_dev, const mla_plan_info* info, void* o_lat,
+                                   float* lse, mla_dims d, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -26,7 +26,7 @@ STATUS_NAMES = {0: "MLA_OK", -1: "MLA_ERR_INVALID", -2: "MLA_ERR_UNSUPPORTED", -
 # Every symbol include/mla.h declares.
 EXPORTS = ("mla_abi_version", "mla_last_error", "mla_set_policy", "mla_set_wait_timeout_ns",
            "mla_check_status", "mla_cache_append", "mla_absorb_q", "mla_plan_capacity", "mla_plan_splits",
-           "mla_workspace_size", "mla_decode_attn", "mla_combine", "mla_out_proj")
+           "mla_workspace_size", "mla_decode_attn", "mla_combine", "mla_out_proj", "mla_decode_attn_noalloc")
 
 
 class MlaError(RuntimeError):
@@ -69,6 +69,7 @@ def _load():
         "mla_decode_attn": (I32, [P, P, P, P, P, I32, I32, I32, I32, F, P, INFO, P, P, P, SZ, D, P]),
         "mla_combine": (I32, [P, INFO, P, SZ, P, P, D, P]),
         "mla_out_proj": (I32, [P, P, P, I32, D, P]),
+        "mla_decode_attn_noalloc": (I32, [P, P, P, P, P, I32, I32, I32, I32, F, P, INFO, P, P, D, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -167,6 +168,14 @@ def mla_combine(plan_dev, info, workspace, workspace_bytes, o_lat, lse, dims, st
 
 def mla_out_proj(o_lat, W_UV, out, T, dims, stream=None):
     _check(_lib.mla_out_proj(_ptr(o_lat), _ptr(W_UV), _ptr(out), T, dims, _stream(stream)), "mla_out_proj")
+
+
+def mla_decode_attn_noalloc(q_lat, q_rope, kv_cache, block_table, seq_lens, B, q_len, max_pages, num_pages,
+                            scale, plan_dev, info, o_lat, lse, dims, stream=None):
+    _check(_lib.mla_decode_attn_noalloc(_ptr(q_lat), _ptr(q_rope), _ptr(kv_cache), _ptr(block_table),
+                                        _ptr(seq_lens), B, q_len, max_pages, num_pages, scale, _ptr(plan_dev),
+                                        ctypes.byref(info), _ptr(o_lat), _ptr(lse), dims, _stream(stream)),
+           "mla_decode_attn_noalloc")
 
 
 def dims_of(spec) -> Dims:

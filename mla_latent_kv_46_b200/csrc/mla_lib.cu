@@ -502,4 +502,59 @@ mla_status mla_combine(const int32_t* plan_dev, const mla_plan_info* info, const
   return launch_check("combine");
 }
 
+// ------------------------------------------------------------------------------- allocation-free decode
+// Scratch for the partial outputs of mla_decode_attn_noalloc. It is a file-scope
+// device array, so every GPU that loads this library holds kNoAllocScratchBytes
+// until the process exits. Host code must not use the symbol as an address: the
+// device address comes from cudaGetSymbolAddress, looked up once per device.
+}  // extern "C"
+
+namespace {
+constexpr size_t kNoAllocScratchBytes = size_t(48) << 20;
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mu;
+void* g_noalloc_ptr[kMaxDevices] = {};
+}  // namespace
+
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+static mla_status noalloc_scratch(void** out) {
+  int dev = 0;
+  MLA_CUDA_TRY(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= kMaxDevices) return fail(MLA_ERR_UNSUPPORTED, "device %d out of range", dev);
+  std::lock_guard<std::mutex> lk(g_noalloc_mu);
+  if (!g_noalloc_ptr[dev]) {
+    void* p = nullptr;
+    MLA_CUDA_TRY(cudaGetSymbolAddress(&p, g_noalloc_scratch));
+    g_noalloc_ptr[dev] = p;
+  }
+  *out = g_noalloc_ptr[dev];
+  return MLA_OK;
+}
+
+extern "C" {
+
+mla_status mla_decode_attn_noalloc(const void* q_lat, const void* q_rope, const void* kv_cache,
+                                   const int32_t* block_table, const int32_t* seq_lens, int32_t B,
+                                   int32_t q_len, int32_t max_pages, int32_t num_pages, float scale,
+                                   const int32_t* plan_dev, const mla_plan_info* info, void* o_lat,
+                                   float* lse, mla_dims d, void* stream) {
+  if (mla_status s = check_dims(d)) return s;
+  if (mla_status s = check_info(info, B, q_len, d)) return s;
+  const size_t need = mla_workspace_size(info, d);
+  if (need > kNoAllocScratchBytes)
+    return fail(MLA_ERR_WORKSPACE,
+                "plan has %d partial outputs needing %zu bytes of scratch; mla_decode_attn_noalloc "
+                "holds at most %zu bytes (use mla_decode_attn with a caller workspace)",
+                info->num_parts, need, kNoAllocScratchBytes);
+  void* ws = nullptr;
+  if (info->num_parts > 0)
+    if (mla_status s = noalloc_scratch(&ws)) return s;
+  if (mla_status s = mla_decode_attn(q_lat, q_rope, kv_cache, block_table, seq_lens, B, q_len, max_pages,
+                                     num_pages, scale, plan_dev, info, o_lat, lse, ws,
+                                     ws ? kNoAllocScratchBytes : 0, d, stream))
+    return s;
+  return mla_combine(plan_dev, info, ws, ws ? kNoAllocScratchBytes : 0, o_lat, lse, d, stream);
+}
+
 }  // extern "C"

@@ -163,3 +163,12 @@ def test_bf16_rounding_is_nearest_even():
     assert got[0] == 1.0 and got[1] == 1.0 and got[2] == 1.0 + 2 ** -6 and got[3] == -2.5
     assert abs(got[4] - 3.140625) < 1e-7
 
+
+def test_noalloc_rejects_plans_beyond_its_scratch():
+    """1000 partial outputs of 64 heads x 512 fp32 need 131 MB, over the 48 MiB the
+    allocation-free entry point holds: refused on the host, before any launch."""
+    info = mla.PlanInfo(num_items=1, num_units=1000, num_slots=1, num_parts=1000, head_groups=1, plan_words=0)
+    with pytest.raises(mla.MlaError) as e:
+        mla.mla_decode_attn_noalloc(16, 16, 16, 16, 16, 1, 1, 1, 1, 0.1, 16, info, 16, None, dims(), stream=0)
+    assert e.value.status == mla._binding.MLA_ERR_WORKSPACE
+    assert "48" in mla.mla_last_error() or "50331648" in mla.mla_last_error()
