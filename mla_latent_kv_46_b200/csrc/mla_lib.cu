@@ -20,6 +20,7 @@
 #include "ptx.cuh"
 #include "simt_kernels.cuh"
 #include "decode_tc.cuh"
+#include "gemm_tc.cuh"
 
 namespace {
 
@@ -100,16 +101,17 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// 2D bf16 tensor [rows][cols] (row pitch `pitch_bytes`), box = 64 rows x 64 cols,
+// 2D bf16 tensor [rows][cols] (row pitch `pitch_bytes`), box = box_rows rows x 64 cols,
 // 128-byte swizzle, zero fill out of bounds.
-mla_status make_map_2d(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows, uint64_t pitch_bytes) {
+mla_status make_map_2d(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows, uint64_t pitch_bytes,
+                       uint32_t box_rows = 64) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return fail(MLA_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
   if (reinterpret_cast<uintptr_t>(base) % 16 != 0)
     return fail(MLA_ERR_INVALID, "tensor base %p is not 16-byte aligned", base);
   const cuuint64_t dims[2] = {cols, rows};
   const cuuint64_t strides[1] = {pitch_bytes};
-  const cuuint32_t box[2] = {64, 64};
+  const cuuint32_t box[2] = {64, box_rows};
   const cuuint32_t estr[2] = {1, 1};
   CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -130,6 +132,30 @@ mla_status ensure_smem_attr(const void* kernel, int bytes) {
   MLA_CUDA_TRY(cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes));
   done.emplace_back(kernel, dev);
   return MLA_OK;
+}
+
+// Geometry the tensor-core projections are instantiated for.
+bool absorb_tc_ok(const mla_dims& d) { return d.dtype == MLA_BF16 && d.Dn == 128 && d.R == 512; }
+bool outproj_tc_ok(const mla_dims& d) { return d.dtype == MLA_BF16 && d.R == 512 && d.Dv == 128; }
+
+template <int KBLK, int N, bool B_MN, int STAGES>
+mla_status launch_proj(const void* A, const void* Bw, void* out, int32_t T, const mla_dims& d, int32_t a_cols,
+                       int32_t b_rows, int32_t b_cols, cudaStream_t st, const char* what) {
+  using C = mla::gemm::Cfg<KBLK, N, B_MN, STAGES>;
+  CUtensorMap ta, tb;
+  if (mla_status s = make_map_2d(&ta, A, (uint64_t)d.H * a_cols, (uint64_t)T, (uint64_t)d.H * a_cols * 2, 128))
+    return s;
+  if (mla_status s = make_map_2d(&tb, Bw, (uint64_t)b_cols, (uint64_t)b_rows, (uint64_t)b_cols * 2, 64)) return s;
+  auto kern = mla::gemm::proj_kernel<KBLK, N, B_MN, STAGES>;
+  if (mla_status s = ensure_smem_attr((const void*)kern, C::kSmemBytes)) return s;
+  mla::gemm::Params p;
+  p.out = static_cast<__nv_bfloat16*>(out);
+  p.T = T;
+  p.H = d.H;
+  p.timeout_ns = g_timeout_ns.load();
+  const dim3 grid(d.H, (T + mla::gemm::kM - 1) / mla::gemm::kM);
+  kern<<<grid, 128, C::kSmemBytes, st>>>(ta, tb, p);
+  return launch_check(what);
 }
 
 int32_t head_groups_for(const mla_dims& d) {
@@ -204,8 +230,12 @@ mla_status mla_absorb_q(const void* q_nope, const void* W_UK, void* q_lat, int32
   if (T < 0) return fail(MLA_ERR_INVALID, "T=%d", T);
   if (T == 0) return ok();
   if (!q_nope || !W_UK || !q_lat) return fail(MLA_ERR_INVALID, "null pointer");
-  if (g_policy.load() == MLA_POLICY_TCGEN05)
-    return fail(MLA_ERR_UNSUPPORTED, "no tensor-core absorb kernel in this build");
+  const int32_t pol = g_policy.load();
+  if (pol == MLA_POLICY_TCGEN05 && !absorb_tc_ok(d))
+    return fail(MLA_ERR_UNSUPPORTED, "tensor-core absorb needs bf16, Dn=128, R=512");
+  if (pol != MLA_POLICY_SIMT && absorb_tc_ok(d))
+    return launch_proj<2, 512, true, 2>(q_nope, W_UK, q_lat, T, d, d.Dn, d.H * d.Dn, d.R, as_stream(stream),
+                                        "absorb_q (tcgen05)");
   const dim3 grid((d.R + 127) / 128, d.H, (T + mla::simt::kTT - 1) / mla::simt::kTT);
   const size_t smem = sizeof(float) * mla::simt::kTT * d.Dn;
   if (smem > 48 * 1024) return fail(MLA_ERR_UNSUPPORTED, "Dn=%d too large", d.Dn);
@@ -227,8 +257,12 @@ mla_status mla_out_proj(const void* o_lat, const void* W_UV, void* out, int32_t 
   if (T < 0) return fail(MLA_ERR_INVALID, "T=%d", T);
   if (T == 0) return ok();
   if (!o_lat || !W_UV || !out) return fail(MLA_ERR_INVALID, "null pointer");
-  if (g_policy.load() == MLA_POLICY_TCGEN05)
-    return fail(MLA_ERR_UNSUPPORTED, "no tensor-core output-projection kernel in this build");
+  const int32_t pol = g_policy.load();
+  if (pol == MLA_POLICY_TCGEN05 && !outproj_tc_ok(d))
+    return fail(MLA_ERR_UNSUPPORTED, "tensor-core output projection needs bf16, R=512, Dv=128");
+  if (pol != MLA_POLICY_SIMT && outproj_tc_ok(d))
+    return launch_proj<8, 128, false, 4>(o_lat, W_UV, out, T, d, d.R, d.H * d.Dv, d.R, as_stream(stream),
+                                         "out_proj (tcgen05)");
   const dim3 grid(d.H, (T + mla::simt::kTT - 1) / mla::simt::kTT);
   const size_t smem = sizeof(float) * mla::simt::kTT * d.R;
   if (smem > 48 * 1024) return fail(MLA_ERR_UNSUPPORTED, "R=%d too large", d.R);

@@ -93,29 +93,37 @@ def test_cache_append_bit_exact(dtype):
 
 # ----------------------------------------------------------------------------- a1 / a7
 
-@pytest.mark.parametrize("case", ["bf16_h64", "bf16_h128", "f32_tiny"])
-def test_absorb_q_matches_oracle(case):
+PROJ_CASES = [("bf16_h64", "simt"), ("bf16_h64", "tcgen05"), ("bf16_h128", "simt"), ("bf16_h128", "tcgen05"),
+              ("bf16_h64_t300", "tcgen05"), ("f32_tiny", "simt")]
+
+
+def proj_case(case):
     if case == "f32_tiny":
-        w = wl.make("tiny_fp32")
-    else:
-        w = wl.make(small_spec(H=64 if case == "bf16_h64" else 128), seed=3, seq_lens=[5] * 37)
+        return wl.make("tiny_fp32")
+    H = 128 if case == "bf16_h128" else 64
+    n = 300 if case.endswith("t300") else 37     # 300 tokens: three 128-row tiles, ragged tail
+    return wl.make(small_spec(H=H), seed=3, seq_lens=[5] * n)
+
+
+@pytest.mark.parametrize("case,policy", PROJ_CASES)
+def test_absorb_q_matches_oracle(case, policy):
+    w = proj_case(case)
     step = dec.DecodeStep(w)
+    run_policy(policy)
     step.absorb()
     torch.cuda.synchronize()
     ref = orc.absorb_q(w["q_nope"], w["W_UK"])
     assert_close(host(step.q_lat), ref, w["spec"].dtype == "f32", "q_lat")
 
 
-@pytest.mark.parametrize("case", ["bf16_h64", "bf16_h128", "f32_tiny"])
-def test_out_proj_matches_oracle(case):
-    if case == "f32_tiny":
-        w = wl.make("tiny_fp32")
-    else:
-        w = wl.make(small_spec(H=64 if case == "bf16_h64" else 128), seed=4, seq_lens=[5] * 37)
+@pytest.mark.parametrize("case,policy", PROJ_CASES)
+def test_out_proj_matches_oracle(case, policy):
+    w = proj_case(case)
     spec = w["spec"]
     step = dec.DecodeStep(w)
     ol = wl.latent_outputs(spec, step.T, seed=4)
     step.o_lat.copy_(dec.to_torch(ol, step.device))
+    run_policy(policy)
     step.project()
     torch.cuda.synchronize()
     ref = orc.out_proj(ol, w["W_UV"])
