@@ -4,8 +4,7 @@
 // unit (query token, page range) of its slot it streams the unit's 64-token pages
 // through shared memory with TMA and runs, per page:
 //   scores   S[h][t]   = sum_k Q[h][k] * KV[t][k]        k over the 576-wide row
-//            tcgen05.mma M=64 (heads) x N=64 (tokens) x K=576, Q read from TMEM,
-//            the page from shared memory, fp32 scores in TMEM
+//            tcgen05.mma M=64 (heads) x N=64 (tokens) x K=576, fp32 in TMEM
 //   softmax  fp32 online softmax per head in registers (4 softmax warps); P goes
 //            to the tensor cores as two bf16 terms, P = P_hi + P_lo
 //   values   O^T[d][h] += sum_t C[t][d] * P[h][t]         d over the 512 latent dims
@@ -16,18 +15,11 @@
 // share each page: QK^T and P.C are dense contractions over the heads.
 //
 // Warp roles (256 threads): warp 0 TMA producer, warp 1 MMA issuer, warp 2 TMEM
-// allocator, warps 4-7 query staging, softmax and epilogue (warp w % 4 owns TMEM
-// lanes 32(w%4)..). Producer and MMA warps walk the schedule warp-wide and issue from
-// one elected lane, so descriptors stay warp-uniform.
+// allocator, warps 4-7 softmax and epilogue (warp w % 4 owns TMEM lanes 32(w%4)..).
 //
-// TMEM (512 columns x 128 lanes):
-//   columns [0,256), all lanes: O^T, four 128-lane x 64-column fp32 tiles (latent
-//     rows 128m..128m+127, one column per head)
-//   columns [256,512), lanes 0-15 of each 32-lane sub-partition: the unit's 64 query
-//     rows, latent part (K=512, bf16 pairs per column), A operand of the score MMA
-//   lanes 16-31 of each sub-partition: columns [256,384) the two score buffers (M=64
-//     accumulators), [384,416) the query rows' rope part (A operand)
-// Shared memory: three page stages (3 x 72 KiB) and the P_hi buffer (8 KiB).
+// TMEM columns: [0,256) O^T, four 128-lane x 64-column fp32 tiles (latent rows
+// 128m..128m+127, one column per head); [256,384) the two 64-column score buffers
+// in the M=64 layout (rows 16j..16j+15 in lanes 32j..32j+15).
 //
 // The four softmax warps meet only on mbarriers (bounded waits), never on named
 // barriers, so a warp that gives up on a timeout cannot strand the others.
@@ -58,14 +50,15 @@ constexpr int kR = 512, kDr = 64, kRow = kR + kDr;
 constexpr int kBox = 64 * 128;        // one TMA box: 64 rows x 64 bf16 = 8 KiB
 constexpr int kBoxes = kRow / 64;     // 9 boxes per 576-wide row block
 constexpr int kTileBytes = kBoxes * kBox;   // 73,728: Q tile or one page
-constexpr int kStages = 3;
+constexpr int kStages = 2;
 constexpr int kPBytes = kHeads * kPage * 2;  // 8 KiB of bf16 probabilities
 
 // shared memory map (offsets from a 1024-aligned base)
-constexpr int kOffKV = 0;
+constexpr int kOffQ = 0;
+constexpr int kOffKV = kOffQ + kTileBytes;
 constexpr int kOffP = kOffKV + kStages * kTileBytes;
-constexpr int kOffBar = kOffP + kPBytes;            // 24 mbarriers
-constexpr int kOffTmem = kOffBar + 24 * 8;
+constexpr int kOffBar = kOffP + kPBytes;            // 16 mbarriers
+constexpr int kOffTmem = kOffBar + 16 * 8;
 constexpr int kOffAbort = kOffTmem + 8;
 constexpr int kOffNeed = kOffAbort + 8;             // uint32[2]
 constexpr int kOffAlpha = kOffNeed + 8;             // float[2][64]
@@ -76,28 +69,25 @@ constexpr int kSmemBytes = kSmemUsed + 1024;        // slack for aligning the ba
 
 // barrier indices
 enum {
-  B_KV_FULL = 0,   // +stage (3)
-  B_KV_EMPTY = 3,  // +stage (3)
-  B_S_FULL = 6,    // +buffer (2)
-  B_S_EMPTY = 8,   // +buffer (2)
-  B_P_FULL = 10,
-  B_O_DONE = 11,
-  B_Q_FULL = 12,   // query rows staged in TMEM (softmax warps)
-  B_Q_EMPTY = 13,  // last score MMA of a unit done
-  B_O_FREE = 14,
-  B_DRAIN = 15,
-  B_GROUP = 16,    // the four softmax warps
-  kNumBars = 17
+  B_KV_FULL = 0,   // +stage
+  B_KV_EMPTY = 2,  // +stage
+  B_S_FULL = 4,    // +buffer
+  B_S_EMPTY = 6,   // +buffer
+  B_P_FULL = 8,
+  B_O_DONE = 9,
+  B_Q_FULL = 10,
+  B_Q_EMPTY = 11,
+  B_O_FREE = 12,
+  B_DRAIN = 13,
+  B_GROUP = 14,    // the four softmax warps
+  kNumBars = 15
 };
 
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColO = 0;
-constexpr uint32_t kColQ = 256;                     // lanes 0-15 per sub-partition
-constexpr uint32_t kColS = 256;                     // lanes 16-31 per sub-partition
-constexpr uint32_t kColQr = 384;                    // lanes 16-31 per sub-partition
-constexpr uint32_t kLaneHi = 16u << 16;             // lane offset of the upper half
+constexpr uint32_t kColS = 256;
 
-constexpr uint32_t kIdescS = ptx::idesc_bf16_f32(64, 64, 0, 0);    // Q (TMEM) x KV^T (K-major)
+constexpr uint32_t kIdescS = ptx::idesc_bf16_f32(64, 64, 0, 0);    // Q (K-major) x KV^T (K-major)
 constexpr uint32_t kIdescO = ptx::idesc_bf16_f32(128, 64, 1, 0);   // C^T (MN-major) x P^T (K-major)
 
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
@@ -158,11 +148,12 @@ __device__ __forceinline__ UnitInfo load_unit(const Params& p, const PlanView& p
 }
 
 __global__ void __launch_bounds__(256, 1)
-decode_kernel(const __grid_constant__ CUtensorMap tm_kv, const Params p) {
+decode_kernel(const __grid_constant__ CUtensorMap tm_qlat, const __grid_constant__ CUtensorMap tm_qrope,
+              const __grid_constant__ CUtensorMap tm_kv, const Params p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sbase = ptx::smem_u32(smem);
-  const uint32_t sKV = sbase + kOffKV, sP = sbase + kOffP;
+  const uint32_t sQ = sbase + kOffQ, sKV = sbase + kOffKV, sP = sbase + kOffP;
   auto bar = [&](int i) { return sbase + kOffBar + 8u * i; };
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kOffAbort);
   float* alpha_s = reinterpret_cast<float*>(smem + kOffAlpha);
@@ -178,17 +169,17 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_kv, const Params p) {
 
   if (threadIdx.x == 0) {
     *abort_flag = 0;
-    for (int s = 0; s < kStages; ++s) {
-      ptx::mbar_init(bar(B_KV_FULL + s), 1);
-      ptx::mbar_init(bar(B_KV_EMPTY + s), 1);
-    }
+    ptx::mbar_init(bar(B_KV_FULL + 0), 1);
+    ptx::mbar_init(bar(B_KV_FULL + 1), 1);
+    ptx::mbar_init(bar(B_KV_EMPTY + 0), 1);
+    ptx::mbar_init(bar(B_KV_EMPTY + 1), 1);
     ptx::mbar_init(bar(B_S_FULL + 0), 1);
     ptx::mbar_init(bar(B_S_FULL + 1), 1);
     ptx::mbar_init(bar(B_S_EMPTY + 0), 4);
     ptx::mbar_init(bar(B_S_EMPTY + 1), 4);
     ptx::mbar_init(bar(B_P_FULL), 4);
     ptx::mbar_init(bar(B_O_DONE), 1);
-    ptx::mbar_init(bar(B_Q_FULL), 4);
+    ptx::mbar_init(bar(B_Q_FULL), 1);
     ptx::mbar_init(bar(B_Q_EMPTY), 1);
     ptx::mbar_init(bar(B_O_FREE), 4);
     ptx::mbar_init(bar(B_DRAIN), 1);
@@ -201,7 +192,11 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_kv, const Params p) {
     ptx::tmem_alloc(sbase + kOffTmem, kTmemCols);
     ptx::tmem_relinquish();
   }
-  if (warp == 0 && lane == 0) ptx::prefetch_tmap(&tm_kv);
+  if (warp == 0 && lane == 0) {
+    ptx::prefetch_tmap(&tm_qlat);
+    ptx::prefetch_tmap(&tm_qrope);
+    ptx::prefetch_tmap(&tm_kv);
+  }
   ptx::tc_fence_before();
   __syncthreads();
   ptx::tc_fence_after();
@@ -223,12 +218,13 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_kv, const Params p) {
 
   if (warp == 0) {
     // ================================================================ TMA producer
+    // The whole warp walks the schedule; one elected lane issues the copies.
     // Loads run kStages pages ahead of the MMAs; an L2 prefetch cursor runs a further
     // kPrefetchPages ahead (across unit boundaries, with the next unit's query rows),
     // so the loads into shared memory mostly hit L2.
     const bool leader = ptx::elect_one();
     const uint64_t pol_stream = ptx::policy_evict_first();
-    uint32_t gpg = 0;
+    uint32_t gpg = 0, nu = 0;
     bool ok = true;
     int32_t pf_ui = u_begin, pf_k = -1;   // prefetch cursor: next page to request into L2
     UnitInfo pf_u = load_unit(p, plan, pf_ui);
@@ -253,8 +249,20 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_kv, const Params p) {
     for (int i = 0; i < kStages + kPrefetchPages; ++i) prefetch_next();
     for (int32_t ui = u_begin; ui < u_end && ok; ++ui) {
       const UnitInfo u = load_unit(p, plan, ui);
+      if (u.npg == 0) continue;
+      if (!wait_all(bar(B_Q_EMPTY), (nu & 1) ^ 1)) {
+        if (leader) fail();
+        ok = false;
+        break;
+      }
+      const int32_t qrow = u.item * H + g * kHeads;
+      if (leader) {
+        ptx::mbar_arrive_expect_tx(bar(B_Q_FULL), kTileBytes);
+        for (int j = 0; j < 8; ++j) ptx::tma_load_2d(sQ + j * kBox, &tm_qlat, bar(B_Q_FULL), 64 * j, qrow);
+        ptx::tma_load_2d(sQ + 8 * kBox, &tm_qrope, bar(B_Q_FULL), 0, qrow);
+      }
       for (int32_t k = 0; k < u.npg; ++k, ++gpg) {
-        const uint32_t st = gpg % kStages, ph = (gpg / kStages) & 1;
+        const uint32_t st = gpg & 1, ph = (gpg >> 1) & 1;
         if (!wait_all(bar(B_KV_EMPTY + st), ph ^ 1)) {
           if (leader) fail();
           ok = false;
@@ -276,22 +284,30 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_kv, const Params p) {
         }
         prefetch_next();
       }
+      ++nu;
     }
     // Loads still in flight land in this CTA's shared memory: wait for them
     // (bounded) before the CTA may exit.
-    for (uint32_t k = (gpg >= kStages ? gpg - kStages : 0); k < gpg; ++k)
-      wait_all(bar(B_KV_FULL + k % kStages), (k / kStages) & 1);
+    for (uint32_t k = (gpg >= 2 ? gpg - 2 : 0); k < gpg; ++k)
+      wait_all(bar(B_KV_FULL + (k & 1)), (k >> 1) & 1);
+    if (nu > 0) wait_all(bar(B_Q_FULL), (nu - 1) & 1);
   } else if (warp == 1) {
     // ================================================================ MMA issuer
+    // The whole warp walks the schedule so the operand descriptors stay warp-uniform;
+    // one elected lane issues the tcgen05 instructions and their commits.
     const bool leader = ptx::elect_one();
+    // Base descriptors; a K step or box adds (byte offset >> 4) to the start-address field.
+    const uint64_t dQ = ptx::sdesc_sw128(sQ, 16, 1024);
     const uint64_t dP = ptx::sdesc_sw128(sP, 16, 1024);
     uint32_t gpg = 0, nu = 0;
     bool ok = true;
     auto gemm_o = [&](uint32_t gp, bool first_of_unit) -> bool {
       if (!wait_all(bar(B_P_FULL), gp & 1)) return false;
-      if (first_of_unit && nu > 0 && !wait_all(bar(B_O_FREE), (nu - 1) & 1)) return false;
+      if (first_of_unit && nu > 0 &&
+          !wait_all(bar(B_O_FREE), (nu - 1) & 1))
+        return false;
       ptx::tc_fence_after();
-      const uint32_t st = gp % kStages;
+      const uint32_t st = gp & 1;
       const uint32_t kv = sKV + st * kTileBytes;
       // A = C^T, MN-major: latent rows 128m.. (boxes 2m, 2m+1), 16 tokens per K step
       const uint64_t dC = ptx::sdesc_sw128(kv, kBox, 1024);
@@ -324,32 +340,27 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_kv, const Params p) {
         break;
       }
       for (int32_t k = 0; k < u.npg; ++k, ++gpg) {
-        const uint32_t st = gpg % kStages, sb = gpg & 1;
-        if (!wait_all(bar(B_KV_FULL + st), (gpg / kStages) & 1) ||
-            !wait_all(bar(B_S_EMPTY + sb), ((gpg >> 1) & 1) ^ 1)) {
+        const uint32_t st = gpg & 1, ph = (gpg >> 1) & 1;
+        if (!wait_all(bar(B_KV_FULL + st), ph) ||
+            !wait_all(bar(B_S_EMPTY + st), ph ^ 1)) {
           if (leader) fail();
           ok = false;
           break;
         }
         ptx::tc_fence_after();
         const uint64_t dK = ptx::sdesc_sw128(sKV + st * kTileBytes, 16, 1024);
-        const uint32_t d_s = tbase + kLaneHi + kColS + 64u * sb;
+        const uint32_t d_s = tbase + kColS + 64u * st;
         if (leader) {
           MLA_TRACE_AT(256 + gpg);
-          // latent part: A = query rows in TMEM (8 columns per 16 K elements)
 #pragma unroll
-          for (int j = 0; j < 8; ++j) {
+          for (int j = 0; j < kBoxes; ++j) {
 #pragma unroll
-            for (int kk = 0; kk < 4; ++kk)
-              ptx::umma_f16_ts(d_s, tbase + kColQ + 32 * j + 8 * kk, dK + (uint64_t)((j * kBox + kk * 32) >> 4),
-                               kIdescS, (j | kk) ? 1u : 0u);
+            for (int kk = 0; kk < 4; ++kk) {
+              const uint64_t off = (uint64_t)((j * kBox + kk * 32) >> 4);
+              ptx::umma_f16_ss(d_s, dQ + off, dK + off, kIdescS, (j | kk) ? 1u : 0u);
+            }
           }
-          // rope part
-#pragma unroll
-          for (int kk = 0; kk < 4; ++kk)
-            ptx::umma_f16_ts(d_s, tbase + kLaneHi + kColQr + 8 * kk, dK + (uint64_t)((8 * kBox + kk * 32) >> 4),
-                             kIdescS, 1u);
-          ptx::umma_commit(bar(B_S_FULL + sb));
+          ptx::umma_commit(bar(B_S_FULL + st));
           if (k == u.npg - 1) ptx::umma_commit(bar(B_Q_EMPTY));
         }
         __syncwarp();
@@ -372,7 +383,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_kv, const Params p) {
     __syncwarp();
     wait_all(bar(B_DRAIN), 0);
   } else if (warp >= 4) {
-    // ================================================================ query staging, softmax, epilogue
+    // ================================================================ softmax + epilogue
     const int sub = warp & 3;          // TMEM sub-partition
     const int sm_tid = threadIdx.x - 128;
     const int r0 = lane >> 2, c2 = 2 * (lane & 3);
@@ -409,62 +420,18 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_kv, const Params p) {
         }
         continue;
       }
-      // ---------------------------------------------------------------- stage the query rows in TMEM
-      // Rows 16*sub + lane/4 (+8) of the group, K elements 16i + 4(lane%4) .. +3 per
-      // 8-column group i: one 8-byte global load each, in the 16x256b register order.
-      {
-        const bool free = wait_all(bar(B_Q_EMPTY), (nu & 1) ^ 1);   // previous unit's scores done
-        if (!free) { fail(); ok = false; break; }
-        ptx::tc_fence_after();
-        const int64_t qrow = (int64_t)u.item * H + g * kHeads;
-        const uint2* qa = reinterpret_cast<const uint2*>(p.q_lat + (qrow + ha) * kR) + (lane & 3);
-        const uint2* qb = reinterpret_cast<const uint2*>(p.q_lat + (qrow + hb) * kR) + (lane & 3);
-#pragma unroll 1
-        for (int half = 0; half < 2; ++half) {
-          uint32_t r[64];
-#pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            const uint2 a = __ldg(qa + 4 * (16 * half + i));
-            const uint2 b = __ldg(qb + 4 * (16 * half + i));
-            r[4 * i + 0] = a.x;
-            r[4 * i + 1] = a.y;
-            r[4 * i + 2] = b.x;
-            r[4 * i + 3] = b.y;
-          }
-          ptx::tmem_st_16x256b_x16(tbase + ((32u * sub) << 16) + kColQ + 128 * half, r);
-        }
-        {
-          const uint2* ra = reinterpret_cast<const uint2*>(p.q_rope + (qrow + ha) * kDr) + (lane & 3);
-          const uint2* rb = reinterpret_cast<const uint2*>(p.q_rope + (qrow + hb) * kDr) + (lane & 3);
-          uint32_t r[16];
-#pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const uint2 a = __ldg(ra + 4 * i);
-            const uint2 b = __ldg(rb + 4 * i);
-            r[4 * i + 0] = a.x;
-            r[4 * i + 1] = a.y;
-            r[4 * i + 2] = b.x;
-            r[4 * i + 3] = b.y;
-          }
-          ptx::tmem_st_16x256b_x4(tbase + ((32u * sub) << 16) + kLaneHi + kColQr, r);
-        }
-        ptx::tmem_wait_st();
-        ptx::tc_fence_before();
-        __syncwarp();
-        if (lane == 0) ptx::mbar_arrive(bar(B_Q_FULL));
-      }
       float m_a = -CUDART_INF_F, m_b = -CUDART_INF_F, l_a = 0.f, l_b = 0.f;
       for (int32_t k = 0; k < u.npg; ++k, ++gpg) {
-        const uint32_t sb = gpg & 1, ph = (gpg >> 1) & 1;
-        const bool got = ptx::mbar_wait_bounded(bar(B_S_FULL + sb), ph, abort_flag, p.timeout_ns);
+        const uint32_t st = gpg & 1, ph = (gpg >> 1) & 1;
+        const bool got = ptx::mbar_wait_bounded(bar(B_S_FULL + st), ph, abort_flag, p.timeout_ns);
         if (!__all_sync(0xffffffffu, got)) { fail(); ok = false; break; }
         ptx::tc_fence_after();
         float v[32];
-        ptx::tmem_ld_16x256b_x8(tbase + ((32u * sub) << 16) + kLaneHi + kColS + 64u * sb, v);
+        ptx::tmem_ld_16x256b_x8(tbase + ((32u * sub) << 16) + kColS + 64u * st, v);
         ptx::tmem_wait_ld();
         ptx::tc_fence_before();
         __syncwarp();
-        if (lane == 0) ptx::mbar_arrive(bar(B_S_EMPTY + sb));
+        if (lane == 0) ptx::mbar_arrive(bar(B_S_EMPTY + st));
 
         // scale to log2 units, mask tokens past the visible end
         const int32_t tok0 = (u.pb + k) * kPage;
@@ -489,24 +456,24 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_kv, const Params p) {
         const float mu_a = need_a ? mx_a : m_a, mu_b = need_b ? mx_b : m_b;
         const float al_a = need_a ? exp2f(m_a - mu_a) : 1.f;   // 0 when m was -inf
         const float al_b = need_b ? exp2f(m_b - mu_b) : 1.f;
-        float* alpha = alpha_s + 64 * sb;
+        float* alpha = alpha_s + 64 * st;
         if ((lane & 3) == 0) {
           alpha[ha] = al_a;
           alpha[hb] = al_b;
         }
-        if (__any_sync(0xffffffffu, need_a || need_b) && lane == 0) need_w[sb] = gpg;
+        if (__any_sync(0xffffffffu, need_a || need_b) && lane == 0) need_w[st] = gpg;
         const float za = (mu_a == -CUDART_INF_F) ? 0.f : mu_a;
         const float zb = (mu_b == -CUDART_INF_F) ? 0.f : mu_b;
         // P split into a bf16 high part and a bf16 remainder: the value MMA runs on
         // both, so P enters the sum with ~16 significant bits instead of 8.
         uint32_t pk[16], pl[16];
-        float sa = 0.f, sbs = 0.f;
+        float sa = 0.f, sb = 0.f;
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
           const float a0 = exp2f(v[4 * i] - za), a1 = exp2f(v[4 * i + 1] - za);
           const float b0 = exp2f(v[4 * i + 2] - zb), b1 = exp2f(v[4 * i + 3] - zb);
           sa += a0 + a1;
-          sbs += b0 + b1;
+          sb += b0 + b1;
           __nv_bfloat162 ha2 = __floats2bfloat162_rn(a0, a1);
           __nv_bfloat162 hb2 = __floats2bfloat162_rn(b0, b1);
           const float2 fa = __bfloat1622float2(ha2), fb = __bfloat1622float2(hb2);
@@ -518,13 +485,13 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_kv, const Params p) {
           pl[2 * i + 1] = *reinterpret_cast<uint32_t*>(&lb2);
         }
         l_a = l_a * al_a + sa;
-        l_b = l_b * al_b + sbs;
+        l_b = l_b * al_b + sb;
         m_a = mu_a;
         m_b = mu_b;
 
         // all alphas and the need word of this page are written
         if (!group_sync()) { fail(); ok = false; break; }
-        const bool any_need = need_w[sb] == gpg;
+        const bool any_need = need_w[st] == gpg;
         // the previous value MMA must be done: it reads P and accumulates O
         const bool prev = gpg == 0 ||
                           ptx::mbar_wait_bounded(bar(B_O_DONE), (gpg - 1) & 1, abort_flag, p.timeout_ns);
@@ -549,7 +516,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_kv, const Params p) {
         // P[h][t] bf16, K-major rows of 64 tokens with the 128-byte swizzle. The high
         // part goes to the P buffer, the remainder to this stage's rope box, which the
         // score MMA has finished with and the next load into this stage waits for.
-        const uint32_t sPlo = sKV + (gpg % kStages) * kTileBytes + 8 * kBox;
+        const uint32_t sPlo = sKV + st * kTileBytes + 8 * kBox;
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
           const uint32_t oa = ha * 128 + (((i ^ (ha & 7)) << 4) | (c2 * 2));

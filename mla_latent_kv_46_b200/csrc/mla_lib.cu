@@ -455,10 +455,9 @@ mla_status mla_decode_attn(const void* q_lat, const void* q_rope, const void* kv
   cudaStream_t st = as_stream(stream);
   if (use_tc_decode(d)) {
     const int64_t T = (int64_t)B * q_len;
-    (void)T;
-    CUtensorMap tk;
-    if (reinterpret_cast<uintptr_t>(q_lat) % 16 || reinterpret_cast<uintptr_t>(q_rope) % 16)
-      return fail(MLA_ERR_INVALID, "q_lat and q_rope must be 16-byte aligned");
+    CUtensorMap tq, tr, tk;
+    if (mla_status s = make_map_2d(&tq, q_lat, d.R, (uint64_t)T * d.H, (uint64_t)d.R * 2)) return s;
+    if (mla_status s = make_map_2d(&tr, q_rope, d.Dr, (uint64_t)T * d.H, (uint64_t)d.Dr * 2)) return s;
     if (mla_status s = make_map_2d(&tk, kv_cache, d.R + d.Dr, (uint64_t)num_pages * d.page_size,
                                    (uint64_t)(d.R + d.Dr) * 2))
       return s;
@@ -481,7 +480,7 @@ mla_status mla_decode_attn(const void* q_lat, const void* q_rope, const void* kv
     p.timeout_ns = g_timeout_ns.load();
     p.trace = g_trace;
     const dim3 grid(info->num_slots * info->head_groups);
-    mla::tc::decode_kernel<<<grid, 256, mla::tc::kSmemBytes, st>>>(tk, p);
+    mla::tc::decode_kernel<<<grid, 256, mla::tc::kSmemBytes, st>>>(tq, tr, tk, p);
     return launch_check("decode_attn (tcgen05)");
   }
   mla::simt::DecodeSimtArgs a;
