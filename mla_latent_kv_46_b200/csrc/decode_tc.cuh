@@ -299,13 +299,13 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_qlat, const __grid_constant
     // Base descriptors; a K step or box adds (byte offset >> 4) to the start-address field.
     const uint64_t dQ = ptx::sdesc_sw128(sQ, 16, 1024);
     const uint64_t dP = ptx::sdesc_sw128(sP, 16, 1024);
-    uint32_t gpg = 0, nu = 0;
+    // Issue order: S(0), then for every page j: V(j) as soon as its probabilities are
+    // ready, then S(j+1). With two stages the load of page j+2 starts only when V(j)
+    // has finished, so V(j) must not queue behind S(j+1), which waits for its own load.
     bool ok = true;
-    auto gemm_o = [&](uint32_t gp, bool first_of_unit) -> bool {
+    auto gemm_o = [&](uint32_t gp, bool first_of_unit, uint32_t nu) -> bool {
       if (!wait_all(bar(B_P_FULL), gp & 1)) return false;
-      if (first_of_unit && nu > 0 &&
-          !wait_all(bar(B_O_FREE), (nu - 1) & 1))
-        return false;
+      if (first_of_unit && nu > 0 && !wait_all(bar(B_O_FREE), (nu - 1) & 1)) return false;
       ptx::tc_fence_after();
       const uint32_t st = gp & 1;
       const uint32_t kv = sKV + st * kTileBytes;
@@ -331,50 +331,60 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_qlat, const __grid_constant
       __syncwarp();
       return true;
     };
+    // Score cursor: unit sui, page sk; gs = global index of the next score page; nq =
+    // non-empty units whose last score MMA has been issued (query tiles consumed).
+    uint32_t gs = 0, nq = 0;
+    int32_t sui = u_begin - 1, sk = 0;
+    UnitInfo su{};
+    auto next_s = [&]() -> bool {
+      if (sui >= u_begin && ++sk < su.npg) return true;
+      while (++sui < u_end) {
+        su = load_unit(p, plan, sui);
+        sk = 0;
+        if (su.npg > 0) return true;
+      }
+      return false;
+    };
+    auto issue_s = [&]() -> bool {
+      if (sk == 0 && !wait_all(bar(B_Q_FULL), nq & 1)) return false;
+      const uint32_t st = gs & 1, ph = (gs >> 1) & 1;
+      if (!wait_all(bar(B_KV_FULL + st), ph) || !wait_all(bar(B_S_EMPTY + st), ph ^ 1)) return false;
+      ptx::tc_fence_after();
+      const uint64_t dK = ptx::sdesc_sw128(sKV + st * kTileBytes, 16, 1024);
+      const uint32_t d_s = tbase + kColS + 64u * st;
+      const bool last = sk == su.npg - 1;
+      if (leader) {
+        MLA_TRACE_AT(256 + gs);
+#pragma unroll
+        for (int j = 0; j < kBoxes; ++j) {
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk) {
+            const uint64_t off = (uint64_t)((j * kBox + kk * 32) >> 4);
+            ptx::umma_f16_ss(d_s, dQ + off, dK + off, kIdescS, (j | kk) ? 1u : 0u);
+          }
+        }
+        ptx::umma_commit(bar(B_S_FULL + st));
+        if (last) ptx::umma_commit(bar(B_Q_EMPTY));
+      }
+      __syncwarp();
+      if (last) ++nq;
+      ++gs;
+      return true;
+    };
+    if (next_s() && !issue_s()) {
+      if (leader) fail();
+      ok = false;
+    }
+    uint32_t gv = 0, nu = 0;
     for (int32_t ui = u_begin; ui < u_end && ok; ++ui) {
       const UnitInfo u = load_unit(p, plan, ui);
       if (u.npg == 0) continue;
-      if (!wait_all(bar(B_Q_FULL), nu & 1)) {
-        if (leader) fail();
-        ok = false;
-        break;
-      }
-      for (int32_t k = 0; k < u.npg; ++k, ++gpg) {
-        const uint32_t st = gpg & 1, ph = (gpg >> 1) & 1;
-        if (!wait_all(bar(B_KV_FULL + st), ph) ||
-            !wait_all(bar(B_S_EMPTY + st), ph ^ 1)) {
+      for (int32_t k = 0; k < u.npg; ++k, ++gv) {
+        if (!gemm_o(gv, k == 0, nu) || (next_s() && !issue_s())) {
           if (leader) fail();
           ok = false;
           break;
         }
-        ptx::tc_fence_after();
-        const uint64_t dK = ptx::sdesc_sw128(sKV + st * kTileBytes, 16, 1024);
-        const uint32_t d_s = tbase + kColS + 64u * st;
-        if (leader) {
-          MLA_TRACE_AT(256 + gpg);
-#pragma unroll
-          for (int j = 0; j < kBoxes; ++j) {
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk) {
-              const uint64_t off = (uint64_t)((j * kBox + kk * 32) >> 4);
-              ptx::umma_f16_ss(d_s, dQ + off, dK + off, kIdescS, (j | kk) ? 1u : 0u);
-            }
-          }
-          ptx::umma_commit(bar(B_S_FULL + st));
-          if (k == u.npg - 1) ptx::umma_commit(bar(B_Q_EMPTY));
-        }
-        __syncwarp();
-        if (k > 0 && !gemm_o(gpg - 1, k == 1)) {
-          if (leader) fail();
-          ok = false;
-          break;
-        }
-      }
-      if (!ok) break;
-      if (!gemm_o(gpg - 1, u.npg == 1)) {
-        if (leader) fail();
-        ok = false;
-        break;
       }
       ++nu;
     }
