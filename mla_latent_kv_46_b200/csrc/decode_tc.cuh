@@ -299,12 +299,14 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_qlat, const __grid_constant
     // Base descriptors; a K step or box adds (byte offset >> 4) to the start-address field.
     const uint64_t dQ = ptx::sdesc_sw128(sQ, 16, 1024);
     const uint64_t dP = ptx::sdesc_sw128(sP, 16, 1024);
-    // Issue order is decided at run time: whichever of "score MMA of the next loaded
-    // page" and "value MMA of the oldest scored page" is ready first goes first. With
-    // two stages the score MMA of page j+1 can run while page j's softmax is computed,
-    // and the value MMA of page j never queues behind a score MMA that waits for a load.
+    // Issue order: S(0), then for every page j: V(j) as soon as its probabilities are
+    // ready, then S(j+1). With two stages the load of page j+2 starts only when V(j)
+    // has finished, so V(j) must not queue behind S(j+1), which waits for its own load.
     bool ok = true;
-    auto gemm_o = [&](uint32_t gp, bool first_of_unit) {
+    auto gemm_o = [&](uint32_t gp, bool first_of_unit, uint32_t nu) -> bool {
+      if (!wait_all(bar(B_P_FULL), gp & 1)) return false;
+      if (first_of_unit && nu > 0 && !wait_all(bar(B_O_FREE), (nu - 1) & 1)) return false;
+      ptx::tc_fence_after();
       const uint32_t st = gp & 1;
       const uint32_t kv = sKV + st * kTileBytes;
       // A = C^T, MN-major: latent rows 128m.. (boxes 2m, 2m+1), 16 tokens per K step
@@ -327,79 +329,64 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_qlat, const __grid_constant
         ptx::umma_commit(bar(B_O_DONE));
       }
       __syncwarp();
+      return true;
     };
-    // Score cursor (unit sui, page sk, global page gs, query tiles consumed nq) and value
-    // cursor (unit vui, page vk, global page gv, units started nu).
-    uint32_t gs = 0, nq = 0, gv = 0, nu = 0;
-    int32_t sui = u_begin - 1, sk = 0, vui = u_begin - 1, vk = 0;
-    UnitInfo su{}, vu{};
-    auto advance = [&](int32_t& ui, int32_t& k, UnitInfo& u) -> bool {
-      if (ui >= u_begin && ++k < u.npg) return true;
-      while (++ui < u_end) {
-        u = load_unit(p, plan, ui);
-        k = 0;
-        if (u.npg > 0) return true;
+    // Score cursor: unit sui, page sk; gs = global index of the next score page; nq =
+    // non-empty units whose last score MMA has been issued (query tiles consumed).
+    uint32_t gs = 0, nq = 0;
+    int32_t sui = u_begin - 1, sk = 0;
+    UnitInfo su{};
+    auto next_s = [&]() -> bool {
+      if (sui >= u_begin && ++sk < su.npg) return true;
+      while (++sui < u_end) {
+        su = load_unit(p, plan, sui);
+        sk = 0;
+        if (su.npg > 0) return true;
       }
       return false;
     };
-    bool s_more = advance(sui, sk, su);
-    bool v_more = advance(vui, vk, vu);
-    auto ready = [&](uint32_t b, uint32_t parity) -> bool {
-      return __all_sync(0xffffffffu, ptx::mbar_try_wait(b, parity));
-    };
-    while (v_more && ok) {
-      bool issued = false;
-      uint64_t t0 = 0;
-      while (!issued) {
-        // score MMA of page gs: at most one page ahead of the value MMAs (two stages)
-        if (s_more && gs <= gv + 1) {
-          const uint32_t st = gs & 1, ph = (gs >> 1) & 1;
-          if ((sk != 0 || ready(bar(B_Q_FULL), nq & 1)) && ready(bar(B_KV_FULL + st), ph) &&
-              ready(bar(B_S_EMPTY + st), ph ^ 1)) {
-            ptx::tc_fence_after();
-            const uint64_t dK = ptx::sdesc_sw128(sKV + st * kTileBytes, 16, 1024);
-            const uint32_t d_s = tbase + kColS + 64u * st;
-            const bool last = sk == su.npg - 1;
-            if (leader) {
-              MLA_TRACE_AT(256 + gs);
+    auto issue_s = [&]() -> bool {
+      if (sk == 0 && !wait_all(bar(B_Q_FULL), nq & 1)) return false;
+      const uint32_t st = gs & 1, ph = (gs >> 1) & 1;
+      if (!wait_all(bar(B_KV_FULL + st), ph) || !wait_all(bar(B_S_EMPTY + st), ph ^ 1)) return false;
+      ptx::tc_fence_after();
+      const uint64_t dK = ptx::sdesc_sw128(sKV + st * kTileBytes, 16, 1024);
+      const uint32_t d_s = tbase + kColS + 64u * st;
+      const bool last = sk == su.npg - 1;
+      if (leader) {
+        MLA_TRACE_AT(256 + gs);
 #pragma unroll
-              for (int j = 0; j < kBoxes; ++j) {
+        for (int j = 0; j < kBoxes; ++j) {
 #pragma unroll
-                for (int kk = 0; kk < 4; ++kk) {
-                  const uint64_t off = (uint64_t)((j * kBox + kk * 32) >> 4);
-                  ptx::umma_f16_ss(d_s, dQ + off, dK + off, kIdescS, (j | kk) ? 1u : 0u);
-                }
-              }
-              ptx::umma_commit(bar(B_S_FULL + st));
-              if (last) ptx::umma_commit(bar(B_Q_EMPTY));
-            }
-            __syncwarp();
-            if (last) ++nq;
-            ++gs;
-            s_more = advance(sui, sk, su);
-            issued = true;
-            break;
+          for (int kk = 0; kk < 4; ++kk) {
+            const uint64_t off = (uint64_t)((j * kBox + kk * 32) >> 4);
+            ptx::umma_f16_ss(d_s, dQ + off, dK + off, kIdescS, (j | kk) ? 1u : 0u);
           }
         }
-        // value MMA of page gv (its scores were issued)
-        if (gv < gs && ready(bar(B_P_FULL), gv & 1) &&
-            (vk != 0 || nu == 0 || ready(bar(B_O_FREE), (nu - 1) & 1))) {
-          ptx::tc_fence_after();
-          gemm_o(gv, vk == 0);
-          const bool last = vk == vu.npg - 1;
-          ++gv;
-          if (last) ++nu;
-          v_more = advance(vui, vk, vu);
-          issued = true;
-          break;
-        }
-        if (t0 == 0) t0 = ptx::globaltimer_ns();
-        if (*abort_flag || ptx::globaltimer_ns() - t0 > p.timeout_ns) {
+        ptx::umma_commit(bar(B_S_FULL + st));
+        if (last) ptx::umma_commit(bar(B_Q_EMPTY));
+      }
+      __syncwarp();
+      if (last) ++nq;
+      ++gs;
+      return true;
+    };
+    if (next_s() && !issue_s()) {
+      if (leader) fail();
+      ok = false;
+    }
+    uint32_t gv = 0, nu = 0;
+    for (int32_t ui = u_begin; ui < u_end && ok; ++ui) {
+      const UnitInfo u = load_unit(p, plan, ui);
+      if (u.npg == 0) continue;
+      for (int32_t k = 0; k < u.npg; ++k, ++gv) {
+        if (!gemm_o(gv, k == 0, nu) || (next_s() && !issue_s())) {
           if (leader) fail();
           ok = false;
           break;
         }
       }
+      ++nu;
     }
     // Let every MMA issued so far finish before TMEM can be released.
     if (leader) ptx::umma_commit(bar(B_DRAIN));
