@@ -113,11 +113,12 @@ struct Params {
 
 // Optional event trace (build with -DMLA_TRACE): per CTA 1024 clock64 values;
 // [0,250) producer load k issued, [256,506) score MMA k issued, [512,762) value
-// MMA k issued, [768,1018) softmax P(k) ready, [1023] kernel start.
+// MMA k issued, [768,890) softmax P(k) ready, [896,1018) scores of page k read
+// from TMEM, [1023] kernel start.
 #ifdef MLA_TRACE
 #define MLA_TRACE_AT(slot)                                                       \
   do {                                                                           \
-    if (p.trace && ((slot) & 255) < 250)                                         \
+    if (p.trace && ((slot) & 255) < 250 && ((slot) < 768 || ((slot) & 127) < 122)) \
       p.trace[(size_t)blockIdx.x * 1024 + (slot)] = (unsigned long long)clock64(); \
   } while (0)
 #else
@@ -442,6 +443,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_qlat, const __grid_constant
         ptx::tc_fence_before();
         __syncwarp();
         if (lane == 0) ptx::mbar_arrive(bar(B_S_EMPTY + st));
+        if (warp == 4 && lane == 0 && gpg < 122) MLA_TRACE_AT(896 + gpg);
 
         // scale to log2 units, mask tokens past the visible end
         const int32_t tok0 = (u.pb + k) * kPage;
@@ -540,7 +542,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_qlat, const __grid_constant
         ptx::tc_fence_before();
         __syncwarp();
         if (lane == 0) ptx::mbar_arrive(bar(B_P_FULL));
-        if (warp == 4 && lane == 0) MLA_TRACE_AT(768 + gpg);
+        if (warp == 4 && lane == 0 && gpg < 122) MLA_TRACE_AT(768 + gpg);
       }
       if (!ok) break;
 
