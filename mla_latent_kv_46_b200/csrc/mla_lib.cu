@@ -21,6 +21,7 @@
 #include "simt_kernels.cuh"
 #include "decode_tc.cuh"
 #include "gemm_tc.cuh"
+#include "decode_pair.cuh"
 
 namespace {
 
@@ -480,6 +481,13 @@ mla_status mla_decode_attn(const void* q_lat, const void* q_rope, const void* kv
     p.timeout_ns = g_timeout_ns.load();
     p.trace = g_trace;
     const dim3 grid(info->num_slots * info->head_groups);
+    if (d.H == mla::pair::kHeads) {
+      // 128 heads: a cluster of two CTAs per slot, each holding half of every page
+      if (mla_status s = ensure_smem_attr((const void*)mla::pair::decode_pair_kernel, mla::pair::kSmemBytes))
+        return s;
+      mla::pair::decode_pair_kernel<<<grid, 256, mla::pair::kSmemBytes, st>>>(tk, tr, p);
+      return launch_check("decode_attn (tcgen05, CTA pair)");
+    }
     mla::tc::decode_kernel<<<grid, 256, mla::tc::kSmemBytes, st>>>(tq, tr, tk, p);
     return launch_check("decode_attn (tcgen05)");
   }
