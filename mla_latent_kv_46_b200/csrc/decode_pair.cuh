@@ -91,6 +91,22 @@ using tc::Params;
 using tc::UnitInfo;
 using tc::load_unit;
 
+// Optional event trace (-DMLA_TRACE): per CTA 1024 clock64 values, 8 regions of 128
+// pages: 0 load issued, 1 score MMA issued, 2 value MMA issued, 3 scores read, 4 peer
+// rows received, 5 previous value MMAs done (P may be written), 6 peer P received,
+// 7 P complete for the MMA; slot 1023 kernel start. Regions 3-7: first owner warp.
+#ifdef MLA_TRACE
+#define PAIR_TRACE(region, page)                                                                   \
+  do {                                                                                             \
+    if (p.trace && (page) < 127)                                                                   \
+      p.trace[(size_t)blockIdx.x * 1024 + 128 * (region) + (page)] = (unsigned long long)clock64(); \
+  } while (0)
+#else
+#define PAIR_TRACE(region, page) \
+  do {                           \
+  } while (0)
+#endif
+
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(256, 1)
 decode_pair_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_constant__ CUtensorMap tm_qrope,
                    const Params p) {
@@ -150,6 +166,9 @@ decode_pair_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_const
   ptx::cluster_sync();   // both CTAs' barriers exist before anyone arrives remotely
   ptx::tc_fence_after();
   const uint32_t tbase = *reinterpret_cast<volatile uint32_t*>(smem + kOffTmem);
+#ifdef MLA_TRACE
+  if (threadIdx.x == 0 && p.trace) p.trace[(size_t)blockIdx.x * 1024 + 1023] = (unsigned long long)clock64();
+#endif
 
   auto fail = [&]() {
     raise_status(kStatusTimeout);
@@ -223,6 +242,7 @@ decode_pair_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_const
         }
         if (leader) {
           const uint32_t dst = sbase + kOffKV + st * kStageBytes;
+          PAIR_TRACE(0, gpg);
           ptx::mbar_arrive_expect_tx(bar(B_KV_FULL + st), stage_tx);
 #pragma unroll
           for (int s = 0; s < 4; ++s)
@@ -267,6 +287,7 @@ decode_pair_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_const
       const uint32_t d_s = tbase + kColS + 64u * sb;
       const bool last = sk == su.npg - 1;
       if (leader) {
+        PAIR_TRACE(1, gs);
 #pragma unroll
         for (int s = 0; s < 4; ++s) {
 #pragma unroll
@@ -295,6 +316,7 @@ decode_pair_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_const
       const uint32_t st = gp % kStages;
       const uint64_t dC = ptx::sdesc_sw128(sbase + kOffKV + st * kStageBytes, kBox, 1024);
       if (leader) {
+        PAIR_TRACE(2, gp);
 #pragma unroll
         for (int m = 0; m < 2; ++m) {
 #pragma unroll
@@ -346,6 +368,7 @@ decode_pair_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_const
     const int h = 32 * sub + lane;                 // this thread's head (TMEM lane)
     const bool owner = (uint32_t)(sub >> 1) == rank;
     const int hl = h - 64 * (sub >> 1);            // index among the owning CTA's 64 heads
+    const bool tracer = owner && (sub & 1) == 0 && lane == 0;
     const uint32_t lane_addr = (32u * sub) << 16;
     uint32_t gpg = 0, nu = 0, ngroup = 0;
     bool ok = true;
@@ -422,6 +445,7 @@ decode_pair_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_const
         ptx::tc_fence_before();
         __syncwarp();
         if (lane == 0) ptx::mbar_arrive(bar(B_S_EMPTY + sb));
+        if (tracer) PAIR_TRACE(3, gpg);
         const uint32_t xslot = sbase + kOffX + sb * kXBytes;
         if (!owner) {
           // ------------------------------------------------ send the peer its heads' partial rows
@@ -439,6 +463,7 @@ decode_pair_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_const
             ok = false;
             break;
           }
+          if (tracer) PAIR_TRACE(4, gpg);
           const volatile float* xs = reinterpret_cast<const volatile float*>(smem + kOffX + sb * kXBytes);
 #pragma unroll
           for (int t = 0; t < kPage; ++t) v[t] += xs[kOwn * t + hl];
@@ -477,6 +502,7 @@ decode_pair_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_const
             ok = false;
             break;
           }
+          if (tracer) PAIR_TRACE(5, gpg);
           // row h of P_hi / P_lo: 64 tokens bf16 = 8 chunks of 16 B, 128-byte swizzle
 #pragma unroll
           for (int part = 0; part < 2; ++part) {
@@ -510,6 +536,7 @@ decode_pair_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_const
           ok = false;
           break;
         }
+        if (tracer) PAIR_TRACE(6, gpg);
         if (!group_sync()) { fail(); ok = false; break; }
         const bool any_need = need_w[sb] == gpg;
         if (any_need && k > 0) {
@@ -539,6 +566,7 @@ decode_pair_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_const
         ptx::tc_fence_before();
         __syncwarp();
         if (lane == 0) ptx::mbar_arrive(bar(B_P_FULL));
+        if (tracer) PAIR_TRACE(7, gpg);
       }
       if (!ok) break;
 
