@@ -104,18 +104,22 @@ EncodeTiledFn encode_fn() {
 
 // 2D bf16 tensor [rows][cols] (row pitch `pitch_bytes`), box = box_rows rows x 64 cols,
 // 128-byte swizzle, zero fill out of bounds.
+// 2-D bf16 tensor map, boxes of box_cols x box_rows; box_cols = 64 uses the 128-byte
+// swizzle, box_cols = 32 the 64-byte swizzle (one box row = one swizzle row).
 mla_status make_map_2d(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows, uint64_t pitch_bytes,
-                       uint32_t box_rows = 64) {
+                       uint32_t box_rows = 64, uint32_t box_cols = 64) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return fail(MLA_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
   if (reinterpret_cast<uintptr_t>(base) % 16 != 0)
     return fail(MLA_ERR_INVALID, "tensor base %p is not 16-byte aligned", base);
   const cuuint64_t dims[2] = {cols, rows};
   const cuuint64_t strides[1] = {pitch_bytes};
-  const cuuint32_t box[2] = {64, box_rows};
+  if (box_cols != 64 && box_cols != 32) return fail(MLA_ERR_INVALID, "unsupported box width %u", box_cols);
+  const cuuint32_t box[2] = {box_cols, box_rows};
   const cuuint32_t estr[2] = {1, 1};
   CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
-                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  box_cols == 64 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return fail(MLA_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
   return MLA_OK;
@@ -482,10 +486,16 @@ mla_status mla_decode_attn(const void* q_lat, const void* q_rope, const void* kv
     p.trace = g_trace;
     const dim3 grid(info->num_slots * info->head_groups);
     if (d.H == mla::pair::kHeads) {
-      // 128 heads: a cluster of two CTAs per slot, each holding half of every page
+      // 128 heads: a cluster of two CTAs per slot, each holding half of every page;
+      // the rope columns travel as two 32-column halves (64-byte swizzle)
+      CUtensorMap tkr, tqr;
+      if (mla_status s = make_map_2d(&tkr, kv_cache, d.R + d.Dr, (uint64_t)num_pages * d.page_size,
+                                     (uint64_t)(d.R + d.Dr) * 2, 64, 32))
+        return s;
+      if (mla_status s = make_map_2d(&tqr, q_rope, d.Dr, (uint64_t)T * d.H, (uint64_t)d.Dr * 2, 64, 32)) return s;
       if (mla_status s = ensure_smem_attr((const void*)mla::pair::decode_pair_kernel, mla::pair::kSmemBytes))
         return s;
-      mla::pair::decode_pair_kernel<<<grid, 256, mla::pair::kSmemBytes, st>>>(tk, tr, p);
+      mla::pair::decode_pair_kernel<<<grid, 256, mla::pair::kSmemBytes, st>>>(tk, tkr, tqr, p);
       return launch_check("decode_attn (tcgen05, CTA pair)");
     }
     mla::tc::decode_kernel<<<grid, 256, mla::tc::kSmemBytes, st>>>(tq, tr, tk, p);
