@@ -488,17 +488,7 @@ decode_pair_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_const
         v[4 * c + 2] = __uint_as_float(a.z) + __uint_as_float(b.z);
         v[4 * c + 3] = __uint_as_float(a.w) + __uint_as_float(b.w);
       }
-      __syncwarp();
-      if (lane == 0) {
-        if (sub == 0) ptx::mbar_arrive_expect_tx(bar(B_X_FULL), kXBytes);   // arm the next page's phase
-        ptx::mbar_arrive_cluster(peer_addr(bar(B_X_EMPTY)));
-      }
-      // ------------------------------------------------ next page's exchange, overlapping this softmax
-      if (ex.valid) {
-        if (!exchange(ex, gpg + 1)) { fail(); ok = false; break; }
-        advance(p, plan, u_end, ex);
-      }
-      // ------------------------------------------------ softmax of head h (identical in both CTAs)
+      // ------------------------------------------------ this page's maximum and reference
       const int32_t tok0 = (u.pb + cur.k) * kPage;
       float mx = -CUDART_INF_F;
       if (tok0 + kPage <= u.ntok) {
@@ -513,6 +503,19 @@ decode_pair_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_const
       }
       mx *= p.scale_log2;
       const bool need = mx > m_run + kRescaleThreshold;
+      // The vote depends on every lane's loaded rows, so all of this warp's reads of X
+      // are complete when lane 0 tells the peer that X may be overwritten.
+      const bool any_need = __any_sync(0xffffffffu, need);
+      if (lane == 0) {
+        if (sub == 0) ptx::mbar_arrive_expect_tx(bar(B_X_FULL), kXBytes);   // arm the next page's phase
+        ptx::mbar_arrive_cluster_relaxed(peer_addr(bar(B_X_EMPTY)));
+      }
+      // ------------------------------------------------ next page's exchange, overlapping this softmax
+      if (ex.valid) {
+        if (!exchange(ex, gpg + 1)) { fail(); ok = false; break; }
+        advance(p, plan, u_end, ex);
+      }
+      // ------------------------------------------------ softmax of head h (identical in both CTAs)
       const float mu = need ? mx : m_run;
       const float al = need ? ptx::ex2(m_run - mu) : 1.f;
       const float nz = (mu == -CUDART_INF_F) ? 0.f : -mu;
@@ -539,7 +542,7 @@ decode_pair_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_const
       if (tracer) PAIR_TRACE(7, gpg);
       ptx::tmem_st_32x32b_x32(tbase + lane_addr + kColP, ph);
       ptx::tmem_st_32x32b_x32(tbase + lane_addr + kColP + 32, pl);
-      if (cur.k > 0 && __any_sync(0xffffffffu, need)) {
+      if (cur.k > 0 && any_need) {
         // a moved reference: O[h][:] *= 2^(m_old - m_new) (1 for heads that kept theirs)
 #pragma unroll 1
         for (int c = 0; c < 8; ++c) {
