@@ -416,36 +416,35 @@ decode_pair_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_const
       if (lane == 0) ptx::mbar_arrive(bar(B_Q_FULL));
       return true;
     };
-    // Exchange step of global page g (cursor c): read S, stage it, copy it to the peer;
-    // after the last page of a unit, stage the next unit's query.
-    auto exchange = [&](const PageCursor& c, uint32_t g) -> bool {
+    // Exchange of global page g, in two steps: read_s moves S from TMEM to registers and
+    // frees the score buffer; send_s stages the rows and copies them to the peer (after
+    // the last page of a unit it also stages the next unit's query).
+    auto read_s = [&](uint32_t g, float (&s)[64]) -> bool {
       if (!wait_all(bar(B_S_FULL), g & 1)) return false;
       if (tracer) PAIR_TRACE(3, g);
       ptx::tc_fence_after();
+      ptx::tmem_ld_32x32b_x64(tbase + lane_addr + kColS, s);
+      ptx::tmem_wait_ld();
+      ptx::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive(bar(B_S_EMPTY));
+      return true;
+    };
+    auto send_s = [&](const PageCursor& c, uint32_t g, const float (&s)[64]) -> bool {
       // the peer has read my previous copy: its X and my staging rows are free
       if (!wait_all_cluster(bar(B_X_EMPTY), (g & 1) ^ 1)) return false;
       if (tracer) PAIR_TRACE(4, g);
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        float s[16];
-        ptx::tmem_ld_32x32b_x16(tbase + lane_addr + kColS + 16 * q, s);
-        ptx::tmem_wait_ld();
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(xo_row + chunk(4 * q + i)),
-                       "r"(__float_as_uint(s[4 * i])), "r"(__float_as_uint(s[4 * i + 1])),
-                       "r"(__float_as_uint(s[4 * i + 2])), "r"(__float_as_uint(s[4 * i + 3]))
-                       : "memory");
-        }
-      }
-      ptx::tc_fence_before();
+      for (int q = 0; q < 16; ++q)
+        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(xo_row + chunk(q)), "r"(__float_as_uint(s[4 * q])),
+                     "r"(__float_as_uint(s[4 * q + 1])), "r"(__float_as_uint(s[4 * q + 2])),
+                     "r"(__float_as_uint(s[4 * q + 3]))
+                     : "memory");
       ptx::fence_proxy_async_smem();
       __syncwarp();
-      if (lane == 0) {
-        ptx::mbar_arrive(bar(B_S_EMPTY));
+      if (lane == 0)
         ptx::bulk_copy_to_cluster(peer_addr(sbase + kOffX + 8192u * sub), sbase + kOffXout + 8192u * sub, 8192u,
                                   peer_addr(bar(B_X_FULL)));
-      }
       if (c.k == c.u.npg - 1) {
         int32_t ui = c.ui;
         UnitInfo nu;
@@ -458,7 +457,8 @@ decode_pair_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_const
     PageCursor ex = cur;
     uint32_t gpg = 0;
     if (cur.valid) {
-      if (!stage_q(cur.u, 0) || !exchange(ex, 0)) { fail(); ok = false; }
+      float s0[64];
+      if (!stage_q(cur.u, 0) || !read_s(0, s0) || !send_s(ex, 0, s0)) { fail(); ok = false; }
       advance(p, plan, u_end, ex);
     }
     float m_run = -CUDART_INF_F, l_run = 0.f;
@@ -469,6 +469,9 @@ decode_pair_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_const
         l_run = 0.f;
       }
       // ------------------------------------------------ full scores of head h: mine + the peer's
+      // the next page's scores leave TMEM first (the score MMA after it can start)
+      float sn[64];
+      if (ex.valid && !read_s(gpg + 1, sn)) { fail(); ok = false; break; }
       if (!wait_all(bar(B_X_FULL), gpg & 1)) { fail(); ok = false; break; }
       if (tracer) PAIR_TRACE(5, gpg);
       float v[64];
@@ -490,16 +493,20 @@ decode_pair_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_const
       }
       // ------------------------------------------------ this page's maximum and reference
       const int32_t tok0 = (u.pb + cur.k) * kPage;
-      float mx = -CUDART_INF_F;
-      if (tok0 + kPage <= u.ntok) {
+      if (tok0 + kPage > u.ntok) {
 #pragma unroll
-        for (int t = 0; t < kPage; ++t) mx = fmaxf(mx, v[t]);
-      } else {
+        for (int t = 0; t < kPage; ++t) v[t] = (tok0 + t < u.ntok) ? v[t] : -CUDART_INF_F;
+      }
+      float mx;
+      {
+        float t8[8];
 #pragma unroll
-        for (int t = 0; t < kPage; ++t) {
-          v[t] = (tok0 + t < u.ntok) ? v[t] : -CUDART_INF_F;
-          mx = fmaxf(mx, v[t]);
+        for (int i = 0; i < 8; ++i) {
+          const float a = fmaxf(fmaxf(v[8 * i], v[8 * i + 1]), fmaxf(v[8 * i + 2], v[8 * i + 3]));
+          const float b = fmaxf(fmaxf(v[8 * i + 4], v[8 * i + 5]), fmaxf(v[8 * i + 6], v[8 * i + 7]));
+          t8[i] = fmaxf(a, b);
         }
+        mx = fmaxf(fmaxf(fmaxf(t8[0], t8[1]), fmaxf(t8[2], t8[3])), fmaxf(fmaxf(t8[4], t8[5]), fmaxf(t8[6], t8[7])));
       }
       mx *= p.scale_log2;
       const bool need = mx > m_run + kRescaleThreshold;
@@ -512,7 +519,7 @@ decode_pair_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_const
       }
       // ------------------------------------------------ next page's exchange, overlapping this softmax
       if (ex.valid) {
-        if (!exchange(ex, gpg + 1)) { fail(); ok = false; break; }
+        if (!send_s(ex, gpg + 1, sn)) { fail(); ok = false; break; }
         advance(p, plan, u_end, ex);
       }
       // ------------------------------------------------ softmax of head h (identical in both CTAs)
@@ -520,12 +527,12 @@ decode_pair_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_const
       const float al = need ? ptx::ex2(m_run - mu) : 1.f;
       const float nz = (mu == -CUDART_INF_F) ? 0.f : -mu;
       uint32_t ph[32], pl[32];
-      float sum = 0.f;
+      float sum4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int i = 0; i < 32; ++i) {
         const float a0 = ptx::ex2(fmaf(v[2 * i], p.scale_log2, nz));
         const float a1 = ptx::ex2(fmaf(v[2 * i + 1], p.scale_log2, nz));
-        sum += a0 + a1;
+        sum4[i & 3] += a0 + a1;
         __nv_bfloat162 hi = __floats2bfloat162_rn(a0, a1);
         const uint32_t hw = *reinterpret_cast<uint32_t*>(&hi);
         __nv_bfloat162 lo =
@@ -533,7 +540,7 @@ decode_pair_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_const
         ph[i] = hw;
         pl[i] = *reinterpret_cast<uint32_t*>(&lo);
       }
-      l_run = l_run * al + sum;
+      l_run = l_run * al + ((sum4[0] + sum4[1]) + (sum4[2] + sum4[3]));
       m_run = mu;
       if (tracer) PAIR_TRACE(6, gpg);
       // ------------------------------------------------ P to TMEM once the previous value MMAs are done
