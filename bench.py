@@ -49,16 +49,24 @@ def load_peaks():
         return dict(FALLBACK_PEAKS), "fallback"
 
 
-def traffic_record(workload):
+def decode_kernel_of(H):
+    """(source file, kernel name) of the tensor-core decode kernel used for H heads."""
+    if H == 128:
+        return "decode_pair.cuh", "mla_decode_attn (tcgen05 decode_pair_kernel, 2-CTA clusters)"
+    return "decode_tc.cuh", "mla_decode_attn (tcgen05 decode_kernel)"
+
+
+def traffic_record(workload, H):
     """DRAM bytes per launch of the decode kernel from a committed ncu summary, valid
     only while the kernel source is unchanged (its sha256 is recorded there)."""
-    src = os.path.join(ROOT, "mla_latent_kv_46_b200", "csrc", "decode_tc.cuh")
+    src_name, _ = decode_kernel_of(H)
+    src = os.path.join(ROOT, "mla_latent_kv_46_b200", "csrc", src_name)
     sha = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
     path = os.path.join(ROOT, "profiles", f"ncu_decode_attn_{workload}.md")
     if not os.path.exists(path):
         return None, sha
     text = open(path).read()
-    m_sha = re.search(r"decode_tc\.cuh sha256\[:16\]:\s*([0-9a-f]{16})", text)
+    m_sha = re.search(re.escape(src_name) + r" sha256\[:16\]:\s*([0-9a-f]{16})", text)
     m_tr = re.search(r"traffic per full launch \(bytes\):\s*([0-9]+)", text)
     if not m_sha or not m_tr or m_sha.group(1) != sha:
         return None, sha
@@ -208,7 +216,9 @@ def workload_config(spec, w, args):
                          else f"{spec.seq_len} each"),
             "cached_tokens": int(np.sum(lens, dtype=np.int64)),
             "l2": f"flushed between timed steps ({L2_FLUSH_BYTES >> 20} MiB write); cache also larger than L2",
-            "parallelism": f"replicas x{args.gpus} (independent sequences per GPU)"}
+            "parallelism": f"replicas x{args.gpus} (independent sequences per GPU)"} | (
+                {"subset": f"first {args.seqs} sequences only (profiling run, not a bench line)"}
+                if getattr(args, "seqs", 0) else {})
 
 
 def run_gpu(args):
@@ -233,7 +243,11 @@ def run_gpu(args):
         torch.cuda.set_device(0)
     dev = torch.device("cuda", torch.cuda.current_device())
     spec = wl.WORKLOADS[args.workload]
-    w = wl.make(spec, seed=rank)
+    if args.seqs:
+        # profiling knob: the first N sequences of the workload only (not a bench line)
+        w = wl.make(spec, seed=rank, seq_lens=wl.seq_lens_of(spec, rank)[:args.seqs])
+    else:
+        w = wl.make(spec, seed=rank)
     step = dec.DecodeStep(w, device=dev)
     mla.mla_set_policy(mla.MLA_POLICY_AUTO)
     stream = torch.cuda.current_stream()
@@ -293,7 +307,9 @@ def run_gpu(args):
     t_hbm = cache_bytes / (peaks["hbm_gbs"] * 1e9)
     t_tc = flops / (peaks["bf16_tflops"] * 1e12)
     bound = "hbm" if t_hbm >= t_tc else "tensor"
-    traffic, sha = traffic_record(spec.name)
+    traffic, sha = traffic_record(spec.name, spec.H)
+    if args.seqs:
+        traffic = None   # the committed figure is for the whole workload
     if bound == "hbm":
         roof = {"bound": "hbm", "achieved": cache_bytes / (attn_ms / 1e3) / 1e9, "peak": peaks["hbm_gbs"],
                 "unit": "GB/s"}
@@ -303,13 +319,13 @@ def run_gpu(args):
     roof["frac"] = roof["achieved"] / roof["peak"]
     roof["traffic"] = traffic
     roof["peak_source"] = f"{peak_src} (MEASURED_PEAKS.json)" if peak_src == "measured" else "fallback"
-    roof["kernel"] = "mla_decode_attn (tcgen05 decode_kernel)"
+    src_name, roof["kernel"] = decode_kernel_of(spec.H)
     roof["algorithmic_bytes_per_launch"] = cache_bytes
     roof["algorithmic_flops_per_launch"] = flops
     roof["roofline_ms"] = 1e3 * max(t_hbm, t_tc)
     roof["frac_of_roofline_time"] = 1e3 * max(t_hbm, t_tc) / attn_ms
     roof["tflops"] = flops / (attn_ms / 1e3) / 1e12
-    roof["decode_tc_sha256_16"] = sha
+    roof["source_sha256_16"] = f"{src_name} {sha}"
 
     # ---------------------------------------------------------------- end to end through the public API
     hostin = dec.HostInputs(step, w)
@@ -347,7 +363,7 @@ def run_gpu(args):
         line = {"metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
                 "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
                 "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-                "config": workload_config(spec, w, argparse.Namespace(gpus=world)),
+                "config": workload_config(spec, w, argparse.Namespace(gpus=world, seqs=args.seqs)),
                 "tflops": world * flops * args.steps / (total_ms_max / 1e3) / 1e12,
                 "per_kernel_ms": {n: per_kernel[n] / args.steps for n in names},
                 "roofline": roof, "cpu_baseline": cpu, "e2e": e2e,
@@ -370,6 +386,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--seqs", type=int, default=0,
+                    help="profiling only: run the first N sequences of the workload")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
