@@ -395,20 +395,22 @@ decode_pair_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_const
       if (!wait_all(bar(B_Q_EMPTY), (n & 1) ^ 1)) return false;
       ptx::tc_fence_after();
       const uint4* src = reinterpret_cast<const uint4*>(p.q_lat + ((int64_t)u.item * H + h) * kR);
+      // two rounds of 16 loads: columns 64c..64c+63 = the 128 contiguous latent dims of
+      // tile c (128r.. for c = 0, 256+128r.. for c = 1), in stage-slot order
 #pragma unroll 1
-      for (int c = 0; c < 4; ++c) {
-        // columns 32c..32c+31 = K pairs of latent dims, in stage-slot order
-        const int dim0 = (c < 2 ? 128 * (int)rank : 256 + 128 * (int)rank) + 64 * (c & 1);
-        uint32_t w[32];
+      for (int c = 0; c < 2; ++c) {
+        const int dim0 = 256 * c + 128 * (int)rank;
+        uint32_t w[2][32];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
+        for (int i = 0; i < 16; ++i) {
           const uint4 v = __ldg(src + dim0 / 8 + i);
-          w[4 * i + 0] = v.x;
-          w[4 * i + 1] = v.y;
-          w[4 * i + 2] = v.z;
-          w[4 * i + 3] = v.w;
+          w[i >> 3][4 * (i & 7) + 0] = v.x;
+          w[i >> 3][4 * (i & 7) + 1] = v.y;
+          w[i >> 3][4 * (i & 7) + 2] = v.z;
+          w[i >> 3][4 * (i & 7) + 3] = v.w;
         }
-        ptx::tmem_st_32x32b_x32(tbase + lane_addr + kColQ + 32 * c, w);
+        ptx::tmem_st_32x32b_x32(tbase + lane_addr + kColQ + 64 * c, w[0]);
+        ptx::tmem_st_32x32b_x32(tbase + lane_addr + kColQ + 64 * c + 32, w[1]);
       }
       ptx::tmem_wait_st();
       ptx::tc_fence_before();
@@ -417,8 +419,7 @@ decode_pair_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_const
       return true;
     };
     // Exchange of global page g, in two steps: read_s moves S from TMEM to registers and
-    // frees the score buffer; send_s stages the rows and copies them to the peer (after
-    // the last page of a unit it also stages the next unit's query).
+    // frees the score buffer; send_s stages the rows and copies them to the peer.
     auto read_s = [&](uint32_t g, float (&s)[64]) -> bool {
       if (!wait_all(bar(B_S_FULL), g & 1)) return false;
       if (tracer) PAIR_TRACE(3, g);
@@ -445,12 +446,66 @@ decode_pair_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_const
       if (lane == 0)
         ptx::bulk_copy_to_cluster(peer_addr(sbase + kOffX + 8192u * sub), sbase + kOffXout + 8192u * sub, 8192u,
                                   peer_addr(bar(B_X_FULL)));
-      if (c.k == c.u.npg - 1) {
-        int32_t ui = c.ui;
-        UnitInfo nu;
-        if (next_nonempty(p, plan, ui, u_end, nu) && !stage_q(nu, c.n + 1)) return false;
-      }
       return true;
+    };
+    // Once the score MMA of a unit's last page is done (its S was read), the query
+    // columns are free: stage the next unit's query so that its first score MMA can go.
+    auto stage_next_q = [&](const PageCursor& c) -> bool {
+      if (c.k != c.u.npg - 1) return true;
+      int32_t ui = c.ui;
+      UnitInfo nu;
+      return !next_nonempty(p, plan, ui, u_end, nu) || stage_q(nu, c.n + 1);
+    };
+    // Epilogue of a unit, run during the next unit's first page (or after the last page
+    // of the slot) once the unit's last value MMAs are done: O[h][:] / l to the output.
+    struct Pending {
+      bool on;
+      bool final_out;
+      int64_t row;
+      float l, m;
+    } pend{false, false, 0, 0.f, 0.f};
+    auto epilogue = [&]() {
+      ptx::tc_fence_after();
+      const float inv_l = pend.l > 0.f ? 1.f / pend.l : 0.f;
+#pragma unroll 1
+      for (int c = 0; c < 8; ++c) {
+        uint32_t o[32];
+        ptx::tmem_ld_32x32b_x32(tbase + lane_addr + kColO + 32 * c, o);
+        ptx::tmem_wait_ld();
+        const int d0 = (c < 4 ? 128 * (int)rank : 256 + 128 * (int)rank) + 32 * (c & 3);
+        if (pend.final_out) {
+          uint4* dst = reinterpret_cast<uint4*>(p.o_lat + pend.row * kR + d0);
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            uint32_t w[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              __nv_bfloat162 b2 = __floats2bfloat162_rn(__uint_as_float(o[8 * q + 2 * i]) * inv_l,
+                                                        __uint_as_float(o[8 * q + 2 * i + 1]) * inv_l);
+              w[i] = *reinterpret_cast<uint32_t*>(&b2);
+            }
+            dst[q] = make_uint4(w[0], w[1], w[2], w[3]);
+          }
+        } else {
+          float4* dst = reinterpret_cast<float4*>(p.o_part + pend.row * kR + d0);
+#pragma unroll
+          for (int q = 0; q < 8; ++q)
+            dst[q] = make_float4(__uint_as_float(o[4 * q]) * inv_l, __uint_as_float(o[4 * q + 1]) * inv_l,
+                                 __uint_as_float(o[4 * q + 2]) * inv_l, __uint_as_float(o[4 * q + 3]) * inv_l);
+        }
+      }
+      if (rank == 0) {
+        const float z = pend.l > 0.f ? (pend.m + log2f(pend.l)) * 0.69314718055994531f : -CUDART_INF_F;
+        if (pend.final_out) {
+          if (p.lse) p.lse[pend.row] = z;
+        } else {
+          p.lse_part[pend.row] = z;
+        }
+      }
+      ptx::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive(bar(B_O_FREE));
+      pend.on = false;
     };
 
     PageCursor cur = first_page(p, plan, u_begin, u_end);
@@ -458,7 +513,7 @@ decode_pair_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_const
     uint32_t gpg = 0;
     if (cur.valid) {
       float s0[64];
-      if (!stage_q(cur.u, 0) || !read_s(0, s0) || !send_s(ex, 0, s0)) { fail(); ok = false; }
+      if (!stage_q(cur.u, 0) || !read_s(0, s0) || !stage_next_q(ex) || !send_s(ex, 0, s0)) { fail(); ok = false; }
       advance(p, plan, u_end, ex);
     }
     float m_run = -CUDART_INF_F, l_run = 0.f;
@@ -471,7 +526,7 @@ decode_pair_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_const
       // ------------------------------------------------ full scores of head h: mine + the peer's
       // the next page's scores leave TMEM first (the score MMA after it can start)
       float sn[64];
-      if (ex.valid && !read_s(gpg + 1, sn)) { fail(); ok = false; break; }
+      if (ex.valid && (!read_s(gpg + 1, sn) || !stage_next_q(ex))) { fail(); ok = false; break; }
       if (!wait_all(bar(B_X_FULL), gpg & 1)) { fail(); ok = false; break; }
       if (tracer) PAIR_TRACE(5, gpg);
       float v[64];
@@ -547,6 +602,7 @@ decode_pair_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_const
       if (gpg > 0 && !wait_all(bar(B_O_DONE), (gpg - 1) & 1)) { fail(); ok = false; break; }
       ptx::tc_fence_after();
       if (tracer) PAIR_TRACE(7, gpg);
+      if (pend.on) epilogue();   // the previous unit's O, before this unit's first value MMA
       ptx::tmem_st_32x32b_x32(tbase + lane_addr + kColP, ph);
       ptx::tmem_st_32x32b_x32(tbase + lane_addr + kColP + 32, pl);
       if (cur.k > 0 && any_need) {
@@ -566,54 +622,21 @@ decode_pair_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_const
       __syncwarp();
       if (lane == 0) ptx::mbar_arrive(bar(B_P_FULL));
 
-      // ---------------------------------------------------------------- epilogue of the unit
       if (cur.k == u.npg - 1) {
-        const bool final_out = u.part < 0;
-        const int64_t row = (final_out ? (int64_t)u.item * H : (int64_t)u.part * H) + h;
-        if (!wait_all(bar(B_O_DONE), gpg & 1)) { fail(); ok = false; break; }
-        ptx::tc_fence_after();
-        const float inv_l = l_run > 0.f ? 1.f / l_run : 0.f;
-#pragma unroll 1
-        for (int c = 0; c < 8; ++c) {
-          uint32_t o[32];
-          ptx::tmem_ld_32x32b_x32(tbase + lane_addr + kColO + 32 * c, o);
-          ptx::tmem_wait_ld();
-          const int d0 = (c < 4 ? 128 * (int)rank : 256 + 128 * (int)rank) + 32 * (c & 3);
-          if (final_out) {
-            uint4* dst = reinterpret_cast<uint4*>(p.o_lat + row * kR + d0);
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-              uint32_t w[4];
-#pragma unroll
-              for (int i = 0; i < 4; ++i) {
-                __nv_bfloat162 b2 = __floats2bfloat162_rn(__uint_as_float(o[8 * q + 2 * i]) * inv_l,
-                                                          __uint_as_float(o[8 * q + 2 * i + 1]) * inv_l);
-                w[i] = *reinterpret_cast<uint32_t*>(&b2);
-              }
-              dst[q] = make_uint4(w[0], w[1], w[2], w[3]);
-            }
-          } else {
-            float4* dst = reinterpret_cast<float4*>(p.o_part + row * kR + d0);
-#pragma unroll
-            for (int q = 0; q < 8; ++q)
-              dst[q] = make_float4(__uint_as_float(o[4 * q]) * inv_l, __uint_as_float(o[4 * q + 1]) * inv_l,
-                                   __uint_as_float(o[4 * q + 2]) * inv_l, __uint_as_float(o[4 * q + 3]) * inv_l);
-          }
-        }
-        if (rank == 0) {
-          const float z = l_run > 0.f ? (m_run + log2f(l_run)) * 0.69314718055994531f : -CUDART_INF_F;
-          if (final_out) {
-            if (p.lse) p.lse[row] = z;
-          } else {
-            p.lse_part[row] = z;
-          }
-        }
-        ptx::tc_fence_before();
-        __syncwarp();
-        if (lane == 0) ptx::mbar_arrive(bar(B_O_FREE));
+        pend.on = true;
+        pend.final_out = u.part < 0;
+        pend.row = (pend.final_out ? (int64_t)u.item * H : (int64_t)u.part * H) + h;
+        pend.l = l_run;
+        pend.m = m_run;
       }
       advance(p, plan, u_end, cur);
       ++gpg;
+    }
+    if (ok && pend.on) {
+      if (wait_all(bar(B_O_DONE), (gpg - 1) & 1))
+        epilogue();
+      else
+        fail();
     }
   }
 

@@ -543,6 +543,16 @@ mla_status mla_combine(const int32_t* plan_dev, const mla_plan_info* info, const
   float *o_part, *lse_part;
   if (mla_status s = split_workspace(info, d, const_cast<void*>(workspace), workspace_bytes, &o_part, &lse_part))
     return s;
+  if (d.R <= 512 && d.R % 4 == 0) {
+    const dim3 gv(info->num_items, (d.H + 3) / 4);
+    if (d.dtype == MLA_BF16)
+      mla::simt::combine_vec_kernel<__nv_bfloat16><<<gv, 128, 0, as_stream(stream)>>>(
+          plan_dev, o_part, lse_part, static_cast<__nv_bfloat16*>(o_lat), lse, d.H, d.R);
+    else
+      mla::simt::combine_vec_kernel<float><<<gv, 128, 0, as_stream(stream)>>>(
+          plan_dev, o_part, lse_part, static_cast<float*>(o_lat), lse, d.H, d.R);
+    return launch_check("combine");
+  }
   const dim3 grid(info->num_items, d.H);
   if (d.dtype == MLA_BF16)
     mla::simt::combine_kernel<__nv_bfloat16><<<grid, 128, 0, as_stream(stream)>>>(

@@ -220,5 +220,66 @@ __global__ void combine_kernel(const int32_t* __restrict__ plan_w, const float* 
   if (threadIdx.x == 0 && lse) lse[(int64_t)item * H + h] = tot > 0.f ? M + logf(tot) : -CUDART_INF_F;
 }
 
+// Same merge, one warp per (item, head), rows of R <= 512 (R % 4 == 0) as float4:
+// grid (num_items, ceil(H / 4)), block 128. Each part's weight is computed once per
+// lane; the parts' rows are accumulated in ascending part order, as above.
+template <typename T>
+__global__ void __launch_bounds__(128) combine_vec_kernel(const int32_t* __restrict__ plan_w,
+                                                          const float* __restrict__ o_part,
+                                                          const float* __restrict__ lse_part,
+                                                          T* __restrict__ o_lat, float* __restrict__ lse,
+                                                          int32_t H, int32_t R) {
+  const PlanView plan{plan_w};
+  const int32_t item = blockIdx.x;
+  const int32_t warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int32_t h = blockIdx.y * 4 + warp;
+  if (h >= H) return;
+  const int32_t first = plan.item_parts()[2 * item], np = plan.item_parts()[2 * item + 1];
+  if (np == 0) return;
+  float M = -CUDART_INF_F;
+  for (int32_t s = 0; s < np; ++s) M = fmaxf(M, lse_part[(int64_t)(first + s) * H + h]);
+  const int32_t nv = R / 4;
+  float4 acc[4];
+#pragma unroll
+  for (int k = 0; k < 4; ++k) acc[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+  float tot = 0.f;
+  for (int32_t s = 0; s < np; ++s) {
+    const float z = lse_part[(int64_t)(first + s) * H + h];
+    const float wgt = (M == -CUDART_INF_F) ? 0.f : expf(z - M);
+    tot += wgt;
+    if (wgt > 0.f) {
+      const float4* src = reinterpret_cast<const float4*>(o_part + ((int64_t)(first + s) * H + h) * R);
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const int32_t i = lane + 32 * k;
+        if (i < nv) {
+          const float4 v = __ldcs(src + i);
+          acc[k].x = fmaf(wgt, v.x, acc[k].x);
+          acc[k].y = fmaf(wgt, v.y, acc[k].y);
+          acc[k].z = fmaf(wgt, v.z, acc[k].z);
+          acc[k].w = fmaf(wgt, v.w, acc[k].w);
+        }
+      }
+    }
+  }
+  const float inv = tot > 0.f ? 1.f / tot : 0.f;
+  T* dst = o_lat + ((int64_t)item * H + h) * R;
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const int32_t i = lane + 32 * k;
+    if (i < nv) {
+      const float4 o = make_float4(acc[k].x * inv, acc[k].y * inv, acc[k].z * inv, acc[k].w * inv);
+      if constexpr (sizeof(T) == 2) {
+        __nv_bfloat162 lo = __floats2bfloat162_rn(o.x, o.y), hi = __floats2bfloat162_rn(o.z, o.w);
+        *reinterpret_cast<uint2*>(dst + 4 * i) =
+            make_uint2(*reinterpret_cast<uint32_t*>(&lo), *reinterpret_cast<uint32_t*>(&hi));
+      } else {
+        *reinterpret_cast<float4*>(dst + 4 * i) = o;
+      }
+    }
+  }
+  if (lane == 0 && lse) lse[(int64_t)item * H + h] = tot > 0.f ? M + logf(tot) : -CUDART_INF_F;
+}
+
 }  // namespace simt
 }  // namespace mla
