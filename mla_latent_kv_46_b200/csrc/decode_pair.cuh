@@ -58,8 +58,9 @@ constexpr int kStages = 4;
 constexpr int kXBytes = kHeads * kPage * 4;        // [128 heads][64 tokens] fp32, chunk-swizzled rows
 
 constexpr int kOffKV = 0;
-constexpr int kOffQr = kOffKV + kStages * kStageBytes;   // rope query half, 128 x 32 bf16
-constexpr int kOffX = kOffQr + 2 * kRopeBox;             // the peer's partial scores
+constexpr int kOffQr = kOffKV + kStages * kStageBytes;   // 2 x rope query half, 128 x 32 bf16
+constexpr int kQrBytes = 2 * kRopeBox;
+constexpr int kOffX = kOffQr + 2 * kQrBytes;             // the peer's partial scores
 constexpr int kOffXout = kOffX + kXBytes;                // mine, staged for the bulk copy
 constexpr int kOffBar = kOffXout + kXBytes;              // 32 mbarriers
 constexpr int kOffTmem = kOffBar + 32 * 8;
@@ -76,11 +77,14 @@ enum {
   B_X_EMPTY = 11,   // the peer's 4 softmax warps have read the X I fill
   B_P_FULL = 12,    // 4 softmax warps: P in TMEM (and O rescaled)
   B_O_DONE = 13,    // value MMAs of a page done
-  B_Q_FULL = 14,    // query staged: 4 warps (latent half to TMEM) + the rope TMA
-  B_Q_EMPTY = 15,   // last score MMA of a unit done
+  B_QT_FULL = 14,   // query latent half staged in TMEM (4 softmax warps)
+  B_QT_EMPTY = 15,  // last score MMA of a unit done: the TMEM query columns are free
   B_O_FREE = 16,    // 4 softmax warps have read O
   B_DRAIN = 17,
-  kNumBars = 18
+  B_QR_FULL = 18,   // +buffer (2): rope query half landed (TMA)
+  B_QR_EMPTY = 20,  // +buffer (2): last score MMA of the unit that used it done
+  B_GROUP = 22,     // the 4 softmax warps (epilogue staging rounds)
+  kNumBars = 23
 };
 
 constexpr uint32_t kTmemCols = 512;
@@ -175,10 +179,15 @@ decode_pair_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_const
     ptx::mbar_init(bar(B_X_EMPTY), 4);
     ptx::mbar_init(bar(B_P_FULL), 4);
     ptx::mbar_init(bar(B_O_DONE), 1);
-    ptx::mbar_init(bar(B_Q_FULL), 5);
-    ptx::mbar_init(bar(B_Q_EMPTY), 1);
+    ptx::mbar_init(bar(B_QT_FULL), 4);
+    ptx::mbar_init(bar(B_QT_EMPTY), 1);
+    for (int b = 0; b < 2; ++b) {
+      ptx::mbar_init(bar(B_QR_FULL + b), 1);
+      ptx::mbar_init(bar(B_QR_EMPTY + b), 1);
+    }
     ptx::mbar_init(bar(B_O_FREE), 4);
     ptx::mbar_init(bar(B_DRAIN), 1);
+    ptx::mbar_init(bar(B_GROUP), 4);
     ptx::fence_mbar_init();
     ptx::mbar_arrive_expect_tx(bar(B_X_FULL), kXBytes);   // armed for the first page
   }
@@ -218,7 +227,7 @@ decode_pair_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_const
     // ================================================================ TMA producer
     const bool leader = ptx::elect_one();
     const uint64_t pol_stream = ptx::policy_evict_first();
-    uint32_t gpg = 0;
+    uint32_t gpg = 0, nq = 0;   // pages and rope-query halves loaded
     bool ok = true;
     // L2 prefetch cursor (CTA 0 prefetches whole pages a few pages ahead)
     PageCursor pf = first_page(p, plan, u_begin, u_end);
@@ -240,18 +249,23 @@ decode_pair_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_const
     PageCursor c = first_page(p, plan, u_begin, u_end);
     while (c.valid && ok) {
       if (c.k == 0) {
-        // this CTA's rope query half for the unit's 128 heads (the previous unit's scores are done)
-        if (!wait_all(bar(B_Q_EMPTY), (c.n & 1) ^ 1)) {
+        // this CTA's rope query half for the unit's 128 heads, into buffer n & 1 (free once
+        // the unit two back has finished its scores: the page stream never waits for the
+        // current unit's scores)
+        const uint32_t qb = c.n & 1;
+        if (!wait_all(bar(B_QR_EMPTY + qb), ((c.n >> 1) & 1) ^ 1)) {
           if (leader) fail();
           ok = false;
           break;
         }
         if (leader) {
           const int32_t qrow = c.u.item * H;
-          ptx::mbar_arrive_expect_tx(bar(B_Q_FULL), 2 * kRopeBox);
-          ptx::tma_load_2d(sbase + kOffQr, &tm_q_rope, bar(B_Q_FULL), 32 * rank, qrow);
-          ptx::tma_load_2d(sbase + kOffQr + kRopeBox, &tm_q_rope, bar(B_Q_FULL), 32 * rank, qrow + 64);
+          const uint32_t dst = sbase + kOffQr + qb * kQrBytes;
+          ptx::mbar_arrive_expect_tx(bar(B_QR_FULL + qb), 2 * kRopeBox);
+          ptx::tma_load_2d(dst, &tm_q_rope, bar(B_QR_FULL + qb), 32 * rank, qrow);
+          ptx::tma_load_2d(dst + kRopeBox, &tm_q_rope, bar(B_QR_FULL + qb), 32 * rank, qrow + 64);
         }
+        ++nq;
       }
       const uint32_t st = gpg % kStages, ph = (gpg / kStages) & 1;
       if (!wait_all(bar(B_KV_EMPTY + st), ph ^ 1)) {
@@ -282,16 +296,21 @@ decode_pair_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_const
     // copies still in flight land in this CTA's shared memory: wait (bounded) for them
     for (uint32_t k = (gpg >= kStages ? gpg - kStages : 0); k < gpg; ++k)
       wait_all(bar(B_KV_FULL + k % kStages), (k / kStages) & 1);
+    for (uint32_t n = (nq >= 2 ? nq - 2 : 0); n < nq; ++n)
+      wait_all(bar(B_QR_FULL + (n & 1)), (n >> 1) & 1);
   } else if (warp == 1) {
     // ================================================================ MMA issuer
     const bool leader = ptx::elect_one();
-    const uint64_t dQr = ptx::sdesc_sw64(sbase + kOffQr, 512);
+
     bool ok = true;
     PageCursor sc = first_page(p, plan, u_begin, u_end);   // next score MMA
     PageCursor vc = sc;                                      // next value MMA
     uint32_t gs = 0, gv = 0;
     auto issue_s = [&]() -> bool {
-      if (sc.k == 0 && !wait_all(bar(B_Q_FULL), sc.n & 1)) return false;
+      const uint32_t qb = sc.n & 1;
+      if (sc.k == 0 && (!wait_all(bar(B_QT_FULL), sc.n & 1) || !wait_all(bar(B_QR_FULL + qb), (sc.n >> 1) & 1)))
+        return false;
+      const uint64_t dQr = ptx::sdesc_sw64(sbase + kOffQr + qb * kQrBytes, 512);
       const uint32_t st = gs % kStages;
       if (!wait_all(bar(B_KV_FULL + st), (gs / kStages) & 1) || !wait_all(bar(B_S_EMPTY), (gs & 1) ^ 1))
         return false;
@@ -314,7 +333,10 @@ decode_pair_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_const
         for (int kk = 0; kk < 2; ++kk)
           ptx::umma_f16_ss(d_s, dQr + (uint64_t)((kk * 32) >> 4), dKr + (uint64_t)((kk * 32) >> 4), kIdescS, 1u);
         ptx::umma_commit(bar(B_S_FULL));
-        if (last) ptx::umma_commit(bar(B_Q_EMPTY));
+        if (last) {
+          ptx::umma_commit(bar(B_QT_EMPTY));
+          ptx::umma_commit(bar(B_QR_EMPTY + qb));
+        }
       }
       __syncwarp();
       advance(p, plan, u_end, sc);
@@ -335,7 +357,9 @@ decode_pair_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_const
           ptx::umma_f16_ts(tbase + kColO, tbase + kColP + 8 * kk, bd, kIdescV, (vc.k == 0 && kk == 0) ? 0u : 1u);
           ptx::umma_f16_ts(tbase + kColO, tbase + kColP + 32 + 8 * kk, bd, kIdescV, 1u);
         }
-        ptx::umma_commit(bar(B_KV_EMPTY + st));
+        // a unit's last page keeps its stage: the epilogue stages the unit's output there
+        // and then frees it
+        if (vc.k != vc.u.npg - 1) ptx::umma_commit(bar(B_KV_EMPTY + st));
         ptx::umma_commit(bar(B_O_DONE));
       }
       __syncwarp();
@@ -392,7 +416,7 @@ decode_pair_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_const
 
     // Stage a unit's query: own latent half of head h, 256 bf16 -> 128 TMEM columns.
     auto stage_q = [&](const UnitInfo& u, uint32_t n) -> bool {
-      if (!wait_all(bar(B_Q_EMPTY), (n & 1) ^ 1)) return false;
+      if (!wait_all(bar(B_QT_EMPTY), (n & 1) ^ 1)) return false;
       ptx::tc_fence_after();
       const uint4* src = reinterpret_cast<const uint4*>(p.q_lat + ((int64_t)u.item * H + h) * kR);
       // two rounds of 16 loads: columns 64c..64c+63 = the 128 contiguous latent dims of
@@ -415,7 +439,7 @@ decode_pair_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_const
       ptx::tmem_wait_st();
       ptx::tc_fence_before();
       __syncwarp();
-      if (lane == 0) ptx::mbar_arrive(bar(B_Q_FULL));
+      if (lane == 0) ptx::mbar_arrive(bar(B_QT_FULL));
       return true;
     };
     // Exchange of global page g, in two steps: read_s moves S from TMEM to registers and
@@ -458,54 +482,97 @@ decode_pair_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_const
     };
     // Epilogue of a unit, run during the next unit's first page (or after the last page
     // of the slot) once the unit's last value MMAs are done: O[h][:] / l to the output.
+    // The rows go out through the unit's last stage (released to the producer at the
+    // end), so that each warp store writes whole 128-byte row segments.
     struct Pending {
       bool on;
       bool final_out;
-      int64_t row;
+      int64_t row0;      // output row of head 0
+      uint32_t stage;    // stage of the unit's last page
       float l, m;
-    } pend{false, false, 0, 0.f, 0.f};
-    auto epilogue = [&]() {
+    } pend{false, false, 0, 0u, 0.f, 0.f};
+    uint32_t ngroup = 0;
+    auto group_sync = [&]() -> bool {
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive(bar(B_GROUP));
+      const bool done = ptx::mbar_wait_bounded(bar(B_GROUP), ngroup & 1, abort_flag, p.timeout_ns);
+      ++ngroup;
+      return __all_sync(0xffffffffu, done);
+    };
+    auto epilogue = [&]() -> bool {
       ptx::tc_fence_after();
       const float inv_l = pend.l > 0.f ? 1.f / pend.l : 0.f;
+      const uint32_t stg = sbase + kOffKV + pend.stage * kStageBytes;
+      // a round stages 128 rows x 128 B (64 bf16 or 32 fp32 columns) in one of two 16 KiB
+      // halves of the stage; row h's 16-byte chunk j sits at j ^ (h & 7)
+      const int rounds = pend.final_out ? 4 : 8;
+      const int cols = pend.final_out ? 64 : 32;
 #pragma unroll 1
-      for (int c = 0; c < 8; ++c) {
-        uint32_t o[32];
-        ptx::tmem_ld_32x32b_x32(tbase + lane_addr + kColO + 32 * c, o);
-        ptx::tmem_wait_ld();
-        const int d0 = (c < 4 ? 128 * (int)rank : 256 + 128 * (int)rank) + 32 * (c & 3);
+      for (int c = 0; c < rounds; ++c) {
+        const uint32_t buf = stg + (uint32_t)(c & 1) * 16384u;
+        uint32_t w[32];
         if (pend.final_out) {
-          uint4* dst = reinterpret_cast<uint4*>(p.o_lat + pend.row * kR + d0);
 #pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            uint32_t w[4];
+          for (int half = 0; half < 2; ++half) {
+            uint32_t o[32];
+            ptx::tmem_ld_32x32b_x32(tbase + lane_addr + kColO + 64 * c + 32 * half, o);
+            ptx::tmem_wait_ld();
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-              __nv_bfloat162 b2 = __floats2bfloat162_rn(__uint_as_float(o[8 * q + 2 * i]) * inv_l,
-                                                        __uint_as_float(o[8 * q + 2 * i + 1]) * inv_l);
-              w[i] = *reinterpret_cast<uint32_t*>(&b2);
+            for (int i = 0; i < 16; ++i) {
+              __nv_bfloat162 b2 =
+                  __floats2bfloat162_rn(__uint_as_float(o[2 * i]) * inv_l, __uint_as_float(o[2 * i + 1]) * inv_l);
+              w[16 * half + i] = *reinterpret_cast<uint32_t*>(&b2);
             }
-            dst[q] = make_uint4(w[0], w[1], w[2], w[3]);
           }
         } else {
-          float4* dst = reinterpret_cast<float4*>(p.o_part + pend.row * kR + d0);
+          ptx::tmem_ld_32x32b_x32(tbase + lane_addr + kColO + 32 * c, w);
+          ptx::tmem_wait_ld();
 #pragma unroll
-          for (int q = 0; q < 8; ++q)
-            dst[q] = make_float4(__uint_as_float(o[4 * q]) * inv_l, __uint_as_float(o[4 * q + 1]) * inv_l,
-                                 __uint_as_float(o[4 * q + 2]) * inv_l, __uint_as_float(o[4 * q + 3]) * inv_l);
+          for (int i = 0; i < 32; ++i) w[i] = __float_as_uint(__uint_as_float(w[i]) * inv_l);
+        }
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(buf + (uint32_t)h * 128u +
+                                                                       (uint32_t)((j ^ (h & 7)) << 4)),
+                       "r"(w[4 * j]), "r"(w[4 * j + 1]), "r"(w[4 * j + 2]), "r"(w[4 * j + 3])
+                       : "memory");
+        if (!group_sync()) return false;
+        // latent column of the round's first TMEM column
+        const int cc = cols * c;
+        const int d0 = (cc < 128 ? 128 * (int)rank + cc : 256 + 128 * (int)rank + (cc - 128));
+#pragma unroll
+        for (int it = 0; it < 8; ++it) {
+          const int row = 32 * sub + 4 * it + (lane >> 3), j = lane & 7;
+          uint4 q;
+          asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                       : "=r"(q.x), "=r"(q.y), "=r"(q.z), "=r"(q.w)
+                       : "r"(buf + (uint32_t)row * 128u + (uint32_t)((j ^ (row & 7)) << 4))
+                       : "memory");
+          if (pend.final_out)
+            *reinterpret_cast<uint4*>(p.o_lat + (pend.row0 + row) * kR + d0 + 8 * j) = q;
+          else
+            *reinterpret_cast<uint4*>(p.o_part + (pend.row0 + row) * kR + d0 + 4 * j) = q;
         }
       }
       if (rank == 0) {
         const float z = pend.l > 0.f ? (pend.m + log2f(pend.l)) * 0.69314718055994531f : -CUDART_INF_F;
         if (pend.final_out) {
-          if (p.lse) p.lse[pend.row] = z;
+          if (p.lse) p.lse[pend.row0 + h] = z;
         } else {
-          p.lse_part[pend.row] = z;
+          p.lse_part[pend.row0 + h] = z;
         }
       }
       ptx::tc_fence_before();
       __syncwarp();
       if (lane == 0) ptx::mbar_arrive(bar(B_O_FREE));
+      // every warp has read the staged rows: the stage goes back to the producer
+      if (!group_sync()) return false;
+      if (sub == 0 && lane == 0) {
+        ptx::fence_proxy_async_smem();   // the staged rows' reads before the next TMA load
+        ptx::mbar_arrive(bar(B_KV_EMPTY + pend.stage));
+      }
       pend.on = false;
+      return true;
     };
 
     PageCursor cur = first_page(p, plan, u_begin, u_end);
@@ -602,7 +669,8 @@ decode_pair_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_const
       if (gpg > 0 && !wait_all(bar(B_O_DONE), (gpg - 1) & 1)) { fail(); ok = false; break; }
       ptx::tc_fence_after();
       if (tracer) PAIR_TRACE(7, gpg);
-      if (pend.on) epilogue();   // the previous unit's O, before this unit's first value MMA
+      // the previous unit's O, before this unit's first value MMA
+      if (pend.on && !epilogue()) { fail(); ok = false; break; }
       ptx::tmem_st_32x32b_x32(tbase + lane_addr + kColP, ph);
       ptx::tmem_st_32x32b_x32(tbase + lane_addr + kColP + 32, pl);
       if (cur.k > 0 && any_need) {
@@ -625,19 +693,15 @@ decode_pair_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_const
       if (cur.k == u.npg - 1) {
         pend.on = true;
         pend.final_out = u.part < 0;
-        pend.row = (pend.final_out ? (int64_t)u.item * H : (int64_t)u.part * H) + h;
+        pend.row0 = pend.final_out ? (int64_t)u.item * H : (int64_t)u.part * H;
+        pend.stage = gpg % kStages;
         pend.l = l_run;
         pend.m = m_run;
       }
       advance(p, plan, u_end, cur);
       ++gpg;
     }
-    if (ok && pend.on) {
-      if (wait_all(bar(B_O_DONE), (gpg - 1) & 1))
-        epilogue();
-      else
-        fail();
-    }
+    if (ok && pend.on && !(wait_all(bar(B_O_DONE), (gpg - 1) & 1) && epilogue())) fail();
   }
 
   ptx::tc_fence_before();
