@@ -37,6 +37,7 @@ METRIC = "MLA decode: cache GB/s and TFLOP/s, fraction of B200 roofline"
 DEFAULT_WORKLOAD = "deepseek_h128_b128_ragged"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 L2_FLUSH_BYTES = 512 << 20
+L2_BYTES = 126 << 20          # B200 L2
 
 
 def load_peaks():
@@ -329,20 +330,37 @@ def run_gpu(args):
 
     # ---------------------------------------------------------------- end to end through the public API
     hostin = dec.HostInputs(step, w)
-    for _ in range(max(3, args.warmup)):
-        dec.run_e2e(step, hostin, stream)
-    torch.cuda.synchronize()
     e2e_steps = args.steps
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e2e_ms = 0.0
     barrier()
-    for k in range(e2e_steps):
-        flush.fill_(k & 0xFF)
-        e0.record(stream)
-        dec.run_e2e(step, hostin, stream)
-        e1.record(stream)
-        e1.synchronize()          # the step's result is on the host
-        e2e_ms += e0.elapsed_time(e1)
+    if cache_bytes > 2 * L2_BYTES:
+        # steps back to back, each one's copies overlapping its neighbours' kernels; the
+        # cache is larger than L2, so no flush is needed between them
+        pipe = dec.PipelinedE2E(step, hostin, stream)
+        for _ in range(max(3, args.warmup)):
+            pipe.enqueue()
+        torch.cuda.synchronize()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e0.record(pipe.copy)
+        last = None
+        for _ in range(e2e_steps):
+            last = pipe.enqueue()
+        last.synchronize()            # the last step's result is on the host
+        e2e_ms = e0.elapsed_time(last)
+        e2e_mode = "pipelined: step k+1's copies in and step k-1's copy out overlap step k"
+    else:
+        for _ in range(max(3, args.warmup)):
+            dec.run_e2e(step, hostin, stream)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e2e_ms = 0.0
+        for k in range(e2e_steps):
+            flush.fill_(k & 0xFF)
+            e0.record(stream)
+            dec.run_e2e(step, hostin, stream)
+            e1.record(stream)
+            e1.synchronize()          # the step's result is on the host
+            e2e_ms += e0.elapsed_time(e1)
+        e2e_mode = "one step at a time, L2 flushed before each"
     barrier()
     mla.mla_check_status()
     if world > 1:
@@ -351,7 +369,7 @@ def run_gpu(args):
         e2e_ms = float(t.item())
     e2e = {"value": world * cache_bytes * e2e_steps / (e2e_ms / 1e3) / 1e9, "unit": "GB/s",
            "h2d_bytes_per_step": hostin.h2d_bytes(step), "d2h_bytes_per_step": hostin.d2h_bytes(),
-           "ms_per_step": e2e_ms / e2e_steps}
+           "ms_per_step": e2e_ms / e2e_steps, "mode": e2e_mode}
 
     line = None
     if rank == 0:

@@ -94,6 +94,17 @@ class DecodeStep:
         self.combine(stream)
         self.project(stream)
 
+    def sibling(self) -> "DecodeStep":
+        """A second set of per-step buffers (queries, new rows, block table, lengths,
+        plan, workspace, intermediates, output) sharing this step's cache and weights."""
+        t = object.__new__(DecodeStep)
+        t.__dict__.update(self.__dict__)
+        for name in ("block_table", "seq_lens", "q_nope", "q_rope", "new_ckr", "q_lat", "o_lat", "lse", "out",
+                     "plan", "workspace"):
+            setattr(t, name, torch.empty_like(getattr(self, name)))
+        t.plan.copy_(self.plan)
+        return t
+
     def launches_per_step(self, append=True) -> int:
         return int(append) + 3 + int(self.info.num_parts > 0)
 
@@ -150,3 +161,61 @@ def run_e2e(step: DecodeStep, host: HostInputs, stream=None):
         step.info = info
         step.run(stream=s)
         host.out.copy_(step.out.view(host.out.dtype), non_blocking=True)
+
+
+class PipelinedE2E:
+    """Consecutive end-to-end steps through the public calls, with host inputs, where
+    step k+1's host-to-device copies and step k-1's device-to-host copy overlap step
+    k's kernels: two sets of per-step device buffers, one stream for copies in and one
+    for copies out beside the compute stream, and events for every hand-over. The host plans step k+1 while the device
+    runs step k, and waits for step k-1's result before it enqueues step k+1 (it
+    consumes results one step behind).
+    """
+
+    def __init__(self, step: DecodeStep, host: HostInputs, stream=None):
+        self.sets = [step, step.sibling()]
+        self.host = host
+        self.comp = stream or torch.cuda.current_stream()
+        self.copy = torch.cuda.Stream(device=step.device)      # host -> device
+        self.copy_out = torch.cuda.Stream(device=step.device)  # device -> host
+        self.plans = [torch.empty_like(host.plan).pin_memory() for _ in range(2)]
+        self.outs = [host.out, torch.empty_like(host.out).pin_memory()]
+        self.inputs_free = [None, None]   # compute of the set's previous step done
+        self.out_read = [None, None]      # device-to-host copy of the set's previous step done
+        self.k = 0
+
+    def enqueue(self):
+        """Plan and enqueue the next step; returns the event of its result on the host."""
+        i = self.k & 1
+        st, host = self.sets[i], self.host
+        if self.k >= 2:
+            self.out_read[i].synchronize()   # the host has the result of step k-2: consume it
+        plan, info = mla.mla_plan_splits(host.seq_lens_np, st.B, st.q_len, st.max_pages, st.dims, st.sms)
+        self.plans[i][:info.plan_words].copy_(torch.from_numpy(plan))
+        ready = torch.cuda.Event()
+        with torch.cuda.stream(self.copy):
+            if self.inputs_free[i] is not None:
+                self.copy.wait_event(self.inputs_free[i])
+            for dst, src in ((st.q_nope, host.q_nope), (st.q_rope, host.q_rope), (st.new_ckr, host.new_ckr)):
+                dst.view(torch.int16 if dst.dtype == torch.bfloat16 else dst.dtype).copy_(src, non_blocking=True)
+            st.block_table.copy_(host.block_table, non_blocking=True)
+            st.seq_lens.copy_(host.seq_lens, non_blocking=True)
+            st.plan[:info.plan_words].copy_(self.plans[i][:info.plan_words], non_blocking=True)
+            ready.record(self.copy)
+        st.info = info
+        done = torch.cuda.Event()
+        with torch.cuda.stream(self.comp):
+            self.comp.wait_event(ready)
+            if self.out_read[i] is not None:
+                self.comp.wait_event(self.out_read[i])   # the output buffer was read back
+            st.run(stream=self.comp)
+            done.record(self.comp)
+        self.inputs_free[i] = done
+        out_read = torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(self.copy_out):
+            self.copy_out.wait_event(done)
+            self.outs[i].copy_(st.out.view(self.outs[i].dtype), non_blocking=True)
+            out_read.record(self.copy_out)
+        self.out_read[i] = out_read
+        self.k += 1
+        return out_read

@@ -232,6 +232,30 @@ def test_whole_step_matches_oracle(policy, H, q_len, lens, sms):
     assert_close(out[long_ctx], exact["out"][long_ctx], False, "out vs definition")
 
 
+@pytest.mark.parametrize("H", [64, 128])
+def test_pipelined_end_to_end_steps_match_device_step(H):
+    """The pipelined end-to-end runner (host inputs, copies overlapping the neighbouring
+    steps' kernels, two buffer sets) returns, step after step, exactly the output of the
+    device-resident step."""
+    spec = small_spec(H=H)
+    w = wl.make(spec, seed=5, seq_lens=[900, 65, 1, 640, 2000])
+    step = dec.DecodeStep(w, sms=9)
+    step.run()
+    torch.cuda.synchronize()
+    want = step.out.view(torch.int16).cpu().clone()
+    hostin = dec.HostInputs(step, w)
+    pipe = dec.PipelinedE2E(step, hostin)
+    for k in range(5):
+        ev = pipe.enqueue()
+        if k >= 1:
+            prev = pipe.outs[(k - 1) & 1]
+            pipe.out_read[(k - 1) & 1].synchronize()
+            assert torch.equal(prev, want), f"step {k - 1}"
+    ev.synchronize()
+    mla.mla_check_status()
+    assert torch.equal(pipe.outs[4 & 1], want)
+
+
 def test_whole_step_tiny_fp32_matches_definition():
     w = wl.make("tiny_fp32")
     step = dec.DecodeStep(w)
