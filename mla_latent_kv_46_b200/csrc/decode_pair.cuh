@@ -55,37 +55,52 @@ constexpr int kBox = 64 * 128;              // 64 rows x 64 bf16, 128-byte swizz
 constexpr int kRopeBox = 64 * 64;           // 64 rows x 32 bf16, 64-byte swizzle
 constexpr int kStageBytes = 4 * kBox + kRopeBox;   // 36 KiB
 constexpr int kStages = 4;
-constexpr int kXBytes = kHeads * kPage * 4;        // [128 heads][64 tokens] fp32, chunk-swizzled rows
+// Exchanged partial scores keep the top 24 bits of each fp32 value: 64 scores of a
+// head = 48 words = 12 chunks of 16 B. Layout of one exchange buffer: [warp 4][chunk 12]
+// [lane 32][16 B], so each warp's 32 heads are one contiguous 6 KiB piece (one bulk copy)
+// and a warp's 16-byte accesses to one chunk are 512 contiguous bytes.
+constexpr int kXWords = 48;
+constexpr int kXWarpBytes = 32 * kXWords * 4;      // 6 KiB
+constexpr int kXBytes = 4 * kXWarpBytes;           // 24 KiB
 
 constexpr int kOffKV = 0;
-constexpr int kOffQr = kOffKV + kStages * kStageBytes;   // 2 x rope query half, 128 x 32 bf16
+constexpr int kQrBufs = 1;                               // rope query half buffers
+constexpr int kOffQr = kOffKV + kStages * kStageBytes;   // rope query half, 128 x 32 bf16
 constexpr int kQrBytes = 2 * kRopeBox;
-constexpr int kOffX = kOffQr + 2 * kQrBytes;             // the peer's partial scores
-constexpr int kOffXout = kOffX + kXBytes;                // mine, staged for the bulk copy
+constexpr int kOffX = kOffQr + kQrBufs * kQrBytes;       // 2 slots: the peer's partial scores
+constexpr int kOffXout = kOffX + 2 * kXBytes;            // mine, staged for the bulk copy
 constexpr int kOffBar = kOffXout + kXBytes;              // 32 mbarriers
 constexpr int kOffTmem = kOffBar + 32 * 8;
 constexpr int kOffAbort = kOffTmem + 8;
 constexpr int kSmemUsed = kOffAbort + 8;
+// The two threads of a head exchange page maxima (and a unit's sums) through the rope box
+// of the page's stage, idle once that page's score MMAs are done: float[2 halves][128]
+// at kOffPairMax (maxima) and kOffPairL (sums) within the stage.
+constexpr int kOffPairMax = 4 * kBox, kOffPairL = kOffPairMax + 2 * 128 * 4;
+constexpr int kThreads = 384;                            // warps 0-3 roles, 4-11 softmax
 constexpr int kSmemBytes = kSmemUsed + 1024;
 
 enum {
-  B_KV_FULL = 0,    // +stage (4)
-  B_KV_EMPTY = 4,   // +stage (4)
-  B_S_FULL = 8,     // score MMAs of a page done
-  B_S_EMPTY = 9,    // 4 softmax warps read S
-  B_X_FULL = 10,    // the peer's partial rows landed in my X (1 local arrival + tx bytes)
-  B_X_EMPTY = 11,   // the peer's 4 softmax warps have read the X I fill
-  B_P_FULL = 12,    // 4 softmax warps: P in TMEM (and O rescaled)
-  B_O_DONE = 13,    // value MMAs of a page done
-  B_QT_FULL = 14,   // query latent half staged in TMEM (4 softmax warps)
-  B_QT_EMPTY = 15,  // last score MMA of a unit done: the TMEM query columns are free
-  B_O_FREE = 16,    // 4 softmax warps have read O
-  B_DRAIN = 17,
-  B_QR_FULL = 18,   // +buffer (2): rope query half landed (TMA)
-  B_QR_EMPTY = 20,  // +buffer (2): last score MMA of the unit that used it done
-  B_GROUP = 22,     // the 4 softmax warps (epilogue staging rounds)
-  kNumBars = 23
+  B_KV_FULL = 0,     // +stage (4)
+  B_KV_EMPTY = 4,    // +stage (4)
+  B_S_FULL = 8,      // score MMAs of a page done
+  B_S_EMPTY = 9,     // 8 softmax warps read S
+  B_X_FULL = 10,     // +slot (2): the peer's partial rows landed (1 local arrival + 24 KiB tx)
+  B_X_EMPTY = 12,    // +slot (2): the peer's 8 softmax warps have read the slot I fill
+  B_XOUT_FREE = 14,  // my previous copy landed in the peer (its watcher warp saw it)
+  B_P_FULL = 15,     // 8 softmax warps: P in TMEM (and O rescaled)
+  B_O_DONE = 16,     // value MMAs of a page done
+  B_QT_FULL = 17,    // query latent half staged in TMEM (8 softmax warps)
+  B_QT_EMPTY = 18,   // last score MMA of a unit done: the TMEM query columns are free
+  B_O_FREE = 19,     // 8 softmax warps have read O
+  B_DRAIN = 20,
+  B_ALL = 21,        // the 8 softmax warps
+  B_PAIR = 22,       // +lane quarter (4): the two softmax warps of a quarter
+  B_QR_FULL = 26,    // +buffer: rope query half landed (TMA)
+  B_QR_EMPTY = 26 + kQrBufs,   // +buffer: last score MMA of the unit that used it done
+  kNumBars = 26 + 2 * kQrBufs
 };
+static_assert(kNumBars <= 32, "barrier area");
 
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColO = 0, kColQ = 256, kColS = 384, kColP = 448;
@@ -150,7 +165,7 @@ __device__ __forceinline__ void advance(const Params& p, const PlanView& plan, i
   c.valid = next_nonempty(p, plan, c.ui, u_end, c.u);
 }
 
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(256, 1)
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 decode_pair_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_constant__ CUtensorMap tm_kv_rope,
                    const __grid_constant__ CUtensorMap tm_q_rope, const Params p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -174,22 +189,27 @@ decode_pair_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_const
       ptx::mbar_init(bar(B_KV_EMPTY + s), 1);
     }
     ptx::mbar_init(bar(B_S_FULL), 1);
-    ptx::mbar_init(bar(B_S_EMPTY), 4);
-    ptx::mbar_init(bar(B_X_FULL), 1);
-    ptx::mbar_init(bar(B_X_EMPTY), 4);
-    ptx::mbar_init(bar(B_P_FULL), 4);
-    ptx::mbar_init(bar(B_O_DONE), 1);
-    ptx::mbar_init(bar(B_QT_FULL), 4);
-    ptx::mbar_init(bar(B_QT_EMPTY), 1);
+    ptx::mbar_init(bar(B_S_EMPTY), 8);
     for (int b = 0; b < 2; ++b) {
+      ptx::mbar_init(bar(B_X_FULL + b), 1);
+      ptx::mbar_init(bar(B_X_EMPTY + b), 8);
+    }
+    ptx::mbar_init(bar(B_XOUT_FREE), 1);
+    ptx::mbar_init(bar(B_P_FULL), 8);
+    ptx::mbar_init(bar(B_O_DONE), 1);
+    ptx::mbar_init(bar(B_QT_FULL), 8);
+    ptx::mbar_init(bar(B_QT_EMPTY), 1);
+    for (int b = 0; b < kQrBufs; ++b) {
       ptx::mbar_init(bar(B_QR_FULL + b), 1);
       ptx::mbar_init(bar(B_QR_EMPTY + b), 1);
     }
-    ptx::mbar_init(bar(B_O_FREE), 4);
+    ptx::mbar_init(bar(B_O_FREE), 8);
     ptx::mbar_init(bar(B_DRAIN), 1);
-    ptx::mbar_init(bar(B_GROUP), 4);
+    ptx::mbar_init(bar(B_ALL), 8);
+    for (int q = 0; q < 4; ++q) ptx::mbar_init(bar(B_PAIR + q), 2);
     ptx::fence_mbar_init();
-    ptx::mbar_arrive_expect_tx(bar(B_X_FULL), kXBytes);   // armed for the first page
+    ptx::mbar_arrive_expect_tx(bar(B_X_FULL), kXBytes);       // armed for pages 0 and 1
+    ptx::mbar_arrive_expect_tx(bar(B_X_FULL + 1), kXBytes);
   }
   if (warp == 2) {
     ptx::tmem_alloc(sbase + kOffTmem, kTmemCols);
@@ -252,8 +272,8 @@ decode_pair_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_const
         // this CTA's rope query half for the unit's 128 heads, into buffer n & 1 (free once
         // the unit two back has finished its scores: the page stream never waits for the
         // current unit's scores)
-        const uint32_t qb = c.n & 1;
-        if (!wait_all(bar(B_QR_EMPTY + qb), ((c.n >> 1) & 1) ^ 1)) {
+        const uint32_t qb = c.n % kQrBufs;
+        if (!wait_all(bar(B_QR_EMPTY + qb), ((c.n / kQrBufs) & 1) ^ 1)) {
           if (leader) fail();
           ok = false;
           break;
@@ -296,8 +316,8 @@ decode_pair_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_const
     // copies still in flight land in this CTA's shared memory: wait (bounded) for them
     for (uint32_t k = (gpg >= kStages ? gpg - kStages : 0); k < gpg; ++k)
       wait_all(bar(B_KV_FULL + k % kStages), (k / kStages) & 1);
-    for (uint32_t n = (nq >= 2 ? nq - 2 : 0); n < nq; ++n)
-      wait_all(bar(B_QR_FULL + (n & 1)), (n >> 1) & 1);
+    for (uint32_t n = (nq >= kQrBufs ? nq - kQrBufs : 0); n < nq; ++n)
+      wait_all(bar(B_QR_FULL + n % kQrBufs), (n / kQrBufs) & 1);
   } else if (warp == 1) {
     // ================================================================ MMA issuer
     const bool leader = ptx::elect_one();
@@ -307,8 +327,9 @@ decode_pair_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_const
     PageCursor vc = sc;                                      // next value MMA
     uint32_t gs = 0, gv = 0;
     auto issue_s = [&]() -> bool {
-      const uint32_t qb = sc.n & 1;
-      if (sc.k == 0 && (!wait_all(bar(B_QT_FULL), sc.n & 1) || !wait_all(bar(B_QR_FULL + qb), (sc.n >> 1) & 1)))
+      const uint32_t qb = sc.n % kQrBufs;
+      if (sc.k == 0 &&
+          (!wait_all(bar(B_QT_FULL), sc.n & 1) || !wait_all(bar(B_QR_FULL + qb), (sc.n / kQrBufs) & 1)))
         return false;
       const uint64_t dQr = ptx::sdesc_sw64(sbase + kOffQr + qb * kQrBytes, 512);
       const uint32_t st = gs % kStages;
@@ -378,18 +399,50 @@ decode_pair_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_const
     if (leader) ptx::umma_commit(bar(B_DRAIN));
     __syncwarp();
     wait_all(bar(B_DRAIN), 0);
+  } else if (warp == 3) {
+    // ================================================================ exchange watcher
+    // A bulk copy into another CTA reports only to the destination's mbarrier: this warp
+    // tells the peer when each of its copies has landed here, so that the peer may refill
+    // the staging rows the copy read.
+    PageCursor c = first_page(p, plan, u_begin, u_end);
+    uint32_t g = 0;
+    while (c.valid) {
+      if (!wait_all(bar(B_X_FULL + (g & 1)), (g >> 1) & 1)) {
+        if (lane == 0) fail();
+        break;
+      }
+      if (lane == 0) ptx::mbar_arrive_cluster_relaxed(peer_addr(bar(B_XOUT_FREE)));
+      advance(p, plan, u_end, c);
+      ++g;
+    }
   } else if (warp >= 4) {
     // ================================================================ query staging, exchange, softmax, epilogue
-    const int sub = warp & 3;
+    // Warp 4 + 4f + q (f = 0, 1; q = 0..3) serves TMEM lane quarter q, i.e. heads 32q..32q+31,
+    // and token half f of every page (tokens 32f..32f+31): the two threads of a head (same
+    // lane in warps 4+q and 8+q) meet on the quarter's pair barrier to combine their
+    // maxima (and, in the epilogue, their sums).
+    const int sw = warp - 4;
+    const int sub = sw & 3, hf = sw >> 2;
     const int h = 32 * sub + lane;                 // this thread's head (TMEM lane)
-    const bool tracer = sub == 0 && lane == 0;
+    const bool tracer = sw == 0 && lane == 0;
     const uint32_t lane_addr = (32u * sub) << 16;
-    // row h of X and of the staging buffer: 64 fp32 = 16 chunks of 16 B, chunk c stored
-    // at (c & 8) | ((c ^ h) & 7) so that 8 consecutive heads hit distinct bank groups
-    const uint32_t x_row = sbase + kOffX + (uint32_t)h * 256u;
-    const uint32_t xo_row = sbase + kOffXout + (uint32_t)h * 256u;
-    auto chunk = [&](int c) -> uint32_t { return (uint32_t)(((c & 8) | ((c ^ h) & 7)) << 4); };
+    // this thread's 6 chunks of 16 B in an exchange buffer (see kXWords): quarter piece
+    // sub, chunks 6f..6f+5, lane; and its warp's 3 KiB run of chunks (one bulk copy)
+    const uint32_t x_lane = (uint32_t)sub * kXWarpBytes + (uint32_t)(6 * hf) * 512u + (uint32_t)lane * 16u;
+    const uint32_t x_run = (uint32_t)sub * kXWarpBytes + (uint32_t)hf * 3072u;
+    const uint32_t xo_lane = sbase + kOffXout + x_lane;
+    auto pair_slot = [&](uint32_t stage, int off) {
+      return reinterpret_cast<volatile float*>(smem + kOffKV + stage * kStageBytes + off);
+    };
+    uint32_t n_pair = 0, n_all = 0;
     bool ok = true;
+    auto bounded_sync = [&](uint32_t b, uint32_t& n) -> bool {
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive(bar(b));
+      const bool done = ptx::mbar_wait_bounded(bar(b), n & 1, abort_flag, p.timeout_ns);
+      ++n;
+      return __all_sync(0xffffffffu, done);
+    };
 
     // Units without a visible token: o = 0 (this CTA's latent half), lse = -inf (CTA 0).
     for (int32_t ui = u_begin; ui < u_end; ++ui) {
@@ -397,7 +450,7 @@ decode_pair_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_const
       if (u.npg > 0) continue;
       const bool final_out = u.part < 0;
       const int64_t row0 = final_out ? (int64_t)u.item * H : (int64_t)u.part * H;
-      for (int e = threadIdx.x - 128; e < kHeads * 256; e += 128) {
+      for (int e = threadIdx.x - 128; e < kHeads * 256; e += kThreads - 128) {
         const int hh = e / 256, j = e % 256;
         const int d = (j < 128 ? 128 * (int)rank : 256 + 128 * (int)rank) + (j & 127);
         if (final_out)
@@ -405,7 +458,7 @@ decode_pair_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_const
         else
           p.o_part[(row0 + hh) * kR + d] = 0.f;
       }
-      if (rank == 0) {
+      if (rank == 0 && hf == 0) {
         if (final_out) {
           if (p.lse) p.lse[row0 + h] = -CUDART_INF_F;
         } else {
@@ -414,62 +467,78 @@ decode_pair_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_const
       }
     }
 
-    // Stage a unit's query: own latent half of head h, 256 bf16 -> 128 TMEM columns.
+    // Stage a unit's query: this thread's 128 of head h's own 256 latent dims
+    // (128r.. for f = 0, 256+128r.. for f = 1) -> TMEM columns 64f..64f+63.
     auto stage_q = [&](const UnitInfo& u, uint32_t n) -> bool {
       if (!wait_all(bar(B_QT_EMPTY), (n & 1) ^ 1)) return false;
       ptx::tc_fence_after();
       const uint4* src = reinterpret_cast<const uint4*>(p.q_lat + ((int64_t)u.item * H + h) * kR);
-      // two rounds of 16 loads: columns 64c..64c+63 = the 128 contiguous latent dims of
-      // tile c (128r.. for c = 0, 256+128r.. for c = 1), in stage-slot order
-#pragma unroll 1
-      for (int c = 0; c < 2; ++c) {
-        const int dim0 = 256 * c + 128 * (int)rank;
-        uint32_t w[2][32];
+      const int dim0 = 256 * hf + 128 * (int)rank;
+      uint32_t w[2][32];
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const uint4 v = __ldg(src + dim0 / 8 + i);
-          w[i >> 3][4 * (i & 7) + 0] = v.x;
-          w[i >> 3][4 * (i & 7) + 1] = v.y;
-          w[i >> 3][4 * (i & 7) + 2] = v.z;
-          w[i >> 3][4 * (i & 7) + 3] = v.w;
-        }
-        ptx::tmem_st_32x32b_x32(tbase + lane_addr + kColQ + 64 * c, w[0]);
-        ptx::tmem_st_32x32b_x32(tbase + lane_addr + kColQ + 64 * c + 32, w[1]);
+      for (int i = 0; i < 16; ++i) {
+        const uint4 v = __ldg(src + dim0 / 8 + i);
+        w[i >> 3][4 * (i & 7) + 0] = v.x;
+        w[i >> 3][4 * (i & 7) + 1] = v.y;
+        w[i >> 3][4 * (i & 7) + 2] = v.z;
+        w[i >> 3][4 * (i & 7) + 3] = v.w;
       }
+      ptx::tmem_st_32x32b_x32(tbase + lane_addr + kColQ + 64 * hf, w[0]);
+      ptx::tmem_st_32x32b_x32(tbase + lane_addr + kColQ + 64 * hf + 32, w[1]);
       ptx::tmem_wait_st();
       ptx::tc_fence_before();
       __syncwarp();
       if (lane == 0) ptx::mbar_arrive(bar(B_QT_FULL));
       return true;
     };
-    // Exchange of global page g, in two steps: read_s moves S from TMEM to registers and
-    // frees the score buffer; send_s stages the rows and copies them to the peer.
-    auto read_s = [&](uint32_t g, float (&s)[64]) -> bool {
+    // Exchange of global page g: move this thread's 32 scores out of TMEM into `own`
+    // (freeing the score buffer), keep the top 24 bits of each, stage them and bulk-copy
+    // this warp's run into the peer's slot g & 1.
+    auto exchange = [&](uint32_t g, float (&own)[32]) -> bool {
       if (!wait_all(bar(B_S_FULL), g & 1)) return false;
       if (tracer) PAIR_TRACE(3, g);
       ptx::tc_fence_after();
-      ptx::tmem_ld_32x32b_x64(tbase + lane_addr + kColS, s);
-      ptx::tmem_wait_ld();
+      {
+        uint32_t r[32];
+        ptx::tmem_ld_32x32b_x32(tbase + lane_addr + kColS + 32 * hf, r);
+        ptx::tmem_wait_ld();
+#pragma unroll
+        for (int t = 0; t < 32; ++t) own[t] = __uint_as_float(r[t]);
+      }
       ptx::tc_fence_before();
       __syncwarp();
       if (lane == 0) ptx::mbar_arrive(bar(B_S_EMPTY));
-      return true;
-    };
-    auto send_s = [&](const PageCursor& c, uint32_t g, const float (&s)[64]) -> bool {
-      // the peer has read my previous copy: its X and my staging rows are free
-      if (!wait_all_cluster(bar(B_X_EMPTY), (g & 1) ^ 1)) return false;
+      // my copy of page g-1 has landed in the peer (the staging rows are free), and the
+      // peer has read its slot g & 1 (page g-2)
+      if (!wait_all(bar(B_XOUT_FREE), (g & 1) ^ 1) ||
+          !wait_all_cluster(bar(B_X_EMPTY + (g & 1)), ((g >> 1) & 1) ^ 1))
+        return false;
       if (tracer) PAIR_TRACE(4, g);
+      ptx::fence_proxy_async_smem();   // the previous copy's reads before these writes
 #pragma unroll
-      for (int q = 0; q < 16; ++q)
-        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(xo_row + chunk(q)), "r"(__float_as_uint(s[4 * q])),
-                     "r"(__float_as_uint(s[4 * q + 1])), "r"(__float_as_uint(s[4 * q + 2])),
-                     "r"(__float_as_uint(s[4 * q + 3]))
-                     : "memory");
+      for (int r = 0; r < 2; ++r) {
+        // 16 values -> 12 words (bytes 1-3 of each value) -> 3 chunks
+        uint32_t w[12];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const float* f = own + 16 * r + 4 * q;
+          const uint32_t a = __float_as_uint(f[0]), b = __float_as_uint(f[1]);
+          const uint32_t c = __float_as_uint(f[2]), d = __float_as_uint(f[3]);
+          w[3 * q] = __byte_perm(a, b, 0x5321);
+          w[3 * q + 1] = __byte_perm(b, c, 0x6532);
+          w[3 * q + 2] = __byte_perm(c, d, 0x7653);
+        }
+#pragma unroll
+        for (int c = 0; c < 3; ++c)
+          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(xo_lane + 512u * (3 * r + c)),
+                       "r"(w[4 * c]), "r"(w[4 * c + 1]), "r"(w[4 * c + 2]), "r"(w[4 * c + 3])
+                       : "memory");
+      }
       ptx::fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0)
-        ptx::bulk_copy_to_cluster(peer_addr(sbase + kOffX + 8192u * sub), sbase + kOffXout + 8192u * sub, 8192u,
-                                  peer_addr(bar(B_X_FULL)));
+        ptx::bulk_copy_to_cluster(peer_addr(sbase + kOffX + (g & 1) * kXBytes + x_run), sbase + kOffXout + x_run,
+                                  3072u, peer_addr(bar(B_X_FULL + (g & 1))));
       return true;
     };
     // Once the score MMA of a unit's last page is done (its S was read), the query
@@ -480,42 +549,39 @@ decode_pair_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_const
       UnitInfo nu;
       return !next_nonempty(p, plan, ui, u_end, nu) || stage_q(nu, c.n + 1);
     };
-    // Epilogue of a unit, run during the next unit's first page (or after the last page
-    // of the slot) once the unit's last value MMAs are done: O[h][:] / l to the output.
-    // The rows go out through the unit's last stage (released to the producer at the
-    // end), so that each warp store writes whole 128-byte row segments.
+    // Epilogue of a unit, run after the next unit's first P (or after the last page of
+    // the slot) once the unit's last value MMAs are done: O[h][:] / l to the output. This
+    // thread holds O columns 128f..128f+127; the warps of token half f stage their rows in
+    // 16 KiB f of the unit's last stage (released to the producer at the end), and a warp
+    // reads back only its own 32 rows, so that each warp store writes whole 128-byte row
+    // segments.
     struct Pending {
       bool on;
       bool final_out;
       int64_t row0;      // output row of head 0
       uint32_t stage;    // stage of the unit's last page
-      float l, m;
+      float l, m;        // this thread's half of l; the shared reference maximum
     } pend{false, false, 0, 0u, 0.f, 0.f};
-    uint32_t ngroup = 0;
-    auto group_sync = [&]() -> bool {
-      __syncwarp();
-      if (lane == 0) ptx::mbar_arrive(bar(B_GROUP));
-      const bool done = ptx::mbar_wait_bounded(bar(B_GROUP), ngroup & 1, abort_flag, p.timeout_ns);
-      ++ngroup;
-      return __all_sync(0xffffffffu, done);
-    };
     auto epilogue = [&]() -> bool {
+      // l = the two halves' sums
+      volatile float* ls = pair_slot(pend.stage, kOffPairL);
+      ls[128 * hf + h] = pend.l;
+      if (!bounded_sync(B_PAIR + sub, n_pair)) return false;
+      const float l = pend.l + ls[128 * (hf ^ 1) + h];
       ptx::tc_fence_after();
-      const float inv_l = pend.l > 0.f ? 1.f / pend.l : 0.f;
-      const uint32_t stg = sbase + kOffKV + pend.stage * kStageBytes;
-      // a round stages 128 rows x 128 B (64 bf16 or 32 fp32 columns) in one of two 16 KiB
-      // halves of the stage; row h's 16-byte chunk j sits at j ^ (h & 7)
-      const int rounds = pend.final_out ? 4 : 8;
+      const float inv_l = l > 0.f ? 1.f / l : 0.f;
+      const uint32_t buf = sbase + kOffKV + pend.stage * kStageBytes + (uint32_t)hf * 16384u;
+      const int rounds = pend.final_out ? 2 : 4;     // 64 bf16 or 32 fp32 columns per round
       const int cols = pend.final_out ? 64 : 32;
 #pragma unroll 1
       for (int c = 0; c < rounds; ++c) {
-        const uint32_t buf = stg + (uint32_t)(c & 1) * 16384u;
+        const int col0 = 128 * hf + cols * c;        // TMEM column of the round
         uint32_t w[32];
         if (pend.final_out) {
 #pragma unroll
           for (int half = 0; half < 2; ++half) {
             uint32_t o[32];
-            ptx::tmem_ld_32x32b_x32(tbase + lane_addr + kColO + 64 * c + 32 * half, o);
+            ptx::tmem_ld_32x32b_x32(tbase + lane_addr + kColO + col0 + 32 * half, o);
             ptx::tmem_wait_ld();
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
@@ -525,21 +591,20 @@ decode_pair_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_const
             }
           }
         } else {
-          ptx::tmem_ld_32x32b_x32(tbase + lane_addr + kColO + 32 * c, w);
+          ptx::tmem_ld_32x32b_x32(tbase + lane_addr + kColO + col0, w);
           ptx::tmem_wait_ld();
 #pragma unroll
           for (int i = 0; i < 32; ++i) w[i] = __float_as_uint(__uint_as_float(w[i]) * inv_l);
         }
+        __syncwarp();   // this warp's previous round has been read back
 #pragma unroll
         for (int j = 0; j < 8; ++j)
           asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(buf + (uint32_t)h * 128u +
                                                                        (uint32_t)((j ^ (h & 7)) << 4)),
                        "r"(w[4 * j]), "r"(w[4 * j + 1]), "r"(w[4 * j + 2]), "r"(w[4 * j + 3])
                        : "memory");
-        if (!group_sync()) return false;
-        // latent column of the round's first TMEM column
-        const int cc = cols * c;
-        const int d0 = (cc < 128 ? 128 * (int)rank + cc : 256 + 128 * (int)rank + (cc - 128));
+        __syncwarp();
+        const int d0 = (col0 < 128 ? 128 * (int)rank + col0 : 256 + 128 * (int)rank + (col0 - 128));
 #pragma unroll
         for (int it = 0; it < 8; ++it) {
           const int row = 32 * sub + 4 * it + (lane >> 3), j = lane & 7;
@@ -554,8 +619,8 @@ decode_pair_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_const
             *reinterpret_cast<uint4*>(p.o_part + (pend.row0 + row) * kR + d0 + 4 * j) = q;
         }
       }
-      if (rank == 0) {
-        const float z = pend.l > 0.f ? (pend.m + log2f(pend.l)) * 0.69314718055994531f : -CUDART_INF_F;
+      if (rank == 0 && hf == 0) {
+        const float z = l > 0.f ? (pend.m + log2f(l)) * 0.69314718055994531f : -CUDART_INF_F;
         if (pend.final_out) {
           if (p.lse) p.lse[pend.row0 + h] = z;
         } else {
@@ -566,8 +631,8 @@ decode_pair_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_const
       __syncwarp();
       if (lane == 0) ptx::mbar_arrive(bar(B_O_FREE));
       // every warp has read the staged rows: the stage goes back to the producer
-      if (!group_sync()) return false;
-      if (sub == 0 && lane == 0) {
+      if (!bounded_sync(B_ALL, n_all)) return false;
+      if (sw == 0 && lane == 0) {
         ptx::fence_proxy_async_smem();   // the staged rows' reads before the next TMA load
         ptx::mbar_arrive(bar(B_KV_EMPTY + pend.stage));
       }
@@ -578,9 +643,9 @@ decode_pair_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_const
     PageCursor cur = first_page(p, plan, u_begin, u_end);
     PageCursor ex = cur;
     uint32_t gpg = 0;
+    float own[32];   // this thread's partial scores for the page read next
     if (cur.valid) {
-      float s0[64];
-      if (!stage_q(cur.u, 0) || !read_s(0, s0) || !stage_next_q(ex) || !send_s(ex, 0, s0)) { fail(); ok = false; }
+      if (!stage_q(cur.u, 0) || !exchange(0, own) || !stage_next_q(ex)) { fail(); ok = false; }
       advance(p, plan, u_end, ex);
     }
     float m_run = -CUDART_INF_F, l_run = 0.f;
@@ -590,68 +655,80 @@ decode_pair_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_const
         m_run = -CUDART_INF_F;
         l_run = 0.f;
       }
-      // ------------------------------------------------ full scores of head h: mine + the peer's
-      // the next page's scores leave TMEM first (the score MMA after it can start)
-      float sn[64];
-      if (ex.valid && (!read_s(gpg + 1, sn) || !stage_next_q(ex))) { fail(); ok = false; break; }
-      if (!wait_all(bar(B_X_FULL), gpg & 1)) { fail(); ok = false; break; }
+      // ------------------------------------------------ the next page's exchange goes first
+      float nxt[32];
+      const bool more = ex.valid;
+      if (more && (!exchange(gpg + 1, nxt) || !stage_next_q(ex))) { fail(); ok = false; break; }
+      // ------------------------------------------------ full scores: mine + the peer's
+      const uint32_t xs = gpg & 1;
+      if (!wait_all(bar(B_X_FULL + xs), (gpg >> 1) & 1)) { fail(); ok = false; break; }
       if (tracer) PAIR_TRACE(5, gpg);
-      float v[64];
+      float v[32];
 #pragma unroll
-      for (int c = 0; c < 16; ++c) {
-        uint4 a, b;
-        asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
-                     : "=r"(a.x), "=r"(a.y), "=r"(a.z), "=r"(a.w)
-                     : "r"(xo_row + chunk(c))
-                     : "memory");
-        asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
-                     : "=r"(b.x), "=r"(b.y), "=r"(b.z), "=r"(b.w)
-                     : "r"(x_row + chunk(c))
-                     : "memory");
-        v[4 * c + 0] = __uint_as_float(a.x) + __uint_as_float(b.x);
-        v[4 * c + 1] = __uint_as_float(a.y) + __uint_as_float(b.y);
-        v[4 * c + 2] = __uint_as_float(a.z) + __uint_as_float(b.z);
-        v[4 * c + 3] = __uint_as_float(a.w) + __uint_as_float(b.w);
+      for (int r = 0; r < 2; ++r) {
+        uint32_t w[12];
+#pragma unroll
+        for (int c = 0; c < 3; ++c)
+          asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                       : "=r"(w[4 * c]), "=r"(w[4 * c + 1]), "=r"(w[4 * c + 2]), "=r"(w[4 * c + 3])
+                       : "r"(sbase + kOffX + xs * kXBytes + x_lane + 512u * (3 * r + c))
+                       : "memory");
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          // the peer's values, bytes 1-3 (byte 0 is noise below the kept precision)
+          const int t = 16 * r + 4 * q;
+          v[t + 0] = own[t + 0] + __uint_as_float(w[3 * q] << 8);
+          v[t + 1] = own[t + 1] + __uint_as_float(__byte_perm(w[3 * q], w[3 * q + 1], 0x5433));
+          v[t + 2] = own[t + 2] + __uint_as_float(__byte_perm(w[3 * q + 1], w[3 * q + 2], 0x4322));
+          v[t + 3] = own[t + 3] + __uint_as_float(w[3 * q + 2]);
+        }
       }
       // ------------------------------------------------ this page's maximum and reference
-      const int32_t tok0 = (u.pb + cur.k) * kPage;
-      if (tok0 + kPage > u.ntok) {
+      const int32_t tok0 = (u.pb + cur.k) * kPage + 32 * hf;
+      if (tok0 + 32 > u.ntok) {
 #pragma unroll
-        for (int t = 0; t < kPage; ++t) v[t] = (tok0 + t < u.ntok) ? v[t] : -CUDART_INF_F;
+        for (int t = 0; t < 32; ++t) v[t] = (tok0 + t < u.ntok) ? v[t] : -CUDART_INF_F;
       }
       float mx;
       {
-        float t8[8];
+        float t4[4];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
+        for (int i = 0; i < 4; ++i) {
           const float a = fmaxf(fmaxf(v[8 * i], v[8 * i + 1]), fmaxf(v[8 * i + 2], v[8 * i + 3]));
           const float b = fmaxf(fmaxf(v[8 * i + 4], v[8 * i + 5]), fmaxf(v[8 * i + 6], v[8 * i + 7]));
-          t8[i] = fmaxf(a, b);
+          t4[i] = fmaxf(a, b);
         }
-        mx = fmaxf(fmaxf(fmaxf(t8[0], t8[1]), fmaxf(t8[2], t8[3])), fmaxf(fmaxf(t8[4], t8[5]), fmaxf(t8[6], t8[7])));
+        mx = fmaxf(fmaxf(t4[0], t4[1]), fmaxf(t4[2], t4[3]));
       }
-      mx *= p.scale_log2;
-      const bool need = mx > m_run + kRescaleThreshold;
-      // The vote depends on every lane's loaded rows, so all of this warp's reads of X
-      // are complete when lane 0 tells the peer that X may be overwritten.
-      const bool any_need = __any_sync(0xffffffffu, need);
+      // The vote depends on every lane's loaded values, so all of this warp's reads of
+      // the slot are complete when lane 0 tells the peer that it may be overwritten.
+      ptx::vote_any_ordered(mx > -CUDART_INF_F);
       if (lane == 0) {
-        if (sub == 0) ptx::mbar_arrive_expect_tx(bar(B_X_FULL), kXBytes);   // arm the next page's phase
-        ptx::mbar_arrive_cluster_relaxed(peer_addr(bar(B_X_EMPTY)));
+        if (sw == 0) ptx::mbar_arrive_expect_tx(bar(B_X_FULL + xs), kXBytes);   // arm the slot's next use
+        ptx::mbar_arrive_cluster_relaxed(peer_addr(bar(B_X_EMPTY + xs)));
       }
-      // ------------------------------------------------ next page's exchange, overlapping this softmax
-      if (ex.valid) {
-        if (!send_s(ex, gpg + 1, sn)) { fail(); ok = false; break; }
+      // the head's maximum over both token halves
+      {
+        volatile float* ms = pair_slot(gpg % kStages, kOffPairMax);
+        ms[128 * hf + h] = mx;
+        if (!bounded_sync(B_PAIR + sub, n_pair)) { fail(); ok = false; break; }
+        mx = fmaxf(mx, ms[128 * (hf ^ 1) + h]) * p.scale_log2;
+      }
+      const bool need = mx > m_run + kRescaleThreshold;
+      const bool any_need = __any_sync(0xffffffffu, need);
+      if (more) {
+#pragma unroll
+        for (int t = 0; t < 32; ++t) own[t] = nxt[t];
         advance(p, plan, u_end, ex);
       }
-      // ------------------------------------------------ softmax of head h (identical in both CTAs)
+      // ------------------------------------------------ softmax of head h, this thread's 32 tokens
       const float mu = need ? mx : m_run;
       const float al = need ? ptx::ex2(m_run - mu) : 1.f;
       const float nz = (mu == -CUDART_INF_F) ? 0.f : -mu;
-      uint32_t ph[32], pl[32];
+      uint32_t ph[16], pl[16];
       float sum4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-      for (int i = 0; i < 32; ++i) {
+      for (int i = 0; i < 16; ++i) {
         const float a0 = ptx::ex2(fmaf(v[2 * i], p.scale_log2, nz));
         const float a1 = ptx::ex2(fmaf(v[2 * i + 1], p.scale_log2, nz));
         sum4[i & 3] += a0 + a1;
@@ -669,26 +746,29 @@ decode_pair_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_const
       if (gpg > 0 && !wait_all(bar(B_O_DONE), (gpg - 1) & 1)) { fail(); ok = false; break; }
       ptx::tc_fence_after();
       if (tracer) PAIR_TRACE(7, gpg);
-      // the previous unit's O, before this unit's first value MMA
-      if (pend.on && !epilogue()) { fail(); ok = false; break; }
-      ptx::tmem_st_32x32b_x32(tbase + lane_addr + kColP, ph);
-      ptx::tmem_st_32x32b_x32(tbase + lane_addr + kColP + 32, pl);
+      ptx::tmem_st_32x32b_x16u(tbase + lane_addr + kColP + 16 * hf, ph);
+      ptx::tmem_st_32x32b_x16u(tbase + lane_addr + kColP + 32 + 16 * hf, pl);
       if (cur.k > 0 && any_need) {
-        // a moved reference: O[h][:] *= 2^(m_old - m_new) (1 for heads that kept theirs)
+        // a moved reference: O[h][:] *= 2^(m_old - m_new) (1 for heads that kept theirs);
+        // this thread scales its 128 columns
 #pragma unroll 1
-        for (int c = 0; c < 8; ++c) {
+        for (int c = 0; c < 4; ++c) {
           uint32_t o[32];
-          ptx::tmem_ld_32x32b_x32(tbase + lane_addr + kColO + 32 * c, o);
+          const uint32_t ta = tbase + lane_addr + kColO + 128 * hf + 32 * c;
+          ptx::tmem_ld_32x32b_x32(ta, o);
           ptx::tmem_wait_ld();
 #pragma unroll
           for (int j = 0; j < 32; ++j) o[j] = __float_as_uint(__uint_as_float(o[j]) * al);
-          ptx::tmem_st_32x32b_x32(tbase + lane_addr + kColO + 32 * c, o);
+          ptx::tmem_st_32x32b_x32(ta, o);
         }
       }
       ptx::tmem_wait_st();
       ptx::tc_fence_before();
+      ptx::fence_proxy_async_smem();   // the rope box's use above before the stage's next load
       __syncwarp();
       if (lane == 0) ptx::mbar_arrive(bar(B_P_FULL));
+      // the previous unit's O; this unit's first value MMA also waits for it (O_FREE)
+      if (pend.on && !epilogue()) { fail(); ok = false; break; }
 
       if (cur.k == u.npg - 1) {
         pend.on = true;

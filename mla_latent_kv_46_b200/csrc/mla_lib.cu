@@ -495,7 +495,7 @@ mla_status mla_decode_attn(const void* q_lat, const void* q_rope, const void* kv
       if (mla_status s = make_map_2d(&tqr, q_rope, d.Dr, (uint64_t)T * d.H, (uint64_t)d.Dr * 2, 64, 32)) return s;
       if (mla_status s = ensure_smem_attr((const void*)mla::pair::decode_pair_kernel, mla::pair::kSmemBytes))
         return s;
-      mla::pair::decode_pair_kernel<<<grid, 256, mla::pair::kSmemBytes, st>>>(tk, tkr, tqr, p);
+      mla::pair::decode_pair_kernel<<<grid, mla::pair::kThreads, mla::pair::kSmemBytes, st>>>(tk, tkr, tqr, p);
       return launch_check("decode_attn (tcgen05, CTA pair)");
     }
     mla::tc::decode_kernel<<<grid, 256, mla::tc::kSmemBytes, st>>>(tq, tr, tk, p);
