@@ -732,12 +732,14 @@ decode_pair_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_const
         const float a0 = ptx::ex2(fmaf(v[2 * i], p.scale_log2, nz));
         const float a1 = ptx::ex2(fmaf(v[2 * i + 1], p.scale_log2, nz));
         sum4[i & 3] += a0 + a1;
-        __nv_bfloat162 hi = __floats2bfloat162_rn(a0, a1);
-        const uint32_t hw = *reinterpret_cast<uint32_t*>(&hi);
-        __nv_bfloat162 lo =
-            __floats2bfloat162_rn(a0 - __uint_as_float(hw << 16), a1 - __uint_as_float(hw & 0xFFFF0000u));
-        ph[i] = hw;
-        pl[i] = *reinterpret_cast<uint32_t*>(&lo);
+        // P_hi = the top 16 bits of p (bf16 truncation), P_lo = the top 16 bits of the
+        // exact remainder: P_hi + P_lo is within 2^-15 of p, with integer and FMA-pipe
+        // operations only (no conversions on the special-function pipe, which the
+        // exponentials already load)
+        const uint32_t u0 = __float_as_uint(a0), u1 = __float_as_uint(a1);
+        ph[i] = __byte_perm(u0, u1, 0x7632);
+        const float r0 = a0 - __uint_as_float(u0 & 0xFFFF0000u), r1 = a1 - __uint_as_float(u1 & 0xFFFF0000u);
+        pl[i] = __byte_perm(__float_as_uint(r0), __float_as_uint(r1), 0x7632);
       }
       l_run = l_run * al + ((sum4[0] + sum4[1]) + (sum4[2] + sum4[3]));
       m_run = mu;

@@ -466,8 +466,8 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_qlat, const __grid_constant
         const bool need_a = mx_a > m_a + kRescaleThreshold;
         const bool need_b = mx_b > m_b + kRescaleThreshold;
         const float mu_a = need_a ? mx_a : m_a, mu_b = need_b ? mx_b : m_b;
-        const float al_a = need_a ? exp2f(m_a - mu_a) : 1.f;   // 0 when m was -inf
-        const float al_b = need_b ? exp2f(m_b - mu_b) : 1.f;
+        const float al_a = need_a ? ptx::ex2(m_a - mu_a) : 1.f;   // 0 when m was -inf
+        const float al_b = need_b ? ptx::ex2(m_b - mu_b) : 1.f;
         float* alpha = alpha_s + 64 * st;
         if ((lane & 3) == 0) {
           alpha[ha] = al_a;
@@ -476,25 +476,25 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_qlat, const __grid_constant
         if (__any_sync(0xffffffffu, need_a || need_b) && lane == 0) need_w[st] = gpg;
         const float za = (mu_a == -CUDART_INF_F) ? 0.f : mu_a;
         const float zb = (mu_b == -CUDART_INF_F) ? 0.f : mu_b;
-        // P split into a bf16 high part and a bf16 remainder: the value MMA runs on
-        // both, so P enters the sum with ~16 significant bits instead of 8.
+        // P split into a bf16 high part (the top 16 bits of p) and a bf16 remainder (the
+        // top 16 bits of p - P_hi): the value MMA runs on both, so P enters the sum
+        // within 2^-15 of p instead of 2^-8; integer operations only, no conversions.
         uint32_t pk[16], pl[16];
         float sa = 0.f, sb = 0.f;
+        auto split = [](float x, float y, uint32_t& hi, uint32_t& lo) {
+          const uint32_t ux = __float_as_uint(x), uy = __float_as_uint(y);
+          hi = __byte_perm(ux, uy, 0x7632);
+          const float rx = x - __uint_as_float(ux & 0xFFFF0000u), ry = y - __uint_as_float(uy & 0xFFFF0000u);
+          lo = __byte_perm(__float_as_uint(rx), __float_as_uint(ry), 0x7632);
+        };
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
-          const float a0 = exp2f(v[4 * i] - za), a1 = exp2f(v[4 * i + 1] - za);
-          const float b0 = exp2f(v[4 * i + 2] - zb), b1 = exp2f(v[4 * i + 3] - zb);
+          const float a0 = ptx::ex2(v[4 * i] - za), a1 = ptx::ex2(v[4 * i + 1] - za);
+          const float b0 = ptx::ex2(v[4 * i + 2] - zb), b1 = ptx::ex2(v[4 * i + 3] - zb);
           sa += a0 + a1;
           sb += b0 + b1;
-          __nv_bfloat162 ha2 = __floats2bfloat162_rn(a0, a1);
-          __nv_bfloat162 hb2 = __floats2bfloat162_rn(b0, b1);
-          const float2 fa = __bfloat1622float2(ha2), fb = __bfloat1622float2(hb2);
-          __nv_bfloat162 la2 = __floats2bfloat162_rn(a0 - fa.x, a1 - fa.y);
-          __nv_bfloat162 lb2 = __floats2bfloat162_rn(b0 - fb.x, b1 - fb.y);
-          pk[2 * i] = *reinterpret_cast<uint32_t*>(&ha2);
-          pk[2 * i + 1] = *reinterpret_cast<uint32_t*>(&hb2);
-          pl[2 * i] = *reinterpret_cast<uint32_t*>(&la2);
-          pl[2 * i + 1] = *reinterpret_cast<uint32_t*>(&lb2);
+          split(a0, a1, pk[2 * i], pl[2 * i]);
+          split(b0, b1, pk[2 * i + 1], pl[2 * i + 1]);
         }
         l_a = l_a * al_a + sa;
         l_b = l_b * al_b + sb;
