@@ -109,8 +109,33 @@ constexpr uint32_t kIdescV = ptx::idesc_bf16_f32(128, 256, 0, 1);   // P (TMEM) 
 constexpr float kRescaleThreshold = 8.0f;
 
 using tc::Params;
-using tc::UnitInfo;
-using tc::load_unit;
+
+// A plan unit for this kernel: 128 rows = the heads of n (1 or 2) consecutive query
+// tokens of sequence b (rows_per_token = H = 128 / n), over pages [pb, pb + npg).
+struct PairUnit {
+  int32_t item, b, pb, npg;
+  int32_t n;           // query tokens
+  int32_t ntok[2];     // tokens each sees (-1: absent)
+  int32_t part[2];     // partial-output index of each, or -1: final result
+};
+
+__device__ __forceinline__ PairUnit load_punit(const Params& p, const PlanView& plan, int32_t idx) {
+  const Unit u = plan.units()[idx];
+  PairUnit r;
+  r.item = u.item;
+  r.b = u.b;
+  r.pb = u.page_begin;
+  r.n = u.pad1 > 1 ? 2 : 1;
+  const int32_t q_len = plan.q_len(), L = p.seq_lens[u.b];
+  r.ntok[0] = visible_tokens(L, q_len, u.item % q_len);
+  r.ntok[1] = r.n > 1 ? visible_tokens(L, q_len, u.item % q_len + 1) : -1;
+  r.part[0] = u.part;
+  r.part[1] = r.n > 1 ? u.pad0 : -1;
+  const int32_t last = (max(r.ntok[0], r.ntok[1]) + kPage - 1) / kPage;   // pages holding visible tokens
+  const int32_t pe = min(u.page_end, min(last, p.max_pages));
+  r.npg = max(0, pe - r.pb);
+  return r;
+}
 
 // Optional event trace (-DMLA_TRACE): per CTA 1024 clock64 values, 8 regions of 128
 // pages: 0 load issued, 1 score MMA issued, 2 value MMA issued, 3 scores complete,
@@ -135,13 +160,13 @@ struct PageCursor {
   int32_t k;         // page within the unit
   uint32_t n;        // ordinal of the unit among the slot's non-empty units
   bool valid;
-  UnitInfo u;
+  PairUnit u;
 };
 
 __device__ __forceinline__ bool next_nonempty(const Params& p, const PlanView& plan, int32_t& ui, int32_t u_end,
-                                              UnitInfo& u) {
+                                              PairUnit& u) {
   while (++ui < u_end) {
-    u = load_unit(p, plan, ui);
+    u = load_punit(p, plan, ui);
     if (u.npg > 0) return true;
   }
   return false;
@@ -180,7 +205,7 @@ decode_pair_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_const
   const PlanView plan{p.plan};
   const int slot = blockIdx.x >> 1;
   const int32_t u_begin = plan.slot_begin()[slot], u_end = plan.slot_begin()[slot + 1];
-  const int32_t H = p.H;   // == 128
+  const int32_t H = p.H;   // 128, or 64 with two query tokens per unit
 
   if (threadIdx.x == 0) {
     *abort_flag = 0;
@@ -255,9 +280,13 @@ decode_pair_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_const
       if (!pf.valid) return;
       if (rank == 0 && leader) {
         if (pf.k == 0) {
+          // the unit's 128 query rows, clipped to the tensor's T * H rows
           const int64_t qrow = (int64_t)pf.u.item * H;
-          ptx::prefetch_l2_bulk(p.q_lat + qrow * kR, kHeads * kR * 2);
-          ptx::prefetch_l2_bulk(p.q_rope + qrow * kDr, kHeads * kDr * 2);
+          const int64_t rows = min((int64_t)kHeads, (int64_t)plan.B() * plan.q_len() * H - qrow);
+          if (rows > 0) {
+            ptx::prefetch_l2_bulk(p.q_lat + qrow * kR, (uint32_t)(rows * kR * 2));
+            ptx::prefetch_l2_bulk(p.q_rope + qrow * kDr, (uint32_t)(rows * kDr * 2));
+          }
         }
         const int32_t page = p.block_table[(int64_t)pf.u.b * p.max_pages + pf.u.pb + pf.k];
         if (page >= 0 && page < p.num_pages)
@@ -444,40 +473,45 @@ decode_pair_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_const
       return __all_sync(0xffffffffu, done);
     };
 
+    // Row h belongs to query token tok_h of a unit (0 for H = 128), head h % H.
+    const int tok_h = h / H;
+
     // Units without a visible token: o = 0 (this CTA's latent half), lse = -inf (CTA 0).
     for (int32_t ui = u_begin; ui < u_end; ++ui) {
-      const UnitInfo u = load_unit(p, plan, ui);
+      const PairUnit u = load_punit(p, plan, ui);
       if (u.npg > 0) continue;
-      const bool final_out = u.part < 0;
-      const int64_t row0 = final_out ? (int64_t)u.item * H : (int64_t)u.part * H;
-      for (int e = threadIdx.x - 128; e < kHeads * 256; e += kThreads - 128) {
-        const int hh = e / 256, j = e % 256;
+      for (int e = threadIdx.x - 128; e < u.n * H * 256; e += kThreads - 128) {
+        const int r = e / 256, j = e % 256, t = r / H;
         const int d = (j < 128 ? 128 * (int)rank : 256 + 128 * (int)rank) + (j & 127);
-        if (final_out)
-          p.o_lat[(row0 + hh) * kR + d] = __float2bfloat16_rn(0.f);
+        const int32_t prt = t ? u.part[1] : u.part[0];
+        if (prt < 0)
+          p.o_lat[((int64_t)(u.item + t) * H + r % H) * kR + d] = __float2bfloat16_rn(0.f);
         else
-          p.o_part[(row0 + hh) * kR + d] = 0.f;
+          p.o_part[((int64_t)prt * H + r % H) * kR + d] = 0.f;
       }
-      if (rank == 0 && hf == 0) {
-        if (final_out) {
-          if (p.lse) p.lse[row0 + h] = -CUDART_INF_F;
+      if (rank == 0 && hf == 0 && tok_h < u.n) {
+        const int32_t prt = tok_h ? u.part[1] : u.part[0];
+        if (prt < 0) {
+          if (p.lse) p.lse[(int64_t)(u.item + tok_h) * H + h % H] = -CUDART_INF_F;
         } else {
-          p.lse_part[row0 + h] = -CUDART_INF_F;
+          p.lse_part[(int64_t)prt * H + h % H] = -CUDART_INF_F;
         }
       }
     }
 
     // Stage a unit's query: this thread's 128 of head h's own 256 latent dims
     // (128r.. for f = 0, 256+128r.. for f = 1) -> TMEM columns 64f..64f+63.
-    auto stage_q = [&](const UnitInfo& u, uint32_t n) -> bool {
+    auto stage_q = [&](const PairUnit& u, uint32_t n) -> bool {
       if (!wait_all(bar(B_QT_EMPTY), (n & 1) ^ 1)) return false;
       ptx::tc_fence_after();
+      // rows of a token the unit does not have stay zero (their scores are never used)
+      const bool present = tok_h < u.n;
       const uint4* src = reinterpret_cast<const uint4*>(p.q_lat + ((int64_t)u.item * H + h) * kR);
       const int dim0 = 256 * hf + 128 * (int)rank;
       uint32_t w[2][32];
 #pragma unroll
       for (int i = 0; i < 16; ++i) {
-        const uint4 v = __ldg(src + dim0 / 8 + i);
+        const uint4 v = present ? __ldg(src + dim0 / 8 + i) : make_uint4(0u, 0u, 0u, 0u);
         w[i >> 3][4 * (i & 7) + 0] = v.x;
         w[i >> 3][4 * (i & 7) + 1] = v.y;
         w[i >> 3][4 * (i & 7) + 2] = v.z;
@@ -546,7 +580,7 @@ decode_pair_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_const
     auto stage_next_q = [&](const PageCursor& c) -> bool {
       if (c.k != c.u.npg - 1) return true;
       int32_t ui = c.ui;
-      UnitInfo nu;
+      PairUnit nu;
       return !next_nonempty(p, plan, ui, u_end, nu) || stage_q(nu, c.n + 1);
     };
     // Epilogue of a unit, run after the next unit's first P (or after the last page of
@@ -557,11 +591,10 @@ decode_pair_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_const
     // segments.
     struct Pending {
       bool on;
-      bool final_out;
-      int64_t row0;      // output row of head 0
-      uint32_t stage;    // stage of the unit's last page
-      float l, m;        // this thread's half of l; the shared reference maximum
-    } pend{false, false, 0, 0u, 0.f, 0.f};
+      int32_t item, n, part0, part1;   // the unit's tokens and their partial-output indices
+      uint32_t stage;                  // stage of the unit's last page
+      float l, m;                      // this thread's half of l; the shared reference maximum
+    } pend{false, 0, 0, -1, -1, 0u, 0.f, 0.f};
     auto epilogue = [&]() -> bool {
       // l = the two halves' sums
       volatile float* ls = pair_slot(pend.stage, kOffPairL);
@@ -571,13 +604,18 @@ decode_pair_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_const
       ptx::tc_fence_after();
       const float inv_l = l > 0.f ? 1.f / l : 0.f;
       const uint32_t buf = sbase + kOffKV + pend.stage * kStageBytes + (uint32_t)hf * 16384u;
-      const int rounds = pend.final_out ? 2 : 4;     // 64 bf16 or 32 fp32 columns per round
-      const int cols = pend.final_out ? 64 : 32;
+      // this warp's 32 rows all belong to token tok_h of the unit: its output rows
+      const bool present = tok_h < pend.n;
+      const int32_t prt = tok_h ? pend.part1 : pend.part0;
+      const bool final_out = prt < 0;
+      const int64_t row0 = (final_out ? (int64_t)(pend.item + tok_h) * H : (int64_t)prt * H) - tok_h * H;
+      const int rounds = final_out ? 2 : 4;     // 64 bf16 or 32 fp32 columns per round
+      const int cols = final_out ? 64 : 32;
 #pragma unroll 1
       for (int c = 0; c < rounds; ++c) {
         const int col0 = 128 * hf + cols * c;        // TMEM column of the round
         uint32_t w[32];
-        if (pend.final_out) {
+        if (final_out) {
 #pragma unroll
           for (int half = 0; half < 2; ++half) {
             uint32_t o[32];
@@ -613,18 +651,19 @@ decode_pair_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_const
                        : "=r"(q.x), "=r"(q.y), "=r"(q.z), "=r"(q.w)
                        : "r"(buf + (uint32_t)row * 128u + (uint32_t)((j ^ (row & 7)) << 4))
                        : "memory");
-          if (pend.final_out)
-            *reinterpret_cast<uint4*>(p.o_lat + (pend.row0 + row) * kR + d0 + 8 * j) = q;
+          if (!present) continue;
+          if (final_out)
+            *reinterpret_cast<uint4*>(p.o_lat + (row0 + row) * kR + d0 + 8 * j) = q;
           else
-            *reinterpret_cast<uint4*>(p.o_part + (pend.row0 + row) * kR + d0 + 4 * j) = q;
+            *reinterpret_cast<uint4*>(p.o_part + (row0 + row) * kR + d0 + 4 * j) = q;
         }
       }
-      if (rank == 0 && hf == 0) {
+      if (rank == 0 && hf == 0 && present) {
         const float z = l > 0.f ? (pend.m + log2f(l)) * 0.69314718055994531f : -CUDART_INF_F;
-        if (pend.final_out) {
-          if (p.lse) p.lse[pend.row0 + h] = z;
+        if (final_out) {
+          if (p.lse) p.lse[row0 + h] = z;
         } else {
-          p.lse_part[pend.row0 + h] = z;
+          p.lse_part[row0 + h] = z;
         }
       }
       ptx::tc_fence_before();
@@ -650,7 +689,8 @@ decode_pair_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_const
     }
     float m_run = -CUDART_INF_F, l_run = 0.f;
     while (cur.valid && ok) {
-      const UnitInfo& u = cur.u;
+      const PairUnit& u = cur.u;
+      const int32_t ntok = tok_h ? u.ntok[1] : u.ntok[0];   // tokens this row sees (-1: no row)
       if (cur.k == 0) {
         m_run = -CUDART_INF_F;
         l_run = 0.f;
@@ -685,9 +725,9 @@ decode_pair_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_const
       }
       // ------------------------------------------------ this page's maximum and reference
       const int32_t tok0 = (u.pb + cur.k) * kPage + 32 * hf;
-      if (tok0 + 32 > u.ntok) {
+      if (tok0 + 32 > ntok) {
 #pragma unroll
-        for (int t = 0; t < 32; ++t) v[t] = (tok0 + t < u.ntok) ? v[t] : -CUDART_INF_F;
+        for (int t = 0; t < 32; ++t) v[t] = (tok0 + t < ntok) ? v[t] : -CUDART_INF_F;
       }
       float mx;
       {
@@ -774,8 +814,10 @@ decode_pair_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_const
 
       if (cur.k == u.npg - 1) {
         pend.on = true;
-        pend.final_out = u.part < 0;
-        pend.row0 = pend.final_out ? (int64_t)u.item * H : (int64_t)u.part * H;
+        pend.item = u.item;
+        pend.n = u.n;
+        pend.part0 = u.part[0];
+        pend.part1 = u.part[1];
         pend.stage = gpg % kStages;
         pend.l = l_run;
         pend.m = m_run;

@@ -163,8 +163,22 @@ mla_status launch_proj(const void* A, const void* Bw, void* out, int32_t T, cons
   return launch_check(what);
 }
 
-int32_t head_groups_for(const mla_dims& d) {
+// The 2-CTA cluster kernel serves 128 rows per cluster: all heads of one query token
+// for H=128, or the heads of two consecutive query tokens of a sequence for H=64
+// (multi-token steps, q_len >= 2), whose rows then share every page.
+bool pair_decode(const mla_dims& d, int32_t q_len) {
+  return use_tc_decode(d) && (d.H == mla::pair::kHeads || (d.H == mla::pair::kHeads / 2 && q_len >= 2));
+}
+
+// CTAs per slot (the plan has num_sms / head_groups slots).
+int32_t head_groups_for(const mla_dims& d, int32_t q_len) {
+  if (pair_decode(d, q_len)) return 2;
   return decode_tc_ok(d) ? d.H / mla::tc::kHeads : 1;
+}
+
+// Query tokens per plan unit (consecutive tokens of one sequence).
+int32_t items_per_unit_for(const mla_dims& d, int32_t q_len) {
+  return pair_decode(d, q_len) ? mla::pair::kHeads / d.H : 1;
 }
 
 }  // namespace
@@ -303,11 +317,11 @@ mla_status mla_plan_splits(const int32_t* seq_lens_host, int32_t B, int32_t q_le
     return fail(MLA_ERR_WORKSPACE, "plan capacity %zu < %zu words", capacity,
                 mla_plan_capacity(B, q_len, num_sms));
   const int32_t ps = d.page_size;
-  const int32_t G = head_groups_for(d);
+  const int32_t G = head_groups_for(d, q_len);
+  const int32_t ipu = items_per_unit_for(d, q_len);
   const int32_t slots_max = std::max(1, num_sms / G);
   const int32_t items = B * q_len;
   std::vector<int32_t> pages(items);
-  int64_t total = 0;
   for (int32_t b = 0; b < B; ++b) {
     const int32_t L = seq_lens_host[b];
     if (L < 0 || (int64_t)L > (int64_t)max_pages * ps)
@@ -316,38 +330,51 @@ mla_status mla_plan_splits(const int32_t* seq_lens_host, int32_t B, int32_t q_le
     for (int32_t i = 0; i < q_len; ++i) {
       const int32_t n = mla::visible_tokens(L, q_len, i);
       pages[b * q_len + i] = (n + ps - 1) / ps;
-      total += pages[b * q_len + i];
     }
   }
+  // Units cover groups of ipu consecutive query tokens of one sequence; a group's page
+  // count is its last token's (which sees the most).
+  int64_t total = 0;
+  const int32_t groups_per_seq = (q_len + ipu - 1) / ipu;
+  auto group_pages = [&](int32_t b, int32_t k) {
+    const int32_t last = std::min(q_len, (k + 1) * ipu) - 1;
+    return pages[b * q_len + last];
+  };
+  for (int32_t b = 0; b < B; ++b)
+    for (int32_t k = 0; k < groups_per_seq; ++k) total += group_pages(b, k);
   // Slot s covers flattened pages [s*total/S, (s+1)*total/S): page counts differ by at most one.
   const int64_t S = std::max<int64_t>(1, std::min<int64_t>(slots_max, total));
   auto bound = [&](int64_t s) { return s * total / S; };
-  struct U { int32_t item, b, pb, pe, slot; };
+  struct U { int32_t item, b, pb, pe, slot, n; };
   std::vector<U> units;
   units.reserve(items + S);
   int32_t slot = 0;
   int64_t flat = 0;  // flattened index of the next page
-  for (int32_t it = 0; it < items; ++it) {
-    const int32_t b = it / q_len;
-    int32_t left = pages[it], pb = 0;
-    if (left == 0) {
-      units.push_back({it, b, 0, 0, slot});
-      continue;
-    }
-    while (left > 0) {
-      while (slot + 1 < S && flat >= bound(slot + 1)) ++slot;
-      const int64_t room = (slot + 1 < S) ? bound(slot + 1) - flat : left;
-      const int32_t take = (int32_t)std::min<int64_t>(left, room);
-      units.push_back({it, b, pb, pb + take, slot});
-      pb += take;
-      left -= take;
-      flat += take;
+  for (int32_t b = 0; b < B; ++b) {
+    for (int32_t k = 0; k < groups_per_seq; ++k) {
+      const int32_t it = b * q_len + k * ipu;
+      const int32_t n = std::min(ipu, q_len - k * ipu);
+      int32_t left = group_pages(b, k), pb = 0;
+      if (left == 0) {
+        units.push_back({it, b, 0, 0, slot, n});
+        continue;
+      }
+      while (left > 0) {
+        while (slot + 1 < S && flat >= bound(slot + 1)) ++slot;
+        const int64_t room = (slot + 1 < S) ? bound(slot + 1) - flat : left;
+        const int32_t take = (int32_t)std::min<int64_t>(left, room);
+        units.push_back({it, b, pb, pb + take, slot, n});
+        pb += take;
+        left -= take;
+        flat += take;
+      }
     }
   }
   const int32_t num_slots = units.empty() ? 0 : units.back().slot + 1;
-  // parts: items with more than one unit
+  // parts: items with more than one unit (every token of a split group is split)
   std::vector<int32_t> count(items, 0);
-  for (const U& u : units) count[u.item]++;
+  for (const U& u : units)
+    for (int32_t j = 0; j < u.n; ++j) count[u.item + j]++;
   std::vector<int32_t> first(items, -1);
   int32_t parts = 0;
   for (int32_t it = 0; it < items; ++it)
@@ -367,19 +394,23 @@ mla_status mla_plan_splits(const int32_t* seq_lens_host, int32_t B, int32_t q_le
   plan_host[6] = G;
   plan_host[7] = d.H;
   plan_host[8] = ps;
+  plan_host[9] = ipu;
   int32_t* uw = plan_host + mla::kPlanHeader;
   std::vector<int32_t> next(items, 0);
   for (size_t k = 0; k < units.size(); ++k) {
     const U& u = units[k];
-    int32_t part = -1;
-    if (count[u.item] > 1) part = first[u.item] + next[u.item]++;
+    int32_t part[2] = {-1, -1};
+    for (int32_t j = 0; j < u.n; ++j)
+      if (count[u.item + j] > 1) part[j] = first[u.item + j] + next[u.item + j]++;
     int32_t* w = uw + mla::kUnitWords * k;
     w[0] = u.item;
     w[1] = u.b;
     w[2] = u.pb;
     w[3] = u.pe;
-    w[4] = part;
+    w[4] = part[0];
     w[5] = u.slot;
+    w[6] = part[1];
+    w[7] = u.n;
   }
   int32_t* sb = uw + mla::kUnitWords * units.size();
   {
@@ -430,9 +461,11 @@ static mla_status check_info(const mla_plan_info* info, int32_t B, int32_t q_len
   if (!info) return fail(MLA_ERR_INVALID, "null plan info");
   if (info->num_items != B * q_len)
     return fail(MLA_ERR_INVALID, "plan covers %d query tokens, call has %d", info->num_items, B * q_len);
-  if (info->head_groups != head_groups_for(d))
-    return fail(MLA_ERR_INVALID, "plan was made for %d head groups, dims need %d", info->head_groups,
-                head_groups_for(d));
+  if (info->head_groups != head_groups_for(d, q_len))
+    return fail(MLA_ERR_INVALID,
+                "plan was made for %d CTAs per slot, these dims, q_len and kernel policy need %d (plan "
+                "again after changing the policy)",
+                info->head_groups, head_groups_for(d, q_len));
   return MLA_OK;
 }
 
@@ -485,7 +518,7 @@ mla_status mla_decode_attn(const void* q_lat, const void* q_rope, const void* kv
     p.timeout_ns = g_timeout_ns.load();
     p.trace = g_trace;
     const dim3 grid(info->num_slots * info->head_groups);
-    if (d.H == mla::pair::kHeads) {
+    if (pair_decode(d, q_len)) {
       // 128 heads: a cluster of two CTAs per slot, each holding half of every page;
       // the rope columns travel as two 32-column halves (64-byte swizzle)
       CUtensorMap tkr, tqr;

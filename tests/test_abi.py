@@ -66,13 +66,23 @@ def test_plan_covers_every_visible_page_once(q_len, sms, H):
     d = dims(H=H)
     plan, info = mla.mla_plan_splits(lens, len(lens), q_len, max_pages, d, sms)
     p = parse_plan(plan)
-    G = H // 64 if H % 64 == 0 else 1
+    # 2-CTA clusters for 128 heads, and for 64 heads with several query tokens (two
+    # consecutive tokens per unit); otherwise one CTA per 64 heads
+    pair = H == 128 or (H == 64 and q_len >= 2)
+    G = 2 if pair else (H // 64 if H % 64 == 0 else 1)
+    per_unit = 128 // H if pair else 1
     assert p["G"] == info.head_groups == G
+    assert plan[9] == per_unit
     assert info.num_slots <= max(1, sms // G)
     cover = {}
-    for (item, b, pb, pe, part, slot, _, _) in p["units"]:
-        assert item // q_len == b
-        cover.setdefault(item, []).append((pb, pe, part, slot))
+    for (item, b, pb, pe, part, slot, part2, n) in p["units"]:
+        assert item // q_len == b and 1 <= n <= per_unit and (item % q_len) % per_unit == 0
+        for j in range(n):
+            # a later token of the group may see more pages than an earlier one
+            L = int(lens[b]); i = item % q_len + j
+            npg = math.ceil(max(0, L - q_len + i + 1) / 64)
+            assert item + j < len(lens) * q_len and (item + j) // q_len == b
+            cover.setdefault(item + j, []).append((pb, min(pe, max(npg, pb)), part if j == 0 else part2, slot))
     slots = p["units"][:, 5]
     assert np.all(np.diff(slots) >= 0)
     for s in range(info.num_slots):

@@ -163,6 +163,18 @@ def test_causal_chunk_attention_matches_oracle(policy):
     attention_case(policy, 64, 5, [70, 5, 129], 6)
 
 
+@pytest.mark.parametrize("sms", [148, 9])
+@pytest.mark.parametrize("q_len", [2, 4])
+def test_paired_token_attention_matches_oracle(q_len, sms):
+    """64 heads, several new tokens: the tensor-core path serves two consecutive tokens
+    of a sequence per 2-CTA cluster (128 rows); the two tokens see different lengths,
+    page ranges are cut between slots, and one sequence is shorter than a page."""
+    step = attention_case("tcgen05", 64, q_len, [300, 64, q_len, 1000, 130], sms)
+    assert step.info.head_groups == 2
+    if sms == 9:
+        assert step.info.num_parts > 0
+
+
 @pytest.mark.parametrize("policy", ["simt", "tcgen05"])
 def test_attention_with_large_logit_offsets(policy):
     """Per-token logit noise of std 4 (the long-context workload's stress): the
@@ -213,6 +225,7 @@ def test_whole_step_matches_oracle(policy, H, q_len, lens, sms):
     step.append()
     step.absorb()
     run_policy(policy)
+    step.replan(step.seq_lens_host)   # the split plan depends on the kernel policy
     step.attend()
     step.combine()
     mla.mla_set_policy(mla.MLA_POLICY_AUTO)
