@@ -506,16 +506,22 @@ decode_pair_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_const
       ptx::tc_fence_after();
       // rows of a token the unit does not have stay zero (their scores are never used)
       const bool present = tok_h < u.n;
-      const uint4* src = reinterpret_cast<const uint4*>(p.q_lat + ((int64_t)u.item * H + h) * kR);
-      const int dim0 = 256 * hf + 128 * (int)rank;
+      // 32-byte loads (one sector each): the 32 lanes read 32 different rows, so each
+      // load instruction costs a transaction per lane and wider loads halve them
+      const __nv_bfloat16* src = p.q_lat + ((int64_t)u.item * H + h) * kR + 256 * hf + 128 * (int)rank;
       uint32_t w[2][32];
 #pragma unroll
-      for (int i = 0; i < 16; ++i) {
-        const uint4 v = present ? __ldg(src + dim0 / 8 + i) : make_uint4(0u, 0u, 0u, 0u);
-        w[i >> 3][4 * (i & 7) + 0] = v.x;
-        w[i >> 3][4 * (i & 7) + 1] = v.y;
-        w[i >> 3][4 * (i & 7) + 2] = v.z;
-        w[i >> 3][4 * (i & 7) + 3] = v.w;
+      for (int i = 0; i < 8; ++i) {
+        uint32_t* d = &w[i >> 2][8 * (i & 3)];
+        if (present) {
+          asm volatile("ld.global.nc.v8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+                       : "=r"(d[0]), "=r"(d[1]), "=r"(d[2]), "=r"(d[3]), "=r"(d[4]), "=r"(d[5]), "=r"(d[6]),
+                         "=r"(d[7])
+                       : "l"(src + 16 * i));
+        } else {
+#pragma unroll
+          for (int k = 0; k < 8; ++k) d[k] = 0u;
+        }
       }
       ptx::tmem_st_32x32b_x32(tbase + lane_addr + kColQ + 64 * hf, w[0]);
       ptx::tmem_st_32x32b_x32(tbase + lane_addr + kColQ + 64 * hf + 32, w[1]);
@@ -616,15 +622,16 @@ decode_pair_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_const
         const int col0 = 128 * hf + cols * c;        // TMEM column of the round
         uint32_t w[32];
         if (final_out) {
+          uint32_t o[2][32];
+          ptx::tmem_ld_32x32b_x32(tbase + lane_addr + kColO + col0, o[0]);
+          ptx::tmem_ld_32x32b_x32(tbase + lane_addr + kColO + col0 + 32, o[1]);
+          ptx::tmem_wait_ld();
 #pragma unroll
           for (int half = 0; half < 2; ++half) {
-            uint32_t o[32];
-            ptx::tmem_ld_32x32b_x32(tbase + lane_addr + kColO + col0 + 32 * half, o);
-            ptx::tmem_wait_ld();
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
-              __nv_bfloat162 b2 =
-                  __floats2bfloat162_rn(__uint_as_float(o[2 * i]) * inv_l, __uint_as_float(o[2 * i + 1]) * inv_l);
+              __nv_bfloat162 b2 = __floats2bfloat162_rn(__uint_as_float(o[half][2 * i]) * inv_l,
+                                                        __uint_as_float(o[half][2 * i + 1]) * inv_l);
               w[16 * half + i] = *reinterpret_cast<uint32_t*>(&b2);
             }
           }
