@@ -271,7 +271,9 @@ decode_pair_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_const
   if (warp == 0) {
     // ================================================================ TMA producer
     const bool leader = ptx::elect_one();
-    const uint64_t pol_stream = ptx::policy_evict_first();
+    // a page is read once per step when every unit has its own sequence (q_len = 1);
+    // with several query tokens per sequence the sequence's other units read it again
+    const uint64_t pol_stream = plan.q_len() > 1 ? ptx::policy_evict_last() : ptx::policy_evict_first();
     uint32_t gpg = 0, nq = 0;   // pages and rope-query halves loaded
     bool ok = true;
     // L2 prefetch cursor (CTA 0 prefetches whole pages a few pages ahead)
