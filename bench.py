@@ -51,17 +51,18 @@ def load_peaks():
         return dict(FALLBACK_PEAKS), "fallback"
 
 
-def decode_kernel_of(H):
-    """(source file, kernel name) of the tensor-core decode kernel used for H heads."""
-    if H == 128:
+def decode_kernel_of(H, q_len):
+    """(source file, kernel name) of the tensor-core decode kernel used for H heads and
+    q_len query tokens per sequence (the library's default policy)."""
+    if H == 128 or (H == 64 and q_len >= 2):
         return "decode_pair.cuh", "mla_decode_attn (tcgen05 decode_pair_kernel, 2-CTA clusters)"
     return "decode_tc.cuh", "mla_decode_attn (tcgen05 decode_kernel)"
 
 
-def traffic_record(workload, H):
+def traffic_record(workload, H, q_len):
     """DRAM bytes per launch of the decode kernel from a committed ncu summary, valid
     only while the kernel source is unchanged (its sha256 is recorded there)."""
-    src_name, _ = decode_kernel_of(H)
+    src_name, _ = decode_kernel_of(H, q_len)
     src = os.path.join(ROOT, "mla_latent_kv_46_b200", "csrc", src_name)
     sha = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
     path = os.path.join(ROOT, "profiles", f"ncu_decode_attn_{workload}.md")
@@ -313,7 +314,7 @@ def run_gpu(args):
     t_hbm = cache_bytes / (peaks["hbm_gbs"] * 1e9)
     t_tc = flops / (peaks["bf16_tflops"] * 1e12)
     bound = "hbm" if t_hbm >= t_tc else "tensor"
-    traffic, sha = traffic_record(spec.name, spec.H)
+    traffic, sha = traffic_record(spec.name, spec.H, spec.q_len)
     if args.seqs:
         traffic = None   # the committed figure is for the whole workload
     if bound == "hbm":
@@ -325,7 +326,7 @@ def run_gpu(args):
     roof["frac"] = roof["achieved"] / roof["peak"]
     roof["traffic"] = traffic
     roof["peak_source"] = f"{peak_src} (MEASURED_PEAKS.json)" if peak_src == "measured" else "fallback"
-    src_name, roof["kernel"] = decode_kernel_of(spec.H)
+    src_name, roof["kernel"] = decode_kernel_of(spec.H, spec.q_len)
     roof["algorithmic_bytes_per_launch"] = cache_bytes
     roof["algorithmic_flops_per_launch"] = flops
     roof["roofline_ms"] = 1e3 * max(t_hbm, t_tc)

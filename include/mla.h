@@ -105,6 +105,15 @@ mla_status mla_set_policy(int32_t policy);
 /* Bound, in nanoseconds, on every wait inside a kernel (default 2e9). */
 mla_status mla_set_wait_timeout_ns(uint64_t ns);
 
+/* Testing hook for the failure path of the tensor-core decode kernels: while set
+ * (ordinal >= 0), the first CTA of each mla_decode_attn launch skips the shared-memory
+ * load of its page with that ordinal (0 = its first page), so the waits on that page
+ * run out after the wait bound (mla_set_wait_timeout_ns), the kernel stops, and
+ * mla_check_status then reports MLA_ERR_TIMEOUT; the outputs of that launch are
+ * undefined. A negative ordinal switches the hook off (the default). Process-wide;
+ * always returns MLA_OK. Nothing in the pages corresponds to it. */
+mla_status mla_debug_drop_page_load(int32_t ordinal);
+
 /* Synchronises `stream`, then reads and clears the device status word of the
  * current device: MLA_OK, MLA_ERR_TIMEOUT (a bounded wait ran out) or
  * MLA_ERR_INVALID (a page id outside the pool was skipped). */

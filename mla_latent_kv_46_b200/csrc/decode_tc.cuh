@@ -109,6 +109,7 @@ struct Params {
   const __nv_bfloat16* q_rope;
   uint64_t timeout_ns;
   unsigned long long* trace;  // per-CTA event clocks, only in builds with MLA_TRACE
+  int32_t drop_load;          // testing hook: CTA 0 skips the load of its page with this ordinal (-1: none)
 };
 
 // Optional event trace (build with -DMLA_TRACE): per CTA 1024 clock64 values;
@@ -275,7 +276,9 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_qlat, const __grid_constant
           page = p.num_pages;  // rows past the tensor: TMA fills zeros
         }
         const uint32_t dst = sKV + st * kTileBytes;
-        if (leader) {
+        // (the testing hook leaves the page's barrier without its load, so that the
+        // waits on it run out and the kernel reports a timeout)
+        if (leader && !(blockIdx.x == 0 && (int32_t)gpg == p.drop_load)) {
           MLA_TRACE_AT(gpg);
           ptx::mbar_arrive_expect_tx(bar(B_KV_FULL + st), kTileBytes);
 #pragma unroll

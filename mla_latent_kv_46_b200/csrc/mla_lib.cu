@@ -29,6 +29,7 @@ thread_local std::string g_last_error;
 std::atomic<int32_t> g_policy{MLA_POLICY_AUTO};
 std::atomic<uint64_t> g_timeout_ns{2000000000ull};
 unsigned long long* g_trace = nullptr;  // event trace buffer (MLA_TRACE builds only)
+std::atomic<int32_t> g_drop_load{-1};   // testing hook, see mla_debug_drop_page_load
 
 mla_status fail(mla_status s, const char* fmt, ...) {
   char buf[512];
@@ -205,6 +206,11 @@ mla_status mla_set_policy(int32_t policy) {
 mla_status mla_set_wait_timeout_ns(uint64_t ns) {
   if (ns == 0) return fail(MLA_ERR_INVALID, "timeout must be positive");
   g_timeout_ns.store(ns);
+  return ok();
+}
+
+mla_status mla_debug_drop_page_load(int32_t ordinal) {
+  g_drop_load.store(ordinal < 0 ? -1 : ordinal);
   return ok();
 }
 
@@ -517,6 +523,7 @@ mla_status mla_decode_attn(const void* q_lat, const void* q_rope, const void* kv
     p.q_rope = static_cast<const __nv_bfloat16*>(q_rope);
     p.timeout_ns = g_timeout_ns.load();
     p.trace = g_trace;
+    p.drop_load = g_drop_load.load();
     const dim3 grid(info->num_slots * info->head_groups);
     if (pair_decode(d, q_len)) {
       // 128 heads: a cluster of two CTAs per slot, each holding half of every page;

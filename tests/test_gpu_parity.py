@@ -339,8 +339,12 @@ def test_full_size_workload_sampled(name):
 
 # ----------------------------------------------------------------------------- failure reporting
 
-def test_bad_page_id_is_reported_not_faulted():
-    w = wl.make(small_spec(H=64), seed=2, seq_lens=[130, 64])
+@pytest.mark.parametrize("H,q_len", [(64, 1), (128, 1), (64, 2)])
+def test_bad_page_id_is_reported_not_faulted(H, q_len):
+    """A block-table entry outside the pool is skipped (the tile reads as zeros) and
+    reported through the status word; the single-CTA kernel (64 heads), the cluster
+    kernel (128 heads) and the cluster kernel with paired query tokens."""
+    w = wl.make(small_spec(H=H, q_len=q_len), seed=2, seq_lens=[130, 64])
     w["block_table"][1, 0] = 10_000          # outside the pool
     step = dec.DecodeStep(w)
     step.run(append=False)
@@ -349,3 +353,51 @@ def test_bad_page_id_is_reported_not_faulted():
         mla.mla_check_status()
     assert e.value.status == mla._binding.MLA_ERR_INVALID
     mla.mla_check_status()                   # cleared
+
+
+@pytest.mark.parametrize("H,q_len", [(64, 1), (128, 1), (64, 2)])
+def test_dropped_page_load_times_out_and_context_stays_usable(H, q_len):
+    """Fault injection without a GPU fault: the first CTA skips one page load (testing
+    hook), its waits run out after a short bound, the kernel stops and the status word
+    reports MLA_ERR_TIMEOUT; afterwards the same context decodes correctly."""
+    spec = small_spec(H=H, q_len=q_len)
+    lens = [700, 300, 129]
+    w = wl.make(spec, seed=4, seq_lens=lens)
+    step = dec.DecodeStep(w, sms=4)
+    ql = wl.latent_queries(spec, step.T, seed=9)
+    step.q_lat.copy_(dec.to_torch(ql, step.device))
+    mla.mla_set_wait_timeout_ns(20_000_000)       # 20 ms
+    mla.mla_debug_drop_page_load(2)
+    try:
+        step.attend()
+        torch.cuda.synchronize()
+        with pytest.raises(mla.MlaError) as e:
+            mla.mla_check_status()
+        assert e.value.status == mla._binding.MLA_ERR_TIMEOUT
+    finally:
+        mla.mla_debug_drop_page_load(-1)
+        mla.mla_set_wait_timeout_ns(2_000_000_000)
+    mla.mla_check_status()                         # cleared
+    step.attend()
+    step.combine()
+    torch.cuda.synchronize()
+    mla.mla_check_status()
+    ref = orc.attend_latent(ql, w["q_rope"], w["kv_cache"], w["block_table"], w["seq_lens"], w["scale"],
+                            q_len=q_len, page_size=spec.page_size)
+    assert_close(host(step.o_lat), ref["o_lat"], False, "o_lat after the injected timeout")
+
+
+@pytest.mark.parametrize("name", ["deepseek_h128_b128_ragged", "causal_chunk_h64_b8_2048p256"])
+def test_decode_is_deterministic(name):
+    """Two runs of the same step give bitwise equal outputs (no atomics, fixed order)."""
+    spec = wl.WORKLOADS[name]
+    lens = wl.seq_lens_of(spec, 0)[:16]
+    w = wl.make(spec, seed=0, seq_lens=lens)
+    step = dec.DecodeStep(w)
+    outs = []
+    for _ in range(2):
+        step.run(append=True)
+        torch.cuda.synchronize()
+        outs.append((step.out.clone(), step.lse.clone()))
+    mla.mla_check_status()
+    assert torch.equal(outs[0][0], outs[1][0]) and torch.equal(outs[0][1], outs[1][1])
