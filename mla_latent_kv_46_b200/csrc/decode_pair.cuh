@@ -5,38 +5,43 @@
 // (128-byte swizzle) and rope dims 32r..32r+31 (64-byte swizzle), so the pair holds
 // each page once. Per page:
 //   partial scores  S_r[h][t] = sum over CTA r's columns of Q[h][k] KV[t][k], all 128
-//                   heads: tcgen05.mma M=128 (heads) x N=64 (tokens); the latent part
+//                   rows: tcgen05.mma M=128 (rows) x N=64 (tokens); the latent part
 //                   takes Q from TMEM, the rope part from shared memory
-//   exchange        each CTA stages its 128 x 64 partial scores in shared memory and
-//                   bulk-copies them into the peer's (DSMEM); S = S_0 + S_1 is then the
-//                   same fp32 value in both CTAs (addition commutes)
-//   softmax         fp32, one thread per head (64 tokens in registers), done by both
-//                   CTAs on identical inputs, so both take the same reference-maximum
-//                   decisions and hold the same P, l and m without exchanging them;
+//   exchange        each CTA encodes its 128 x 64 partial scores as 16-bit codes with
+//                   one scale per 32 values (see kXRunBytes), stages them in shared
+//                   memory and bulk-copies them into the peer's single receive slot
+//                   (DSMEM, 17 KiB each way); each CTA adds its own exact partial and the
+//                   peer's decoded one, so the two sums agree to 2^-16 of the largest
+//                   partial in a block of 32
+//   softmax         fp32, two threads per row (32 tokens each), in both CTAs; each CTA
+//                   keeps its own reference maximum, P, l and m, so each output half is
+//                   normalised consistently with the P it was summed with;
 //                   P = P_hi + P_lo (two bf16 parts) is written to TMEM
 //   values          O[h][d] += sum_t P[h][t] C[t][d] over CTA r's 256 latent columns:
-//                   tcgen05.mma M=128 (heads) x N=256 x K=16, P from TMEM, C from the
+//                   tcgen05.mma M=128 (rows) x N=256 x K=16, P from TMEM, C from the
 //                   stage (N-major), 4 K-steps x 2 parts per page
-// So each CTA streams half a page through its shared memory, every MMA has M=128, the
-// value MMA reads only C from shared memory, and the only cross-CTA traffic is one
-// 32 KiB score exchange each way per page.
+// So each CTA streams half a page through its shared memory, every MMA has M=128 and
+// the value MMA reads only C from shared memory.
 //
-// The softmax warps issue page j+1's exchange before page j's softmax, so the copy
-// overlaps the exponentials; the MMA warp therefore runs the score MMAs two pages
-// ahead of the value MMAs (order S0 S1 S2 V0 S3 V1 ...), with four stages of pages.
+// The softmax warps read page j's exchange slot, release it and issue page j+1's
+// exchange before page j's exponentials, so the copy overlaps them; the MMA warp runs
+// the score MMAs two pages ahead of the value MMAs (order S0 S1 S2 V0 S3 V1 ...). Five
+// stages of pages: the loop that sets the page period (a stage's load, that page's
+// scores, the softmax that needs them, the value MMAs that free the stage) spans
+// stages - 1 page periods, so the small exchange buffers buy the fifth stage.
 //
-// Warp roles (256 threads): warp 0 TMA producer, warp 1 MMA issuer, warp 2 TMEM
-// allocator, warps 4-7 query staging, exchange, softmax, epilogue. Warp w (4-7)
-// accesses TMEM lanes 32(w%4).., i.e. heads 32(w%4)..+31; each softmax thread owns
-// one head's row of S, P and O.
+// Warp roles (384 threads): warp 0 TMA producer, warp 1 MMA issuer, warp 2 TMEM
+// allocator, warp 3 exchange watcher, warps 4-11 query staging, exchange, softmax and
+// epilogue. Warps 4+q and 8+q access TMEM lanes 32q..32q+31 (rows 32q..), each thread
+// half of one row's tokens.
 //
-// TMEM (512 columns, lane = head): [0,256) O, fp32, CTA r's latent columns in box
+// TMEM (512 columns, lane = row): [0,256) O, fp32, CTA r's latent columns in box
 // order; [256,384) the query's own latent half (bf16 pairs); [384,448) S; [448,480)
 // P_hi, [480,512) P_lo (bf16 pairs).
 //
-// Online softmax with a lazily moved per-head reference maximum (moved only when a
+// Online softmax with a lazily moved per-row reference maximum (moved only when a
 // page's maximum exceeds it by more than 2^8); a moved reference rescales that
-// head's O row.
+// row's O.
 //
 // Every wait is bounded; a CTA that gives up raises the device status word and the
 // peer's waits on it run out the same way. Both CTAs meet in a cluster barrier
@@ -54,21 +59,22 @@ constexpr int kPage = 64, kR = 512, kDr = 64, kRow = kR + kDr;
 constexpr int kBox = 64 * 128;              // 64 rows x 64 bf16, 128-byte swizzle
 constexpr int kRopeBox = 64 * 64;           // 64 rows x 32 bf16, 64-byte swizzle
 constexpr int kStageBytes = 4 * kBox + kRopeBox;   // 36 KiB
-constexpr int kStages = 4;
-// Exchanged partial scores keep the top 24 bits of each fp32 value: 64 scores of a
-// head = 48 words = 12 chunks of 16 B. Layout of one exchange buffer: [warp 4][chunk 12]
-// [lane 32][16 B], so each warp's 32 heads are one contiguous 6 KiB piece (one bulk copy)
-// and a warp's 16-byte accesses to one chunk are 512 contiguous bytes.
-constexpr int kXWords = 48;
-constexpr int kXWarpBytes = 32 * kXWords * 4;      // 6 KiB
-constexpr int kXBytes = 4 * kXWarpBytes;           // 24 KiB
+constexpr int kStages = 5;
+// Exchanged partial scores, per softmax thread (one row, one token half: 32 values v_t):
+// 16-bit codes c_t = round(v_t * 32767 / a) + 32768 with a = max |v_t|, and the decode
+// step a / 32767 (fp32), so every value is kept to within 2^-16 of its block's largest
+// magnitude. Layout of the exchange buffer: per softmax warp one contiguous run (one
+// bulk copy) of [chunk 4][lane 32][16 B] codes followed by [lane 32] fp32 steps; a
+// warp's 16-byte accesses to one chunk are 512 contiguous bytes.
+constexpr int kXRunBytes = 4 * 512 + 32 * 4;       // 2176
+constexpr int kXBytes = 8 * kXRunBytes;            // 17 KiB
 
 constexpr int kOffKV = 0;
 constexpr int kQrBufs = 1;                               // rope query half buffers
 constexpr int kOffQr = kOffKV + kStages * kStageBytes;   // rope query half, 128 x 32 bf16
 constexpr int kQrBytes = 2 * kRopeBox;
-constexpr int kOffX = kOffQr + kQrBufs * kQrBytes;       // 2 slots: the peer's partial scores
-constexpr int kOffXout = kOffX + 2 * kXBytes;            // mine, staged for the bulk copy
+constexpr int kOffX = kOffQr + kQrBufs * kQrBytes;       // the peer's partial scores
+constexpr int kOffXout = kOffX + kXBytes;                // mine, staged for the bulk copy
 constexpr int kOffBar = kOffXout + kXBytes;              // 32 mbarriers
 constexpr int kOffTmem = kOffBar + 32 * 8;
 constexpr int kOffAbort = kOffTmem + 8;
@@ -81,26 +87,27 @@ constexpr int kThreads = 384;                            // warps 0-3 roles, 4-1
 constexpr int kSmemBytes = kSmemUsed + 1024;
 
 enum {
-  B_KV_FULL = 0,     // +stage (4)
-  B_KV_EMPTY = 4,    // +stage (4)
-  B_S_FULL = 8,      // score MMAs of a page done
-  B_S_EMPTY = 9,     // 8 softmax warps read S
-  B_X_FULL = 10,     // +slot (2): the peer's partial rows landed (1 local arrival + 24 KiB tx)
-  B_X_EMPTY = 12,    // +slot (2): the peer's 8 softmax warps have read the slot I fill
-  B_XOUT_FREE = 14,  // my previous copy landed in the peer (its watcher warp saw it)
-  B_P_FULL = 15,     // 8 softmax warps: P in TMEM (and O rescaled)
-  B_O_DONE = 16,     // value MMAs of a page done
-  B_QT_FULL = 17,    // query latent half staged in TMEM (8 softmax warps)
-  B_QT_EMPTY = 18,   // last score MMA of a unit done: the TMEM query columns are free
-  B_O_FREE = 19,     // 8 softmax warps have read O
-  B_DRAIN = 20,
-  B_ALL = 21,        // the 8 softmax warps
-  B_PAIR = 22,       // +lane quarter (4): the two softmax warps of a quarter
-  B_QR_FULL = 26,    // +buffer: rope query half landed (TMA)
-  B_QR_EMPTY = 26 + kQrBufs,   // +buffer: last score MMA of the unit that used it done
-  kNumBars = 26 + 2 * kQrBufs
+  B_KV_FULL = 0,                // +stage
+  B_KV_EMPTY = kStages,         // +stage
+  B_S_FULL = 2 * kStages,       // score MMAs of a page done
+  B_S_EMPTY,                    // 8 softmax warps read S
+  B_X_FULL,                     // the peer's partial scores landed (1 local arrival + 17 KiB tx)
+  B_X_EMPTY,                    // the peer's 8 softmax warps have read the slot I fill
+  B_XOUT_FREE,                  // my previous copy landed in the peer (its watcher warp saw it)
+  B_P_FULL,                     // 8 softmax warps: P in TMEM (and O rescaled)
+  B_O_DONE,                     // value MMAs of a page done
+  B_QT_FULL,                    // query latent half staged in TMEM (8 softmax warps)
+  B_QT_EMPTY,                   // last score MMA of a unit done: the TMEM query columns are free
+  B_O_FREE,                     // 8 softmax warps have read O
+  B_DRAIN,
+  B_ALL,                        // the 8 softmax warps
+  B_PAIR,                       // +lane quarter (4): the two softmax warps of a quarter
+  B_QR_FULL = B_PAIR + 4,       // +buffer: rope query half landed (TMA)
+  B_QR_EMPTY = B_QR_FULL + kQrBufs,   // +buffer: last score MMA of the unit that used it done
+  kNumBars = B_QR_EMPTY + kQrBufs
 };
 static_assert(kNumBars <= 32, "barrier area");
+static_assert(kSmemBytes <= 232448, "shared memory of one CTA");
 
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColO = 0, kColQ = 256, kColS = 384, kColP = 448;
@@ -215,10 +222,8 @@ decode_pair_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_const
     }
     ptx::mbar_init(bar(B_S_FULL), 1);
     ptx::mbar_init(bar(B_S_EMPTY), 8);
-    for (int b = 0; b < 2; ++b) {
-      ptx::mbar_init(bar(B_X_FULL + b), 1);
-      ptx::mbar_init(bar(B_X_EMPTY + b), 8);
-    }
+    ptx::mbar_init(bar(B_X_FULL), 1);
+    ptx::mbar_init(bar(B_X_EMPTY), 8);
     ptx::mbar_init(bar(B_XOUT_FREE), 1);
     ptx::mbar_init(bar(B_P_FULL), 8);
     ptx::mbar_init(bar(B_O_DONE), 1);
@@ -233,8 +238,7 @@ decode_pair_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_const
     ptx::mbar_init(bar(B_ALL), 8);
     for (int q = 0; q < 4; ++q) ptx::mbar_init(bar(B_PAIR + q), 2);
     ptx::fence_mbar_init();
-    ptx::mbar_arrive_expect_tx(bar(B_X_FULL), kXBytes);       // armed for pages 0 and 1
-    ptx::mbar_arrive_expect_tx(bar(B_X_FULL + 1), kXBytes);
+    ptx::mbar_arrive_expect_tx(bar(B_X_FULL), kXBytes);       // armed for page 0
   }
   if (warp == 2) {
     ptx::tmem_alloc(sbase + kOffTmem, kTmemCols);
@@ -440,7 +444,7 @@ decode_pair_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_const
     PageCursor c = first_page(p, plan, u_begin, u_end);
     uint32_t g = 0;
     while (c.valid) {
-      if (!wait_all(bar(B_X_FULL + (g & 1)), (g >> 1) & 1)) {
+      if (!wait_all(bar(B_X_FULL), g & 1)) {
         if (lane == 0) fail();
         break;
       }
@@ -459,10 +463,11 @@ decode_pair_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_const
     const int h = 32 * sub + lane;                 // this thread's head (TMEM lane)
     const bool tracer = sw == 0 && lane == 0;
     const uint32_t lane_addr = (32u * sub) << 16;
-    // this thread's 6 chunks of 16 B in an exchange buffer (see kXWords): quarter piece
-    // sub, chunks 6f..6f+5, lane; and its warp's 3 KiB run of chunks (one bulk copy)
-    const uint32_t x_lane = (uint32_t)sub * kXWarpBytes + (uint32_t)(6 * hf) * 512u + (uint32_t)lane * 16u;
-    const uint32_t x_run = (uint32_t)sub * kXWarpBytes + (uint32_t)hf * 3072u;
+    // this warp's run in an exchange buffer (one bulk copy), this thread's first chunk
+    // of codes and its decode step there (see kXRunBytes)
+    const uint32_t x_run = (uint32_t)sw * kXRunBytes;
+    const uint32_t x_lane = x_run + (uint32_t)lane * 16u;
+    const uint32_t x_step = x_run + 2048u + (uint32_t)lane * 4u;
     const uint32_t xo_lane = sbase + kOffXout + x_lane;
     auto pair_slot = [&](uint32_t stage, int off) {
       return reinterpret_cast<volatile float*>(smem + kOffKV + stage * kStageBytes + off);
@@ -513,22 +518,26 @@ decode_pair_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_const
       // 32-byte loads (one sector each): the 32 lanes read 32 different rows, so each
       // load instruction costs a transaction per lane and wider loads halve them
       const __nv_bfloat16* src = p.q_lat + ((int64_t)u.item * H + h) * kR + 256 * hf + 128 * (int)rank;
-      uint32_t w[2][32];
+      // (two rounds of 32 words, so that the staging holds few registers next to the
+      // softmax's scores)
+#pragma unroll 1
+      for (int half = 0; half < 2; ++half) {
+        uint32_t w[32];
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        uint32_t* d = &w[i >> 2][8 * (i & 3)];
-        if (present) {
-          asm volatile("ld.global.nc.v8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
-                       : "=r"(d[0]), "=r"(d[1]), "=r"(d[2]), "=r"(d[3]), "=r"(d[4]), "=r"(d[5]), "=r"(d[6]),
-                         "=r"(d[7])
-                       : "l"(src + 16 * i));
-        } else {
+        for (int i = 0; i < 4; ++i) {
+          uint32_t* d = &w[8 * i];
+          if (present) {
+            asm volatile("ld.global.nc.v8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+                         : "=r"(d[0]), "=r"(d[1]), "=r"(d[2]), "=r"(d[3]), "=r"(d[4]), "=r"(d[5]), "=r"(d[6]),
+                           "=r"(d[7])
+                         : "l"(src + 64 * half + 16 * i));
+          } else {
 #pragma unroll
-          for (int k = 0; k < 8; ++k) d[k] = 0u;
+            for (int k = 0; k < 8; ++k) d[k] = 0u;
+          }
         }
+        ptx::tmem_st_32x32b_x32(tbase + lane_addr + kColQ + 64 * hf + 32 * half, w);
       }
-      ptx::tmem_st_32x32b_x32(tbase + lane_addr + kColQ + 64 * hf, w[0]);
-      ptx::tmem_st_32x32b_x32(tbase + lane_addr + kColQ + 64 * hf + 32, w[1]);
       ptx::tmem_wait_st();
       ptx::tc_fence_before();
       __syncwarp();
@@ -536,8 +545,8 @@ decode_pair_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_const
       return true;
     };
     // Exchange of global page g: move this thread's 32 scores out of TMEM into `own`
-    // (freeing the score buffer), keep the top 24 bits of each, stage them and bulk-copy
-    // this warp's run into the peer's slot g & 1.
+    // (freeing the score buffer), encode them (see kXRunBytes), stage them and bulk-copy
+    // this warp's run into the peer's slot.
     auto exchange = [&](uint32_t g, float (&own)[32]) -> bool {
       if (!wait_all(bar(B_S_FULL), g & 1)) return false;
       if (tracer) PAIR_TRACE(3, g);
@@ -553,36 +562,37 @@ decode_pair_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_const
       __syncwarp();
       if (lane == 0) ptx::mbar_arrive(bar(B_S_EMPTY));
       // my copy of page g-1 has landed in the peer (the staging rows are free), and the
-      // peer has read its slot g & 1 (page g-2)
-      if (!wait_all(bar(B_XOUT_FREE), (g & 1) ^ 1) ||
-          !wait_all_cluster(bar(B_X_EMPTY + (g & 1)), ((g >> 1) & 1) ^ 1))
+      // peer has read it from its slot
+      if (!wait_all(bar(B_XOUT_FREE), (g & 1) ^ 1) || !wait_all_cluster(bar(B_X_EMPTY), (g & 1) ^ 1))
         return false;
       if (tracer) PAIR_TRACE(4, g);
       ptx::fence_proxy_async_smem();   // the previous copy's reads before these writes
+      // codes: v * (32767 / a) rounded to an integer by adding 1.5 * 2^23 + 2^15 (the sum's
+      // unit in the last place is 1), whose low 16 bits are then round(v * 32767 / a) + 32768
+      float a = 0.f;
 #pragma unroll
-      for (int r = 0; r < 2; ++r) {
-        // 16 values -> 12 words (bytes 1-3 of each value) -> 3 chunks
-        uint32_t w[12];
+      for (int t = 0; t < 32; ++t) a = fmaxf(a, fabsf(own[t]));
+      const float enc = a > 1e-30f ? 32767.f / a : 0.f;   // (smaller partials are sent as 0)
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const float* f = own + 16 * r + 4 * q;
-          const uint32_t a = __float_as_uint(f[0]), b = __float_as_uint(f[1]);
-          const uint32_t c = __float_as_uint(f[2]), d = __float_as_uint(f[3]);
-          w[3 * q] = __byte_perm(a, b, 0x5321);
-          w[3 * q + 1] = __byte_perm(b, c, 0x6532);
-          w[3 * q + 2] = __byte_perm(c, d, 0x7653);
+      for (int c = 0; c < 4; ++c) {
+        uint32_t w[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const float lo = fmaf(own[8 * c + 2 * i], enc, 12615680.f);
+          const float hi = fmaf(own[8 * c + 2 * i + 1], enc, 12615680.f);
+          w[i] = __byte_perm(__float_as_uint(lo), __float_as_uint(hi), 0x5410);
         }
-#pragma unroll
-        for (int c = 0; c < 3; ++c)
-          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(xo_lane + 512u * (3 * r + c)),
-                       "r"(w[4 * c]), "r"(w[4 * c + 1]), "r"(w[4 * c + 2]), "r"(w[4 * c + 3])
-                       : "memory");
+        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(xo_lane + 512u * c), "r"(w[0]), "r"(w[1]),
+                     "r"(w[2]), "r"(w[3])
+                     : "memory");
       }
+      asm volatile("st.shared.f32 [%0], %1;" ::"r"(sbase + kOffXout + x_step), "f"(a * (1.f / 32767.f))
+                   : "memory");
       ptx::fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0)
-        ptx::bulk_copy_to_cluster(peer_addr(sbase + kOffX + (g & 1) * kXBytes + x_run), sbase + kOffXout + x_run,
-                                  3072u, peer_addr(bar(B_X_FULL + (g & 1))));
+        ptx::bulk_copy_to_cluster(peer_addr(sbase + kOffX + x_run), sbase + kOffXout + x_run, (uint32_t)kXRunBytes,
+                                  peer_addr(bar(B_X_FULL)));
       return true;
     };
     // Once the score MMA of a unit's last page is done (its S was read), the query
@@ -706,32 +716,29 @@ decode_pair_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_const
         m_run = -CUDART_INF_F;
         l_run = 0.f;
       }
-      // ------------------------------------------------ the next page's exchange goes first
-      float nxt[32];
-      const bool more = ex.valid;
-      if (more && (!exchange(gpg + 1, nxt) || !stage_next_q(ex))) { fail(); ok = false; break; }
       // ------------------------------------------------ full scores: mine + the peer's
-      const uint32_t xs = gpg & 1;
-      if (!wait_all(bar(B_X_FULL + xs), (gpg >> 1) & 1)) { fail(); ok = false; break; }
+      if (!wait_all(bar(B_X_FULL), gpg & 1)) { fail(); ok = false; break; }
       if (tracer) PAIR_TRACE(5, gpg);
       float v[32];
+      {
+        float step;
+        asm volatile("ld.shared.f32 %0, [%1];" : "=f"(step) : "r"(sbase + kOffX + x_step) : "memory");
 #pragma unroll
-      for (int r = 0; r < 2; ++r) {
-        uint32_t w[12];
-#pragma unroll
-        for (int c = 0; c < 3; ++c)
+        for (int c = 0; c < 4; ++c) {
+          uint32_t w[4];
           asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
-                       : "=r"(w[4 * c]), "=r"(w[4 * c + 1]), "=r"(w[4 * c + 2]), "=r"(w[4 * c + 3])
-                       : "r"(sbase + kOffX + xs * kXBytes + x_lane + 512u * (3 * r + c))
+                       : "=r"(w[0]), "=r"(w[1]), "=r"(w[2]), "=r"(w[3])
+                       : "r"(sbase + kOffX + x_lane + 512u * c)
                        : "memory");
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          // the peer's values, bytes 1-3 (byte 0 is noise below the kept precision)
-          const int t = 16 * r + 4 * q;
-          v[t + 0] = own[t + 0] + __uint_as_float(w[3 * q] << 8);
-          v[t + 1] = own[t + 1] + __uint_as_float(__byte_perm(w[3 * q], w[3 * q + 1], 0x5433));
-          v[t + 2] = own[t + 2] + __uint_as_float(__byte_perm(w[3 * q + 1], w[3 * q + 2], 0x4322));
-          v[t + 3] = own[t + 3] + __uint_as_float(w[3 * q + 2]);
+          for (int i = 0; i < 4; ++i) {
+            // a code under the exponent and leading bits of 1.5 * 2^23 is that float plus
+            // the code; less the code's offset of 2^15 it is the peer's value / step
+            const float lo = __uint_as_float(__byte_perm(w[i], 0x4B400000u, 0x7610)) - 12615680.f;
+            const float hi = __uint_as_float(__byte_perm(w[i], 0x4B400000u, 0x7632)) - 12615680.f;
+            v[8 * c + 2 * i] = fmaf(lo, step, own[8 * c + 2 * i]);
+            v[8 * c + 2 * i + 1] = fmaf(hi, step, own[8 * c + 2 * i + 1]);
+          }
         }
       }
       // ------------------------------------------------ this page's maximum and reference
@@ -755,9 +762,14 @@ decode_pair_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_const
       // the slot are complete when lane 0 tells the peer that it may be overwritten.
       ptx::vote_any_ordered(mx > -CUDART_INF_F);
       if (lane == 0) {
-        if (sw == 0) ptx::mbar_arrive_expect_tx(bar(B_X_FULL + xs), kXBytes);   // arm the slot's next use
-        ptx::mbar_arrive_cluster_relaxed(peer_addr(bar(B_X_EMPTY + xs)));
+        if (sw == 0) ptx::mbar_arrive_expect_tx(bar(B_X_FULL), kXBytes);   // arm the slot's next use
+        ptx::mbar_arrive_cluster_relaxed(peer_addr(bar(B_X_EMPTY)));
       }
+      // ------------------------------------------------ the next page's exchange (the slot is
+      // free once both CTAs have read it), overlapping this page's exponentials; `own` is
+      // dead once v holds the sums and takes the next page's partial scores
+      const bool more = ex.valid;
+      if (more && (!exchange(gpg + 1, own) || !stage_next_q(ex))) { fail(); ok = false; break; }
       // the head's maximum over both token halves
       {
         volatile float* ms = pair_slot(gpg % kStages, kOffPairMax);
@@ -767,11 +779,7 @@ decode_pair_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_const
       }
       const bool need = mx > m_run + kRescaleThreshold;
       const bool any_need = __any_sync(0xffffffffu, need);
-      if (more) {
-#pragma unroll
-        for (int t = 0; t < 32; ++t) own[t] = nxt[t];
-        advance(p, plan, u_end, ex);
-      }
+      if (more) advance(p, plan, u_end, ex);
       // ------------------------------------------------ softmax of head h, this thread's 32 tokens
       const float mu = need ? mx : m_run;
       const float al = need ? ptx::ex2(m_run - mu) : 1.f;
