@@ -10,7 +10,9 @@
 //   exchange        each CTA encodes its 128 x 64 partial scores as 16-bit codes with
 //                   one scale per 32 values (see kXRunBytes), stages them in shared
 //                   memory and bulk-copies them into the peer's single receive slot
-//                   (DSMEM, 17 KiB each way); each CTA adds its own exact partial and the
+//                   (DSMEM, 17 KiB each way, one 2,176-byte run per softmax warp with
+//                   its own pair of barriers, so softmax warp w of one CTA waits only
+//                   for warp w of the other); each CTA adds its own exact partial and the
 //                   peer's decoded one, so the two sums agree to 2^-16 of the largest
 //                   partial in a block of 32
 //   softmax         fp32, two threads per row (32 tokens each), in both CTAs; each CTA
@@ -31,8 +33,7 @@
 // stages - 1 page periods, so the small exchange buffers buy the fifth stage.
 //
 // Warp roles (384 threads): warp 0 TMA producer, warp 1 MMA issuer, warp 2 TMEM
-// allocator, warp 3 exchange watcher, warps 4-11 query staging, exchange, softmax and
-// epilogue. Warps 4+q and 8+q access TMEM lanes 32q..32q+31 (rows 32q..), each thread
+// allocator, warp 3 idle, warps 4-11 query staging, exchange, softmax and epilogue. Warps 4+q and 8+q access TMEM lanes 32q..32q+31 (rows 32q..), each thread
 // half of one row's tokens.
 //
 // TMEM (512 columns, lane = row): [0,256) O, fp32, CTA r's latent columns in box
@@ -75,8 +76,8 @@ constexpr int kOffQr = kOffKV + kStages * kStageBytes;   // rope query half, 128
 constexpr int kQrBytes = 2 * kRopeBox;
 constexpr int kOffX = kOffQr + kQrBufs * kQrBytes;       // the peer's partial scores
 constexpr int kOffXout = kOffX + kXBytes;                // mine, staged for the bulk copy
-constexpr int kOffBar = kOffXout + kXBytes;              // 32 mbarriers
-constexpr int kOffTmem = kOffBar + 32 * 8;
+constexpr int kOffBar = kOffXout + kXBytes;              // 64 mbarriers
+constexpr int kOffTmem = kOffBar + 64 * 8;
 constexpr int kOffAbort = kOffTmem + 8;
 constexpr int kSmemUsed = kOffAbort + 8;
 // The two threads of a head exchange page maxima (and a unit's sums) through the rope box
@@ -91,10 +92,11 @@ enum {
   B_KV_EMPTY = kStages,         // +stage
   B_S_FULL = 2 * kStages,       // score MMAs of a page done
   B_S_EMPTY,                    // 8 softmax warps read S
-  B_X_FULL,                     // the peer's partial scores landed (1 local arrival + 17 KiB tx)
-  B_X_EMPTY,                    // the peer's 8 softmax warps have read the slot I fill
-  B_XOUT_FREE,                  // my previous copy landed in the peer (its watcher warp saw it)
-  B_P_FULL,                     // 8 softmax warps: P in TMEM (and O rescaled)
+  B_X_FULL,                     // +softmax warp (8): the peer's run for this warp landed
+                                // (1 local arrival + one run of tx bytes)
+  B_X_EMPTY = B_X_FULL + 8,     // +softmax warp (8): the peer's warp has read the run I fill
+                                // (and so my copy of it has landed: my staging run is free)
+  B_P_FULL = B_X_EMPTY + 8,                     // 8 softmax warps: P in TMEM (and O rescaled)
   B_O_DONE,                     // value MMAs of a page done
   B_QT_FULL,                    // query latent half staged in TMEM (8 softmax warps)
   B_QT_EMPTY,                   // last score MMA of a unit done: the TMEM query columns are free
@@ -106,7 +108,7 @@ enum {
   B_QR_EMPTY = B_QR_FULL + kQrBufs,   // +buffer: last score MMA of the unit that used it done
   kNumBars = B_QR_EMPTY + kQrBufs
 };
-static_assert(kNumBars <= 32, "barrier area");
+static_assert(kNumBars <= 64, "barrier area");
 static_assert(kSmemBytes <= 232448, "shared memory of one CTA");
 
 constexpr uint32_t kTmemCols = 512;
@@ -222,9 +224,10 @@ decode_pair_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_const
     }
     ptx::mbar_init(bar(B_S_FULL), 1);
     ptx::mbar_init(bar(B_S_EMPTY), 8);
-    ptx::mbar_init(bar(B_X_FULL), 1);
-    ptx::mbar_init(bar(B_X_EMPTY), 8);
-    ptx::mbar_init(bar(B_XOUT_FREE), 1);
+    for (int w = 0; w < 8; ++w) {
+      ptx::mbar_init(bar(B_X_FULL + w), 1);
+      ptx::mbar_init(bar(B_X_EMPTY + w), 1);
+    }
     ptx::mbar_init(bar(B_P_FULL), 8);
     ptx::mbar_init(bar(B_O_DONE), 1);
     ptx::mbar_init(bar(B_QT_FULL), 8);
@@ -238,7 +241,7 @@ decode_pair_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_const
     ptx::mbar_init(bar(B_ALL), 8);
     for (int q = 0; q < 4; ++q) ptx::mbar_init(bar(B_PAIR + q), 2);
     ptx::fence_mbar_init();
-    ptx::mbar_arrive_expect_tx(bar(B_X_FULL), kXBytes);       // armed for page 0
+    for (int w = 0; w < 8; ++w) ptx::mbar_arrive_expect_tx(bar(B_X_FULL + w), kXRunBytes);   // page 0
   }
   if (warp == 2) {
     ptx::tmem_alloc(sbase + kOffTmem, kTmemCols);
@@ -436,22 +439,6 @@ decode_pair_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_const
     if (leader) ptx::umma_commit(bar(B_DRAIN));
     __syncwarp();
     wait_all(bar(B_DRAIN), 0);
-  } else if (warp == 3) {
-    // ================================================================ exchange watcher
-    // A bulk copy into another CTA reports only to the destination's mbarrier: this warp
-    // tells the peer when each of its copies has landed here, so that the peer may refill
-    // the staging rows the copy read.
-    PageCursor c = first_page(p, plan, u_begin, u_end);
-    uint32_t g = 0;
-    while (c.valid) {
-      if (!wait_all(bar(B_X_FULL), g & 1)) {
-        if (lane == 0) fail();
-        break;
-      }
-      if (lane == 0) ptx::mbar_arrive_cluster_relaxed(peer_addr(bar(B_XOUT_FREE)));
-      advance(p, plan, u_end, c);
-      ++g;
-    }
   } else if (warp >= 4) {
     // ================================================================ query staging, exchange, softmax, epilogue
     // Warp 4 + 4f + q (f = 0, 1; q = 0..3) serves TMEM lane quarter q, i.e. heads 32q..32q+31,
@@ -561,10 +548,9 @@ decode_pair_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_const
       ptx::tc_fence_before();
       __syncwarp();
       if (lane == 0) ptx::mbar_arrive(bar(B_S_EMPTY));
-      // my copy of page g-1 has landed in the peer (the staging rows are free), and the
-      // peer has read it from its slot
-      if (!wait_all(bar(B_XOUT_FREE), (g & 1) ^ 1) || !wait_all_cluster(bar(B_X_EMPTY), (g & 1) ^ 1))
-        return false;
+      // the peer's warp has read page g-1 from its slot, so my copy of it has landed and
+      // the staging run is free
+      if (!wait_all_cluster(bar(B_X_EMPTY + sw), (g & 1) ^ 1)) return false;
       if (tracer) PAIR_TRACE(4, g);
       ptx::fence_proxy_async_smem();   // the previous copy's reads before these writes
       // codes: v * (32767 / a) rounded to an integer by adding 1.5 * 2^23 + 2^15 (the sum's
@@ -592,7 +578,7 @@ decode_pair_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_const
       __syncwarp();
       if (lane == 0)
         ptx::bulk_copy_to_cluster(peer_addr(sbase + kOffX + x_run), sbase + kOffXout + x_run, (uint32_t)kXRunBytes,
-                                  peer_addr(bar(B_X_FULL)));
+                                  peer_addr(bar(B_X_FULL + sw)));
       return true;
     };
     // Once the score MMA of a unit's last page is done (its S was read), the query
@@ -717,7 +703,7 @@ decode_pair_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_const
         l_run = 0.f;
       }
       // ------------------------------------------------ full scores: mine + the peer's
-      if (!wait_all(bar(B_X_FULL), gpg & 1)) { fail(); ok = false; break; }
+      if (!wait_all(bar(B_X_FULL + sw), gpg & 1)) { fail(); ok = false; break; }
       if (tracer) PAIR_TRACE(5, gpg);
       float v[32];
       {
@@ -762,8 +748,8 @@ decode_pair_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_const
       // the slot are complete when lane 0 tells the peer that it may be overwritten.
       ptx::vote_any_ordered(mx > -CUDART_INF_F);
       if (lane == 0) {
-        if (sw == 0) ptx::mbar_arrive_expect_tx(bar(B_X_FULL), kXBytes);   // arm the slot's next use
-        ptx::mbar_arrive_cluster_relaxed(peer_addr(bar(B_X_EMPTY)));
+        ptx::mbar_arrive_expect_tx(bar(B_X_FULL + sw), kXRunBytes);   // arm the run's next use
+        ptx::mbar_arrive_cluster_relaxed(peer_addr(bar(B_X_EMPTY + sw)));
       }
       // ------------------------------------------------ the next page's exchange (the slot is
       // free once both CTAs have read it), overlapping this page's exponentials; `own` is
