@@ -10,12 +10,12 @@
 //   exchange        each CTA encodes its 128 x 64 partial scores as 16-bit codes with
 //                   one scale per 32 values (see kXRunBytes), stages them in shared
 //                   memory and bulk-copies them into the peer's single receive slot
-//                   (DSMEM, 17 KiB each way, one 2,176-byte run per softmax warp with
-//                   its own pair of barriers, so softmax warp w of one CTA waits only
-//                   for warp w of the other); each CTA adds its own exact partial and the
-//                   peer's decoded one, so the two sums agree to 2^-16 of the largest
-//                   partial in a block of 32
-//   softmax         fp32, two threads per row (32 tokens each), in both CTAs; each CTA
+//                   (DSMEM, 17-18 KiB each way, one run per softmax warp with its own
+//                   pair of barriers, so softmax warp w of one CTA waits only for warp w
+//                   of the other); each CTA adds its own exact partial and the peer's
+//                   decoded one, so the two sums agree to 2^-16 of the largest partial
+//                   in a thread's block
+//   softmax         fp32, kTG threads per row (64 / kTG tokens each), in both CTAs; each CTA
 //                   keeps its own reference maximum, P, l and m, so each output half is
 //                   normalised consistently with the P it was summed with;
 //                   P = P_hi + P_lo (two bf16 parts) is written to TMEM
@@ -25,16 +25,19 @@
 // So each CTA streams half a page through its shared memory, every MMA has M=128 and
 // the value MMA reads only C from shared memory.
 //
-// The softmax warps read page j's exchange slot, release it and issue page j+1's
-// exchange before page j's exponentials, so the copy overlaps them; the MMA warp runs
-// the score MMAs two pages ahead of the value MMAs (order S0 S1 S2 V0 S3 V1 ...). Five
-// stages of pages: the loop that sets the page period (a stage's load, that page's
-// scores, the softmax that needs them, the value MMAs that free the stage) spans
-// stages - 1 page periods, so the small exchange buffers buy the fifth stage.
+// The softmax warps read page j's exchange slot, release it, post their part of page
+// j's row maxima to the other warps of their lane quarter and issue page j+1's
+// exchange, then combine the maxima and run page j's exponentials, so the copy and the
+// other warps' skew overlap work; the MMA warp runs the score MMAs two pages ahead of the value MMAs (order S0 S1
+// S2 V0 S3 V1 ...). Five stages of pages (the small exchange buffers buy the fifth).
 //
-// Warp roles (384 threads): warp 0 TMA producer, warp 1 MMA issuer, warp 2 TMEM
-// allocator, warp 3 idle, warps 4-11 query staging, exchange, softmax and epilogue. Warps 4+q and 8+q access TMEM lanes 32q..32q+31 (rows 32q..), each thread
-// half of one row's tokens.
+// Warp roles: warp 0 TMA producer, warp 1 MMA issuer (and TMEM allocator), then
+// 4 x kTG softmax warps (query staging, exchange, softmax, epilogue): 8 warps of 32
+// tokens per row by default (320 threads), or 16 warps of 16 with
+// MLA_PAIR_TOKEN_GROUPS=4 (576 threads, 96 registers each). The per-page chain of a
+// softmax warp is mostly fixed latency (TMEM loads and stores, barrier round trips,
+// proxy fences), so halving its arithmetic with twice the warps does not shorten it,
+// and the 96-register build spills: 16 warps measured slower.
 //
 // TMEM (512 columns, lane = row): [0,256) O, fp32, CTA r's latent columns in box
 // order; [256,384) the query's own latent half (bf16 pairs); [384,448) S; [448,480)
@@ -61,14 +64,24 @@ constexpr int kBox = 64 * 128;              // 64 rows x 64 bf16, 128-byte swizz
 constexpr int kRopeBox = 64 * 64;           // 64 rows x 32 bf16, 64-byte swizzle
 constexpr int kStageBytes = 4 * kBox + kRopeBox;   // 36 KiB
 constexpr int kStages = 5;
-// Exchanged partial scores, per softmax thread (one row, one token half: 32 values v_t):
+// Softmax warps: kTG per TMEM lane quarter, each thread one row and kTokT of a page's
+// tokens (token group tg = tokens kTokT*tg ..).
+#ifndef MLA_PAIR_TOKEN_GROUPS
+#define MLA_PAIR_TOKEN_GROUPS 2
+#endif
+constexpr int kTG = MLA_PAIR_TOKEN_GROUPS;
+static_assert(kTG == 2 || kTG == 4, "token groups");
+constexpr int kTokT = kPage / kTG;            // tokens per softmax thread
+constexpr int kSoftWarps = 4 * kTG;
+// Exchanged partial scores, per softmax thread (one row, one token group: kTokT values v_t):
 // 16-bit codes c_t = round(v_t * 32767 / a) + 32768 with a = max |v_t|, and the decode
 // step a / 32767 (fp32), so every value is kept to within 2^-16 of its block's largest
 // magnitude. Layout of the exchange buffer: per softmax warp one contiguous run (one
-// bulk copy) of [chunk 4][lane 32][16 B] codes followed by [lane 32] fp32 steps; a
-// warp's 16-byte accesses to one chunk are 512 contiguous bytes.
-constexpr int kXRunBytes = 4 * 512 + 32 * 4;       // 2176
-constexpr int kXBytes = 8 * kXRunBytes;            // 17 KiB
+// bulk copy) of [chunk kXChunks][lane 32][16 B] codes followed by [lane 32] fp32 steps;
+// a warp's 16-byte accesses to one chunk are 512 contiguous bytes.
+constexpr int kXChunks = kTokT / 8;
+constexpr int kXRunBytes = kXChunks * 512 + 32 * 4;   // 2176 (kTG 2) or 1152 (kTG 4)
+constexpr int kXBytes = kSoftWarps * kXRunBytes;      // 17 or 18 KiB
 
 constexpr int kOffKV = 0;
 constexpr int kQrBufs = 1;                               // rope query half buffers
@@ -80,30 +93,32 @@ constexpr int kOffBar = kOffXout + kXBytes;              // 64 mbarriers
 constexpr int kOffTmem = kOffBar + 64 * 8;
 constexpr int kOffAbort = kOffTmem + 8;
 constexpr int kSmemUsed = kOffAbort + 8;
-// The two threads of a head exchange page maxima (and a unit's sums) through the rope box
-// of the page's stage, idle once that page's score MMAs are done: float[2 halves][128]
-// at kOffPairMax (maxima) and kOffPairL (sums) within the stage.
-constexpr int kOffPairMax = 4 * kBox, kOffPairL = kOffPairMax + 2 * 128 * 4;
-constexpr int kThreads = 384;                            // warps 0-3 roles, 4-11 softmax
+// The kTG threads of a row exchange page maxima (and a unit's sums) through the rope box
+// of the page's stage, idle once that page's score MMAs are done: float[kTG][128] at
+// kOffPairMax (maxima) and kOffPairL (sums) within the stage.
+constexpr int kOffPairMax = 4 * kBox, kOffPairL = kOffPairMax + kTG * 128 * 4;
+static_assert(kOffPairL + kTG * 128 * 4 <= kStageBytes, "pair scratch in the rope box");
+constexpr int kRoleWarps = 2;                            // warp 0 TMA producer, warp 1 MMA
+constexpr int kThreads = 32 * (kRoleWarps + kSoftWarps);
 constexpr int kSmemBytes = kSmemUsed + 1024;
 
 enum {
   B_KV_FULL = 0,                // +stage
   B_KV_EMPTY = kStages,         // +stage
   B_S_FULL = 2 * kStages,       // score MMAs of a page done
-  B_S_EMPTY,                    // 8 softmax warps read S
-  B_X_FULL,                     // +softmax warp (8): the peer's run for this warp landed
+  B_S_EMPTY,                    // the softmax warps read S
+  B_X_FULL,                     // +softmax warp: the peer's run for this warp landed
                                 // (1 local arrival + one run of tx bytes)
-  B_X_EMPTY = B_X_FULL + 8,     // +softmax warp (8): the peer's warp has read the run I fill
-                                // (and so my copy of it has landed: my staging run is free)
-  B_P_FULL = B_X_EMPTY + 8,                     // 8 softmax warps: P in TMEM (and O rescaled)
+  B_X_EMPTY = B_X_FULL + kSoftWarps,   // +softmax warp: the peer's warp has read the run I
+                                // fill (and so my copy of it has landed: my staging run is free)
+  B_P_FULL = B_X_EMPTY + kSoftWarps,   // the softmax warps: P in TMEM (and O rescaled)
   B_O_DONE,                     // value MMAs of a page done
-  B_QT_FULL,                    // query latent half staged in TMEM (8 softmax warps)
+  B_QT_FULL,                    // query latent half staged in TMEM (the softmax warps)
   B_QT_EMPTY,                   // last score MMA of a unit done: the TMEM query columns are free
-  B_O_FREE,                     // 8 softmax warps have read O
+  B_O_FREE,                     // the softmax warps have read O
   B_DRAIN,
-  B_ALL,                        // the 8 softmax warps
-  B_PAIR,                       // +lane quarter (4): the two softmax warps of a quarter
+  B_ALL,                        // the softmax warps
+  B_PAIR,                       // +lane quarter (4): the kTG softmax warps of a quarter
   B_QR_FULL = B_PAIR + 4,       // +buffer: rope query half landed (TMA)
   B_QR_EMPTY = B_QR_FULL + kQrBufs,   // +buffer: last score MMA of the unit that used it done
   kNumBars = B_QR_EMPTY + kQrBufs
@@ -223,27 +238,27 @@ decode_pair_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_const
       ptx::mbar_init(bar(B_KV_EMPTY + s), 1);
     }
     ptx::mbar_init(bar(B_S_FULL), 1);
-    ptx::mbar_init(bar(B_S_EMPTY), 8);
-    for (int w = 0; w < 8; ++w) {
+    ptx::mbar_init(bar(B_S_EMPTY), kSoftWarps);
+    for (int w = 0; w < kSoftWarps; ++w) {
       ptx::mbar_init(bar(B_X_FULL + w), 1);
       ptx::mbar_init(bar(B_X_EMPTY + w), 1);
     }
-    ptx::mbar_init(bar(B_P_FULL), 8);
+    ptx::mbar_init(bar(B_P_FULL), kSoftWarps);
     ptx::mbar_init(bar(B_O_DONE), 1);
-    ptx::mbar_init(bar(B_QT_FULL), 8);
+    ptx::mbar_init(bar(B_QT_FULL), kSoftWarps);
     ptx::mbar_init(bar(B_QT_EMPTY), 1);
     for (int b = 0; b < kQrBufs; ++b) {
       ptx::mbar_init(bar(B_QR_FULL + b), 1);
       ptx::mbar_init(bar(B_QR_EMPTY + b), 1);
     }
-    ptx::mbar_init(bar(B_O_FREE), 8);
+    ptx::mbar_init(bar(B_O_FREE), kSoftWarps);
     ptx::mbar_init(bar(B_DRAIN), 1);
-    ptx::mbar_init(bar(B_ALL), 8);
-    for (int q = 0; q < 4; ++q) ptx::mbar_init(bar(B_PAIR + q), 2);
+    ptx::mbar_init(bar(B_ALL), kSoftWarps);
+    for (int q = 0; q < 4; ++q) ptx::mbar_init(bar(B_PAIR + q), kTG);
     ptx::fence_mbar_init();
-    for (int w = 0; w < 8; ++w) ptx::mbar_arrive_expect_tx(bar(B_X_FULL + w), kXRunBytes);   // page 0
+    for (int w = 0; w < kSoftWarps; ++w) ptx::mbar_arrive_expect_tx(bar(B_X_FULL + w), kXRunBytes);   // page 0
   }
-  if (warp == 2) {
+  if (warp == 1) {
     ptx::tmem_alloc(sbase + kOffTmem, kTmemCols);
     ptx::tmem_relinquish();
   }
@@ -439,14 +454,15 @@ decode_pair_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_const
     if (leader) ptx::umma_commit(bar(B_DRAIN));
     __syncwarp();
     wait_all(bar(B_DRAIN), 0);
-  } else if (warp >= 4) {
+  } else if (warp >= kRoleWarps) {
     // ================================================================ query staging, exchange, softmax, epilogue
-    // Warp 4 + 4f + q (f = 0, 1; q = 0..3) serves TMEM lane quarter q, i.e. heads 32q..32q+31,
-    // and token half f of every page (tokens 32f..32f+31): the two threads of a head (same
-    // lane in warps 4+q and 8+q) meet on the quarter's pair barrier to combine their
-    // maxima (and, in the epilogue, their sums).
-    const int sw = warp - 4;
-    const int sub = sw & 3, hf = sw >> 2;
+    // Softmax warp sw = warp - kRoleWarps serves TMEM lane quarter q = warp % 4 (the only
+    // quarter a warp reaches), i.e. rows 32q..32q+31, and token group g = sw / 4 of every
+    // page (tokens kTokT*g ..): the kTG threads of a row (same lane in the kTG warps of
+    // the quarter) meet on the quarter's pair barrier to combine their maxima (and, in
+    // the epilogue, their sums).
+    const int sw = warp - kRoleWarps;
+    const int sub = warp & 3, tg = sw >> 2;
     const int h = 32 * sub + lane;                 // this thread's head (TMEM lane)
     const bool tracer = sw == 0 && lane == 0;
     const uint32_t lane_addr = (32u * sub) << 16;
@@ -454,7 +470,7 @@ decode_pair_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_const
     // of codes and its decode step there (see kXRunBytes)
     const uint32_t x_run = (uint32_t)sw * kXRunBytes;
     const uint32_t x_lane = x_run + (uint32_t)lane * 16u;
-    const uint32_t x_step = x_run + 2048u + (uint32_t)lane * 4u;
+    const uint32_t x_step = x_run + (uint32_t)kXChunks * 512u + (uint32_t)lane * 4u;
     const uint32_t xo_lane = sbase + kOffXout + x_lane;
     auto pair_slot = [&](uint32_t stage, int off) {
       return reinterpret_cast<volatile float*>(smem + kOffKV + stage * kStageBytes + off);
@@ -468,6 +484,16 @@ decode_pair_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_const
       ++n;
       return __all_sync(0xffffffffu, done);
     };
+    // the same in two halves, with other work between the arrival and the wait
+    auto sync_arrive = [&](uint32_t b) {
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive(bar(b));
+    };
+    auto sync_wait = [&](uint32_t b, uint32_t& n) -> bool {
+      const bool done = ptx::mbar_wait_bounded(bar(b), n & 1, abort_flag, p.timeout_ns);
+      ++n;
+      return __all_sync(0xffffffffu, done);
+    };
 
     // Row h belongs to query token tok_h of a unit (0 for H = 128), head h % H.
     const int tok_h = h / H;
@@ -476,7 +502,7 @@ decode_pair_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_const
     for (int32_t ui = u_begin; ui < u_end; ++ui) {
       const PairUnit u = load_punit(p, plan, ui);
       if (u.npg > 0) continue;
-      for (int e = threadIdx.x - 128; e < u.n * H * 256; e += kThreads - 128) {
+      for (int e = threadIdx.x - 32 * kRoleWarps; e < u.n * H * 256; e += kThreads - 32 * kRoleWarps) {
         const int r = e / 256, j = e % 256, t = r / H;
         const int d = (j < 128 ? 128 * (int)rank : 256 + 128 * (int)rank) + (j & 127);
         const int32_t prt = t ? u.part[1] : u.part[0];
@@ -485,7 +511,7 @@ decode_pair_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_const
         else
           p.o_part[((int64_t)prt * H + r % H) * kR + d] = 0.f;
       }
-      if (rank == 0 && hf == 0 && tok_h < u.n) {
+      if (rank == 0 && tg == 0 && tok_h < u.n) {
         const int32_t prt = tok_h ? u.part[1] : u.part[0];
         if (prt < 0) {
           if (p.lse) p.lse[(int64_t)(u.item + tok_h) * H + h % H] = -CUDART_INF_F;
@@ -495,20 +521,21 @@ decode_pair_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_const
       }
     }
 
-    // Stage a unit's query: this thread's 128 of head h's own 256 latent dims
-    // (128r.. for f = 0, 256+128r.. for f = 1) -> TMEM columns 64f..64f+63.
+    // Stage a unit's query: this thread's 256 / kTG of row h's own 256 latent dims, box
+    // slots 4g/kTG .. (slot s: dims 128r + 64s for s < 2, 256 + 128r + 64(s-2) above) ->
+    // TMEM columns 32s.. of the query block.
     auto stage_q = [&](const PairUnit& u, uint32_t n) -> bool {
       if (!wait_all(bar(B_QT_EMPTY), (n & 1) ^ 1)) return false;
       ptx::tc_fence_after();
       // rows of a token the unit does not have stay zero (their scores are never used)
       const bool present = tok_h < u.n;
       // 32-byte loads (one sector each): the 32 lanes read 32 different rows, so each
-      // load instruction costs a transaction per lane and wider loads halve them
-      const __nv_bfloat16* src = p.q_lat + ((int64_t)u.item * H + h) * kR + 256 * hf + 128 * (int)rank;
-      // (two rounds of 32 words, so that the staging holds few registers next to the
-      // softmax's scores)
+      // load instruction costs a transaction per lane and wider loads halve them; one box
+      // slot (32 words) per round, so that the staging holds few registers
 #pragma unroll 1
-      for (int half = 0; half < 2; ++half) {
+      for (int s = (4 / kTG) * tg; s < (4 / kTG) * (tg + 1); ++s) {
+        const int d0 = s < 2 ? 128 * (int)rank + 64 * s : 256 + 128 * (int)rank + 64 * (s - 2);
+        const __nv_bfloat16* src = p.q_lat + ((int64_t)u.item * H + h) * kR + d0;
         uint32_t w[32];
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
@@ -517,13 +544,13 @@ decode_pair_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_const
             asm volatile("ld.global.nc.v8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
                          : "=r"(d[0]), "=r"(d[1]), "=r"(d[2]), "=r"(d[3]), "=r"(d[4]), "=r"(d[5]), "=r"(d[6]),
                            "=r"(d[7])
-                         : "l"(src + 64 * half + 16 * i));
+                         : "l"(src + 16 * i));
           } else {
 #pragma unroll
             for (int k = 0; k < 8; ++k) d[k] = 0u;
           }
         }
-        ptx::tmem_st_32x32b_x32(tbase + lane_addr + kColQ + 64 * hf + 32 * half, w);
+        ptx::tmem_st_32x32b_x32(tbase + lane_addr + kColQ + 32 * s, w);
       }
       ptx::tmem_wait_st();
       ptx::tc_fence_before();
@@ -531,19 +558,19 @@ decode_pair_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_const
       if (lane == 0) ptx::mbar_arrive(bar(B_QT_FULL));
       return true;
     };
-    // Exchange of global page g: move this thread's 32 scores out of TMEM into `own`
+    // Exchange of global page g: move this thread's kTokT scores out of TMEM into `own`
     // (freeing the score buffer), encode them (see kXRunBytes), stage them and bulk-copy
     // this warp's run into the peer's slot.
-    auto exchange = [&](uint32_t g, float (&own)[32]) -> bool {
+    auto exchange = [&](uint32_t g, float (&own)[kTokT]) -> bool {
       if (!wait_all(bar(B_S_FULL), g & 1)) return false;
       if (tracer) PAIR_TRACE(3, g);
       ptx::tc_fence_after();
       {
-        uint32_t r[32];
-        ptx::tmem_ld_32x32b_x32(tbase + lane_addr + kColS + 32 * hf, r);
+        uint32_t r[kTokT];
+        ptx::tmem_ld_cols<kTokT>(tbase + lane_addr + kColS + kTokT * tg, r);
         ptx::tmem_wait_ld();
 #pragma unroll
-        for (int t = 0; t < 32; ++t) own[t] = __uint_as_float(r[t]);
+        for (int t = 0; t < kTokT; ++t) own[t] = __uint_as_float(r[t]);
       }
       ptx::tc_fence_before();
       __syncwarp();
@@ -557,10 +584,11 @@ decode_pair_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_const
       // unit in the last place is 1), whose low 16 bits are then round(v * 32767 / a) + 32768
       float a = 0.f;
 #pragma unroll
-      for (int t = 0; t < 32; ++t) a = fmaxf(a, fabsf(own[t]));
-      const float enc = a > 1e-30f ? 32767.f / a : 0.f;   // (smaller partials are sent as 0)
+      for (int t = 0; t < kTokT; ++t) a = fmaxf(a, fabsf(own[t]));
+      // (an approximate quotient: |v| * enc stays below 32767.5; smaller partials are sent as 0)
+      const float enc = a > 1e-30f ? __fdividef(32767.f, a) : 0.f;
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
+      for (int c = 0; c < kXChunks; ++c) {
         uint32_t w[4];
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
@@ -591,72 +619,76 @@ decode_pair_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_const
     };
     // Epilogue of a unit, run after the next unit's first P (or after the last page of
     // the slot) once the unit's last value MMAs are done: O[h][:] / l to the output. This
-    // thread holds O columns 128f..128f+127; the warps of token half f stage their rows in
-    // 16 KiB f of the unit's last stage (released to the producer at the end), and a warp
-    // reads back only its own 32 rows, so that each warp store writes whole 128-byte row
-    // segments.
+    // thread holds O columns (256/kTG)g ..; the warps of token group g stage their rows
+    // (kRowB bytes per row and round) in the g-th 128 x kRowB block of the unit's last
+    // stage (released to the producer at the end), and a warp reads back only its own 32
+    // rows, so that each warp store writes whole row segments.
     struct Pending {
       bool on;
       int32_t item, n, part0, part1;   // the unit's tokens and their partial-output indices
       uint32_t stage;                  // stage of the unit's last page
-      float l, m;                      // this thread's half of l; the shared reference maximum
+      float l, m;                      // this thread's part of l; the shared reference maximum
     } pend{false, 0, 0, -1, -1, 0u, 0.f, 0.f};
     auto epilogue = [&]() -> bool {
-      // l = the two halves' sums
+      // l = the token groups' sums, added in group order (the same value in each thread of a row)
       volatile float* ls = pair_slot(pend.stage, kOffPairL);
-      ls[128 * hf + h] = pend.l;
+      ls[128 * tg + h] = pend.l;
       if (!bounded_sync(B_PAIR + sub, n_pair)) return false;
-      const float l = pend.l + ls[128 * (hf ^ 1) + h];
+      float l = 0.f;
+#pragma unroll
+      for (int t = 0; t < kTG; ++t) l += ls[128 * t + h];
       ptx::tc_fence_after();
       const float inv_l = l > 0.f ? 1.f / l : 0.f;
-      const uint32_t buf = sbase + kOffKV + pend.stage * kStageBytes + (uint32_t)hf * 16384u;
+      constexpr int kRowB = 256 / kTG;   // staged bytes per row and round
+      constexpr int kCh = kRowB / 16;    // 16-byte chunks per staged row
+      const uint32_t buf = sbase + kOffKV + pend.stage * kStageBytes + (uint32_t)tg * (128u * kRowB);
       // this warp's 32 rows all belong to token tok_h of the unit: its output rows
       const bool present = tok_h < pend.n;
       const int32_t prt = tok_h ? pend.part1 : pend.part0;
       const bool final_out = prt < 0;
       const int64_t row0 = (final_out ? (int64_t)(pend.item + tok_h) * H : (int64_t)prt * H) - tok_h * H;
-      const int rounds = final_out ? 2 : 4;     // 64 bf16 or 32 fp32 columns per round
-      const int cols = final_out ? 64 : 32;
+      const int rounds = final_out ? 2 : 4;                  // (256/kTG) columns in kRowB-byte rows
+      const int cols = final_out ? kRowB / 2 : kRowB / 4;    // O columns per round
 #pragma unroll 1
       for (int c = 0; c < rounds; ++c) {
-        const int col0 = 128 * hf + cols * c;        // TMEM column of the round
-        uint32_t w[32];
+        const int col0 = (256 / kTG) * tg + cols * c;        // TMEM column of the round
+        uint32_t w[kRowB / 4];
         if (final_out) {
-          uint32_t o[2][32];
-          ptx::tmem_ld_32x32b_x32(tbase + lane_addr + kColO + col0, o[0]);
-          ptx::tmem_ld_32x32b_x32(tbase + lane_addr + kColO + col0 + 32, o[1]);
+          uint32_t o[kRowB / 64][32];
+#pragma unroll
+          for (int k = 0; k < kRowB / 64; ++k) ptx::tmem_ld_32x32b_x32(tbase + lane_addr + kColO + col0 + 32 * k, o[k]);
           ptx::tmem_wait_ld();
 #pragma unroll
-          for (int half = 0; half < 2; ++half) {
+          for (int k = 0; k < kRowB / 64; ++k) {
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
-              __nv_bfloat162 b2 = __floats2bfloat162_rn(__uint_as_float(o[half][2 * i]) * inv_l,
-                                                        __uint_as_float(o[half][2 * i + 1]) * inv_l);
-              w[16 * half + i] = *reinterpret_cast<uint32_t*>(&b2);
+              __nv_bfloat162 b2 = __floats2bfloat162_rn(__uint_as_float(o[k][2 * i]) * inv_l,
+                                                        __uint_as_float(o[k][2 * i + 1]) * inv_l);
+              w[16 * k + i] = *reinterpret_cast<uint32_t*>(&b2);
             }
           }
         } else {
-          ptx::tmem_ld_32x32b_x32(tbase + lane_addr + kColO + col0, w);
+          ptx::tmem_ld_cols<kRowB / 4>(tbase + lane_addr + kColO + col0, w);
           ptx::tmem_wait_ld();
 #pragma unroll
-          for (int i = 0; i < 32; ++i) w[i] = __float_as_uint(__uint_as_float(w[i]) * inv_l);
+          for (int i = 0; i < kRowB / 4; ++i) w[i] = __float_as_uint(__uint_as_float(w[i]) * inv_l);
         }
         __syncwarp();   // this warp's previous round has been read back
 #pragma unroll
-        for (int j = 0; j < 8; ++j)
-          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(buf + (uint32_t)h * 128u +
-                                                                       (uint32_t)((j ^ (h & 7)) << 4)),
+        for (int j = 0; j < kCh; ++j)
+          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(buf + (uint32_t)h * kRowB +
+                                                                       (uint32_t)((j ^ (h & (kCh - 1))) << 4)),
                        "r"(w[4 * j]), "r"(w[4 * j + 1]), "r"(w[4 * j + 2]), "r"(w[4 * j + 3])
                        : "memory");
         __syncwarp();
         const int d0 = (col0 < 128 ? 128 * (int)rank + col0 : 256 + 128 * (int)rank + (col0 - 128));
 #pragma unroll
-        for (int it = 0; it < 8; ++it) {
-          const int row = 32 * sub + 4 * it + (lane >> 3), j = lane & 7;
+        for (int it = 0; it < kCh; ++it) {
+          const int row = 32 * sub + (32 / kCh) * it + lane / kCh, j = lane % kCh;
           uint4 q;
           asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
                        : "=r"(q.x), "=r"(q.y), "=r"(q.z), "=r"(q.w)
-                       : "r"(buf + (uint32_t)row * 128u + (uint32_t)((j ^ (row & 7)) << 4))
+                       : "r"(buf + (uint32_t)row * kRowB + (uint32_t)((j ^ (row & (kCh - 1))) << 4))
                        : "memory");
           if (!present) continue;
           if (final_out)
@@ -665,7 +697,7 @@ decode_pair_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_const
             *reinterpret_cast<uint4*>(p.o_part + (row0 + row) * kR + d0 + 4 * j) = q;
         }
       }
-      if (rank == 0 && hf == 0 && present) {
+      if (rank == 0 && tg == 0 && present) {
         const float z = l > 0.f ? (pend.m + log2f(l)) * 0.69314718055994531f : -CUDART_INF_F;
         if (final_out) {
           if (p.lse) p.lse[row0 + h] = z;
@@ -689,7 +721,7 @@ decode_pair_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_const
     PageCursor cur = first_page(p, plan, u_begin, u_end);
     PageCursor ex = cur;
     uint32_t gpg = 0;
-    float own[32];   // this thread's partial scores for the page read next
+    float own[kTokT];   // this thread's partial scores for the page read next
     if (cur.valid) {
       if (!stage_q(cur.u, 0) || !exchange(0, own) || !stage_next_q(ex)) { fail(); ok = false; }
       advance(p, plan, u_end, ex);
@@ -705,12 +737,12 @@ decode_pair_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_const
       // ------------------------------------------------ full scores: mine + the peer's
       if (!wait_all(bar(B_X_FULL + sw), gpg & 1)) { fail(); ok = false; break; }
       if (tracer) PAIR_TRACE(5, gpg);
-      float v[32];
+      float v[kTokT];
       {
         float step;
         asm volatile("ld.shared.f32 %0, [%1];" : "=f"(step) : "r"(sbase + kOffX + x_step) : "memory");
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
+        for (int c = 0; c < kXChunks; ++c) {
           uint32_t w[4];
           asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
                        : "=r"(w[0]), "=r"(w[1]), "=r"(w[2]), "=r"(w[3])
@@ -728,21 +760,23 @@ decode_pair_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_const
         }
       }
       // ------------------------------------------------ this page's maximum and reference
-      const int32_t tok0 = (u.pb + cur.k) * kPage + 32 * hf;
-      if (tok0 + 32 > ntok) {
+      const int32_t tok0 = (u.pb + cur.k) * kPage + kTokT * tg;
+      if (tok0 + kTokT > ntok) {
 #pragma unroll
-        for (int t = 0; t < 32; ++t) v[t] = (tok0 + t < ntok) ? v[t] : -CUDART_INF_F;
+        for (int t = 0; t < kTokT; ++t) v[t] = (tok0 + t < ntok) ? v[t] : -CUDART_INF_F;
       }
       float mx;
       {
-        float t4[4];
+        float t8[kTokT / 8];
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
+        for (int i = 0; i < kTokT / 8; ++i) {
           const float a = fmaxf(fmaxf(v[8 * i], v[8 * i + 1]), fmaxf(v[8 * i + 2], v[8 * i + 3]));
           const float b = fmaxf(fmaxf(v[8 * i + 4], v[8 * i + 5]), fmaxf(v[8 * i + 6], v[8 * i + 7]));
-          t4[i] = fmaxf(a, b);
+          t8[i] = fmaxf(a, b);
         }
-        mx = fmaxf(fmaxf(t4[0], t4[1]), fmaxf(t4[2], t4[3]));
+        mx = t8[0];
+#pragma unroll
+        for (int i = 1; i < kTokT / 8; ++i) mx = fmaxf(mx, t8[i]);
       }
       // The vote depends on every lane's loaded values, so all of this warp's reads of
       // the slot are complete when lane 0 tells the peer that it may be overwritten.
@@ -751,29 +785,32 @@ decode_pair_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_const
         ptx::mbar_arrive_expect_tx(bar(B_X_FULL + sw), kXRunBytes);   // arm the run's next use
         ptx::mbar_arrive_cluster_relaxed(peer_addr(bar(B_X_EMPTY + sw)));
       }
+      // this group's maximum to the quarter's other warps; theirs are read after the
+      // exchange below
+      volatile float* ms = pair_slot(gpg % kStages, kOffPairMax);
+      ms[128 * tg + h] = mx;
+      sync_arrive(B_PAIR + sub);
       // ------------------------------------------------ the next page's exchange (the slot is
       // free once both CTAs have read it), overlapping this page's exponentials; `own` is
       // dead once v holds the sums and takes the next page's partial scores
       const bool more = ex.valid;
       if (more && (!exchange(gpg + 1, own) || !stage_next_q(ex))) { fail(); ok = false; break; }
-      // the head's maximum over both token halves
-      {
-        volatile float* ms = pair_slot(gpg % kStages, kOffPairMax);
-        ms[128 * hf + h] = mx;
-        if (!bounded_sync(B_PAIR + sub, n_pair)) { fail(); ok = false; break; }
-        mx = fmaxf(mx, ms[128 * (hf ^ 1) + h]) * p.scale_log2;
-      }
+      // the row's maximum over the token groups
+      if (!sync_wait(B_PAIR + sub, n_pair)) { fail(); ok = false; break; }
+#pragma unroll
+      for (int t = 0; t < kTG; ++t) mx = fmaxf(mx, ms[128 * t + h]);
+      mx *= p.scale_log2;
       const bool need = mx > m_run + kRescaleThreshold;
       const bool any_need = __any_sync(0xffffffffu, need);
       if (more) advance(p, plan, u_end, ex);
-      // ------------------------------------------------ softmax of head h, this thread's 32 tokens
+      // ------------------------------------------------ softmax of row h, this thread's kTokT tokens
       const float mu = need ? mx : m_run;
       const float al = need ? ptx::ex2(m_run - mu) : 1.f;
       const float nz = (mu == -CUDART_INF_F) ? 0.f : -mu;
-      uint32_t ph[16], pl[16];
+      uint32_t ph[kTokT / 2], pl[kTokT / 2];
       float sum4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-      for (int i = 0; i < 16; ++i) {
+      for (int i = 0; i < kTokT / 2; ++i) {
         const float a0 = ptx::ex2(fmaf(v[2 * i], p.scale_log2, nz));
         const float a1 = ptx::ex2(fmaf(v[2 * i + 1], p.scale_log2, nz));
         sum4[i & 3] += a0 + a1;
@@ -793,15 +830,15 @@ decode_pair_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_const
       if (gpg > 0 && !wait_all(bar(B_O_DONE), (gpg - 1) & 1)) { fail(); ok = false; break; }
       ptx::tc_fence_after();
       if (tracer) PAIR_TRACE(7, gpg);
-      ptx::tmem_st_32x32b_x16u(tbase + lane_addr + kColP + 16 * hf, ph);
-      ptx::tmem_st_32x32b_x16u(tbase + lane_addr + kColP + 32 + 16 * hf, pl);
+      ptx::tmem_st_cols<kTokT / 2>(tbase + lane_addr + kColP + (kTokT / 2) * tg, ph);
+      ptx::tmem_st_cols<kTokT / 2>(tbase + lane_addr + kColP + 32 + (kTokT / 2) * tg, pl);
       if (cur.k > 0 && any_need) {
-        // a moved reference: O[h][:] *= 2^(m_old - m_new) (1 for heads that kept theirs);
-        // this thread scales its 128 columns
+        // a moved reference: O[h][:] *= 2^(m_old - m_new) (1 for rows that kept theirs);
+        // this thread scales its 256 / kTG columns
 #pragma unroll 1
-        for (int c = 0; c < 4; ++c) {
+        for (int c = 0; c < 8 / kTG; ++c) {
           uint32_t o[32];
-          const uint32_t ta = tbase + lane_addr + kColO + 128 * hf + 32 * c;
+          const uint32_t ta = tbase + lane_addr + kColO + (256 / kTG) * tg + 32 * c;
           ptx::tmem_ld_32x32b_x32(ta, o);
           ptx::tmem_wait_ld();
 #pragma unroll
@@ -835,7 +872,7 @@ decode_pair_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_const
 
   ptx::tc_fence_before();
   __syncthreads();
-  if (warp == 2) {
+  if (warp == 1) {
     ptx::tc_fence_after();
     ptx::tmem_dealloc(tbase, kTmemCols);
   }

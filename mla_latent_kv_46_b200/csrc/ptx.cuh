@@ -316,6 +316,34 @@ __device__ __forceinline__ void tmem_st_32x32b_x16u(uint32_t taddr, const uint32
       : "memory");
 }
 
+__device__ __forceinline__ void tmem_ld_32x32b_x16u(uint32_t taddr, uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_st_32x32b_x8u(uint32_t taddr, const uint32_t (&r)[8]) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(taddr), "r"(r[0]),
+               "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
+               : "memory");
+}
+// Row-wise TMEM access of N consecutive 32-bit columns (32x32b shape, one lane per thread).
+template <int N>
+__device__ __forceinline__ void tmem_ld_cols(uint32_t taddr, uint32_t (&r)[N]) {
+  static_assert(N == 16 || N == 32, "columns");
+  if constexpr (N == 32) tmem_ld_32x32b_x32(taddr, r);
+  else tmem_ld_32x32b_x16u(taddr, r);
+}
+template <int N>
+__device__ __forceinline__ void tmem_st_cols(uint32_t taddr, const uint32_t (&r)[N]) {
+  static_assert(N == 8 || N == 16 || N == 32, "columns");
+  if constexpr (N == 32) tmem_st_32x32b_x32(taddr, r);
+  else if constexpr (N == 16) tmem_st_32x32b_x16u(taddr, r);
+  else tmem_st_32x32b_x8u(taddr, r);
+}
+
 // ------------------------------------------------------------------ UMMA descriptors
 // Shared-memory matrix descriptor, 128-byte swizzle (atoms of 8 rows x 128 B,
 // the layout TMA writes with CU_TENSOR_MAP_SWIZZLE_128B from a 1024-B aligned base):
