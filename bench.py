@@ -213,17 +213,44 @@ def run_reference(args):
 
 # ----------------------------------------------------------------------------- GPU arm
 
-def workload_config(spec, w, args):
+def reduce_over_ranks(world, device, sums=(), maxes=()):
+    """Sums and maxima of per-rank numbers over all ranks of the default process group, in
+    float64 on `device` (identity on one rank). Every rank makes the same calls in the same
+    order: one all-reduce for the sums, one for the maxima."""
+    sums, maxes = [float(x) for x in sums], [float(x) for x in maxes]
+    if world == 1:
+        return sums, maxes
+    import torch
+    import torch.distributed as dist
+    out = []
+    for vals, op in ((sums, dist.ReduceOp.SUM), (maxes, dist.ReduceOp.MAX)):
+        if vals:
+            t = torch.tensor(vals, dtype=torch.float64, device=device)
+            dist.all_reduce(t, op=op)
+            vals = t.cpu().tolist()
+        out.append(vals)
+    return out[0], out[1]
+
+
+def workload_config(spec, w, args, job_tokens=None):
+    """The line's `config`: rank 0's batch, plus the whole job's when several ranks run
+    (rank r decodes the batch generated with seed r)."""
     lens = w["seq_lens"]
-    return {"workload": spec.name, "B": int(len(lens)), "H": spec.H, "kv_lora_rank": spec.R, "rope_dim": spec.Dr,
-            "D_nope": spec.Dn, "D_v": spec.Dv, "q_len": spec.q_len, "page_size": spec.page_size,
-            "seq_lens": (f"uniform in [{spec.ragged[0]},{spec.ragged[1]}], seed 0" if spec.ragged
-                         else f"{spec.seq_len} each"),
-            "cached_tokens": int(np.sum(lens, dtype=np.int64)),
-            "l2": f"flushed between timed steps ({L2_FLUSH_BYTES >> 20} MiB write); cache also larger than L2",
-            "parallelism": f"replicas x{args.gpus} (independent sequences per GPU)"} | (
-                {"subset": f"first {args.seqs} sequences only (profiling run, not a bench line)"}
-                if getattr(args, "seqs", 0) else {})
+    seed = "seed 0" if args.gpus == 1 else "seed = rank of each replica"
+    cfg = {"workload": spec.name, "B": int(len(lens)), "H": spec.H, "kv_lora_rank": spec.R, "rope_dim": spec.Dr,
+           "D_nope": spec.Dn, "D_v": spec.Dv, "q_len": spec.q_len, "page_size": spec.page_size,
+           "seq_lens": (f"uniform in [{spec.ragged[0]},{spec.ragged[1]}], {seed}" if spec.ragged
+                        else f"{spec.seq_len} each"),
+           "cached_tokens": int(np.sum(lens, dtype=np.int64)),
+           "l2": f"flushed between timed steps ({L2_FLUSH_BYTES >> 20} MiB write); cache also larger than L2",
+           "parallelism": f"replicas x{args.gpus} (independent sequences per GPU)"}
+    if args.gpus > 1:
+        cfg["global_batch"] = int(len(lens)) * args.gpus
+        if job_tokens is not None:
+            cfg["cached_tokens_all_ranks"] = int(job_tokens)
+    if getattr(args, "seqs", 0):
+        cfg["subset"] = f"first {args.seqs} sequences only (profiling run, not a bench line)"
+    return cfg
 
 
 def run_gpu(args):
@@ -296,17 +323,15 @@ def run_gpu(args):
             per_kernel[n] += e[i].elapsed_time(e[i + 1])
         attend_ms.append(e[2].elapsed_time(e[3]))
         step_ms.append(e[0].elapsed_time(e[-1]))
-    total_ms = float(sum(step_ms))
-    total_ms_max = total_ms
-    if world > 1:
-        t = torch.tensor([total_ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms_max = float(t.item())
-
+    # this rank's batch; the job's work is the sum over ranks (each rank decodes its own
+    # ragged batch) and its time the slowest rank's
     cache_bytes = wl.cache_bytes(spec, w["seq_lens"])
     flops = wl.attention_flops(spec, w["seq_lens"])
+    tokens = int(np.sum(w["seq_lens"], dtype=np.int64))
+    (job_bytes, job_flops, job_tokens), (total_ms_max,) = reduce_over_ranks(
+        world, dev, (cache_bytes, flops, tokens), (float(sum(step_ms)),))
     ms_per_step = total_ms_max / args.steps
-    value = world * cache_bytes * args.steps / (total_ms_max / 1e3) / 1e9
+    value = job_bytes * args.steps / (total_ms_max / 1e3) / 1e9
 
     # ---------------------------------------------------------------- roofline of the decode kernel
     peaks, peak_src = load_peaks()
@@ -375,11 +400,8 @@ def run_gpu(args):
         e2e_mode = "one step at a time, L2 flushed before each"
     barrier()
     mla.mla_check_status()
-    if world > 1:
-        t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
-    e2e = {"value": world * cache_bytes * e2e_steps / (e2e_ms / 1e3) / 1e9, "unit": "GB/s",
+    _, (e2e_ms,) = reduce_over_ranks(world, dev, (), (e2e_ms,))
+    e2e = {"value": job_bytes * e2e_steps / (e2e_ms / 1e3) / 1e9, "unit": "GB/s",
            "h2d_bytes_per_step": hostin.h2d_bytes(step), "d2h_bytes_per_step": hostin.d2h_bytes(),
            "ms_per_step": e2e_ms / e2e_steps, "mode": e2e_mode}
 
@@ -396,8 +418,8 @@ def run_gpu(args):
         line = {"metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
                 "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
                 "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-                "config": workload_config(spec, w, argparse.Namespace(gpus=world, seqs=args.seqs)),
-                "tflops": world * flops * args.steps / (total_ms_max / 1e3) / 1e12,
+                "config": workload_config(spec, w, argparse.Namespace(gpus=world, seqs=args.seqs), job_tokens),
+                "tflops": job_flops * args.steps / (total_ms_max / 1e3) / 1e12,
                 "per_kernel_ms": {n: per_kernel[n] / args.steps for n in names},
                 "roofline": roof, "cpu_baseline": cpu, "e2e": e2e,
                 "gpu_launches": step.launches_per_step() * args.steps,
