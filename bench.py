@@ -53,8 +53,8 @@ def load_peaks():
 def decode_kernel_of(H, q_len):
     """(source file, kernel name) of the tensor-core decode kernel used for H heads and
     q_len query tokens per sequence (the library's default policy)."""
-    if H == 128 or (H == 64 and q_len >= 2):
-        return "decode_pair.cuh", "mla_decode_attn (tcgen05 decode_pair_kernel, 2-CTA clusters)"
+    if H in (64, 128):
+        return "decode_2sm.cuh", "mla_decode_attn (tcgen05 cta_group::2 decode_2sm_kernel, SM pairs)"
     return "decode_tc.cuh", "mla_decode_attn (tcgen05 decode_kernel)"
 
 
@@ -186,7 +186,7 @@ def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return 0
-    from mla_latent_kv_46_b200 import workloads as wl
+    from inputs import workloads as wl
     spec = wl.WORKLOADS[args.workload]
     w = wl.make(spec, seed=0)
     per_step_budget = 4.0
@@ -260,7 +260,7 @@ def run_gpu(args):
     __graft_entry__.build()
     import mla_latent_kv_46_b200 as mla
     from mla_latent_kv_46_b200 import decoder as dec
-    from mla_latent_kv_46_b200 import workloads as wl
+    from inputs import workloads as wl
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))

@@ -2,8 +2,8 @@
 
 The compute lives in libmla.so (C ABI: include/mla.h; CUDA sources in csrc/).
 This package is its Python binding (`_binding`, the C names), a step driver
-(`decoder`), the seeded synthetic workloads (`workloads`) and the in-tree build
-(`build`). Importing it fails loudly if libmla.so has not been built: there is
+(`decoder`) and the in-tree build (`build`); the seeded synthetic inputs live in
+the top-level `inputs` package. Importing it fails loudly if libmla.so has not been built: there is
 no CPU or library fallback.
 """
 from ._binding import *  # noqa: F401,F403

@@ -185,6 +185,6 @@ def mla_decode_attn_noalloc(q_lat, q_rope, kv_cache, block_table, seq_lens, B, q
 
 
 def dims_of(spec) -> Dims:
-    """Dims from a workloads.WorkloadSpec."""
+    """Dims from an inputs.workloads.WorkloadSpec."""
     return Dims(spec.H, spec.Dn, spec.Dr, spec.Dv, spec.R, spec.page_size,
                 MLA_BF16 if spec.dtype == "bf16" else MLA_F32)

@@ -1,0 +1,820 @@
+// decode_2sm.cuh -- MLA decode attention on a pair of SMs (tcgen05 cta_group::2).
+//
+// A cluster of two CTAs serves one slot of the split plan. The pair holds 128 query
+// rows: CTA r owns rows 64r..64r+63, i.e. heads 64r.. of one query token for H=128,
+// or the 64 heads of the unit's token r for H=64 (two consecutive query tokens of a
+// sequence per unit; with one token, CTA 1's rows are idle). For every 64-token page
+// of a unit the even CTA issues, for both CTAs at once:
+//   scores  S = Q . KV^T         tcgen05.mma.cta_group::2 M=128 (rows) x N=64 (tokens)
+//                                x K=576; CTA r brings its 64 query rows and the page's
+//                                tokens 32r..32r+31 (all 576 columns), and receives its
+//                                rows' scores for all 64 tokens
+//   values  O^T += C^T . P^T     tcgen05.mma.cta_group::2 M=256 (latent) x N=128 (rows)
+//                                x K=64, twice (latent 0-255, 256-511); CTA r brings the
+//                                page's 64 tokens of its own 128 latent columns of each
+//                                half (128r.. and 256+128r..) and its rows' P, and
+//                                receives O^T for those latent columns and all 128 rows
+// The tensor cores combine the two CTAs' operands. Each CTA holds complete scores for
+// its own rows, so the softmax runs once per row, in the CTA that owns it; the value
+// MMA runs at full rate (128 rows per SM), while the score MMA, with 64 rows per SM,
+// runs at half rate. The price of splitting the work this way is that each CTA also
+// stages its own latent half of the page's other 32 tokens (per page a CTA stages
+// 36 + 32 KiB; the pair reads 72 KiB of HBM, the rest is a second read of lines the
+// peer loads at the same time, served by L2), and that each CTA's O^T holds every row:
+// the rows' rescale factors (per page) and 1 / l (per unit) go to both CTAs.
+//
+// TMEM (512 columns, both CTAs):
+//   [0,256)   O^T: lane L of region lh (columns 128lh..) is latent 256lh + 128r + L, one
+//             column per row of the pair (rows 0-63 the even CTA's, 64-127 the odd's)
+//   [256,320) two score buffers of 32 columns (a pair MMA with M=128 holds row m of the
+//             CTA in lanes m and 64+m): lane half h holds tokens 32h..32h+31
+//   [320,512) the score MMA's A operand for latent columns 0-383 of the query (bf16
+//             pairs, 32 columns per 64 dims), row m in lanes m and 64+m
+// Shared memory: the query's latent columns 384-511 and rope (three 64-row boxes),
+// three score-operand slots (the page's own 32 tokens x 576: nine 32-row boxes), two
+// value-operand slots (64 tokens x own 256 latent: eight 32-row boxes), P as bf16
+// (K-major, 64 rows x 64 tokens) and its remainder P_lo.
+//
+// P enters the value MMA in bf16 (round to nearest). Where one token can carry a
+// large share of a row's weight, one bf16 rounding of P moves the output by more than
+// the bf16 tolerance, so the value MMA is issued a second time with P_lo = bf16(p -
+// bf16(p)) on the pages where some row of the pair has max_t p_t > l / 16 (l the
+// row's running sum so far, of which each thread knows its own half: a conservative
+// test). Elsewhere the single rounding is well inside the tolerance.
+//
+// Online softmax with a lazily moved per-row reference maximum, moved only when a
+// page's maximum exceeds it by more than 2^24 (p and the fp32 sums stay far inside
+// their range below that); a moved reference rescales the row's column of O^T in both
+// CTAs.
+//
+// Warp roles (256 threads per CTA): warp 0 loads the query's shared-memory part and
+// the score operands, warp 2 the value operands, warp 1 allocates TMEM and (even CTA)
+// issues the MMAs, warps 4-7 stage the query's TMEM part, run the softmax and the
+// epilogue (warp w reaches TMEM lanes 32(w%4)..).
+//
+// Barriers that gate an MMA live in the even CTA: both CTAs' TMA loads count their
+// bytes there, and the odd CTA's warps arrive there remotely: arrivals that only
+// report finished TMEM reads are relaxed; P's arrival has CTA-scope release (the data
+// is in the arriving CTA's own shared memory) and the odd CTA's P_lo requests travel
+// as st.async words whose bytes complete on the same barrier. Rescale factors and 1 / l
+// travel the same way to a barrier of the receiving CTA. MMA completion is committed
+// to both CTAs. Every wait is bounded; a CTA that gives up raises the device status
+// word and sets both CTAs' abort flags.
+#pragma once
+
+#include "common.cuh"
+#include "ptx.cuh"
+#include "decode_tc.cuh"
+
+namespace mla {
+namespace duo {
+
+constexpr int kRows = 128;             // MMA rows of the pair
+constexpr int kCtaRows = 64;           // rows per CTA
+constexpr int kPage = 64, kR = 512, kDr = 64, kRow = kR + kDr;
+constexpr int kChunks = kRow / 64;     // 64-column chunks of a row (8 latent + rope)
+constexpr int kQTmemChunks = 6;        // query chunks held in TMEM (latent 0-383)
+constexpr int kQSmemChunks = kChunks - kQTmemChunks;   // latent 384-511 and rope
+constexpr int kBox32 = 32 * 128;       // 32 rows x 64 bf16, 128-byte swizzle
+constexpr int kBox64 = 64 * 128;       // 64 rows x 64 bf16
+constexpr int kQBytes = kQSmemChunks * kBox64;     // 24,576
+constexpr int kQKSlotBytes = kChunks * kBox32;     // 36,864
+constexpr int kPVSlotBytes = 8 * kBox32;           // 32,768
+constexpr int kQKSlots = 3, kPVSlots = 2;
+constexpr int kPBytes = kCtaRows * kPage * 2;      // 8,192
+constexpr int kSoftWarps = 4;
+constexpr int kFirstSoftWarp = 4;
+constexpr int kThreads = 32 * (kFirstSoftWarp + kSoftWarps);
+
+constexpr int kOffQ = 0;
+constexpr int kOffQK = kOffQ + kQBytes;
+constexpr int kOffPV = kOffQK + kQKSlots * kQKSlotBytes;
+constexpr int kOffP = kOffPV + kPVSlots * kPVSlotBytes;   // P_hi, then P_lo
+constexpr int kOffBar = kOffP + 2 * kPBytes;              // 32 mbarriers
+constexpr int kOffXmax = kOffBar + 32 * 8;                // float[2][128]: row maxima of the lane halves
+constexpr int kOffXl = kOffXmax + 2 * 128 * 4;            // float[128]: row sums of the lane halves
+constexpr int kOffFlag = kOffXl + 128 * 4;                // uint32[4][8] (even CTA): P_lo wanted, per tile % 4
+                                                          // and softmax warp (0-3 even CTA, 4-7 odd CTA)
+constexpr int kOffXal = kOffFlag + 4 * 8 * 4;             // float[2][128]: the pair's rescale factors, per row
+constexpr int kOffXflg = kOffXal + 2 * 128 * 4;           // uint32[2][4]: a moved reference among 32 rows
+constexpr int kOffXinv = kOffXflg + 2 * 4 * 4;            // float[128]: the pair's 1 / l, per row
+constexpr int kOffTmem = kOffXinv + 128 * 4;
+constexpr int kOffAbort = kOffTmem + 8;
+constexpr int kSmemUsed = kOffAbort + 8;
+constexpr int kSmemBytes = kSmemUsed + 1024;
+static_assert(kSmemBytes <= 232448, "shared memory of one CTA");
+
+enum {
+  B_QK_FULL = 0,                   // +slot (even CTA): score operands of both CTAs landed
+  B_QK_EMPTY = B_QK_FULL + 3,      // +slot: score MMAs that read the slot done
+  B_PV_FULL = B_QK_EMPTY + 3,      // +slot (even CTA): value operands landed
+  B_PV_EMPTY = B_PV_FULL + 2,      // +slot: value MMAs that read the slot done
+  B_Q_FULL = B_PV_EMPTY + 2,       // (even CTA) the unit's query in both CTAs: TMA bytes of the
+                                   // shared-memory part, one arrival per softmax warp for TMEM
+  B_Q_EMPTY,                       // last score MMA of a unit done
+  B_S_FULL,                        // +buffer: score MMAs done
+  B_S_EMPTY = B_S_FULL + 2,        // +buffer (even CTA): both CTAs' softmax warps read S
+  B_P_FULL = B_S_EMPTY + 2,        // (even CTA) P of both CTAs in shared memory, O rescaled
+  B_O_DONE,                        // value MMAs of a page done
+  B_O_FREE,                        // (even CTA) both CTAs' epilogues have read O
+  B_PAIR,                          // +1: the two softmax warps of rows 0-31 / 32-63
+  B_AL_FULL = B_PAIR + 2,          // +buffer: both CTAs' rescale factors of a page (local arrivals,
+                                   // the peer's words as transaction bytes)
+  B_LX_FULL = B_AL_FULL + 2,       // both CTAs' 1 / l of a unit (likewise)
+  B_DRAIN,
+  kNumBars
+};
+static_assert(kNumBars <= 32, "barrier area");
+static_assert(kQKSlots <= 3 && kPVSlots <= 2, "barrier slots");
+
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kColO = 0, kColS = 256, kColQ = 320;
+static_assert(kColQ + 32 * kQTmemChunks <= kTmemCols, "TMEM columns");
+constexpr uint32_t kIdescS = ptx::idesc_bf16_f32(128, 64, 0, 0);    // Q (K-major) x KV^T (K-major)
+constexpr uint32_t kIdescV = ptx::idesc_bf16_f32(256, 128, 1, 0);   // C^T (M-major) x P^T (K-major)
+// log2 units: p stays below 2^24, far inside the range of the bf16 P and of the fp32
+// sums (at most 2^24 x 2^17 tokens x |c|), so the reference moves (and O is rescaled)
+// only when a row's maximum jumps by that much, which almost never happens
+constexpr float kRescaleThreshold = 24.0f;
+constexpr uint32_t kAlBytes = 64 * 4 + 2 * 4;   // one CTA's rescale factors and votes
+constexpr float kLoShare = 16.0f;           // P_lo wanted when 16 * max p > l
+
+using tc::Params;
+
+// A plan unit: the rows of n (1 or 2) consecutive query tokens of sequence b over
+// pages [pb, pb + npg).
+struct Unit2 {
+  int32_t item, b, pb, npg, n;
+  int32_t ntok[2];   // tokens each token sees (-1: absent)
+  int32_t part[2];   // partial-output index of each token, or -1: final result
+};
+
+__device__ __forceinline__ Unit2 load_unit2(const Params& p, const PlanView& plan, int32_t idx) {
+  const Unit u = plan.units()[idx];
+  Unit2 r;
+  r.item = u.item;
+  r.b = u.b;
+  r.pb = u.page_begin;
+  r.n = u.pad1 > 1 ? 2 : 1;
+  const int32_t q_len = plan.q_len(), L = p.seq_lens[u.b];
+  r.ntok[0] = visible_tokens(L, q_len, u.item % q_len);
+  r.ntok[1] = r.n > 1 ? visible_tokens(L, q_len, u.item % q_len + 1) : -1;
+  r.part[0] = u.part;
+  r.part[1] = r.n > 1 ? u.pad0 : -1;
+  const int32_t last = (max(r.ntok[0], r.ntok[1]) + kPage - 1) / kPage;
+  const int32_t pe = min(u.page_end, min(last, p.max_pages));
+  r.npg = max(0, pe - r.pb);
+  return r;
+}
+
+// Optional event trace (-DMLA_TRACE): per CTA 1024 clock64 values, 16 regions of 64
+// tiles: 0 score operand load issued, 1 value operand load issued, 2 score operand
+// landed (MMA warp), 3 score MMA issued, 4 P of both CTAs ready (MMA warp), 5 value
+// MMA issued, 6 scores read (softmax warp 4), 7 P stored (softmax warp 4), 8 value
+// operand landed (MMA warp), 9 query staged in TMEM (softmax warp 4, per unit); slot
+// 1020 the SM id, 1021 the global timer at start, 1022 clock at exit, 1023 at start.
+#ifdef MLA_TRACE
+#define DUO_TRACE(region, g)                                                                     \
+  do {                                                                                           \
+    if (p.trace && (g) < 60)                                                                     \
+      p.trace[(size_t)blockIdx.x * 1024 + 64 * (region) + (g)] = (unsigned long long)clock64(); \
+  } while (0)
+#else
+#define DUO_TRACE(region, g) \
+  do {                       \
+  } while (0)
+#endif
+
+// Walks the pages of a slot's non-empty units in order.
+struct Cursor {
+  int32_t ui, k;
+  uint32_t n;   // ordinal of the unit among the slot's non-empty units
+  bool valid;
+  Unit2 u;
+};
+
+__device__ __forceinline__ bool next_unit(const Params& p, const PlanView& plan, int32_t& ui, int32_t u_end,
+                                          Unit2& u) {
+  while (++ui < u_end) {
+    u = load_unit2(p, plan, ui);
+    if (u.npg > 0) return true;
+  }
+  return false;
+}
+
+__device__ __forceinline__ Cursor first_page(const Params& p, const PlanView& plan, int32_t u_begin,
+                                             int32_t u_end) {
+  Cursor c;
+  c.ui = u_begin - 1;
+  c.k = 0;
+  c.n = 0;
+  c.valid = next_unit(p, plan, c.ui, u_end, c.u);
+  return c;
+}
+
+__device__ __forceinline__ void advance(const Params& p, const PlanView& plan, int32_t u_end, Cursor& c) {
+  if (!c.valid) return;
+  if (++c.k < c.u.npg) return;
+  c.k = 0;
+  ++c.n;
+  c.valid = next_unit(p, plan, c.ui, u_end, c.u);
+}
+
+__device__ __forceinline__ int32_t page_id(const Params& p, const Unit2& u, int32_t k, bool report) {
+  int32_t page = p.block_table[(int64_t)u.b * p.max_pages + u.pb + k];
+  if (page < 0 || page >= p.num_pages) {
+    if (report) raise_status(kStatusBadPage);
+    page = p.num_pages;   // rows past the tensor: the loads fill zeros
+  }
+  return page;
+}
+
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
+decode_2sm_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_constant__ CUtensorMap tm_q,
+                  const __grid_constant__ CUtensorMap tm_qr, const Params p) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sbase = ptx::smem_u32(smem);
+  const uint32_t rank = ptx::cluster_rank();
+  const bool even = rank == 0;
+  auto bar = [&](int i) { return sbase + kOffBar + 8u * i; };
+  auto lead = [&](uint32_t local) { return ptx::map_peer(local, 0); };   // the even CTA's copy
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kOffAbort);
+  volatile uint32_t* lo_flag = reinterpret_cast<volatile uint32_t*>(smem + kOffFlag);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const PlanView plan{p.plan};
+  const int slot = blockIdx.x >> 1;
+  const int32_t u_begin = plan.slot_begin()[slot], u_end = plan.slot_begin()[slot + 1];
+  const int32_t H = p.H;   // 128, or 64 with up to two query tokens per unit
+  const int64_t TH = (int64_t)plan.B() * plan.q_len() * H;   // query rows
+
+  if (threadIdx.x == 0) {
+    *abort_flag = 0;
+    for (int i = 0; i < 32; ++i) lo_flag[i] = 0u;
+    for (int s = 0; s < kQKSlots; ++s) {
+      ptx::mbar_init(bar(B_QK_FULL + s), 1);
+      ptx::mbar_init(bar(B_QK_EMPTY + s), 1);
+    }
+    for (int s = 0; s < kPVSlots; ++s) {
+      ptx::mbar_init(bar(B_PV_FULL + s), 1);
+      ptx::mbar_init(bar(B_PV_EMPTY + s), 1);
+    }
+    for (int s = 0; s < 2; ++s) {
+      ptx::mbar_init(bar(B_S_FULL + s), 1);
+      ptx::mbar_init(bar(B_S_EMPTY + s), 2 * kSoftWarps);
+    }
+    ptx::mbar_init(bar(B_Q_FULL), 1 + 2 * kSoftWarps);
+    ptx::mbar_init(bar(B_Q_EMPTY), 1);
+    ptx::mbar_init(bar(B_P_FULL), 2 * kSoftWarps);
+    ptx::mbar_init(bar(B_O_DONE), 1);
+    ptx::mbar_init(bar(B_O_FREE), 2 * kSoftWarps);
+    ptx::mbar_init(bar(B_PAIR), 2);
+    ptx::mbar_init(bar(B_PAIR + 1), 2);
+    ptx::mbar_init(bar(B_AL_FULL), 2);
+    ptx::mbar_init(bar(B_AL_FULL + 1), 2);
+    ptx::mbar_init(bar(B_LX_FULL), 2);
+    ptx::mbar_init(bar(B_DRAIN), 1);
+    ptx::fence_mbar_init();
+  }
+  if (warp == 1) {
+    ptx::tmem_alloc_pair(sbase + kOffTmem, kTmemCols);
+    ptx::tmem_relinquish_pair();
+  }
+  if (warp == 0 && lane == 0) {
+    ptx::prefetch_tmap(&tm_kv);
+    ptx::prefetch_tmap(&tm_q);
+    ptx::prefetch_tmap(&tm_qr);
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::cluster_sync();   // both CTAs' barriers exist before anyone arrives, loads or issues
+  ptx::tc_fence_after();
+  const uint32_t tbase = *reinterpret_cast<volatile uint32_t*>(smem + kOffTmem);
+#ifdef MLA_TRACE
+  if (threadIdx.x == 0 && p.trace) {
+    uint32_t smid;
+    asm volatile("mov.u32 %0, %%smid;" : "=r"(smid));
+    unsigned long long* tr = p.trace + (size_t)blockIdx.x * 1024;
+    tr[1020] = smid;
+    tr[1021] = ptx::globaltimer_ns();
+    tr[1023] = (unsigned long long)clock64();
+  }
+#endif
+
+  auto fail = [&]() {
+    raise_status(kStatusTimeout);
+    *abort_flag = 1;
+    ptx::st_cluster_u32(ptx::map_peer(sbase + kOffAbort, rank ^ 1u), 1u);
+  };
+  auto wait_all = [&](uint32_t b, uint32_t parity) -> bool {
+    return __all_sync(0xffffffffu, ptx::mbar_wait_cluster_bounded(b, parity, abort_flag, p.timeout_ns));
+  };
+
+  if (warp == 0 || warp == 2) {
+    // ================================================================ TMA producers
+    // warp 0: the query's shared-memory part per unit and each page's score operand (own
+    // 32 tokens x 576); warp 2: each page's value operand (64 tokens x own 256 latent)
+    const bool leader = ptx::elect_one();
+    const bool qk = warp == 0;
+    const int nslots = qk ? kQKSlots : kPVSlots;
+    Cursor c = first_page(p, plan, u_begin, u_end);
+    // L2 prefetch cursor (even CTA, warp 0): whole pages a few pages ahead, and the next
+    // units' query rows when the cursor enters them
+    Cursor pf = c;
+    auto prefetch_one = [&]() {
+      if (!pf.valid) return;
+      if (even && leader) {
+        if (pf.k == 0) {
+          const int64_t qrow = (int64_t)pf.u.item * H;
+          const int64_t rows = min((int64_t)kRows, TH - qrow);
+          if (rows > 0) {
+            ptx::prefetch_l2_bulk(p.q_lat + qrow * kR, (uint32_t)(rows * kR * 2));
+            ptx::prefetch_l2_bulk(p.q_rope + qrow * kDr, (uint32_t)(rows * kDr * 2));
+          }
+        }
+        const int32_t page = page_id(p, pf.u, pf.k, false);
+        if (page < p.num_pages) ptx::prefetch_l2_bulk(p.kv + (int64_t)page * kPage * kRow, kPage * kRow * 2);
+      }
+      advance(p, plan, u_end, pf);
+    };
+    if (qk)
+      for (int i = 0; i < 6; ++i) prefetch_one();
+    uint32_t g = 0, nq = 0;
+    bool ok = true;
+    while (c.valid && ok) {
+      if (qk && c.k == 0) {
+        if (!wait_all(bar(B_Q_EMPTY), (nq & 1) ^ 1)) { if (leader) fail(); ok = false; break; }
+        if (leader) {
+          if (even) ptx::mbar_arrive_expect_tx(bar(B_Q_FULL), 2 * kQBytes);
+          const int32_t qrow = c.u.item * H + kCtaRows * (int32_t)rank;   // rows past the tensor read zeros
+#pragma unroll 1
+          for (int ch = 0; ch < kQSmemChunks - 1; ++ch)
+            ptx::tma_load_2d_pair(sbase + kOffQ + ch * kBox64, &tm_q, lead(bar(B_Q_FULL)),
+                                  64 * (kQTmemChunks + ch), qrow);
+          ptx::tma_load_2d_pair(sbase + kOffQ + (kQSmemChunks - 1) * kBox64, &tm_qr, lead(bar(B_Q_FULL)), 0,
+                                qrow);
+        }
+        ++nq;
+      }
+      const uint32_t s = g % nslots, ph = (g / nslots) & 1;
+      if (!wait_all(bar((qk ? B_QK_EMPTY : B_PV_EMPTY) + s), ph ^ 1)) { if (leader) fail(); ok = false; break; }
+      const int32_t page = page_id(p, c.u, c.k, leader && qk);
+      // (the testing hook leaves the page's barrier without the even CTA's load: the waits
+      // on it run out and the kernel reports a timeout)
+      const bool drop = qk && blockIdx.x == 0 && (int32_t)g == p.drop_load;
+      if (leader) {
+        if (qk) {
+          DUO_TRACE(0, g);
+          if (even) ptx::mbar_arrive_expect_tx(bar(B_QK_FULL + s), 2 * kQKSlotBytes);
+          if (!drop) {
+            const uint32_t dst = sbase + kOffQK + s * kQKSlotBytes;
+#pragma unroll 1
+            for (int ch = 0; ch < kChunks; ++ch)
+              ptx::tma_load_2d_pair(dst + ch * kBox32, &tm_kv, lead(bar(B_QK_FULL + s)), 64 * ch,
+                                    page * kPage + 32 * (int32_t)rank);
+          }
+        } else {
+          DUO_TRACE(1, g);
+          if (even) ptx::mbar_arrive_expect_tx(bar(B_PV_FULL + s), 2 * kPVSlotBytes);
+          const uint32_t dst = sbase + kOffPV + s * kPVSlotBytes;
+          // box (hh, th, b) at ((hh * 2 + th) * 2 + b): latent block 4hh + 2r + b, tokens 32th..
+#pragma unroll 1
+          for (int i = 0; i < 8; ++i) {
+            const int hh = i >> 2, th = (i >> 1) & 1, b = i & 1;
+            ptx::tma_load_2d_pair(dst + i * kBox32, &tm_kv, lead(bar(B_PV_FULL + s)),
+                                  64 * (4 * hh + 2 * (int)rank + b), page * kPage + 32 * th);
+          }
+        }
+      }
+      if (qk) prefetch_one();
+      advance(p, plan, u_end, c);
+      ++g;
+    }
+    // The even CTA's barriers count both CTAs' loads: before the pair exits, wait (bounded)
+    // for the phases armed last, so no copy is still landing in either CTA.
+    if (even) {
+      for (uint32_t k = (g >= (uint32_t)nslots ? g - nslots : 0); k < g; ++k)
+        wait_all(bar((qk ? B_QK_FULL : B_PV_FULL) + k % nslots), (k / nslots) & 1);
+      if (qk && nq > 0) wait_all(bar(B_Q_FULL), (nq - 1) & 1);
+    }
+  } else if (warp == 1) {
+    // ================================================================ MMA issuer (even CTA)
+    if (even) {
+      const bool leader = ptx::elect_one();
+      bool ok = true;
+      Cursor qc = first_page(p, plan, u_begin, u_end);   // next score MMA
+      Cursor vc = qc;                                     // next value MMA
+      uint32_t gq = 0, gv = 0;
+      auto issue_s = [&]() -> bool {
+        if (qc.k == 0 && !wait_all(bar(B_Q_FULL), qc.n & 1)) return false;
+        const uint32_t s = gq % kQKSlots, ph = (gq / kQKSlots) & 1, sb = gq & 1;
+        if (!wait_all(bar(B_QK_FULL + s), ph)) return false;
+        if (leader) DUO_TRACE(2, gq);
+        if (!wait_all(bar(B_S_EMPTY + sb), ((gq >> 1) & 1) ^ 1)) return false;
+        ptx::tc_fence_after();
+        const uint32_t kvs = sbase + kOffQK + s * kQKSlotBytes;
+        const uint32_t d_s = tbase + kColS + 32u * sb;
+        if (leader) {
+          DUO_TRACE(3, gq);
+#pragma unroll 1
+          for (int ch = 0; ch < kChunks; ++ch) {
+            const uint64_t dk = ptx::sdesc_sw128(kvs + ch * kBox32, 16, 1024);
+            if (ch < kQTmemChunks) {
+#pragma unroll
+              for (int kk = 0; kk < 4; ++kk)
+                ptx::umma_pair_ts(d_s, tbase + kColQ + 32u * ch + 8u * kk, dk + (uint64_t)(2 * kk), kIdescS,
+                                  (ch | kk) ? 1u : 0u);
+            } else {
+              const uint64_t dq = ptx::sdesc_sw128(sbase + kOffQ + (ch - kQTmemChunks) * kBox64, 16, 1024);
+#pragma unroll
+              for (int kk = 0; kk < 4; ++kk)
+                ptx::umma_pair_ss(d_s, dq + (uint64_t)(2 * kk), dk + (uint64_t)(2 * kk), kIdescS, 1u);
+            }
+          }
+          ptx::umma_commit_pair(bar(B_QK_EMPTY + s), 3);
+          ptx::umma_commit_pair(bar(B_S_FULL + sb), 3);
+          if (qc.k == qc.u.npg - 1) ptx::umma_commit_pair(bar(B_Q_EMPTY), 3);
+        }
+        __syncwarp();
+        advance(p, plan, u_end, qc);
+        ++gq;
+        return true;
+      };
+      auto issue_v = [&]() -> bool {
+        if (!wait_all(bar(B_P_FULL), gv & 1)) return false;
+        if (leader) DUO_TRACE(4, gv);
+        if (vc.k == 0 && vc.n > 0 && !wait_all(bar(B_O_FREE), (vc.n - 1) & 1)) return false;
+        const uint32_t s = gv % kPVSlots, ph = (gv / kPVSlots) & 1;
+        if (!wait_all(bar(B_PV_FULL + s), ph)) return false;
+        if (leader) DUO_TRACE(8, gv);
+        uint32_t want_lo = 0;
+#pragma unroll
+        for (int w = 0; w < 2 * kSoftWarps; ++w) want_lo |= lo_flag[8 * (gv & 3) + w];
+        ptx::tc_fence_after();
+        const uint32_t pvs = sbase + kOffPV + s * kPVSlotBytes;
+        if (leader) {
+          DUO_TRACE(5, gv);
+#pragma unroll 1
+          for (int part = 0; part < (want_lo ? 2 : 1); ++part) {
+            const uint64_t dp = ptx::sdesc_sw128(sbase + kOffP + part * kPBytes, 16, 1024);
+#pragma unroll
+            for (int lh = 0; lh < 2; ++lh) {
+#pragma unroll
+              for (int kk = 0; kk < 4; ++kk) {
+                // O^T[latent][row] += C^T[latent][t] P^T[t][row], tokens 16kk..16kk+15: box
+                // pair (lh, kk / 2) at rows 16 (kk % 2) holds this CTA's 128 latent rows
+                const uint64_t dc =
+                    ptx::sdesc_sw128(pvs + ((lh * 2 + (kk >> 1)) * 2) * kBox32 + (kk & 1) * 2048, kBox32, 1024);
+                ptx::umma_pair_ss(tbase + kColO + 128u * lh, dc, dp + (uint64_t)(2 * kk), kIdescV,
+                                  (part == 0 && vc.k == 0 && kk == 0) ? 0u : 1u);
+              }
+            }
+          }
+          ptx::umma_commit_pair(bar(B_PV_EMPTY + s), 3);
+          ptx::umma_commit_pair(bar(B_O_DONE), 3);
+        }
+        __syncwarp();
+        advance(p, plan, u_end, vc);
+        ++gv;
+        return true;
+      };
+      // S(0), then per page j: S(j+1), V(j)
+      if (qc.valid && !issue_s()) { if (leader) fail(); ok = false; }
+      while (vc.valid && ok) {
+        if (qc.valid && !issue_s()) { if (leader) fail(); ok = false; break; }
+        if (!issue_v()) { if (leader) fail(); ok = false; break; }
+      }
+      if (leader) ptx::umma_commit_pair(bar(B_DRAIN), 1);
+      __syncwarp();
+      wait_all(bar(B_DRAIN), 0);
+    }
+  } else if (warp >= kFirstSoftWarp) {
+    // ================================================================ query staging, softmax, epilogue
+    const int sw = warp - kFirstSoftWarp;         // softmax warp 0-3
+    const int q = warp & 3;                       // TMEM lane quarter
+    const int L = 32 * q + lane;                  // this thread's TMEM lane
+    // scores: row m of the CTA, tokens 32h..32h+31 of the page (h = lane half); O^T: latent
+    // row 256lh + 128 rank + L of region lh, one column per row of the pair
+    const int m = L & 63, half = L >> 6;
+    const int prow = kCtaRows * (int)rank + m;    // this thread's score row among the pair's 128
+    const uint32_t lane_addr = (32u * q) << 16;
+    const int tok = H == kRows ? 0 : (int)rank;   // the unit's query token this CTA's rows belong to
+    volatile float* xmax = reinterpret_cast<volatile float*>(smem + kOffXmax);
+    volatile float* xl = reinterpret_cast<volatile float*>(smem + kOffXl);
+    volatile float* xal = reinterpret_cast<volatile float*>(smem + kOffXal);
+    volatile uint32_t* xflg = reinterpret_cast<volatile uint32_t*>(smem + kOffXflg);
+    volatile float* xinv = reinterpret_cast<volatile float*>(smem + kOffXinv);
+    auto peer = [&](uint32_t local) { return ptx::map_peer(local, rank ^ 1u); };
+    uint32_t n_pair = 0, n_lx = 0;
+    bool ok = true;
+    // the two warps of rows 32(q&1).. (lane halves 0 and 1) meet on B_PAIR + (q & 1)
+    auto pair_sync = [&]() -> bool {
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive(bar(B_PAIR + (q & 1)));
+      const bool done = ptx::mbar_wait_bounded(bar(B_PAIR + (q & 1)), n_pair & 1, abort_flag, p.timeout_ns);
+      ++n_pair;
+      return __all_sync(0xffffffffu, done);
+    };
+    // arrivals on the even CTA's barriers that only report finished TMEM reads
+    auto arrive_read = [&](int b) {
+      if (even) ptx::mbar_arrive(bar(b));
+      else ptx::mbar_arrive_cluster_relaxed(lead(bar(b)));
+    };
+    // query row of the pair's row n (H=64: rows 64.. are the unit's second token)
+    auto qrow_of = [&](int32_t item, int n) -> int64_t { return (int64_t)item * H + n; };
+
+    // Units without a visible token: o = 0, lse = -inf for this CTA's latent half of the
+    // pair's rows (this thread: latent rows 128 rank + L and 256 + 128 rank + L).
+    for (int32_t ui = u_begin; ui < u_end; ++ui) {
+      const Unit2 u = load_unit2(p, plan, ui);
+      if (u.npg > 0) continue;
+      for (int n = 0; n < kRows; ++n) {
+        const int tn = H == kRows ? 0 : n / kCtaRows;
+        if (tn >= u.n) continue;
+        const int64_t row = qrow_of(u.item, n);
+        const int32_t prt = u.part[tn];
+        for (int lh = 0; lh < 2; ++lh) {
+          const int d = 256 * lh + 128 * (int)rank + L;
+          if (prt < 0) p.o_lat[row * kR + d] = __float2bfloat16_rn(0.f);
+          else p.o_part[((int64_t)prt * H + row % H) * kR + d] = 0.f;
+        }
+      }
+      if (half == 0 && tok < u.n) {
+        const int64_t row = qrow_of(u.item, prow);
+        const int32_t prt = u.part[tok];
+        if (prt < 0) { if (p.lse) p.lse[row] = -CUDART_INF_F; }
+        else p.lse_part[(int64_t)prt * H + row % H] = -CUDART_INF_F;
+      }
+    }
+
+    // The TMEM part of a unit's query (latent 0-383 of this thread's score row, both lane
+    // halves hold it), once the previous unit's last score MMA is done.
+    auto stage_q = [&](const Unit2& u, uint32_t n) -> bool {
+      if (!wait_all(bar(B_Q_EMPTY), (n & 1) ^ 1)) return false;
+      ptx::tc_fence_after();
+      const int64_t row = qrow_of(u.item, prow);
+      const bool inside = row < TH;   // rows past the query tensor (an absent token) stay zero
+      const __nv_bfloat16* src = p.q_lat + row * kR;
+#pragma unroll 1
+      for (int ch = 0; ch < kQTmemChunks; ++ch) {
+        uint32_t w[32];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          uint32_t* d = &w[8 * i];
+          if (inside) {
+            asm volatile("ld.global.nc.v8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+                         : "=r"(d[0]), "=r"(d[1]), "=r"(d[2]), "=r"(d[3]), "=r"(d[4]), "=r"(d[5]), "=r"(d[6]),
+                           "=r"(d[7])
+                         : "l"(src + 64 * ch + 16 * i));
+          } else {
+#pragma unroll
+            for (int k = 0; k < 8; ++k) d[k] = 0u;
+          }
+        }
+        ptx::tmem_st_32x32b_x32(tbase + lane_addr + kColQ + 32u * ch, w);
+      }
+      ptx::tmem_wait_st();
+      ptx::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) {
+        if (even) ptx::mbar_arrive(bar(B_Q_FULL));
+        else ptx::mbar_arrive_cluster(lead(bar(B_Q_FULL)));
+      }
+      if (sw == 0 && lane == 0) DUO_TRACE(9, n);
+      return true;
+    };
+
+    struct Pending {
+      bool on;
+      int32_t item, n, part0, part1;
+      float l, m;
+    } pend{false, 0, 0, -1, -1, 0.f, 0.f};
+    // O^T[:, row] / l_row to the output, once the unit's last value MMAs are done: the row's
+    // owner CTA adds its two threads' sums and publishes 1 / l to both CTAs; every thread
+    // then writes its two latent rows for all of the pair's rows.
+    auto epilogue = [&](uint32_t g_last) -> bool {
+      if (!wait_all(bar(B_O_DONE), g_last & 1)) return false;
+      ptx::tc_fence_after();
+      xl[L] = pend.l;
+      if (!pair_sync()) return false;
+      if (half == 0) {
+        const float l = pend.l + xl[L ^ 64];   // half 0 + half 1
+        const float inv_l = l > 0.f ? 1.f / l : 0.f;
+        xinv[prow] = inv_l;
+        const uint32_t xa = sbase + kOffXinv + 4u * prow;
+        ptx::st_async_u32(peer(xa), __float_as_uint(inv_l), peer(bar(B_LX_FULL)));
+        if (tok < pend.n) {
+          const int64_t row = qrow_of(pend.item, prow);
+          const int32_t prt = tok ? pend.part1 : pend.part0;
+          const float z = l > 0.f ? (pend.m + log2f(l)) * 0.69314718055994531f : -CUDART_INF_F;
+          if (prt < 0) { if (p.lse) p.lse[row] = z; }
+          else p.lse_part[(int64_t)prt * H + row % H] = z;
+        }
+        __syncwarp();
+        if (lane == 0) {
+          if (sw == 0) ptx::mbar_arrive_expect_tx(bar(B_LX_FULL), 4u * kCtaRows);   // the peer's words
+          else ptx::mbar_arrive(bar(B_LX_FULL));
+        }
+      }
+      const bool got = ptx::mbar_wait_cluster_bounded(bar(B_LX_FULL), n_lx & 1, abort_flag, p.timeout_ns);
+      ++n_lx;
+      if (!__all_sync(0xffffffffu, got)) return false;
+#pragma unroll 1
+      for (int c = 0; c < 8; ++c) {
+        uint32_t o[32];
+        ptx::tmem_ld_32x32b_x32(tbase + lane_addr + kColO + 32u * c, o);
+        ptx::tmem_wait_ld();
+        const int lh = c >> 2, n0 = 32 * (c & 3);
+        const int d = 256 * lh + 128 * (int)rank + L;   // this thread's latent row
+        const int tn = H == kRows ? 0 : n0 / kCtaRows;  // the 32 rows' query token
+        if (tn >= pend.n) continue;
+        const int32_t prt = tn ? pend.part1 : pend.part0;
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+          const int64_t row = qrow_of(pend.item, n0 + j);
+          const float v = __uint_as_float(o[j]) * xinv[n0 + j];
+          if (prt < 0) p.o_lat[row * kR + d] = __float2bfloat16_rn(v);
+          else p.o_part[((int64_t)prt * H + row % H) * kR + d] = v;
+        }
+      }
+      ptx::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) arrive_read(B_O_FREE);
+      pend.on = false;
+      return true;
+    };
+
+    Cursor cur = first_page(p, plan, u_begin, u_end);
+    if (cur.valid && !stage_q(cur.u, 0)) { fail(); ok = false; }
+    uint32_t g = 0;
+    float m_ref = -CUDART_INF_F, l_part = 0.f;
+    while (cur.valid && ok) {
+      const Unit2& u = cur.u;
+      if (cur.k == 0) {
+        if (pend.on && !epilogue(g - 1)) { fail(); ok = false; break; }
+        m_ref = -CUDART_INF_F;
+        l_part = 0.f;
+      }
+      const int32_t ntok = tok < u.n ? max(u.ntok[tok], 0) : 0;
+      // ------------------------------------------------ this thread's 32 scores
+      const uint32_t sb = g & 1;
+      if (!wait_all(bar(B_S_FULL + sb), (g >> 1) & 1)) { fail(); ok = false; break; }
+      ptx::tc_fence_after();
+      if (sw == 0 && lane == 0) DUO_TRACE(6, g);
+      float v[32];
+      {
+        uint32_t r[32];
+        ptx::tmem_ld_32x32b_x32(tbase + lane_addr + kColS + 32u * sb, r);
+        ptx::tmem_wait_ld();
+#pragma unroll
+        for (int t = 0; t < 32; ++t) v[t] = __uint_as_float(r[t]);
+      }
+      ptx::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) arrive_read(B_S_EMPTY + sb);
+      // the unit's last score MMA is done: stage the next unit's query
+      if (cur.k == u.npg - 1) {
+        int32_t ui = cur.ui;
+        Unit2 nu;
+        if (next_unit(p, plan, ui, u_end, nu) && !stage_q(nu, cur.n + 1)) { fail(); ok = false; break; }
+      }
+      const int32_t tok0 = (u.pb + cur.k) * kPage + 32 * half;
+      if (tok0 + 32 > ntok) {
+#pragma unroll
+        for (int t = 0; t < 32; ++t) v[t] = (tok0 + t < ntok) ? v[t] : -CUDART_INF_F;
+      }
+      float mx;
+      {
+        float a[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+          a[i] = fmaxf(fmaxf(fmaxf(v[8 * i], v[8 * i + 1]), fmaxf(v[8 * i + 2], v[8 * i + 3])),
+                       fmaxf(fmaxf(v[8 * i + 4], v[8 * i + 5]), fmaxf(v[8 * i + 6], v[8 * i + 7])));
+        mx = fmaxf(fmaxf(a[0], a[1]), fmaxf(a[2], a[3]));
+      }
+      // ------------------------------------------------ the row's maximum over both lane halves
+      xmax[128 * (g & 1) + L] = mx;
+      if (!pair_sync()) { fail(); ok = false; break; }
+      const float mrow = fmaxf(mx, xmax[128 * (g & 1) + (L ^ 64)]) * p.scale_log2;
+      const bool need = mrow > m_ref + kRescaleThreshold;
+      const float mu = need ? mrow : m_ref;
+      const float al = need ? ptx::ex2(m_ref - mu) : 1.f;
+      const float nz = (mu == -CUDART_INF_F) ? 0.f : -mu;
+      // ------------------------------------------------ the rows' rescale factors to both CTAs
+      // (each CTA's O^T holds every row of the pair); one thread per row sends its factor
+      const uint32_t ab = g & 1;
+      if (half == 0) {
+        const uint32_t xa = sbase + kOffXal + 4u * (128 * ab + prow);
+        xal[128 * ab + prow] = al;
+        ptx::st_async_u32(peer(xa), __float_as_uint(al), peer(bar(B_AL_FULL + ab)));
+        const uint32_t moved = __any_sync(0xffffffffu, need && cur.k > 0) ? 1u : 0u;
+        if (lane == 0) {
+          const uint32_t fi = 4 * ab + 2 * rank + (q & 1);
+          xflg[fi] = moved;
+          ptx::st_async_u32(peer(sbase + kOffXflg + 4u * fi), moved, peer(bar(B_AL_FULL + ab)));
+        }
+        __syncwarp();
+        if (lane == 0) {
+          if (sw == 0) ptx::mbar_arrive_expect_tx(bar(B_AL_FULL + ab), kAlBytes);   // the peer's words
+          else ptx::mbar_arrive(bar(B_AL_FULL + ab));
+        }
+      }
+      // ------------------------------------------------ p = 2^(x - m), its bf16 rounding and remainder
+      uint32_t ph[16], pl[16];
+      float sum4[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        const float a0 = ptx::ex2(fmaf(v[2 * i], p.scale_log2, nz));
+        const float a1 = ptx::ex2(fmaf(v[2 * i + 1], p.scale_log2, nz));
+        sum4[i & 3] += a0 + a1;
+        __nv_bfloat162 h2 = __floats2bfloat162_rn(a0, a1);
+        ph[i] = *reinterpret_cast<uint32_t*>(&h2);
+        const float r0 = a0 - __uint_as_float(ph[i] << 16), r1 = a1 - __uint_as_float(ph[i] & 0xFFFF0000u);
+        __nv_bfloat162 l2 = __floats2bfloat162_rn(r0, r1);
+        pl[i] = *reinterpret_cast<uint32_t*>(&l2);
+      }
+      l_part = l_part * al + ((sum4[0] + sum4[1]) + (sum4[2] + sum4[3]));
+      m_ref = mu;
+      const float pmax = ptx::ex2(fmaf(mx, p.scale_log2, nz));
+      const bool want_lo = pmax * kLoShare > l_part;
+      // ------------------------------------------------ P to shared memory once the previous value MMAs are done
+      if (g > 0 && cur.k != 0 && !wait_all(bar(B_O_DONE), (g - 1) & 1)) { fail(); ok = false; break; }
+      if (!wait_all(bar(B_AL_FULL + ab), (g >> 1) & 1)) { fail(); ok = false; break; }
+      ptx::tc_fence_after();
+      if (xflg[4 * ab] | xflg[4 * ab + 1] | xflg[4 * ab + 2] | xflg[4 * ab + 3]) {
+        // a moved reference: O^T[:, row] *= 2^(m_old - m_new) for every row of the pair (1 for
+        // rows that kept theirs); this thread scales its two latent rows
+#pragma unroll 1
+        for (int c = 0; c < 8; ++c) {
+          uint32_t o[32];
+          const uint32_t ta = tbase + lane_addr + kColO + 32u * c;
+          ptx::tmem_ld_32x32b_x32(ta, o);
+          ptx::tmem_wait_ld();
+#pragma unroll
+          for (int j = 0; j < 32; ++j)
+            o[j] = __float_as_uint(__uint_as_float(o[j]) * xal[128 * ab + 32 * (c & 3) + j]);
+          ptx::tmem_st_32x32b_x32(ta, o);
+        }
+        ptx::tmem_wait_st();
+      }
+      {
+        // row m, tokens 32h..32h+31 = 16-byte chunks 4h..4h+3 of the 128-byte row (128-byte swizzle)
+        const uint32_t prow_s = sbase + kOffP + (uint32_t)m * 128u;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const uint32_t off = (uint32_t)(((4 * half + i) ^ (m & 7)) << 4);
+          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(prow_s + off), "r"(ph[4 * i]),
+                       "r"(ph[4 * i + 1]), "r"(ph[4 * i + 2]), "r"(ph[4 * i + 3])
+                       : "memory");
+          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(prow_s + kPBytes + off), "r"(pl[4 * i]),
+                       "r"(pl[4 * i + 1]), "r"(pl[4 * i + 2]), "r"(pl[4 * i + 3])
+                       : "memory");
+        }
+      }
+      ptx::fence_proxy_async_smem();
+      ptx::tc_fence_before();
+      const uint32_t any_lo = __any_sync(0xffffffffu, want_lo) ? 1u : 0u;
+      __syncwarp();   // every lane's P stores before lane 0's release
+      if (sw == 0 && lane == 0) DUO_TRACE(7, g);
+      if (lane == 0) {
+        const uint32_t fa = sbase + kOffFlag + 4u * (8 * (g & 3) + 4 * rank + sw);
+        if (even) {
+          lo_flag[8 * (g & 3) + sw] = any_lo;
+          if (sw == 0) ptx::mbar_arrive_expect_tx(bar(B_P_FULL), 4u * kSoftWarps);   // the odd CTA's words
+          else ptx::mbar_arrive(bar(B_P_FULL));
+        } else {
+          ptx::st_async_u32(lead(fa), any_lo, lead(bar(B_P_FULL)));
+          ptx::mbar_arrive_remote(lead(bar(B_P_FULL)));
+        }
+      }
+      if (cur.k == u.npg - 1) {
+        pend.on = true;
+        pend.item = u.item;
+        pend.n = u.n;
+        pend.part0 = u.part[0];
+        pend.part1 = u.part[1];
+        pend.l = l_part;
+        pend.m = m_ref;
+      }
+      advance(p, plan, u_end, cur);
+      ++g;
+    }
+    if (ok && pend.on && !epilogue(g - 1)) fail();
+  }
+
+  ptx::tc_fence_before();
+  __syncthreads();
+#ifdef MLA_TRACE
+  if (threadIdx.x == 0 && p.trace) p.trace[(size_t)blockIdx.x * 1024 + 1022] = (unsigned long long)clock64();
+#endif
+  ptx::cluster_sync();   // the even CTA's MMAs, commits and loads for both CTAs are done
+  if (warp == 1) {
+    ptx::tc_fence_after();
+    ptx::tmem_dealloc_pair(tbase, kTmemCols);
+  }
+  ptx::cluster_sync();
+}
+
+}  // namespace duo
+}  // namespace mla

@@ -21,7 +21,7 @@
 #include "simt_kernels.cuh"
 #include "decode_tc.cuh"
 #include "gemm_tc.cuh"
-#include "decode_pair.cuh"
+#include "decode_2sm.cuh"
 
 namespace {
 
@@ -164,11 +164,12 @@ mla_status launch_proj(const void* A, const void* Bw, void* out, int32_t T, cons
   return launch_check(what);
 }
 
-// The 2-CTA cluster kernel serves 128 rows per cluster: all heads of one query token
-// for H=128, or the heads of two consecutive query tokens of a sequence for H=64
-// (multi-token steps, q_len >= 2), whose rows then share every page.
+// The SM-pair kernel serves 128 rows per cluster: all heads of one query token for
+// H=128, or the heads of up to two consecutive query tokens of a sequence for H=64
+// (with one query token per sequence the odd CTA's rows are idle).
 bool pair_decode(const mla_dims& d, int32_t q_len) {
-  return use_tc_decode(d) && (d.H == mla::pair::kHeads || (d.H == mla::pair::kHeads / 2 && q_len >= 2));
+  (void)q_len;
+  return use_tc_decode(d) && (d.H == mla::duo::kRows || d.H == mla::duo::kRows / 2);
 }
 
 // CTAs per slot (the plan has num_sms / head_groups slots).
@@ -179,7 +180,7 @@ int32_t head_groups_for(const mla_dims& d, int32_t q_len) {
 
 // Query tokens per plan unit (consecutive tokens of one sequence).
 int32_t items_per_unit_for(const mla_dims& d, int32_t q_len) {
-  return pair_decode(d, q_len) ? mla::pair::kHeads / d.H : 1;
+  return pair_decode(d, q_len) && q_len >= 2 ? mla::duo::kRows / d.H : 1;
 }
 
 }  // namespace
@@ -526,17 +527,16 @@ mla_status mla_decode_attn(const void* q_lat, const void* q_rope, const void* kv
     p.drop_load = g_drop_load.load();
     const dim3 grid(info->num_slots * info->head_groups);
     if (pair_decode(d, q_len)) {
-      // 128 heads: a cluster of two CTAs per slot, each holding half of every page;
-      // the rope columns travel as two 32-column halves (64-byte swizzle)
-      CUtensorMap tkr, tqr;
-      if (mla_status s = make_map_2d(&tkr, kv_cache, d.R + d.Dr, (uint64_t)num_pages * d.page_size,
-                                     (uint64_t)(d.R + d.Dr) * 2, 64, 32))
+      // a pair of SMs per slot: 32-row boxes of the cache (half a page), 64-row boxes of
+      // the queries (one CTA's rows)
+      CUtensorMap tk32;
+      if (mla_status s = make_map_2d(&tk32, kv_cache, d.R + d.Dr, (uint64_t)num_pages * d.page_size,
+                                     (uint64_t)(d.R + d.Dr) * 2, 32, 64))
         return s;
-      if (mla_status s = make_map_2d(&tqr, q_rope, d.Dr, (uint64_t)T * d.H, (uint64_t)d.Dr * 2, 64, 32)) return s;
-      if (mla_status s = ensure_smem_attr((const void*)mla::pair::decode_pair_kernel, mla::pair::kSmemBytes))
+      if (mla_status s = ensure_smem_attr((const void*)mla::duo::decode_2sm_kernel, mla::duo::kSmemBytes))
         return s;
-      mla::pair::decode_pair_kernel<<<grid, mla::pair::kThreads, mla::pair::kSmemBytes, st>>>(tk, tkr, tqr, p);
-      return launch_check("decode_attn (tcgen05, CTA pair)");
+      mla::duo::decode_2sm_kernel<<<grid, mla::duo::kThreads, mla::duo::kSmemBytes, st>>>(tk32, tq, tr, p);
+      return launch_check("decode_attn (tcgen05, SM pair)");
     }
     mla::tc::decode_kernel<<<grid, 256, mla::tc::kSmemBytes, st>>>(tq, tr, tk, p);
     return launch_check("decode_attn (tcgen05)");

@@ -158,6 +158,90 @@ __device__ __forceinline__ void bulk_copy_to_cluster(uint32_t dst_cluster, uint3
                : "memory");
 }
 
+// ------------------------------------------------------------------ CTA pairs (tcgen05 cta_group::2)
+// 2D tiled load into this CTA's shared memory whose completion (bytes) is counted on
+// an mbarrier that may live in either CTA of the pair (`bar_cluster` is a
+// shared::cluster address, e.g. from map_peer). No multicast: each CTA loads its own.
+__device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const CUtensorMap* map, uint32_t bar_cluster,
+                                                 int32_t x, int32_t y) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4}], [%2];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar_cluster), "r"(x), "r"(y)
+      : "memory");
+}
+// Arrive on an mbarrier of either CTA of the cluster, ordering this thread's earlier
+// memory operations (and what it has observed) before the arrival at cluster scope.
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t bar_cluster) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(bar_cluster) : "memory");
+}
+__device__ __forceinline__ void st_cluster_u32(uint32_t addr_cluster, uint32_t v) {
+  asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(addr_cluster), "r"(v) : "memory");
+}
+// Arrive on an mbarrier of either CTA of the cluster with release semantics at CTA
+// scope: orders this thread's earlier writes to its own CTA's shared memory (made
+// visible to the async proxy by fence.proxy.async) before the arrival. Much cheaper
+// than a cluster-scope release, which waits for cluster-wide visibility.
+__device__ __forceinline__ void mbar_arrive_remote(uint32_t bar_cluster) {
+  asm volatile("mbarrier.arrive.release.cta.shared::cluster.b64 _, [%0];" ::"r"(bar_cluster) : "memory");
+}
+// 4-byte store into a shared-memory word of another CTA of the cluster whose completion
+// is counted (4 transaction bytes) on an mbarrier of that CTA: whoever sees the
+// barrier's phase complete also sees the word.
+__device__ __forceinline__ void st_async_u32(uint32_t addr_cluster, uint32_t v, uint32_t bar_cluster) {
+  asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.u32 [%0], %1, [%2];" ::"r"(addr_cluster),
+               "r"(v), "r"(bar_cluster)
+               : "memory");
+}
+// D[tmem] (+)= A[tmem] * B[smem desc] over the CTA pair (kind::f16), issued by one thread
+// of the even CTA: CTA r's A rows (its M/2 rows) come from its own TMEM at a_tmem,
+// duplicated in lane halves (row m in lanes m and 64 + m), K elements 2c, 2c+1 packed in
+// column c; B as for umma_pair_ss.
+__device__ __forceinline__ void umma_pair_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
+                                             uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+// TMEM allocation shared by the two CTAs of a pair: issued by the same warp in both.
+__device__ __forceinline__ void tmem_alloc_pair(uint32_t holder_smem, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(holder_smem),
+               "r"(ncols)
+               : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish_pair() {
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+// D[tmem] (+)= A[smem desc] * B[smem desc] over the CTA pair (kind::f16, bf16 in, fp32
+// accumulate), issued by one thread of the even CTA: CTA r supplies rows
+// [M/2 r, M/2 (r+1)) of A and columns [N/2 r, N/2 (r+1)) of B from its own shared
+// memory at the descriptors' addresses, and receives its M/2 rows of D (all N columns)
+// in its own TMEM.
+__device__ __forceinline__ void umma_pair_ss(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                             uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+// Arrive once on the mbarrier at shared offset `bar` in each CTA of `cta_mask` when every
+// tcgen05 operation issued so far by this thread is done.
+__device__ __forceinline__ void umma_commit_pair(uint32_t bar, uint16_t cta_mask) {
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(
+          bar),
+      "h"(cta_mask)
+      : "memory");
+}
+
 // Warp vote kept in program order (volatile): an instruction after it issues only once
 // every lane's predicate, and whatever it was computed from, is available.
 __device__ __forceinline__ uint32_t vote_any_ordered(bool pred) {

@@ -4,7 +4,7 @@ TEST INFRASTRUCTURE. Only ``tests/``, ``__graft_entry__.smoke()`` and the
 ``cpu_baseline`` / ``--impl reference`` legs of ``bench.py`` may import it. The
 library (``mla_latent_kv_46_b200``) never imports it and shares no code with it;
 the only thing both sides use is the seeded input generator
-(``mla_latent_kv_46_b200.workloads``), which holds no attention arithmetic.
+(``inputs.workloads``), which holds no attention arithmetic and imports only numpy.
 
 Sources (page title, then the section used):
   [GatedMLA]  kimi-k3 docs, "GatedMLA" (attention/gated_mla): "Projection geometry

@@ -8,6 +8,11 @@ if ROOT not in sys.path:
 
 def pytest_configure(config):
     config.addinivalue_line("markers", "gpu: needs a CUDA device (B200, sm_100a)")
-    # (re)build libmla.so if a source is newer, before any test imports the package
+    # (Re)build libmla.so if a source is newer, before any test imports the package.
+    # Compiling loads nothing; a missing toolchain must not stop the oracle's tests,
+    # which never import the package: the library's own tests then fail on import.
     import __graft_entry__
-    __graft_entry__._builder().build(force=False)
+    try:
+        __graft_entry__._builder().build(force=False)
+    except Exception as e:  # noqa: BLE001
+        print(f"conftest: libmla.so not built ({e})")

@@ -12,7 +12,7 @@ import numpy as np
 import pytest
 
 import mla_latent_kv_46_b200 as mla
-from mla_latent_kv_46_b200 import workloads as wl
+from inputs import workloads as wl
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 HEADER = os.path.join(ROOT, "include", "mla.h")
@@ -66,11 +66,11 @@ def test_plan_covers_every_visible_page_once(q_len, sms, H):
     d = dims(H=H)
     plan, info = mla.mla_plan_splits(lens, len(lens), q_len, max_pages, d, sms)
     p = parse_plan(plan)
-    # 2-CTA clusters for 128 heads, and for 64 heads with several query tokens (two
-    # consecutive tokens per unit); otherwise one CTA per 64 heads
-    pair = H == 128 or (H == 64 and q_len >= 2)
+    # SM pairs (2-CTA clusters) for 128 and 64 heads, with two consecutive tokens per
+    # unit for 64 heads and several query tokens; otherwise one CTA per 64 heads
+    pair = H in (64, 128)
     G = 2 if pair else (H // 64 if H % 64 == 0 else 1)
-    per_unit = 128 // H if pair else 1
+    per_unit = 128 // H if pair and q_len >= 2 else 1
     assert p["G"] == info.head_groups == G
     assert plan[9] == per_unit
     assert info.num_slots <= max(1, sms // G)
@@ -115,8 +115,8 @@ def test_plan_balances_pages_over_slots():
     for u in p["units"]:
         per[u[5]] += u[3] - u[2]
     assert per.sum() == 64 * 64
-    assert per.max() <= math.ceil(4096 / 148)
-    assert info.num_slots == 148
+    assert per.max() <= math.ceil(4096 / 74)
+    assert info.num_slots == 74     # one SM pair per slot
 
 
 def test_plan_rejects_too_long_sequences_and_small_buffers():
@@ -177,7 +177,7 @@ def test_bf16_rounding_is_nearest_even():
 def test_noalloc_rejects_plans_beyond_its_scratch():
     """1000 partial outputs of 64 heads x 512 fp32 need 131 MB, over the 48 MiB the
     allocation-free entry point holds: refused on the host, before any launch."""
-    info = mla.PlanInfo(num_items=1, num_units=1000, num_slots=1, num_parts=1000, head_groups=1, plan_words=0)
+    info = mla.PlanInfo(num_items=1, num_units=1000, num_slots=1, num_parts=1000, head_groups=2, plan_words=0)
     with pytest.raises(mla.MlaError) as e:
         mla.mla_decode_attn_noalloc(16, 16, 16, 16, 16, 1, 1, 1, 1, 0.1, 16, info, 16, None, dims(), stream=0)
     assert e.value.status == mla._binding.MLA_ERR_WORKSPACE

@@ -56,7 +56,7 @@ def fake_root(tmp_path, monkeypatch):
     src_dir = tmp_path / "mla_latent_kv_46_b200" / "csrc"
     src_dir.mkdir(parents=True)
     (tmp_path / "profiles").mkdir()
-    src = src_dir / "decode_pair.cuh"
+    src = src_dir / "decode_2sm.cuh"
     src.write_text("// kernel v1\n")
     monkeypatch.setattr(bench, "ROOT", str(tmp_path))
     return tmp_path, src
@@ -64,7 +64,7 @@ def fake_root(tmp_path, monkeypatch):
 
 def _profile(root, sha, traffic):
     (root / "profiles" / "ncu_decode_attn_wl.md").write_text(
-        f"Kernel source: decode_pair.cuh sha256[:16]: {sha}\n"
+        f"Kernel source: decode_2sm.cuh sha256[:16]: {sha}\n"
         f"| traffic per full launch (bytes): {traffic} | x |\n")
 
 
@@ -90,6 +90,7 @@ def test_traffic_needs_a_summary_of_that_workload(fake_root):
 
 
 def test_decode_kernel_follows_the_library_dispatch():
-    assert bench.decode_kernel_of(128, 1)[0] == "decode_pair.cuh"
-    assert bench.decode_kernel_of(64, 2)[0] == "decode_pair.cuh"
-    assert bench.decode_kernel_of(64, 1)[0] == "decode_tc.cuh"
+    assert bench.decode_kernel_of(128, 1)[0] == "decode_2sm.cuh"
+    assert bench.decode_kernel_of(64, 2)[0] == "decode_2sm.cuh"
+    assert bench.decode_kernel_of(64, 1)[0] == "decode_2sm.cuh"
+    assert bench.decode_kernel_of(192, 1)[0] == "decode_tc.cuh"

@@ -6,8 +6,10 @@ fp32 storage: |got - ref| <= 1e-5. Cache append is bit-exact.
 
 Small cases span several pages and a ragged tail and include empty sequences; both
 kernel policies (SIMT CUDA cores, tcgen05 tensor cores) run where the geometry allows.
-The full-size workloads run in the launch configuration the benchmark times and are
-checked on sampled (query, head) outputs the oracle computes one by one.
+The full-size workloads run in the launch configuration the benchmark times and every
+(query, head) output is checked: against the fp64 absorbed pipeline for the decode
+workloads (plus a non-absorbed sample holding the longest sequence), against the full
+causal forward for the multi-token chunk.
 """
 import math
 
@@ -17,7 +19,7 @@ import torch
 
 import mla_latent_kv_46_b200 as mla
 from mla_latent_kv_46_b200 import decoder as dec
-from mla_latent_kv_46_b200 import workloads as wl
+from inputs import workloads as wl
 from oracle import mla_oracle as orc
 
 pytestmark = pytest.mark.gpu
@@ -298,43 +300,71 @@ def test_incremental_gpu_decode_equals_full_causal_tiny():
         assert_close(host(step.out)[0], full[n - 1], True, f"prefix {n}")
 
 
-# ----------------------------------------------------------------------------- full-size workloads, sampled
+# ----------------------------------------------------------------------------- full-size workloads, every output
 
 FULL = ["kimi_h64_b64_l4096", "deepseek_h128_b128_ragged", "longctx_h64_b4_l131072",
         "causal_chunk_h64_b8_2048p256"]
 
 
-@pytest.mark.parametrize("name", FULL)
-def test_full_size_workload_sampled(name):
+def _full_step(name):
+    """The whole step (append included) at full size, in the launch configuration the
+    benchmark times; returns the workload (cache as after the append) and host outputs."""
     spec = wl.WORKLOADS[name]
     w = wl.make(spec, seed=0, new_rows_in_cache=False)
     step = dec.DecodeStep(w)
     step.run(append=True)
     torch.cuda.synchronize()
     mla.mla_check_status()
-    out, lse = host(step.out), host(step.lse)
+    out, lse, o_lat = host(step.out), host(step.lse), host(step.o_lat)
+    del step
+    torch.cuda.empty_cache()
+    return wl.make(spec, seed=0), out, lse, o_lat
+
+
+@pytest.mark.parametrize("name", FULL[:3])
+def test_full_size_workload_every_output(name):
+    """Every (query, head) of the workload against the fp64 absorbed pipeline with the
+    kernels' two bf16 stores (q_lat, o_lat) rounded the same way: out, lse and o_lat,
+    elementwise at the bf16 bound. That oracle is pinned to the non-absorbed definition
+    (tests/test_oracle.py); here the definition itself is checked too, on a sample that
+    always holds the longest sequence (for the long-context workload: 131,072 tokens
+    with per-token logit noise of std 4)."""
+    spec = wl.WORKLOADS[name]
+    full, out, lse, o_lat = _full_step(name)
+    args = (full["q_nope"], full["q_rope"], full["kv_cache"], full["block_table"], full["seq_lens"],
+            full["W_UK"], full["W_UV"], full["scale"])
+    mixed = orc.decode_absorbed(*args, q_len=spec.q_len, page_size=spec.page_size, intermediates="bf16")
+    assert_close(out, mixed["out"], False, f"{name} out, every query and head")
+    assert_close(lse, mixed["lse"], False, f"{name} lse, every query and head")
+    assert_close(o_lat, mixed["o_lat"], False, f"{name} o_lat, every query and head")
+    lens = np.asarray(full["seq_lens"])
     rng = np.random.default_rng(123)
-    seqs = sorted(rng.choice(len(w["seq_lens"]), size=min(2, len(w["seq_lens"])), replace=False).tolist())
+    seqs = sorted({int(np.argmax(lens))} | set(rng.choice(len(lens), size=min(2, len(lens)),
+                                                          replace=False).tolist()))
     heads = sorted(rng.choice(spec.H, size=2, replace=False).tolist())
-    full = wl.make(spec, seed=0)   # the cache as it must be after the append
-    if spec.all_query_positions:
-        for b in seqs[:1]:
-            L = int(w["seq_lens"][b])
-            rows = orc.to_f64(wl.sequence_rows(spec, b, L, seed=0))
-            qn, qr = full["all_queries"][b]
-            ref = orc.full_causal(rows[:, :spec.R], rows[:, spec.R:], qn, qr, w["W_UK"], w["W_UV"], w["scale"],
-                                  heads=heads)
-            got = out[b * spec.q_len:(b + 1) * spec.q_len]
-            assert_close(got[:, heads], ref[L - spec.q_len:, heads], False, f"{name} b={b}")
-        return
-    ref = orc.decode_nonabsorbed(full["q_nope"], full["q_rope"], full["kv_cache"], full["block_table"],
-                                 full["seq_lens"], full["W_UK"], full["W_UV"], full["scale"], q_len=spec.q_len,
-                                 page_size=spec.page_size, seqs=seqs, heads=heads)
+    ref = orc.decode_nonabsorbed(*args, q_len=spec.q_len, page_size=spec.page_size, seqs=seqs, heads=heads)
     for b in seqs:
         for h in heads:
-            assert_close(out[b, h], ref["out"][b, h], False, f"{name} out b={b} h={h}")
-            assert_close(lse[b, h], ref["lse"][b, h], False, f"{name} lse b={b} h={h}")
-    assert np.all(np.isfinite(out))
+            assert_close(out[b, h], ref["out"][b, h], False, f"{name} out vs definition b={b} h={h}")
+            assert_close(lse[b, h], ref["lse"][b, h], False, f"{name} lse vs definition b={b} h={h}")
+
+
+def test_full_size_causal_chunk_every_output():
+    """All 8 sequences x 64 heads x 256 new tokens of the multi-token causal chunk
+    against the oracle's full causal forward over all 2304 positions (the definition:
+    rebuilt per-head K and V, causal softmax), the last 256 rows of each."""
+    name = FULL[3]
+    spec = wl.WORKLOADS[name]
+    full, out, lse, o_lat = _full_step(name)
+    for b in range(len(full["seq_lens"])):
+        L = int(full["seq_lens"][b])
+        rows = orc.to_f64(wl.sequence_rows(spec, b, L, seed=0))
+        qn, qr = full["all_queries"][b]
+        ref = orc.full_causal(rows[:, :spec.R], rows[:, spec.R:], qn, qr, full["W_UK"], full["W_UV"],
+                              full["scale"])
+        got = out[b * spec.q_len:(b + 1) * spec.q_len]
+        assert_close(got, ref[L - spec.q_len:], False, f"{name} b={b}, every new token and head")
+    assert np.all(np.isfinite(lse))
 
 
 # ----------------------------------------------------------------------------- failure reporting

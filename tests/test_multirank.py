@@ -27,7 +27,7 @@ def _rank_main(rank, port, out):
     dist.init_process_group("gloo", rank=rank, world_size=WORLD, timeout=datetime.timedelta(seconds=60))
     try:
         import bench
-        from mla_latent_kv_46_b200 import workloads as wl
+        from inputs import workloads as wl
 
         spec = wl.WORKLOADS[WORKLOAD]
         lens = wl.seq_lens_of(spec, rank)            # the batch bench.py gives rank r: seed r

@@ -14,7 +14,7 @@ import numpy as np
 import pytest
 import torch
 
-from mla_latent_kv_46_b200 import workloads as wl
+from inputs import workloads as wl
 from oracle import ledger, loops
 from oracle import mla_oracle as orc
 

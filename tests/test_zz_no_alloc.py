@@ -18,7 +18,7 @@ import torch
 
 import mla_latent_kv_46_b200 as mla
 from mla_latent_kv_46_b200 import decoder as dec
-from mla_latent_kv_46_b200 import workloads as wl
+from inputs import workloads as wl
 
 pytestmark = pytest.mark.gpu
 
