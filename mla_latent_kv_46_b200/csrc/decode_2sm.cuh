@@ -26,14 +26,15 @@
 // TMEM (512 columns, both CTAs):
 //   [0,256)   O^T: lane L of region lh (columns 128lh..) is latent 256lh + 128r + L, one
 //             column per row of the pair (rows 0-63 the even CTA's, 64-127 the odd's)
-//   [256,320) two score buffers of 32 columns (a pair MMA with M=128 holds row m of the
-//             CTA in lanes m and 64+m): lane half h holds tokens 32h..32h+31
-//   [320,512) the score MMA's A operand for latent columns 0-383 of the query (bf16
+//   [256,288) the score buffer (a pair MMA with M=128 holds row m of the CTA in lanes m
+//             and 64+m): lane half h holds tokens 32h..32h+31
+//   [288,512) the score MMA's A operand for latent columns 0-447 of the query (bf16
 //             pairs, 32 columns per 64 dims), row m in lanes m and 64+m
-// Shared memory: the query's latent columns 384-511 and rope (three 64-row boxes),
-// three score-operand slots (the page's own 32 tokens x 576: nine 32-row boxes), two
-// value-operand slots (64 tokens x own 256 latent: eight 32-row boxes), P as bf16
-// (K-major, 64 rows x 64 tokens) and its remainder P_lo.
+// Shared memory: the query's latent columns 448-511 and rope (two 64-row boxes), three
+// score-operand slots (the page's own 32 tokens x 576: nine 32-row boxes), two
+// value-operand slots (64 tokens x own 256 latent: eight 32-row boxes), and two
+// buffers of P as bf16 (K-major, 64 rows x 64 tokens) with its remainder P_lo, so that
+// page g's P is written while page g-1's value MMAs read the other buffer.
 //
 // P enters the value MMA in bf16 (round to nearest). Where one token can carry a
 // large share of a row's weight, one bf16 rounding of P moves the output by more than
@@ -73,11 +74,11 @@ constexpr int kRows = 128;             // MMA rows of the pair
 constexpr int kCtaRows = 64;           // rows per CTA
 constexpr int kPage = 64, kR = 512, kDr = 64, kRow = kR + kDr;
 constexpr int kChunks = kRow / 64;     // 64-column chunks of a row (8 latent + rope)
-constexpr int kQTmemChunks = 6;        // query chunks held in TMEM (latent 0-383)
-constexpr int kQSmemChunks = kChunks - kQTmemChunks;   // latent 384-511 and rope
+constexpr int kQTmemChunks = 7;        // query chunks held in TMEM (latent 0-447)
+constexpr int kQSmemChunks = kChunks - kQTmemChunks;   // latent 448-511 and rope
 constexpr int kBox32 = 32 * 128;       // 32 rows x 64 bf16, 128-byte swizzle
 constexpr int kBox64 = 64 * 128;       // 64 rows x 64 bf16
-constexpr int kQBytes = kQSmemChunks * kBox64;     // 24,576
+constexpr int kQBytes = kQSmemChunks * kBox64;     // 16,384
 constexpr int kQKSlotBytes = kChunks * kBox32;     // 36,864
 constexpr int kPVSlotBytes = 8 * kBox32;           // 32,768
 constexpr int kQKSlots = 3, kPVSlots = 2;
@@ -89,8 +90,8 @@ constexpr int kThreads = 32 * (kFirstSoftWarp + kSoftWarps);
 constexpr int kOffQ = 0;
 constexpr int kOffQK = kOffQ + kQBytes;
 constexpr int kOffPV = kOffQK + kQKSlots * kQKSlotBytes;
-constexpr int kOffP = kOffPV + kPVSlots * kPVSlotBytes;   // P_hi, then P_lo
-constexpr int kOffBar = kOffP + 2 * kPBytes;              // 32 mbarriers
+constexpr int kOffP = kOffPV + kPVSlots * kPVSlotBytes;   // two buffers of P_hi then P_lo
+constexpr int kOffBar = kOffP + 4 * kPBytes;              // 32 mbarriers
 constexpr int kOffXmax = kOffBar + 32 * 8;                // float[2][128]: row maxima of the lane halves
 constexpr int kOffXl = kOffXmax + 2 * 128 * 4;            // float[128]: row sums of the lane halves
 constexpr int kOffFlag = kOffXl + 128 * 4;                // uint32[4][8] (even CTA): P_lo wanted, per tile % 4
@@ -112,15 +113,16 @@ enum {
   B_Q_FULL = B_PV_EMPTY + 2,       // (even CTA) the unit's query in both CTAs: TMA bytes of the
                                    // shared-memory part, one arrival per softmax warp for TMEM
   B_Q_EMPTY,                       // last score MMA of a unit done
-  B_S_FULL,                        // +buffer: score MMAs done
-  B_S_EMPTY = B_S_FULL + 2,        // +buffer (even CTA): both CTAs' softmax warps read S
-  B_P_FULL = B_S_EMPTY + 2,        // (even CTA) P of both CTAs in shared memory, O rescaled
-  B_O_DONE,                        // value MMAs of a page done
-  B_O_FREE,                        // (even CTA) both CTAs' epilogues have read O
+  B_S_FULL,                        // score MMAs done
+  B_S_EMPTY,                       // (even CTA) both CTAs' softmax warps read S
+  B_P_FULL,                        // (even CTA) P of both CTAs in shared memory, O rescaled
+  B_O_DONE,                        // +P buffer: value MMAs that read the buffer done
+  B_O_FREE = B_O_DONE + 2,                        // (even CTA) both CTAs' epilogues have read O
   B_PAIR,                          // +1: the two softmax warps of rows 0-31 / 32-63
   B_AL_FULL = B_PAIR + 2,          // +buffer: both CTAs' rescale factors of a page (local arrivals,
                                    // the peer's words as transaction bytes)
   B_LX_FULL = B_AL_FULL + 2,       // both CTAs' 1 / l of a unit (likewise)
+  B_ALL4,                          // the four softmax warps (epilogue staging)
   B_DRAIN,
   kNumBars
 };
@@ -128,7 +130,7 @@ static_assert(kNumBars <= 32, "barrier area");
 static_assert(kQKSlots <= 3 && kPVSlots <= 2, "barrier slots");
 
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColO = 0, kColS = 256, kColQ = 320;
+constexpr uint32_t kColO = 0, kColS = 256, kColQ = 288;
 static_assert(kColQ + 32 * kQTmemChunks <= kTmemCols, "TMEM columns");
 constexpr uint32_t kIdescS = ptx::idesc_bf16_f32(128, 64, 0, 0);    // Q (K-major) x KV^T (K-major)
 constexpr uint32_t kIdescV = ptx::idesc_bf16_f32(256, 128, 1, 0);   // C^T (M-major) x P^T (K-major)
@@ -171,8 +173,11 @@ __device__ __forceinline__ Unit2 load_unit2(const Params& p, const PlanView& pla
 // tiles: 0 score operand load issued, 1 value operand load issued, 2 score operand
 // landed (MMA warp), 3 score MMA issued, 4 P of both CTAs ready (MMA warp), 5 value
 // MMA issued, 6 scores read (softmax warp 4), 7 P stored (softmax warp 4), 8 value
-// operand landed (MMA warp), 9 query staged in TMEM (softmax warp 4, per unit); slot
-// 1020 the SM id, 1021 the global timer at start, 1022 clock at exit, 1023 at start.
+// operand landed (MMA warp), 9 query staged in TMEM (softmax warp 4, per unit), 10 and
+// 11 epilogue start and end (softmax warp 4, per unit), 12 unit's query ready and 13
+// the previous unit's O read (MMA warp, per unit), 14 epilogue: both CTAs' 1 / l
+// received; slot 1020 the SM id, 1021 the global timer at start, 1022 clock at exit,
+// 1023 at start.
 #ifdef MLA_TRACE
 #define DUO_TRACE(region, g)                                                                     \
   do {                                                                                           \
@@ -260,20 +265,20 @@ decode_2sm_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_consta
       ptx::mbar_init(bar(B_PV_FULL + s), 1);
       ptx::mbar_init(bar(B_PV_EMPTY + s), 1);
     }
-    for (int s = 0; s < 2; ++s) {
-      ptx::mbar_init(bar(B_S_FULL + s), 1);
-      ptx::mbar_init(bar(B_S_EMPTY + s), 2 * kSoftWarps);
-    }
+    ptx::mbar_init(bar(B_S_FULL), 1);
+    ptx::mbar_init(bar(B_S_EMPTY), 2 * kSoftWarps);
     ptx::mbar_init(bar(B_Q_FULL), 1 + 2 * kSoftWarps);
     ptx::mbar_init(bar(B_Q_EMPTY), 1);
     ptx::mbar_init(bar(B_P_FULL), 2 * kSoftWarps);
     ptx::mbar_init(bar(B_O_DONE), 1);
+    ptx::mbar_init(bar(B_O_DONE + 1), 1);
     ptx::mbar_init(bar(B_O_FREE), 2 * kSoftWarps);
     ptx::mbar_init(bar(B_PAIR), 2);
     ptx::mbar_init(bar(B_PAIR + 1), 2);
     ptx::mbar_init(bar(B_AL_FULL), 2);
     ptx::mbar_init(bar(B_AL_FULL + 1), 2);
     ptx::mbar_init(bar(B_LX_FULL), 2);
+    ptx::mbar_init(bar(B_ALL4), kSoftWarps);
     ptx::mbar_init(bar(B_DRAIN), 1);
     ptx::fence_mbar_init();
   }
@@ -313,50 +318,15 @@ decode_2sm_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_consta
 
   if (warp == 0 || warp == 2) {
     // ================================================================ TMA producers
-    // warp 0: the query's shared-memory part per unit and each page's score operand (own
-    // 32 tokens x 576); warp 2: each page's value operand (64 tokens x own 256 latent)
+    // warp 0: each page's score operand (own 32 tokens x 576); warp 2: each page's value
+    // operand (64 tokens x own 256 latent)
     const bool leader = ptx::elect_one();
     const bool qk = warp == 0;
     const int nslots = qk ? kQKSlots : kPVSlots;
     Cursor c = first_page(p, plan, u_begin, u_end);
-    // L2 prefetch cursor (even CTA, warp 0): whole pages a few pages ahead, and the next
-    // units' query rows when the cursor enters them
-    Cursor pf = c;
-    auto prefetch_one = [&]() {
-      if (!pf.valid) return;
-      if (even && leader) {
-        if (pf.k == 0) {
-          const int64_t qrow = (int64_t)pf.u.item * H;
-          const int64_t rows = min((int64_t)kRows, TH - qrow);
-          if (rows > 0) {
-            ptx::prefetch_l2_bulk(p.q_lat + qrow * kR, (uint32_t)(rows * kR * 2));
-            ptx::prefetch_l2_bulk(p.q_rope + qrow * kDr, (uint32_t)(rows * kDr * 2));
-          }
-        }
-        const int32_t page = page_id(p, pf.u, pf.k, false);
-        if (page < p.num_pages) ptx::prefetch_l2_bulk(p.kv + (int64_t)page * kPage * kRow, kPage * kRow * 2);
-      }
-      advance(p, plan, u_end, pf);
-    };
-    if (qk)
-      for (int i = 0; i < 6; ++i) prefetch_one();
-    uint32_t g = 0, nq = 0;
+    uint32_t g = 0;
     bool ok = true;
     while (c.valid && ok) {
-      if (qk && c.k == 0) {
-        if (!wait_all(bar(B_Q_EMPTY), (nq & 1) ^ 1)) { if (leader) fail(); ok = false; break; }
-        if (leader) {
-          if (even) ptx::mbar_arrive_expect_tx(bar(B_Q_FULL), 2 * kQBytes);
-          const int32_t qrow = c.u.item * H + kCtaRows * (int32_t)rank;   // rows past the tensor read zeros
-#pragma unroll 1
-          for (int ch = 0; ch < kQSmemChunks - 1; ++ch)
-            ptx::tma_load_2d_pair(sbase + kOffQ + ch * kBox64, &tm_q, lead(bar(B_Q_FULL)),
-                                  64 * (kQTmemChunks + ch), qrow);
-          ptx::tma_load_2d_pair(sbase + kOffQ + (kQSmemChunks - 1) * kBox64, &tm_qr, lead(bar(B_Q_FULL)), 0,
-                                qrow);
-        }
-        ++nq;
-      }
       const uint32_t s = g % nslots, ph = (g / nslots) & 1;
       if (!wait_all(bar((qk ? B_QK_EMPTY : B_PV_EMPTY) + s), ph ^ 1)) { if (leader) fail(); ok = false; break; }
       const int32_t page = page_id(p, c.u, c.k, leader && qk);
@@ -387,17 +357,50 @@ decode_2sm_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_consta
           }
         }
       }
-      if (qk) prefetch_one();
       advance(p, plan, u_end, c);
       ++g;
     }
     // The even CTA's barriers count both CTAs' loads: before the pair exits, wait (bounded)
     // for the phases armed last, so no copy is still landing in either CTA.
-    if (even) {
+    if (even)
       for (uint32_t k = (g >= (uint32_t)nslots ? g - nslots : 0); k < g; ++k)
         wait_all(bar((qk ? B_QK_FULL : B_PV_FULL) + k % nslots), (k / nslots) & 1);
-      if (qk && nq > 0) wait_all(bar(B_Q_FULL), (nq - 1) & 1);
+  } else if (warp == 3) {
+    // ================================================================ the query's shared-memory part
+    // per unit (latent 448-511 and rope of the CTA's 64 rows), once the previous unit's
+    // last score MMA is done; the even CTA also prefetches the next unit's query rows
+    // into L2 for the softmax warps, which stage the TMEM part
+    const bool leader = ptx::elect_one();
+    int32_t ui = u_begin - 1;
+    Unit2 u;
+    uint32_t nq = 0;
+    bool have = next_unit(p, plan, ui, u_end, u);
+    while (have) {
+      Unit2 nu;
+      int32_t ni = ui;
+      const bool more = next_unit(p, plan, ni, u_end, nu);
+      if (even && leader && more) {
+        const int64_t qrow = (int64_t)nu.item * H;
+        const int64_t rows = min((int64_t)kRows, TH - qrow);
+        if (rows > 0) ptx::prefetch_l2_bulk(p.q_lat + qrow * kR, (uint32_t)(rows * kR * 2));
+      }
+      if (!wait_all(bar(B_Q_EMPTY), (nq & 1) ^ 1)) { if (leader) fail(); break; }
+      if (leader) {
+        if (even) ptx::mbar_arrive_expect_tx(bar(B_Q_FULL), 2 * kQBytes);
+        const int32_t qrow = u.item * H + kCtaRows * (int32_t)rank;   // rows past the tensor read zeros
+#pragma unroll 1
+        for (int ch = 0; ch < kQSmemChunks - 1; ++ch)
+          ptx::tma_load_2d_pair(sbase + kOffQ + ch * kBox64, &tm_q, lead(bar(B_Q_FULL)),
+                                64 * (kQTmemChunks + ch), qrow);
+        ptx::tma_load_2d_pair(sbase + kOffQ + (kQSmemChunks - 1) * kBox64, &tm_qr, lead(bar(B_Q_FULL)), 0,
+                              qrow);
+      }
+      ++nq;
+      ui = ni;
+      u = nu;
+      have = more;
     }
+    if (even && nq > 0) wait_all(bar(B_Q_FULL), (nq - 1) & 1);
   } else if (warp == 1) {
     // ================================================================ MMA issuer (even CTA)
     if (even) {
@@ -408,13 +411,14 @@ decode_2sm_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_consta
       uint32_t gq = 0, gv = 0;
       auto issue_s = [&]() -> bool {
         if (qc.k == 0 && !wait_all(bar(B_Q_FULL), qc.n & 1)) return false;
-        const uint32_t s = gq % kQKSlots, ph = (gq / kQKSlots) & 1, sb = gq & 1;
+        if (qc.k == 0 && leader) DUO_TRACE(12, qc.n);
+        const uint32_t s = gq % kQKSlots, ph = (gq / kQKSlots) & 1;
         if (!wait_all(bar(B_QK_FULL + s), ph)) return false;
         if (leader) DUO_TRACE(2, gq);
-        if (!wait_all(bar(B_S_EMPTY + sb), ((gq >> 1) & 1) ^ 1)) return false;
+        if (!wait_all(bar(B_S_EMPTY), (gq & 1) ^ 1)) return false;   // both CTAs read S(gq - 1)
         ptx::tc_fence_after();
         const uint32_t kvs = sbase + kOffQK + s * kQKSlotBytes;
-        const uint32_t d_s = tbase + kColS + 32u * sb;
+        const uint32_t d_s = tbase + kColS;
         if (leader) {
           DUO_TRACE(3, gq);
 #pragma unroll 1
@@ -433,7 +437,7 @@ decode_2sm_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_consta
             }
           }
           ptx::umma_commit_pair(bar(B_QK_EMPTY + s), 3);
-          ptx::umma_commit_pair(bar(B_S_FULL + sb), 3);
+          ptx::umma_commit_pair(bar(B_S_FULL), 3);
           if (qc.k == qc.u.npg - 1) ptx::umma_commit_pair(bar(B_Q_EMPTY), 3);
         }
         __syncwarp();
@@ -445,6 +449,7 @@ decode_2sm_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_consta
         if (!wait_all(bar(B_P_FULL), gv & 1)) return false;
         if (leader) DUO_TRACE(4, gv);
         if (vc.k == 0 && vc.n > 0 && !wait_all(bar(B_O_FREE), (vc.n - 1) & 1)) return false;
+        if (vc.k == 0 && leader) DUO_TRACE(13, vc.n);
         const uint32_t s = gv % kPVSlots, ph = (gv / kPVSlots) & 1;
         if (!wait_all(bar(B_PV_FULL + s), ph)) return false;
         if (leader) DUO_TRACE(8, gv);
@@ -457,7 +462,7 @@ decode_2sm_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_consta
           DUO_TRACE(5, gv);
 #pragma unroll 1
           for (int part = 0; part < (want_lo ? 2 : 1); ++part) {
-            const uint64_t dp = ptx::sdesc_sw128(sbase + kOffP + part * kPBytes, 16, 1024);
+            const uint64_t dp = ptx::sdesc_sw128(sbase + kOffP + (2 * (gv & 1) + part) * kPBytes, 16, 1024);
 #pragma unroll
             for (int lh = 0; lh < 2; ++lh) {
 #pragma unroll
@@ -472,7 +477,7 @@ decode_2sm_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_consta
             }
           }
           ptx::umma_commit_pair(bar(B_PV_EMPTY + s), 3);
-          ptx::umma_commit_pair(bar(B_O_DONE), 3);
+          ptx::umma_commit_pair(bar(B_O_DONE + (gv & 1)), 3);
         }
         __syncwarp();
         advance(p, plan, u_end, vc);
@@ -506,7 +511,7 @@ decode_2sm_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_consta
     volatile uint32_t* xflg = reinterpret_cast<volatile uint32_t*>(smem + kOffXflg);
     volatile float* xinv = reinterpret_cast<volatile float*>(smem + kOffXinv);
     auto peer = [&](uint32_t local) { return ptx::map_peer(local, rank ^ 1u); };
-    uint32_t n_pair = 0, n_lx = 0;
+    uint32_t n_pair = 0, n_lx = 0, n_all4 = 0;
     bool ok = true;
     // the two warps of rows 32(q&1).. (lane halves 0 and 1) meet on B_PAIR + (q & 1)
     auto pair_sync = [&]() -> bool {
@@ -514,6 +519,14 @@ decode_2sm_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_consta
       if (lane == 0) ptx::mbar_arrive(bar(B_PAIR + (q & 1)));
       const bool done = ptx::mbar_wait_bounded(bar(B_PAIR + (q & 1)), n_pair & 1, abort_flag, p.timeout_ns);
       ++n_pair;
+      return __all_sync(0xffffffffu, done);
+    };
+    // the four softmax warps of this CTA
+    auto all4_sync = [&]() -> bool {
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive(bar(B_ALL4));
+      const bool done = ptx::mbar_wait_bounded(bar(B_ALL4), n_all4 & 1, abort_flag, p.timeout_ns);
+      ++n_all4;
       return __all_sync(0xffffffffu, done);
     };
     // arrivals on the even CTA's barriers that only report finished TMEM reads
@@ -557,22 +570,26 @@ decode_2sm_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_consta
       const bool inside = row < TH;   // rows past the query tensor (an absent token) stay zero
       const __nv_bfloat16* src = p.q_lat + row * kR;
 #pragma unroll 1
-      for (int ch = 0; ch < kQTmemChunks; ++ch) {
-        uint32_t w[32];
+      for (int ch = 0; ch < kQTmemChunks; ch += 2) {
+        uint32_t w[2][32];
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          uint32_t* d = &w[8 * i];
-          if (inside) {
-            asm volatile("ld.global.nc.v8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
-                         : "=r"(d[0]), "=r"(d[1]), "=r"(d[2]), "=r"(d[3]), "=r"(d[4]), "=r"(d[5]), "=r"(d[6]),
-                           "=r"(d[7])
-                         : "l"(src + 64 * ch + 16 * i));
-          } else {
+        for (int h = 0; h < 2; ++h) {
 #pragma unroll
-            for (int k = 0; k < 8; ++k) d[k] = 0u;
+          for (int i = 0; i < 4; ++i) {
+            uint32_t* d = &w[h][8 * i];
+            if (inside && ch + h < kQTmemChunks) {
+              asm volatile("ld.global.nc.v8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+                           : "=r"(d[0]), "=r"(d[1]), "=r"(d[2]), "=r"(d[3]), "=r"(d[4]), "=r"(d[5]), "=r"(d[6]),
+                             "=r"(d[7])
+                           : "l"(src + 64 * (ch + h) + 16 * i));
+            } else {
+#pragma unroll
+              for (int k = 0; k < 8; ++k) d[k] = 0u;
+            }
           }
         }
-        ptx::tmem_st_32x32b_x32(tbase + lane_addr + kColQ + 32u * ch, w);
+        ptx::tmem_st_32x32b_x32(tbase + lane_addr + kColQ + 32u * ch, w[0]);
+        if (ch + 1 < kQTmemChunks) ptx::tmem_st_32x32b_x32(tbase + lane_addr + kColQ + 32u * (ch + 1), w[1]);
       }
       ptx::tmem_wait_st();
       ptx::tc_fence_before();
@@ -593,9 +610,11 @@ decode_2sm_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_consta
     // O^T[:, row] / l_row to the output, once the unit's last value MMAs are done: the row's
     // owner CTA adds its two threads' sums and publishes 1 / l to both CTAs; every thread
     // then writes its two latent rows for all of the pair's rows.
+    uint32_t n_ep = 0;
     auto epilogue = [&](uint32_t g_last) -> bool {
-      if (!wait_all(bar(B_O_DONE), g_last & 1)) return false;
+      if (!wait_all(bar(B_O_DONE + (g_last & 1)), (g_last >> 1) & 1)) return false;
       ptx::tc_fence_after();
+      if (sw == 0 && lane == 0) DUO_TRACE(10, n_ep);
       xl[L] = pend.l;
       if (!pair_sync()) return false;
       if (half == 0) {
@@ -620,26 +639,88 @@ decode_2sm_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_consta
       const bool got = ptx::mbar_wait_cluster_bounded(bar(B_LX_FULL), n_lx & 1, abort_flag, p.timeout_ns);
       ++n_lx;
       if (!__all_sync(0xffffffffu, got)) return false;
+      if (sw == 0 && lane == 0) DUO_TRACE(14, n_ep);
+      // Two 32-row chunks of O^T per round (32 rows x this CTA's 128 latent columns of one
+      // half each): scale, stage them row-major in the idle P buffers, then write whole row
+      // segments with 16-byte stores (bf16 final rows: 256 B each, fp32 partial rows: 512 B).
 #pragma unroll 1
-      for (int c = 0; c < 8; ++c) {
-        uint32_t o[32];
-        ptx::tmem_ld_32x32b_x32(tbase + lane_addr + kColO + 32u * c, o);
-        ptx::tmem_wait_ld();
-        const int lh = c >> 2, n0 = 32 * (c & 3);
-        const int d = 256 * lh + 128 * (int)rank + L;   // this thread's latent row
-        const int tn = H == kRows ? 0 : n0 / kCtaRows;  // the 32 rows' query token
-        if (tn >= pend.n) continue;
-        const int32_t prt = tn ? pend.part1 : pend.part0;
+      for (int c2 = 0; c2 < 8; c2 += 2) {
+        bool any_rows = false;
 #pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          const int64_t row = qrow_of(pend.item, n0 + j);
-          const float v = __uint_as_float(o[j]) * xinv[n0 + j];
-          if (prt < 0) p.o_lat[row * kR + d] = __float2bfloat16_rn(v);
-          else p.o_part[((int64_t)prt * H + row % H) * kR + d] = v;
+        for (int h = 0; h < 2; ++h) {
+          const int c = c2 + h, n0 = 32 * (c & 3);
+          const int tn = H == kRows ? 0 : n0 / kCtaRows;   // the 32 rows' query token
+          if (tn >= pend.n) continue;                       // (the same for every thread)
+          any_rows = true;
+          const bool fin = (tn ? pend.part1 : pend.part0) < 0;
+          const uint32_t tile = sbase + kOffP + (uint32_t)h * (2 * kPBytes);
+          uint32_t o[32];
+          ptx::tmem_ld_32x32b_x32(tbase + lane_addr + kColO + 32u * c, o);
+          float inv[32];
+#pragma unroll
+          for (int k = 0; k < 8; ++k)
+            asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
+                         : "=f"(inv[4 * k]), "=f"(inv[4 * k + 1]), "=f"(inv[4 * k + 2]), "=f"(inv[4 * k + 3])
+                         : "r"(sbase + kOffXinv + 4u * (n0 + 4 * k)));
+          ptx::tmem_wait_ld();
+          if (fin) {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+              const __nv_bfloat16 bv = __float2bfloat16_rn(__uint_as_float(o[j]) * inv[j]);
+              asm volatile("st.shared.b16 [%0], %1;" ::"r"(tile + (uint32_t)(j * 256 + 2 * L)),
+                           "h"(*reinterpret_cast<const unsigned short*>(&bv))
+                           : "memory");
+            }
+          } else {
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+              asm volatile("st.shared.f32 [%0], %1;" ::"r"(tile + (uint32_t)(j * 512 + 4 * L)),
+                           "f"(__uint_as_float(o[j]) * inv[j])
+                           : "memory");
+          }
         }
+        if (!any_rows) continue;
+        if (!all4_sync()) return false;
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const int c = c2 + h, lh = c >> 2, n0 = 32 * (c & 3);
+          const int tn = H == kRows ? 0 : n0 / kCtaRows;
+          if (tn >= pend.n) continue;
+          const int32_t prt = tn ? pend.part1 : pend.part0;
+          const uint32_t tile = sbase + kOffP + (uint32_t)h * (2 * kPBytes);
+          const int d0 = 256 * lh + 128 * (int)rank;   // this CTA's latent run of the half
+          if (prt < 0) {
+            // warp sw: rows 8sw..8sw+7, two rows per instruction (16 lanes x 16 B each)
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+              const int r = 8 * sw + 2 * k + (lane >> 4), piece = lane & 15;
+              uint4 v;
+              asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                           : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                           : "r"(tile + (uint32_t)(r * 256 + 16 * piece))
+                           : "memory");
+              *reinterpret_cast<uint4*>(p.o_lat + qrow_of(pend.item, n0 + r) * kR + d0 + 8 * piece) = v;
+            }
+          } else {
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+              const int r = 8 * sw + k;
+              uint4 v;
+              asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                           : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                           : "r"(tile + (uint32_t)(r * 512 + 16 * lane))
+                           : "memory");
+              const int64_t row = qrow_of(pend.item, n0 + r);
+              *reinterpret_cast<uint4*>(p.o_part + ((int64_t)prt * H + row % H) * kR + d0 + 4 * lane) = v;
+            }
+          }
+        }
+        if (!all4_sync()) return false;   // the tiles are read before the next round overwrites them
       }
       ptx::tc_fence_before();
       __syncwarp();
+      if (sw == 0 && lane == 0) DUO_TRACE(11, n_ep);
+      ++n_ep;
       if (lane == 0) arrive_read(B_O_FREE);
       pend.on = false;
       return true;
@@ -658,21 +739,20 @@ decode_2sm_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_consta
       }
       const int32_t ntok = tok < u.n ? max(u.ntok[tok], 0) : 0;
       // ------------------------------------------------ this thread's 32 scores
-      const uint32_t sb = g & 1;
-      if (!wait_all(bar(B_S_FULL + sb), (g >> 1) & 1)) { fail(); ok = false; break; }
+      if (!wait_all(bar(B_S_FULL), g & 1)) { fail(); ok = false; break; }
       ptx::tc_fence_after();
       if (sw == 0 && lane == 0) DUO_TRACE(6, g);
       float v[32];
       {
         uint32_t r[32];
-        ptx::tmem_ld_32x32b_x32(tbase + lane_addr + kColS + 32u * sb, r);
+        ptx::tmem_ld_32x32b_x32(tbase + lane_addr + kColS, r);
         ptx::tmem_wait_ld();
 #pragma unroll
         for (int t = 0; t < 32; ++t) v[t] = __uint_as_float(r[t]);
       }
       ptx::tc_fence_before();
       __syncwarp();
-      if (lane == 0) arrive_read(B_S_EMPTY + sb);
+      if (lane == 0) arrive_read(B_S_EMPTY);
       // the unit's last score MMA is done: stage the next unit's query
       if (cur.k == u.npg - 1) {
         int32_t ui = cur.ui;
@@ -739,10 +819,14 @@ decode_2sm_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_consta
       const float pmax = ptx::ex2(fmaf(mx, p.scale_log2, nz));
       const bool want_lo = pmax * kLoShare > l_part;
       // ------------------------------------------------ P to shared memory once the previous value MMAs are done
-      if (g > 0 && cur.k != 0 && !wait_all(bar(B_O_DONE), (g - 1) & 1)) { fail(); ok = false; break; }
+      // P buffer g % 2 was last read by the value MMAs of page g - 2
+      if (g >= 2 && cur.k != 0 && !wait_all(bar(B_O_DONE + (g & 1)), ((g >> 1) & 1) ^ 1)) { fail(); ok = false; break; }
       if (!wait_all(bar(B_AL_FULL + ab), (g >> 1) & 1)) { fail(); ok = false; break; }
       ptx::tc_fence_after();
       if (xflg[4 * ab] | xflg[4 * ab + 1] | xflg[4 * ab + 2] | xflg[4 * ab + 3]) {
+        // O^T is stable once page g - 1's value MMAs are done
+        if (!wait_all(bar(B_O_DONE + ((g - 1) & 1)), ((g - 1) >> 1) & 1)) { fail(); ok = false; break; }
+        ptx::tc_fence_after();
         // a moved reference: O^T[:, row] *= 2^(m_old - m_new) for every row of the pair (1 for
         // rows that kept theirs); this thread scales its two latent rows
 #pragma unroll 1
@@ -760,7 +844,7 @@ decode_2sm_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_consta
       }
       {
         // row m, tokens 32h..32h+31 = 16-byte chunks 4h..4h+3 of the 128-byte row (128-byte swizzle)
-        const uint32_t prow_s = sbase + kOffP + (uint32_t)m * 128u;
+        const uint32_t prow_s = sbase + kOffP + 2u * kPBytes * (g & 1) + (uint32_t)m * 128u;
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
           const uint32_t off = (uint32_t)(((4 * half + i) ^ (m & 7)) << 4);

@@ -178,6 +178,12 @@ int32_t head_groups_for(const mla_dims& d, int32_t q_len) {
   return decode_tc_ok(d) ? d.H / mla::tc::kHeads : 1;
 }
 
+// Work a unit costs beyond its pages, in pages, for the split planner: the SM-pair
+// kernel stages each unit's query, runs its epilogue and refills its load pipeline at the
+// unit's boundaries (measured at about six pages' time); the other kernels are planned on
+// pages alone.
+double unit_cost_pages(const mla_dims& d, int32_t q_len) { return pair_decode(d, q_len) ? 6.0 : 0.0; }
+
 // Query tokens per plan unit (consecutive tokens of one sequence).
 int32_t items_per_unit_for(const mla_dims& d, int32_t q_len) {
   return pair_decode(d, q_len) && q_len >= 2 ? mla::duo::kRows / d.H : 1;
@@ -349,31 +355,77 @@ mla_status mla_plan_splits(const int32_t* seq_lens_host, int32_t B, int32_t q_le
   };
   for (int32_t b = 0; b < B; ++b)
     for (int32_t k = 0; k < groups_per_seq; ++k) total += group_pages(b, k);
-  // Slot s covers flattened pages [s*total/S, (s+1)*total/S): page counts differ by at most one.
-  const int64_t S = std::max<int64_t>(1, std::min<int64_t>(slots_max, total));
-  auto bound = [&](int64_t s) { return s * total / S; };
   struct U { int32_t item, b, pb, pe, slot, n; };
   std::vector<U> units;
+  const int64_t S = std::max<int64_t>(1, std::min<int64_t>(slots_max, total));
   units.reserve(items + S);
-  int32_t slot = 0;
-  int64_t flat = 0;  // flattened index of the next page
-  for (int32_t b = 0; b < B; ++b) {
-    for (int32_t k = 0; k < groups_per_seq; ++k) {
-      const int32_t it = b * q_len + k * ipu;
-      const int32_t n = std::min(ipu, q_len - k * ipu);
-      int32_t left = group_pages(b, k), pb = 0;
-      if (left == 0) {
-        units.push_back({it, b, 0, 0, slot, n});
-        continue;
+  const double cost = unit_cost_pages(d, q_len);
+  if (cost <= 0.0) {
+    // Slot s covers flattened pages [s*total/S, (s+1)*total/S): page counts differ by at most one.
+    auto bound = [&](int64_t s) { return s * total / S; };
+    int32_t slot = 0;
+    int64_t flat = 0;  // flattened index of the next page
+    for (int32_t b = 0; b < B; ++b) {
+      for (int32_t k = 0; k < groups_per_seq; ++k) {
+        const int32_t it = b * q_len + k * ipu;
+        const int32_t n = std::min(ipu, q_len - k * ipu);
+        int32_t left = group_pages(b, k), pb = 0;
+        if (left == 0) {
+          units.push_back({it, b, 0, 0, slot, n});
+          continue;
+        }
+        while (left > 0) {
+          while (slot + 1 < S && flat >= bound(slot + 1)) ++slot;
+          const int64_t room = (slot + 1 < S) ? bound(slot + 1) - flat : left;
+          const int32_t take = (int32_t)std::min<int64_t>(left, room);
+          units.push_back({it, b, pb, pb + take, slot, n});
+          pb += take;
+          left -= take;
+          flat += take;
+        }
       }
-      while (left > 0) {
-        while (slot + 1 < S && flat >= bound(slot + 1)) ++slot;
-        const int64_t room = (slot + 1 < S) ? bound(slot + 1) - flat : left;
-        const int32_t take = (int32_t)std::min<int64_t>(left, room);
-        units.push_back({it, b, pb, pb + take, slot, n});
-        pb += take;
-        left -= take;
-        flat += take;
+    }
+  } else {
+    // Every unit also costs `cost` pages of work (its query, its epilogue, a pipeline
+    // refill): slots get equal shares of pages + cost * units, assuming one unit per
+    // non-empty group plus one more for each slot boundary that cuts a group.
+    int64_t groups = 0;
+    for (int32_t b = 0; b < B; ++b)
+      for (int32_t k = 0; k < groups_per_seq; ++k) groups += group_pages(b, k) > 0;
+    const double share = ((double)total + cost * (double)(groups + S - 1)) / (double)S;
+    // slot s ends where the work assigned so far reaches (s + 1) * share
+    int32_t slot = 0;
+    bool slot_used = false;
+    double acc = 0.0;
+    for (int32_t b = 0; b < B; ++b) {
+      for (int32_t k = 0; k < groups_per_seq; ++k) {
+        const int32_t it = b * q_len + k * ipu;
+        const int32_t n = std::min(ipu, q_len - k * ipu);
+        int32_t left = group_pages(b, k), pb = 0;
+        if (left == 0) {
+          units.push_back({it, b, 0, 0, slot, n});
+          continue;
+        }
+        while (left > 0) {
+          const bool last_slot = slot + 1 >= S;
+          // no room left here even for one page: the next slot
+          if (!last_slot && slot_used && acc + cost + 1.0 > (slot + 1) * share + 0.5) {
+            ++slot;
+            slot_used = false;
+            continue;
+          }
+          const double room = (slot + 1) * share - acc - cost;
+          const int32_t take = last_slot ? left : (int32_t)std::min<double>(left, std::max(1.0, std::floor(room + 0.5)));
+          units.push_back({it, b, pb, pb + take, slot, n});
+          slot_used = true;
+          pb += take;
+          left -= take;
+          acc += cost + take;
+          if (!last_slot && acc >= (slot + 1) * share - 0.5) {
+            ++slot;
+            slot_used = false;
+          }
+        }
       }
     }
   }

@@ -107,16 +107,45 @@ def test_plan_covers_every_visible_page_once(q_len, sms, H):
     assert parts_seen == set(range(info.num_parts))
 
 
-def test_plan_balances_pages_over_slots():
-    lens = np.full(64, 4096, np.int32)
-    plan, info = mla.mla_plan_splits(lens, 64, 1, 64, dims(), 148)
+UNIT_COST = 6.0   # pages of work the SM-pair kernel spends per unit beyond its pages
+
+
+def slot_loads(plan, info):
     p = parse_plan(plan)
-    per = np.zeros(info.num_slots, np.int64)
+    pages = np.zeros(info.num_slots, np.int64)
+    units = np.zeros(info.num_slots, np.int64)
     for u in p["units"]:
-        per[u[5]] += u[3] - u[2]
-    assert per.sum() == 64 * 64
-    assert per.max() <= math.ceil(4096 / 74)
-    assert info.num_slots == 74     # one SM pair per slot
+        pages[u[5]] += u[3] - u[2]
+        units[u[5]] += u[3] > u[2]
+    return pages, units
+
+
+@pytest.mark.parametrize("lens", [np.full(64, 4096, np.int32),
+                                  np.random.default_rng(0).integers(512, 16385, 128).astype(np.int32)])
+def test_plan_balances_pages_and_units_over_pair_slots(lens):
+    """SM-pair plans (H=64/128): one slot per pair of SMs, and every slot's work, its
+    pages plus a fixed cost per unit, within one unit's cost (and a page) of an equal share."""
+    H = 64 if lens[0] == 4096 else 128
+    plan, info = mla.mla_plan_splits(lens, len(lens), 1, 256, dims(H=H), 148)
+    pages, units = slot_loads(plan, info)
+    total = int(np.sum((lens + 63) // 64))
+    assert pages.sum() == total
+    assert info.num_slots == 74
+    groups = len(lens)
+    share = (total + UNIT_COST * (groups + 74 - 1)) / 74
+    work = pages + UNIT_COST * units
+    assert work.max() <= share + UNIT_COST + 1, (work.max(), share)
+
+
+def test_plan_balances_pages_for_the_single_cta_kernel():
+    """Other head counts (one CTA per 64 heads) are planned on pages alone: slots differ
+    by at most one page."""
+    lens = np.full(64, 4096, np.int32)
+    plan, info = mla.mla_plan_splits(lens, 64, 1, 64, dims(H=192), 148)
+    pages, _ = slot_loads(plan, info)
+    assert pages.sum() == 64 * 64
+    assert info.num_slots == 148 // 3
+    assert pages.max() - pages.min() <= 1
 
 
 def test_plan_rejects_too_long_sequences_and_small_buffers():

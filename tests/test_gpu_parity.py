@@ -155,7 +155,8 @@ def attention_case(policy, H, q_len, lens, sms, noise=0.0):
 @pytest.mark.parametrize("H", [64, 128])
 @pytest.mark.parametrize("sms", [148, 9])
 def test_decode_attention_matches_oracle(policy, H, sms):
-    step = attention_case(policy, H, 1, SMALL_LENS, sms)
+    # with few slots a 2000-token sequence is cut between slots: partial outputs + combine
+    step = attention_case(policy, H, 1, SMALL_LENS + ([2000] if sms == 9 else []), sms)
     if sms == 9:
         assert step.info.num_parts > 0   # the combine ran
 
