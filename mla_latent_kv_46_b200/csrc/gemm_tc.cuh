@@ -5,12 +5,14 @@
 //   outproj  out[t][h][:]   = o_lat[t][h][:] @ W_UV[h]^T    A [T x R] (K-major),
 //            B = W_UV[h] [Dv x R]: N rows, K = R contiguous (K-major)
 //
-// One CTA computes a 128-row tile of tokens for one head: TMA streams 64-wide K blocks
-// of A and B into a ring of stages (128-byte swizzle), one elected lane issues
-// tcgen05.mma (M=128, N <= 256 per instruction, fp32 accumulators in TMEM), and the four
-// warps read the accumulators back with tcgen05.ld (warp w owns rows 32w..32w+31) and
-// store bf16 rows. Both projections read their weights once per token tile; at decode
-// sizes (T <= 128) they are bound by the weight bytes.
+// One CTA computes a 128-row tile of tokens x N output columns (block blockIdx.z of the
+// output row) for one head: TMA streams 64-wide K blocks of A and B into a ring of stages
+// (128-byte swizzle), one elected lane issues tcgen05.mma (M=128, N <= 256 per
+// instruction, fp32 accumulators in TMEM), and the four warps read the accumulators back
+// with tcgen05.ld (warp w owns rows 32w..32w+31) and store bf16 rows. Both projections
+// read their weights once per token tile; at decode sizes (T <= 128) they are bound by
+// the weight bytes, so the absorb's 512 output columns are cut into blocks to spread the
+// weight reads over more CTAs than there are heads.
 #pragma once
 
 #include "common.cuh"
@@ -23,8 +25,9 @@ constexpr int kM = 128;           // token rows per CTA
 constexpr int kKB = 64;           // K elements per block (one 128-byte swizzle row)
 
 struct Params {
-  __nv_bfloat16* out;             // [T][H][N]
+  __nv_bfloat16* out;             // [T][H][n_total]
   int32_t T, H;
+  int32_t n_total;                // output row width (N x gridDim.z)
   uint64_t timeout_ns;
 };
 
@@ -53,7 +56,7 @@ proj_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
   const uint32_t tmem_holder = sbase + C::kOffBar + 8u * (2 * STAGES + 2);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kOffBar + 8 * (2 * STAGES + 3));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int h = blockIdx.x, m0 = blockIdx.y * kM;
+  const int h = blockIdx.x, m0 = blockIdx.y * kM, n0 = blockIdx.z * N;
 
   if (threadIdx.x == 0) {
     *abort_flag = 0;
@@ -96,12 +99,12 @@ proj_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
           // B block: 64 K rows (head h's rows kb*64..) x N columns, as N/64 boxes
 #pragma unroll
           for (int j = 0; j < N / 64; ++j)
-            ptx::tma_load_2d(sb + j * (64 * 128), &tmB, bar(s), 64 * j, h * (KBLK * kKB) + kb * kKB);
+            ptx::tma_load_2d(sb + j * (64 * 128), &tmB, bar(s), n0 + 64 * j, h * (KBLK * kKB) + kb * kKB);
         } else {
           // B block: N rows (head h's rows) x 64 K columns
 #pragma unroll
           for (int j = 0; j < N / 64; ++j)
-            ptx::tma_load_2d(sb + j * (64 * 128), &tmB, bar(s), kb * kKB, h * N + 64 * j);
+            ptx::tma_load_2d(sb + j * (64 * 128), &tmB, bar(s), kb * kKB, h * p.n_total + n0 + 64 * j);
         }
       }
     }
@@ -165,7 +168,7 @@ proj_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
           __nv_bfloat162 b2 = __floats2bfloat162_rn(v[2 * j], v[2 * j + 1]);
           w[j] = *reinterpret_cast<uint32_t*>(&b2);
         }
-        uint4* dst = reinterpret_cast<uint4*>(p.out + ((int64_t)row * p.H + h) * N + c);
+        uint4* dst = reinterpret_cast<uint4*>(p.out + ((int64_t)row * p.H + h) * p.n_total + n0 + c);
         dst[0] = pk[0];
         dst[1] = pk[1];
       }

@@ -146,7 +146,7 @@ bool outproj_tc_ok(const mla_dims& d) { return d.dtype == MLA_BF16 && d.R == 512
 
 template <int KBLK, int N, bool B_MN, int STAGES>
 mla_status launch_proj(const void* A, const void* Bw, void* out, int32_t T, const mla_dims& d, int32_t a_cols,
-                       int32_t b_rows, int32_t b_cols, cudaStream_t st, const char* what) {
+                       int32_t b_rows, int32_t b_cols, int32_t n_total, cudaStream_t st, const char* what) {
   using C = mla::gemm::Cfg<KBLK, N, B_MN, STAGES>;
   CUtensorMap ta, tb;
   if (mla_status s = make_map_2d(&ta, A, (uint64_t)d.H * a_cols, (uint64_t)T, (uint64_t)d.H * a_cols * 2, 128))
@@ -158,8 +158,9 @@ mla_status launch_proj(const void* A, const void* Bw, void* out, int32_t T, cons
   p.out = static_cast<__nv_bfloat16*>(out);
   p.T = T;
   p.H = d.H;
+  p.n_total = n_total;
   p.timeout_ns = g_timeout_ns.load();
-  const dim3 grid(d.H, (T + mla::gemm::kM - 1) / mla::gemm::kM);
+  const dim3 grid(d.H, (T + mla::gemm::kM - 1) / mla::gemm::kM, n_total / N);
   kern<<<grid, 128, C::kSmemBytes, st>>>(ta, tb, p);
   return launch_check(what);
 }
@@ -243,6 +244,15 @@ mla_status mla_cache_append(void* kv_cache, const int32_t* block_table, const in
   if (B == 0) return ok();
   if (!kv_cache || !block_table || !seq_lens || !new_ckr) return fail(MLA_ERR_INVALID, "null pointer");
   const int32_t row = d.R + d.Dr;
+  const size_t row_bytes = (size_t)row * (d.dtype == MLA_BF16 ? 2 : 4);
+  if (row_bytes % 16 == 0 && reinterpret_cast<uintptr_t>(kv_cache) % 16 == 0 &&
+      reinterpret_cast<uintptr_t>(new_ckr) % 16 == 0) {
+    const int32_t items = B * q_len;
+    mla::simt::cache_append_vec_kernel<<<(items + 3) / 4, 128, 0, as_stream(stream)>>>(
+        static_cast<uint4*>(kv_cache), block_table, seq_lens, static_cast<const uint4*>(new_ckr), items, q_len,
+        max_pages, num_pages, (int32_t)(row_bytes / 16), d.page_size);
+    return launch_check("cache_append");
+  }
   const dim3 grid(B * q_len);
   if (d.dtype == MLA_BF16)
     mla::simt::cache_append_kernel<__nv_bfloat16><<<grid, 128, 0, as_stream(stream)>>>(
@@ -266,7 +276,7 @@ mla_status mla_absorb_q(const void* q_nope, const void* W_UK, void* q_lat, int32
   if (pol == MLA_POLICY_TCGEN05 && !absorb_tc_ok(d))
     return fail(MLA_ERR_UNSUPPORTED, "tensor-core absorb needs bf16, Dn=128, R=512");
   if (pol != MLA_POLICY_SIMT && absorb_tc_ok(d))
-    return launch_proj<2, 512, true, 2>(q_nope, W_UK, q_lat, T, d, d.Dn, d.H * d.Dn, d.R, as_stream(stream),
+    return launch_proj<2, 128, true, 2>(q_nope, W_UK, q_lat, T, d, d.Dn, d.H * d.Dn, d.R, d.R, as_stream(stream),
                                         "absorb_q (tcgen05)");
   const dim3 grid((d.R + 127) / 128, d.H, (T + mla::simt::kTT - 1) / mla::simt::kTT);
   const size_t smem = sizeof(float) * mla::simt::kTT * d.Dn;
@@ -293,7 +303,7 @@ mla_status mla_out_proj(const void* o_lat, const void* W_UV, void* out, int32_t 
   if (pol == MLA_POLICY_TCGEN05 && !outproj_tc_ok(d))
     return fail(MLA_ERR_UNSUPPORTED, "tensor-core output projection needs bf16, R=512, Dv=128");
   if (pol != MLA_POLICY_SIMT && outproj_tc_ok(d))
-    return launch_proj<8, 128, false, 4>(o_lat, W_UV, out, T, d, d.R, d.H * d.Dv, d.R, as_stream(stream),
+    return launch_proj<8, 128, false, 6>(o_lat, W_UV, out, T, d, d.R, d.H * d.Dv, d.R, d.Dv, as_stream(stream),
                                          "out_proj (tcgen05)");
   const dim3 grid(d.H, (T + mla::simt::kTT - 1) / mla::simt::kTT);
   const size_t smem = sizeof(float) * mla::simt::kTT * d.R;

@@ -9,7 +9,34 @@ namespace mla {
 namespace simt {
 
 // ------------------------------------------------------------------ a2: cache append
-// One block per new row: kv[page][pos % ps][:] = new_ckr[b*q_len + i][:].
+// One warp per new row, 16-byte copies (rows whose byte size is a multiple of 16):
+// kv[page][pos % ps][:] = new_ckr[b*q_len + i][:].
+__global__ void __launch_bounds__(128) cache_append_vec_kernel(uint4* __restrict__ kv, const int32_t* __restrict__ block_table,
+                                                               const int32_t* __restrict__ seq_lens,
+                                                               const uint4* __restrict__ new_ckr, int32_t items,
+                                                               int32_t q_len, int32_t max_pages, int32_t num_pages,
+                                                               int32_t row_vec, int32_t page_size) {
+  const int32_t item = blockIdx.x * 4 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
+  if (item >= items) return;
+  const int32_t b = item / q_len, i = item % q_len;
+  const int32_t pos = seq_lens[b] - q_len + i;
+  if (pos < 0) return;
+  const int32_t pidx = pos / page_size;
+  if (pidx >= max_pages) {
+    if (lane == 0) raise_status(kStatusBadPage);
+    return;
+  }
+  const int32_t page = block_table[(int64_t)b * max_pages + pidx];
+  if (page < 0 || page >= num_pages) {
+    if (lane == 0) raise_status(kStatusBadPage);
+    return;
+  }
+  uint4* dst = kv + ((int64_t)page * page_size + pos % page_size) * row_vec;
+  const uint4* src = new_ckr + (int64_t)item * row_vec;
+  for (int32_t e = lane; e < row_vec; e += 32) dst[e] = src[e];
+}
+
+// One block per new row, element copies (any row width).
 template <typename T>
 __global__ void cache_append_kernel(T* __restrict__ kv, const int32_t* __restrict__ block_table,
                                     const int32_t* __restrict__ seq_lens,
@@ -243,22 +270,33 @@ __global__ void __launch_bounds__(128) combine_vec_kernel(const int32_t* __restr
 #pragma unroll
   for (int k = 0; k < 4; ++k) acc[k] = make_float4(0.f, 0.f, 0.f, 0.f);
   float tot = 0.f;
-  for (int32_t s = 0; s < np; ++s) {
-    const float z = lse_part[(int64_t)(first + s) * H + h];
-    const float wgt = (M == -CUDART_INF_F) ? 0.f : expf(z - M);
-    tot += wgt;
-    if (wgt > 0.f) {
-      const float4* src = reinterpret_cast<const float4*>(o_part + ((int64_t)(first + s) * H + h) * R);
+  // parts two at a time, so that each lane has eight 16-byte loads in flight (a part with
+  // no visible token holds zeros and weighs 0)
+  for (int32_t s = 0; s < np; s += 2) {
+    const bool two = s + 1 < np;
+    float wgt[2];
+    float4 v[2][4];
+#pragma unroll
+    for (int q = 0; q < 2; ++q) {
+      const int32_t ps = first + s + (q && two ? 1 : 0);
+      const float z = lse_part[(int64_t)ps * H + h];
+      wgt[q] = (q && !two) || M == -CUDART_INF_F ? 0.f : expf(z - M);
+      const float4* src = reinterpret_cast<const float4*>(o_part + ((int64_t)ps * H + h) * R);
 #pragma unroll
       for (int k = 0; k < 4; ++k) {
         const int32_t i = lane + 32 * k;
-        if (i < nv) {
-          const float4 v = __ldcs(src + i);
-          acc[k].x = fmaf(wgt, v.x, acc[k].x);
-          acc[k].y = fmaf(wgt, v.y, acc[k].y);
-          acc[k].z = fmaf(wgt, v.z, acc[k].z);
-          acc[k].w = fmaf(wgt, v.w, acc[k].w);
-        }
+        v[q][k] = i < nv ? __ldcs(src + i) : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+    }
+#pragma unroll
+    for (int q = 0; q < 2; ++q) {
+      tot += wgt[q];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        acc[k].x = fmaf(wgt[q], v[q][k].x, acc[k].x);
+        acc[k].y = fmaf(wgt[q], v[q][k].y, acc[k].y);
+        acc[k].z = fmaf(wgt[q], v[q][k].z, acc[k].z);
+        acc[k].w = fmaf(wgt[q], v[q][k].w, acc[k].w);
       }
     }
   }

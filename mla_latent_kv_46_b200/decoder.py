@@ -53,6 +53,9 @@ class DecodeStep:
         self.o_lat = torch.empty((self.T, H, R), dtype=dt, device=d)
         self.lse = torch.empty((self.T, H), dtype=torch.float32, device=d)
         self.out = torch.empty((self.T, H, Dv), dtype=dt, device=d)
+        # the cache append and the query absorption are independent: the append runs on
+        # this side stream beside the absorption, and the decode waits for both
+        self.side = torch.cuda.Stream(device=d)
         self.replan(self.seq_lens_host)
 
     def replan(self, seq_lens_host: np.ndarray, stream=None):
@@ -85,11 +88,20 @@ class DecodeStep:
     def project(self, stream=None):
         mla.mla_out_proj(self.o_lat, self.W_UV, self.out, self.T, self.dims, stream)
 
+    def append_and_absorb(self, stream=None):
+        """a2 on the side stream beside a1 on `stream`; `stream` then waits for both."""
+        s = stream or torch.cuda.current_stream(self.device)
+        self.side.wait_stream(s)               # the step's inputs are in place
+        self.append(self.side)
+        self.absorb(s)
+        s.wait_stream(self.side)
+
     def run(self, append=True, stream=None):
-        """The whole step on device-resident inputs: a2, a1, a3-a5, a6, a7."""
+        """The whole step on device-resident inputs: a2 (beside a1), a1, a3-a5, a6, a7."""
         if append:
-            self.append(stream)
-        self.absorb(stream)
+            self.append_and_absorb(stream)
+        else:
+            self.absorb(stream)
         self.attend(stream)
         self.combine(stream)
         self.project(stream)
