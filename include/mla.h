@@ -52,7 +52,7 @@
 extern "C" {
 #endif
 
-#define MLA_ABI_VERSION 1
+#define MLA_ABI_VERSION 2
 
 typedef enum {
   MLA_OK = 0,
@@ -92,6 +92,8 @@ typedef struct {
   int32_t num_parts;    /* units whose result is partial and needs mla_combine */
   int32_t head_groups;  /* heads are processed in groups of H / head_groups */
   int32_t plan_words;   /* int32 words of the plan buffer in use */
+  int32_t max_pages;    /* block_table row length the plan's page ranges were cut for;
+                           mla_decode_attn(_noalloc) rejects a call with another one */
 } mla_plan_info;
 
 int32_t mla_abi_version(void);
@@ -105,18 +107,21 @@ mla_status mla_set_policy(int32_t policy);
 /* Bound, in nanoseconds, on every wait inside a kernel (default 2e9). */
 mla_status mla_set_wait_timeout_ns(uint64_t ns);
 
-/* Testing hook for the failure path of the tensor-core decode kernels: while set
+/* TEST-ONLY hook for the failure path of the tensor-core decode kernels: while set
  * (ordinal >= 0), the first CTA of each mla_decode_attn launch skips the shared-memory
  * load of its page with that ordinal (0 = its first page), so the waits on that page
  * run out after the wait bound (mla_set_wait_timeout_ns), the kernel stops, and
  * mla_check_status then reports MLA_ERR_TIMEOUT; the outputs of that launch are
  * undefined. A negative ordinal switches the hook off (the default). Process-wide;
- * always returns MLA_OK. Nothing in the pages corresponds to it. */
+ * always returns MLA_OK. Nothing in the pages corresponds to it. Production code
+ * never sets it: while it is set, mla_check_status returns MLA_ERR_INVALID even
+ * when no kernel reported a problem, so a hook left on cannot go unnoticed. */
 mla_status mla_debug_drop_page_load(int32_t ordinal);
 
 /* Synchronises `stream`, then reads and clears the device status word of the
  * current device: MLA_OK, MLA_ERR_TIMEOUT (a bounded wait ran out) or
- * MLA_ERR_INVALID (a page id outside the pool was skipped). */
+ * MLA_ERR_INVALID (a page id outside the pool was skipped, or the test-only
+ * mla_debug_drop_page_load hook is still set; mla_last_error says which). */
 mla_status mla_check_status(void* stream);
 
 /* ---------------------------------------------------------------- a2: cache append
@@ -139,6 +144,12 @@ mla_status mla_absorb_q(const void* q_nope, const void* W_UK, void* q_lat, int32
                         void* stream);
 
 /* ---------------------------------------------------------------- split planning (host)
+ * The pages fix what a decode step computes, not how the work of a batch of
+ * sequences is spread over the GPU. Splitting a query's cached tokens into ranges
+ * and merging the ranges' results exactly by their log-sum-exp is the flash-decoding
+ * reading of the softmax: softmax over a union of token sets equals the
+ * lse-weighted mix of the softmaxes over each set (the merge identity written out
+ * in mla_combine below). The plan, its workspace and the combine serve that split.
  * Upper bound, in int32 words, of the plan buffer for these sizes. */
 size_t mla_plan_capacity(int32_t B, int32_t q_len, int32_t num_sms);
 
@@ -154,7 +165,9 @@ mla_status mla_plan_splits(const int32_t* seq_lens_host, int32_t B, int32_t q_le
                            mla_plan_info* info);
 
 /* Bytes of workspace mla_decode_attn / mla_combine need for this plan: fp32
- * partials [num_parts][H][R] followed by fp32 lse [num_parts][H]. */
+ * partials [num_parts][H][R] followed by fp32 lse [num_parts][H] (one partial
+ * o_lat and lse per unit of a split query, the inputs of the merge identity
+ * above). Returns 0 for a null info or invalid dims. */
 size_t mla_workspace_size(const mla_plan_info* info, mla_dims d);
 
 /* ---------------------------------------------------------------- a3-a5: decode attention
@@ -176,7 +189,10 @@ mla_status mla_decode_attn(const void* q_lat, const void* q_rope, const void* kv
                            void* stream);
 
 /* ---------------------------------------------------------------- a6: split-KV combine
- * For each query whose work was split: m = max_s lse_s, w_s = exp(lse_s - m),
+ * The exact merge of softmax results over disjoint token sets (the pages' attention,
+ * GatedMLA "Observe logits, then compute causal attention", is one softmax over all
+ * visible tokens; the merge restores it from the per-range results):
+ * for each query whose work was split: m = max_s lse_s, w_s = exp(lse_s - m),
  * o_lat = sum_s w_s o_s / sum_s w_s, lse = m + log sum_s w_s (parts with
  * lse = -inf weigh 0). Writes o_lat (dtype) and lse (fp32, may be NULL) of those
  * queries only. A no-op launch-free call when info->num_parts == 0.              */
@@ -193,8 +209,8 @@ mla_status mla_out_proj(const void* o_lat, const void* W_UV, void* out, int32_t 
 
 /* ---------------------------------------------------------------- allocation-free decode
  * The pages describe no counterpart of this call; it exists for callers that cannot
- * allocate device memory: code running inside a CUDA-graph capture or another
- * framework's fixed memory pool, or a host environment with no allocator exposed.
+ * allocate device memory: code inside another framework's fixed memory pool, or a
+ * host environment with no allocator exposed.
  * It computes exactly what mla_decode_attn followed by mla_combine computes, final
  * o_lat and lse for every query, but keeps the partial outputs of split queries in
  * a scratch array that the library owns: a file-scope device array of 48 MiB
@@ -204,9 +220,10 @@ mla_status mla_out_proj(const void* o_lat, const void* W_UV, void* out, int32_t 
  *  - A plan whose partials need more than 48 MiB (mla_workspace_size) is rejected
  *    with MLA_ERR_WORKSPACE before any launch: fewer num_sms or fewer splits, or
  *    mla_decode_attn with a caller workspace, serve those.
- *  - The first call on each device looks up the array's device address
- *    (cudaGetSymbolAddress) with that device current; make that first call before
- *    any stream capture.
+ *  - The first call in each CUDA context looks up the array's device address
+ *    (cudaGetSymbolAddress) in that context. The address is kept per context (its
+ *    driver context id), so a context that is destroyed and created again (for
+ *    instance after cudaDeviceReset) gets a fresh lookup, never a stale address.
  *  - Every call on a device shares the one array, which keeps the last call's
  *    contents. Nothing in it has to start at zero: each partial is written before it
  *    is read in the same call. Calls that overlap on the GPU (concurrent streams)

@@ -47,7 +47,8 @@ class Dims(ctypes.Structure):
 
 class PlanInfo(ctypes.Structure):
     _fields_ = [("num_items", ctypes.c_int32), ("num_units", ctypes.c_int32), ("num_slots", ctypes.c_int32),
-                ("num_parts", ctypes.c_int32), ("head_groups", ctypes.c_int32), ("plan_words", ctypes.c_int32)]
+                ("num_parts", ctypes.c_int32), ("head_groups", ctypes.c_int32), ("plan_words", ctypes.c_int32),
+                ("max_pages", ctypes.c_int32)]
 
 
 def _load():

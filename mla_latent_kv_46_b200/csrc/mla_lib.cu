@@ -230,6 +230,9 @@ mla_status mla_check_status(void* stream) {
   if (v & mla::kStatusTimeout) return fail(MLA_ERR_TIMEOUT, "a kernel wait ran out (status 0x%x)", v);
   if (v & mla::kStatusBadPage)
     return fail(MLA_ERR_INVALID, "a block_table entry was outside [0, num_pages) (status 0x%x)", v);
+  if (g_drop_load.load() >= 0)
+    return fail(MLA_ERR_INVALID, "the test-only mla_debug_drop_page_load hook is still set (ordinal %d)",
+                g_drop_load.load());
   return ok();
 }
 
@@ -500,6 +503,7 @@ mla_status mla_plan_splits(const int32_t* seq_lens_host, int32_t B, int32_t q_le
   info->num_parts = parts;
   info->head_groups = G;
   info->plan_words = (int32_t)words;
+  info->max_pages = max_pages;
   return ok();
 }
 
@@ -526,10 +530,14 @@ static mla_status split_workspace(const mla_plan_info* info, const mla_dims& d, 
   return MLA_OK;
 }
 
-static mla_status check_info(const mla_plan_info* info, int32_t B, int32_t q_len, const mla_dims& d) {
+static mla_status check_info(const mla_plan_info* info, int32_t B, int32_t q_len, int32_t max_pages,
+                             const mla_dims& d) {
   if (!info) return fail(MLA_ERR_INVALID, "null plan info");
   if (info->num_items != B * q_len)
     return fail(MLA_ERR_INVALID, "plan covers %d query tokens, call has %d", info->num_items, B * q_len);
+  // the plan's page ranges index block_table rows of the length it was cut for
+  if (info->max_pages != max_pages)
+    return fail(MLA_ERR_INVALID, "plan was made for max_pages=%d, call has %d", info->max_pages, max_pages);
   if (info->head_groups != head_groups_for(d, q_len))
     return fail(MLA_ERR_INVALID,
                 "plan was made for %d CTAs per slot, these dims, q_len and kernel policy need %d (plan "
@@ -550,7 +558,7 @@ mla_status mla_decode_attn(const void* q_lat, const void* q_rope, const void* kv
     return fail(MLA_ERR_INVALID, "bad sizes B=%d q_len=%d max_pages=%d num_pages=%d", B, q_len, max_pages,
                 num_pages);
   if (!(scale > 0.f) || !std::isfinite(scale)) return fail(MLA_ERR_INVALID, "scale must be positive");
-  if (mla_status s = check_info(info, B, q_len, d)) return s;
+  if (mla_status s = check_info(info, B, q_len, max_pages, d)) return s;
   if (B == 0 || info->num_units == 0) return ok();
   if (!q_lat || !q_rope || !kv_cache || !block_table || !seq_lens || !plan_dev || !o_lat)
     return fail(MLA_ERR_INVALID, "null pointer");
@@ -670,29 +678,54 @@ mla_status mla_combine(const int32_t* plan_dev, const mla_plan_info* info, const
 // Scratch for the partial outputs of mla_decode_attn_noalloc. It is a file-scope
 // device array, so every GPU that loads this library holds kNoAllocScratchBytes
 // until the process exits. Host code must not use the symbol as an address: the
-// device address comes from cudaGetSymbolAddress, looked up once per device.
+// device address comes from cudaGetSymbolAddress, looked up once per CUDA context
+// and kept under the context's driver id (unique for the life of the process), so a
+// context created again after a reset is looked up afresh.
 }  // extern "C"
 
 namespace {
 constexpr size_t kNoAllocScratchBytes = size_t(48) << 20;
-constexpr int kMaxDevices = 64;
+typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
+typedef CUresult (*CtxGetIdFn)(CUcontext, unsigned long long*);
 std::mutex g_noalloc_mu;
-void* g_noalloc_ptr[kMaxDevices] = {};
+std::vector<std::pair<unsigned long long, void*>> g_noalloc_ptr;   // (context id, scratch address)
+
+template <typename Fn>
+Fn driver_fn(const char* name) {
+  void* p = nullptr;
+  cudaDriverEntryPointQueryResult q;
+  if (cudaGetDriverEntryPoint(name, &p, cudaEnableDefault, &q) == cudaSuccess && q == cudaDriverEntryPointSuccess)
+    return reinterpret_cast<Fn>(p);
+  return nullptr;
+}
 }  // namespace
 
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
 
 static mla_status noalloc_scratch(void** out) {
-  int dev = 0;
-  MLA_CUDA_TRY(cudaGetDevice(&dev));
-  if (dev < 0 || dev >= kMaxDevices) return fail(MLA_ERR_UNSUPPORTED, "device %d out of range", dev);
-  std::lock_guard<std::mutex> lk(g_noalloc_mu);
-  if (!g_noalloc_ptr[dev]) {
+  static const CtxGetCurrentFn get_current = driver_fn<CtxGetCurrentFn>("cuCtxGetCurrent");
+  static const CtxGetIdFn get_id = driver_fn<CtxGetIdFn>("cuCtxGetId");
+  if (!get_current || !get_id) return fail(MLA_ERR_CUDA, "cuCtxGetCurrent / cuCtxGetId not available");
+  CUcontext ctx = nullptr;
+  if (get_current(&ctx) != CUDA_SUCCESS || !ctx) {
+    // no context yet on this thread: the runtime makes the device's primary context
+    // current on its first call that needs one
     void* p = nullptr;
     MLA_CUDA_TRY(cudaGetSymbolAddress(&p, g_noalloc_scratch));
-    g_noalloc_ptr[dev] = p;
+    if (get_current(&ctx) != CUDA_SUCCESS || !ctx) return fail(MLA_ERR_CUDA, "no current CUDA context");
   }
-  *out = g_noalloc_ptr[dev];
+  unsigned long long id = 0;
+  if (get_id(ctx, &id) != CUDA_SUCCESS) return fail(MLA_ERR_CUDA, "cuCtxGetId failed");
+  std::lock_guard<std::mutex> lk(g_noalloc_mu);
+  for (const auto& e : g_noalloc_ptr)
+    if (e.first == id) {
+      *out = e.second;
+      return MLA_OK;
+    }
+  void* p = nullptr;
+  MLA_CUDA_TRY(cudaGetSymbolAddress(&p, g_noalloc_scratch));
+  g_noalloc_ptr.emplace_back(id, p);
+  *out = p;
   return MLA_OK;
 }
 
@@ -704,7 +737,7 @@ mla_status mla_decode_attn_noalloc(const void* q_lat, const void* q_rope, const 
                                    const int32_t* plan_dev, const mla_plan_info* info, void* o_lat,
                                    float* lse, mla_dims d, void* stream) {
   if (mla_status s = check_dims(d)) return s;
-  if (mla_status s = check_info(info, B, q_len, d)) return s;
+  if (mla_status s = check_info(info, B, q_len, max_pages, d)) return s;
   const size_t need = mla_workspace_size(info, d);
   if (need > kNoAllocScratchBytes)
     return fail(MLA_ERR_WORKSPACE,

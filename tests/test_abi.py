@@ -34,7 +34,7 @@ def test_library_exports_every_declared_symbol():
 
 
 def test_abi_version_and_error_text():
-    assert mla.mla_abi_version() == 1
+    assert mla.mla_abi_version() == 2
     with pytest.raises(mla.MlaError) as e:
         mla.mla_set_policy(7)
     assert e.value.status == mla._binding.MLA_ERR_INVALID
@@ -206,8 +206,28 @@ def test_bf16_rounding_is_nearest_even():
 def test_noalloc_rejects_plans_beyond_its_scratch():
     """1000 partial outputs of 64 heads x 512 fp32 need 131 MB, over the 48 MiB the
     allocation-free entry point holds: refused on the host, before any launch."""
-    info = mla.PlanInfo(num_items=1, num_units=1000, num_slots=1, num_parts=1000, head_groups=2, plan_words=0)
+    info = mla.PlanInfo(num_items=1, num_units=1000, num_slots=1, num_parts=1000, head_groups=2, plan_words=0,
+                        max_pages=1)
     with pytest.raises(mla.MlaError) as e:
         mla.mla_decode_attn_noalloc(16, 16, 16, 16, 16, 1, 1, 1, 1, 0.1, 16, info, 16, None, dims(), stream=0)
     assert e.value.status == mla._binding.MLA_ERR_WORKSPACE
     assert "48" in mla.mla_last_error() or "50331648" in mla.mla_last_error()
+
+
+def test_plan_records_max_pages_and_decode_rejects_another():
+    """The plan's page ranges index block_table rows of the max_pages it was cut for;
+    a decode call with a shorter (or longer) row is refused on the host before any
+    launch, so the kernels never index past a row."""
+    d = dims(H=128)
+    lens = np.array([700, 64, 1], np.int32)
+    plan, info = mla.mla_plan_splits(lens, 3, 1, 12, d, 148)
+    assert info.max_pages == 12
+    for mp in (11, 13):
+        with pytest.raises(mla.MlaError) as e:
+            mla.mla_decode_attn(16, 16, 16, 16, 16, 3, 1, mp, 100, 0.1, 16, info, 16, None, None, 0, d,
+                                stream=0)
+        assert e.value.status == mla._binding.MLA_ERR_INVALID
+        assert "max_pages" in mla.mla_last_error()
+        with pytest.raises(mla.MlaError) as e:
+            mla.mla_decode_attn_noalloc(16, 16, 16, 16, 16, 3, 1, mp, 100, 0.1, 16, info, 16, None, d, stream=0)
+        assert "max_pages" in mla.mla_last_error()

@@ -418,6 +418,21 @@ def test_dropped_page_load_times_out_and_context_stays_usable(H, q_len):
     assert_close(host(step.o_lat), ref["o_lat"], False, "o_lat after the injected timeout")
 
 
+def test_check_status_reports_a_test_hook_left_set():
+    """The drop-page hook is test-only: while it is set, mla_check_status fails even
+    though no kernel reported anything, and passes again once it is switched off."""
+    mla.mla_check_status()
+    mla.mla_debug_drop_page_load(0)
+    try:
+        with pytest.raises(mla.MlaError) as e:
+            mla.mla_check_status()
+        assert e.value.status == mla._binding.MLA_ERR_INVALID
+        assert "mla_debug_drop_page_load" in mla.mla_last_error()
+    finally:
+        mla.mla_debug_drop_page_load(-1)
+    mla.mla_check_status()
+
+
 @pytest.mark.parametrize("name", ["deepseek_h128_b128_ragged", "causal_chunk_h64_b8_2048p256"])
 def test_decode_is_deterministic(name):
     """Two runs of the same step give bitwise equal outputs (no atomics, fixed order)."""
