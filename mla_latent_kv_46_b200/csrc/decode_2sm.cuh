@@ -91,8 +91,9 @@ constexpr int kOffQ = 0;
 constexpr int kOffQK = kOffQ + kQBytes;
 constexpr int kOffPV = kOffQK + kQKSlots * kQKSlotBytes;
 constexpr int kOffP = kOffPV + kPVSlots * kPVSlotBytes;   // two buffers of P_hi then P_lo
-constexpr int kOffBar = kOffP + 4 * kPBytes;              // 32 mbarriers
-constexpr int kOffXmax = kOffBar + 32 * 8;                // float[2][128]: row maxima of the lane halves
+constexpr int kMaxBars = 32;
+constexpr int kOffBar = kOffP + 4 * kPBytes;              // kMaxBars mbarriers
+constexpr int kOffXmax = kOffBar + kMaxBars * 8;          // float[2][128]: row maxima of the lane halves
 constexpr int kOffXl = kOffXmax + 2 * 128 * 4;            // float[128]: row sums of the lane halves
 constexpr int kOffFlag = kOffXl + 128 * 4;                // uint32[4][8] (even CTA): P_lo wanted, per tile % 4
                                                           // and softmax warp (0-3 even CTA, 4-7 odd CTA)
@@ -126,7 +127,7 @@ enum {
   B_DRAIN,
   kNumBars
 };
-static_assert(kNumBars <= 32, "barrier area");
+static_assert(kNumBars <= kMaxBars, "barrier area");
 static_assert(kQKSlots <= 3 && kPVSlots <= 2, "barrier slots");
 
 constexpr uint32_t kTmemCols = 512;
@@ -236,7 +237,8 @@ __device__ __forceinline__ int32_t page_id(const Params& p, const Unit2& u, int3
 
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 decode_2sm_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_constant__ CUtensorMap tm_q,
-                  const __grid_constant__ CUtensorMap tm_qr, const Params p) {
+                  const __grid_constant__ CUtensorMap tm_qr, const __grid_constant__ CUtensorMap tm_o,
+                  const __grid_constant__ CUtensorMap tm_op, const Params p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sbase = ptx::smem_u32(smem);
@@ -290,6 +292,8 @@ decode_2sm_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_consta
     ptx::prefetch_tmap(&tm_kv);
     ptx::prefetch_tmap(&tm_q);
     ptx::prefetch_tmap(&tm_qr);
+    ptx::prefetch_tmap(&tm_o);
+    ptx::prefetch_tmap(&tm_op);
   }
   ptx::tc_fence_before();
   __syncthreads();
@@ -335,6 +339,8 @@ decode_2sm_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_consta
       const bool drop = qk && blockIdx.x == 0 && (int32_t)g == p.drop_load;
       if (leader) {
         if (qk) {
+          // all nine boxes of the page at once (issued together, the page's rows are read
+          // from DRAM together)
           DUO_TRACE(0, g);
           if (even) ptx::mbar_arrive_expect_tx(bar(B_QK_FULL + s), 2 * kQKSlotBytes);
           if (!drop) {
@@ -360,11 +366,16 @@ decode_2sm_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_consta
       advance(p, plan, u_end, c);
       ++g;
     }
-    // The even CTA's barriers count both CTAs' loads: before the pair exits, wait (bounded)
-    // for the phases armed last, so no copy is still landing in either CTA.
-    if (even)
-      for (uint32_t k = (g >= (uint32_t)nslots ? g - nslots : 0); k < g; ++k)
-        wait_all(bar((qk ? B_QK_FULL : B_PV_FULL) + k % nslots), (k / nslots) & 1);
+    // The even CTA's barriers count both CTAs' loads: before the pair exits, wait for the
+    // phases armed last, so no copy is still landing in either CTA. These waits ignore the
+    // abort flag (copies in flight land within microseconds) and stop at the wait bound;
+    // after one runs out (a phase that cannot complete) the rest are skipped.
+    if (even) {
+      bool landed = true;
+      for (uint32_t k = (g >= (uint32_t)nslots ? g - nslots : 0); k < g && landed; ++k)
+        landed = __all_sync(0xffffffffu, ptx::mbar_wait_cluster_timed(bar((qk ? B_QK_FULL : B_PV_FULL) + k % nslots),
+                                                                      (k / nslots) & 1, p.timeout_ns));
+    }
   } else if (warp == 3) {
     // ================================================================ the query's shared-memory part
     // per unit (latent 448-511 and rope of the CTA's 64 rows), once the previous unit's
@@ -640,89 +651,67 @@ decode_2sm_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_consta
       ++n_lx;
       if (!__all_sync(0xffffffffu, got)) return false;
       if (sw == 0 && lane == 0) DUO_TRACE(14, n_ep);
-      // Two 32-row chunks of O^T per round (32 rows x this CTA's 128 latent columns of one
-      // half each): scale, stage them row-major in the idle P buffers, then write whole row
-      // segments with 16-byte stores (bf16 final rows: 256 B each, fp32 partial rows: 512 B).
+      // Each warp writes its own 32 latent columns (latent rows of its TMEM lane quarter)
+      // of each 32-row chunk of O^T: scale by 1 / l, stage the 32 x 32 block row-major in
+      // one of the warp's two tiles in the idle P buffers, and hand it to a TMA store
+      // (bf16 final rows, fp32 partial rows). The stores run in the background; a tile is
+      // restaged once the store two chunks back has read it.
+      const uint32_t tiles = sbase + kOffP + (uint32_t)sw * kPBytes;   // 2 x 4 KiB
+      uint32_t nst = 0;
 #pragma unroll 1
-      for (int c2 = 0; c2 < 8; c2 += 2) {
-        bool any_rows = false;
+      for (int c = 0; c < 8; ++c) {
+        const int lh = c >> 2, n0 = 32 * (c & 3);
+        const int tn = H == kRows ? 0 : n0 / kCtaRows;   // the 32 rows' query token
+        if (tn >= pend.n) continue;                       // (the same for every thread)
+        const int32_t prt = tn ? pend.part1 : pend.part0;
+        uint32_t o[32];
+        ptx::tmem_ld_32x32b_x32(tbase + lane_addr + kColO + 32u * c, o);
+        float inv[32];
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          const int c = c2 + h, n0 = 32 * (c & 3);
-          const int tn = H == kRows ? 0 : n0 / kCtaRows;   // the 32 rows' query token
-          if (tn >= pend.n) continue;                       // (the same for every thread)
-          any_rows = true;
-          const bool fin = (tn ? pend.part1 : pend.part0) < 0;
-          const uint32_t tile = sbase + kOffP + (uint32_t)h * (2 * kPBytes);
-          uint32_t o[32];
-          ptx::tmem_ld_32x32b_x32(tbase + lane_addr + kColO + 32u * c, o);
-          float inv[32];
+        for (int k = 0; k < 8; ++k)
+          asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
+                       : "=f"(inv[4 * k]), "=f"(inv[4 * k + 1]), "=f"(inv[4 * k + 2]), "=f"(inv[4 * k + 3])
+                       : "r"(sbase + kOffXinv + 4u * (n0 + 4 * k)));
+        if (nst >= 2 && lane == 0) ptx::bulk_wait_group_read<1>();   // the tile's previous store read it
+        ptx::tmem_wait_ld();
+        __syncwarp();
+        const uint32_t tile = tiles + (nst & 1) * (uint32_t)kPBytes / 2;
+        if (prt < 0) {
 #pragma unroll
-          for (int k = 0; k < 8; ++k)
-            asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
-                         : "=f"(inv[4 * k]), "=f"(inv[4 * k + 1]), "=f"(inv[4 * k + 2]), "=f"(inv[4 * k + 3])
-                         : "r"(sbase + kOffXinv + 4u * (n0 + 4 * k)));
-          ptx::tmem_wait_ld();
-          if (fin) {
-#pragma unroll
-            for (int j = 0; j < 32; ++j) {
-              const __nv_bfloat16 bv = __float2bfloat16_rn(__uint_as_float(o[j]) * inv[j]);
-              asm volatile("st.shared.b16 [%0], %1;" ::"r"(tile + (uint32_t)(j * 256 + 2 * L)),
-                           "h"(*reinterpret_cast<const unsigned short*>(&bv))
-                           : "memory");
-            }
-          } else {
-#pragma unroll
-            for (int j = 0; j < 32; ++j)
-              asm volatile("st.shared.f32 [%0], %1;" ::"r"(tile + (uint32_t)(j * 512 + 4 * L)),
-                           "f"(__uint_as_float(o[j]) * inv[j])
-                           : "memory");
+          for (int j = 0; j < 32; ++j) {
+            const __nv_bfloat16 bv = __float2bfloat16_rn(__uint_as_float(o[j]) * inv[j]);
+            asm volatile("st.shared.b16 [%0], %1;" ::"r"(tile + (uint32_t)(j * 64 + 2 * lane)),
+                         "h"(*reinterpret_cast<const unsigned short*>(&bv))
+                         : "memory");
           }
+        } else {
+#pragma unroll
+          for (int j = 0; j < 32; ++j)
+            asm volatile("st.shared.f32 [%0], %1;" ::"r"(tile + (uint32_t)(j * 128 + 4 * lane)),
+                         "f"(__uint_as_float(o[j]) * inv[j])
+                         : "memory");
         }
-        if (!any_rows) continue;
-        if (!all4_sync()) return false;
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          const int c = c2 + h, lh = c >> 2, n0 = 32 * (c & 3);
-          const int tn = H == kRows ? 0 : n0 / kCtaRows;
-          if (tn >= pend.n) continue;
-          const int32_t prt = tn ? pend.part1 : pend.part0;
-          const uint32_t tile = sbase + kOffP + (uint32_t)h * (2 * kPBytes);
-          const int d0 = 256 * lh + 128 * (int)rank;   // this CTA's latent run of the half
-          if (prt < 0) {
-            // warp sw: rows 8sw..8sw+7, two rows per instruction (16 lanes x 16 B each)
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-              const int r = 8 * sw + 2 * k + (lane >> 4), piece = lane & 15;
-              uint4 v;
-              asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
-                           : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-                           : "r"(tile + (uint32_t)(r * 256 + 16 * piece))
-                           : "memory");
-              *reinterpret_cast<uint4*>(p.o_lat + qrow_of(pend.item, n0 + r) * kR + d0 + 8 * piece) = v;
-            }
-          } else {
-#pragma unroll
-            for (int k = 0; k < 8; ++k) {
-              const int r = 8 * sw + k;
-              uint4 v;
-              asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
-                           : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-                           : "r"(tile + (uint32_t)(r * 512 + 16 * lane))
-                           : "memory");
-              const int64_t row = qrow_of(pend.item, n0 + r);
-              *reinterpret_cast<uint4*>(p.o_part + ((int64_t)prt * H + row % H) * kR + d0 + 4 * lane) = v;
-            }
-          }
+        ptx::fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          const int x = 256 * lh + 128 * (int)rank + 32 * q;   // this warp's latent columns
+          const int64_t row0 = qrow_of(pend.item, n0);
+          if (prt < 0) ptx::tma_store_2d(&tm_o, tile, x, (int32_t)row0);
+          else ptx::tma_store_2d(&tm_op, tile, x, (int32_t)((int64_t)prt * H + row0 % H));
+          ptx::bulk_commit_group();
         }
-        if (!all4_sync()) return false;   // the tiles are read before the next round overwrites them
+        ++nst;
       }
+      // O^T is read: the next unit's value MMAs may overwrite it
       ptx::tc_fence_before();
       __syncwarp();
       if (sw == 0 && lane == 0) DUO_TRACE(11, n_ep);
       ++n_ep;
       if (lane == 0) arrive_read(B_O_FREE);
       pend.on = false;
+      // every warp's tiles are read before P is written into those buffers again
+      if (lane == 0) ptx::bulk_wait_group_read<0>();
+      if (!all4_sync()) return false;
       return true;
     };
 
@@ -885,6 +874,7 @@ decode_2sm_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_consta
       ++g;
     }
     if (ok && pend.on && !epilogue(g - 1)) fail();
+    if (lane == 0) ptx::bulk_wait_group<0>();   // this warp's output stores are complete
   }
 
   ptx::tc_fence_before();

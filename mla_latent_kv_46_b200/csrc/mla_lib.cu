@@ -126,6 +126,25 @@ mla_status make_map_2d(CUtensorMap* m, const void* base, uint64_t cols, uint64_t
   return MLA_OK;
 }
 
+// 2-D tensor map without swizzle (boxes stored row-major in shared memory), for the
+// decode kernel's output stores: bf16 or fp32 elements, boxes of box_cols x box_rows.
+mla_status make_store_map_2d(CUtensorMap* m, const void* base, bool f32, uint64_t cols, uint64_t rows,
+                             uint64_t pitch_bytes, uint32_t box_cols, uint32_t box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return fail(MLA_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+  if (reinterpret_cast<uintptr_t>(base) % 16 != 0)
+    return fail(MLA_ERR_INVALID, "tensor base %p is not 16-byte aligned", base);
+  const cuuint64_t dims[2] = {cols, rows};
+  const cuuint64_t strides[1] = {pitch_bytes};
+  const cuuint32_t box[2] = {box_cols, box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(m, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+                  const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(MLA_ERR_CUDA, "cuTensorMapEncodeTiled (store map) failed (%d)", (int)r);
+  return MLA_OK;
+}
+
 // Per-device one-time kernel attributes (large dynamic shared memory).
 mla_status ensure_smem_attr(const void* kernel, int bytes) {
   static std::mutex mu;
@@ -599,13 +618,24 @@ mla_status mla_decode_attn(const void* q_lat, const void* q_rope, const void* kv
     if (pair_decode(d, q_len)) {
       // a pair of SMs per slot: 32-row boxes of the cache (half a page), 64-row boxes of
       // the queries (one CTA's rows)
-      CUtensorMap tk32;
+      CUtensorMap tk32, to, top;
       if (mla_status s = make_map_2d(&tk32, kv_cache, d.R + d.Dr, (uint64_t)num_pages * d.page_size,
                                      (uint64_t)(d.R + d.Dr) * 2, 32, 64))
         return s;
+      // output stores: 32 x 32 blocks of final rows (bf16) and of partial rows (fp32)
+      if (mla_status s = make_store_map_2d(&to, o_lat, false, d.R, (uint64_t)T * d.H, (uint64_t)d.R * 2, 32, 32))
+        return s;
+      if (info->num_parts > 0) {
+        if (mla_status s = make_store_map_2d(&top, o_part, true, d.R, (uint64_t)info->num_parts * d.H,
+                                             (uint64_t)d.R * 4, 32, 32))
+          return s;
+      } else {
+        top = to;   // never used: the plan has no partial outputs
+      }
       if (mla_status s = ensure_smem_attr((const void*)mla::duo::decode_2sm_kernel, mla::duo::kSmemBytes))
         return s;
-      mla::duo::decode_2sm_kernel<<<grid, mla::duo::kThreads, mla::duo::kSmemBytes, st>>>(tk32, tq, tr, p);
+      mla::duo::decode_2sm_kernel<<<grid, mla::duo::kThreads, mla::duo::kSmemBytes, st>>>(tk32, tq, tr, to, top,
+                                                                                          p);
       return launch_check("decode_attn (tcgen05, SM pair)");
     }
     mla::tc::decode_kernel<<<grid, 256, mla::tc::kSmemBytes, st>>>(tq, tr, tk, p);
