@@ -202,7 +202,10 @@ int32_t head_groups_for(const mla_dims& d, int32_t q_len) {
 // kernel stages each unit's query, runs its epilogue and refills its load pipeline at the
 // unit's boundaries (measured at about six pages' time); the other kernels are planned on
 // pages alone.
-double unit_cost_pages(const mla_dims& d, int32_t q_len) { return pair_decode(d, q_len) ? 6.0 : 0.0; }
+// Work the SM-pair kernel spends on a unit beyond its pages, in pages: a unit boundary
+// (the next query staged in TMEM, the previous unit's epilogue, the pipeline refilled)
+// measured ~18.9K cycles against ~2.45K per page in steady state on B200.
+double unit_cost_pages(const mla_dims& d, int32_t q_len) { return pair_decode(d, q_len) ? 7.5 : 0.0; }
 
 // Query tokens per plan unit (consecutive tokens of one sequence).
 int32_t items_per_unit_for(const mla_dims& d, int32_t q_len) {
@@ -419,47 +422,55 @@ mla_status mla_plan_splits(const int32_t* seq_lens_host, int32_t B, int32_t q_le
     }
   } else {
     // Every unit also costs `cost` pages of work (its query, its epilogue, a pipeline
-    // refill): slots get equal shares of pages + cost * units, assuming one unit per
-    // non-empty group plus one more for each slot boundary that cuts a group.
-    int64_t groups = 0;
-    for (int32_t b = 0; b < B; ++b)
-      for (int32_t k = 0; k < groups_per_seq; ++k) groups += group_pages(b, k) > 0;
-    const double share = ((double)total + cost * (double)(groups + S - 1)) / (double)S;
-    // slot s ends where the work assigned so far reaches (s + 1) * share
-    int32_t slot = 0;
-    bool slot_used = false;
-    double acc = 0.0;
-    for (int32_t b = 0; b < B; ++b) {
-      for (int32_t k = 0; k < groups_per_seq; ++k) {
-        const int32_t it = b * q_len + k * ipu;
-        const int32_t n = std::min(ipu, q_len - k * ipu);
-        int32_t left = group_pages(b, k), pb = 0;
-        if (left == 0) {
-          units.push_back({it, b, 0, 0, slot, n});
-          continue;
-        }
-        while (left > 0) {
-          const bool last_slot = slot + 1 >= S;
-          // no room left here even for one page: the next slot
-          if (!last_slot && slot_used && acc + cost + 1.0 > (slot + 1) * share + 0.5) {
-            ++slot;
-            slot_used = false;
+    // refill). Units are laid out in order and each slot takes work up to a capacity C
+    // (a group is cut where a slot fills up); C is the smallest capacity whose fill
+    // needs at most S slots, found by bisection, so the heaviest slot is as light as
+    // this contiguous layout allows.
+    auto fill = [&](double C, bool emit) -> int64_t {
+      int64_t slot = 0;
+      double acc = 0.0;
+      bool used = false;
+      for (int32_t b = 0; b < B; ++b) {
+        for (int32_t k = 0; k < groups_per_seq; ++k) {
+          const int32_t it = b * q_len + k * ipu;
+          const int32_t n = std::min(ipu, q_len - k * ipu);
+          int32_t left = group_pages(b, k), pb = 0;
+          if (left == 0) {
+            if (emit) units.push_back({it, b, 0, 0, (int32_t)slot, n});
             continue;
           }
-          const double room = (slot + 1) * share - acc - cost;
-          const int32_t take = last_slot ? left : (int32_t)std::min<double>(left, std::max(1.0, std::floor(room + 0.5)));
-          units.push_back({it, b, pb, pb + take, slot, n});
-          slot_used = true;
-          pb += take;
-          left -= take;
-          acc += cost + take;
-          if (!last_slot && acc >= (slot + 1) * share - 0.5) {
-            ++slot;
-            slot_used = false;
+          while (left > 0) {
+            const double room = C - acc - cost;
+            if (used && room < 1.0) {   // not even one more page fits: the next slot
+              ++slot;
+              acc = 0.0;
+              used = false;
+              continue;
+            }
+            const int32_t take = (int32_t)std::min<double>(left, std::max(1.0, std::floor(room)));
+            if (emit) units.push_back({it, b, pb, pb + take, (int32_t)slot, n});
+            used = true;
+            pb += take;
+            left -= take;
+            acc += cost + take;
           }
         }
       }
+      return slot + 1;
+    };
+    int64_t groups = 0;
+    for (int32_t b = 0; b < B; ++b)
+      for (int32_t k = 0; k < groups_per_seq; ++k) groups += group_pages(b, k) > 0;
+    // below lo the pages and one cost per group do not fit in S slots; hi fits in one
+    double lo = ((double)total + cost * (double)groups) / (double)S - 1.0;
+    double hi = (double)total + cost * (double)(groups + S) + 1.0;
+    lo = std::max(lo, cost);
+    for (int it = 0; it < 48 && hi - lo > 0.25; ++it) {
+      const double mid = 0.5 * (lo + hi);
+      if (fill(mid, false) <= S) hi = mid;
+      else lo = mid;
     }
+    fill(hi, true);
   }
   const int32_t num_slots = units.empty() ? 0 : units.back().slot + 1;
   // parts: items with more than one unit (every token of a split group is split)

@@ -107,7 +107,7 @@ def test_plan_covers_every_visible_page_once(q_len, sms, H):
     assert parts_seen == set(range(info.num_parts))
 
 
-UNIT_COST = 6.0   # pages of work the SM-pair kernel spends per unit beyond its pages
+UNIT_COST = 7.5   # pages of work the SM-pair kernel spends per unit beyond its pages
 
 
 def slot_loads(plan, info):
