@@ -28,9 +28,11 @@
  *    Calls are asynchronous on it.
  *  - Arguments are validated before any launch. On error the call returns a
  *    negative mla_status, launches nothing, and mla_last_error() describes why.
- *  - dtype MLA_BF16: q_nope, q_rope, W_UK, W_UV, kv_cache, new_ckr, q_lat, o_lat and
- *    out are bf16 (RN-even conversions); accumulation is fp32. MLA_F32: all fp32.
- *    Partial outputs and log-sum-exp values are always fp32.
+ *  - dtype MLA_BF16: q_nope, q_rope, W_UK, W_UV, kv_cache, new_ckr, q_lat and out are
+ *    bf16 (RN-even conversions); accumulation is fp32. MLA_F32: all fp32. The latent
+ *    output o_lat, partial outputs and log-sum-exp values are fp32 for both dtypes
+ *    (o_lat enters the output projection in full: with only a few visible tokens a
+ *    bf16 o_lat alone would move `out` by more than a bf16 rounding).
  *  - A cache row is [c (R) ; k_rope (Dr)]; k_rope is stored already rotated.
  *    seq_lens[b] counts cached tokens of sequence b INCLUDING its q_len new ones.
  *    Query i (0 <= i < q_len) of sequence b sits at position seq_lens[b]-q_len+i
@@ -52,7 +54,7 @@
 extern "C" {
 #endif
 
-#define MLA_ABI_VERSION 2
+#define MLA_ABI_VERSION 3
 
 typedef enum {
   MLA_OK = 0,
@@ -177,7 +179,7 @@ size_t mla_workspace_size(const mla_plan_info* info, mla_dims d);
  * (the absorbed form of the GatedMLA attention; scale = 1/sqrt(Dn+Dr) there).
  *   q_lat [B*q_len][H][R], q_rope [B*q_len][H][Dr], kv_cache as above (dtype)
  *   plan_dev: device copy of the mla_plan_splits buffer; info: its host summary
- *   o_lat [B*q_len][H][R] dtype and lse [B*q_len][H] fp32 (lse may be NULL):
+ *   o_lat [B*q_len][H][R] fp32 and lse [B*q_len][H] fp32 (lse may be NULL):
  *   written for queries whose work is one unit; others go to the workspace.
  *   workspace: >= mla_workspace_size bytes, 256-byte aligned (may be NULL when
  *   the plan has no parts).                                                       */
@@ -195,7 +197,7 @@ mla_status mla_decode_attn(const void* q_lat, const void* q_rope, const void* kv
  * for each query whose work was split: m = max_s lse_s, w_s = exp(lse_s - m),
  * o_lat = sum_s w_s o_s / sum_s w_s, lse = m + log sum_s w_s (parts with
  * lse = -inf weigh 0). Writes o_lat (dtype) and lse (fp32, may be NULL) of those
- * queries only. A no-op launch-free call when info->num_parts == 0.              */
+ * queries only (both fp32). A no-op launch-free call when info->num_parts == 0.      */
 mla_status mla_combine(const int32_t* plan_dev, const mla_plan_info* info, const void* workspace,
                        size_t workspace_bytes, void* o_lat, float* lse, mla_dims d, void* stream);
 
@@ -203,7 +205,9 @@ mla_status mla_combine(const int32_t* plan_dev, const mla_plan_info* info, const
  * out[t][h][:] = W_UV[h] @ o_lat[t][h][:]  (the value up-projection folded into
  * the output side; GatedMLA "Output projection and optional gate" applies Wo and
  * the gate after this, outside this library).
- *   o_lat [T][H][R], W_UV [H][Dv][R]  ->  out [T][H][Dv]             all dtype      */
+ *   o_lat [T][H][R] fp32, W_UV [H][Dv][R] dtype  ->  out [T][H][Dv] dtype
+ * (bf16 on the tensor cores: each fp32 o_lat element enters as bf16 hi + lo, two MMAs
+ * per K step, so o_lat keeps ~16 significant bits; fp32 accumulation)              */
 mla_status mla_out_proj(const void* o_lat, const void* W_UV, void* out, int32_t T, mla_dims d,
                         void* stream);
 

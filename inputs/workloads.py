@@ -249,7 +249,9 @@ def latent_queries(spec: WorkloadSpec, T: int, seed: int = 0) -> np.ndarray:
     return _store(spec, g.standard_normal((T, spec.H, spec.R), dtype=np.float32) * np.float32(0.5))
 
 
-def latent_outputs(spec: WorkloadSpec, T: int, seed: int = 0) -> np.ndarray:
-    """Seeded stand-in for a latent attention output, [T, H, R]: entries N(0, 0.1^2)."""
+def latent_outputs(spec: WorkloadSpec, T: int, seed: int = 0, fp32: bool = False) -> np.ndarray:
+    """Seeded stand-in for a latent attention output, [T, H, R]: entries N(0, 0.1^2),
+    in the workload's storage dtype, or as float32 values when `fp32`."""
     g = _rng(seed, 7)
-    return _store(spec, g.standard_normal((T, spec.H, spec.R), dtype=np.float32) * np.float32(0.1))
+    x = g.standard_normal((T, spec.H, spec.R), dtype=np.float32) * np.float32(0.1)
+    return x if fp32 else _store(spec, x)

@@ -560,7 +560,7 @@ decode_2sm_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_consta
         const int32_t prt = u.part[tn];
         for (int lh = 0; lh < 2; ++lh) {
           const int d = 256 * lh + 128 * (int)rank + L;
-          if (prt < 0) p.o_lat[row * kR + d] = __float2bfloat16_rn(0.f);
+          if (prt < 0) p.o_lat[row * kR + d] = 0.f;
           else p.o_part[((int64_t)prt * H + row % H) * kR + d] = 0.f;
         }
       }
@@ -652,10 +652,10 @@ decode_2sm_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_consta
       if (!__all_sync(0xffffffffu, got)) return false;
       if (sw == 0 && lane == 0) DUO_TRACE(14, n_ep);
       // Each warp writes its own 32 latent columns (latent rows of its TMEM lane quarter)
-      // of each 32-row chunk of O^T: scale by 1 / l, stage the 32 x 32 block row-major in
-      // one of the warp's two tiles in the idle P buffers, and hand it to a TMA store
-      // (bf16 final rows, fp32 partial rows). The stores run in the background; a tile is
-      // restaged once the store two chunks back has read it.
+      // of each 32-row chunk of O^T: scale by 1 / l, stage two 16-row fp32 blocks row-major
+      // in the warp's two tiles in the idle P buffers, and hand each to a TMA store (final
+      // rows to o_lat, partial rows to the workspace). The stores run in the background; a
+      // tile is restaged once the store two blocks back has read it.
       const uint32_t tiles = sbase + kOffP + (uint32_t)sw * kPBytes;   // 2 x 4 KiB
       uint32_t nst = 0;
 #pragma unroll 1
@@ -672,35 +672,29 @@ decode_2sm_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_consta
           asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
                        : "=f"(inv[4 * k]), "=f"(inv[4 * k + 1]), "=f"(inv[4 * k + 2]), "=f"(inv[4 * k + 3])
                        : "r"(sbase + kOffXinv + 4u * (n0 + 4 * k)));
-        if (nst >= 2 && lane == 0) ptx::bulk_wait_group_read<1>();   // the tile's previous store read it
         ptx::tmem_wait_ld();
-        __syncwarp();
-        const uint32_t tile = tiles + (nst & 1) * (uint32_t)kPBytes / 2;
-        if (prt < 0) {
+        const int x = 256 * lh + 128 * (int)rank + 32 * q;   // this warp's latent columns
+        const int64_t row0 = qrow_of(pend.item, n0);
+        const CUtensorMap* map = prt < 0 ? &tm_o : &tm_op;
+        const int64_t y0 = prt < 0 ? row0 : (int64_t)prt * H + row0 % H;
 #pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            const __nv_bfloat16 bv = __float2bfloat16_rn(__uint_as_float(o[j]) * inv[j]);
-            asm volatile("st.shared.b16 [%0], %1;" ::"r"(tile + (uint32_t)(j * 64 + 2 * lane)),
-                         "h"(*reinterpret_cast<const unsigned short*>(&bv))
-                         : "memory");
-          }
-        } else {
+        for (int hr = 0; hr < 2; ++hr) {
+          if (nst >= 2 && lane == 0) ptx::bulk_wait_group_read<1>();   // the tile's previous store read it
+          __syncwarp();
+          const uint32_t tile = tiles + (nst & 1) * (uint32_t)kPBytes / 2;
 #pragma unroll
-          for (int j = 0; j < 32; ++j)
+          for (int j = 0; j < 16; ++j)
             asm volatile("st.shared.f32 [%0], %1;" ::"r"(tile + (uint32_t)(j * 128 + 4 * lane)),
-                         "f"(__uint_as_float(o[j]) * inv[j])
+                         "f"(__uint_as_float(o[16 * hr + j]) * inv[16 * hr + j])
                          : "memory");
+          ptx::fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            ptx::tma_store_2d(map, tile, x, (int32_t)(y0 + 16 * hr));
+            ptx::bulk_commit_group();
+          }
+          ++nst;
         }
-        ptx::fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) {
-          const int x = 256 * lh + 128 * (int)rank + 32 * q;   // this warp's latent columns
-          const int64_t row0 = qrow_of(pend.item, n0);
-          if (prt < 0) ptx::tma_store_2d(&tm_o, tile, x, (int32_t)row0);
-          else ptx::tma_store_2d(&tm_op, tile, x, (int32_t)((int64_t)prt * H + row0 % H));
-          ptx::bulk_commit_group();
-        }
-        ++nst;
       }
       // O^T is read: the next unit's value MMAs may overwrite it
       ptx::tc_fence_before();

@@ -100,7 +100,7 @@ struct Params {
   int32_t num_pages;
   int32_t H;
   float scale_log2;           // softmax scale * log2(e)
-  __nv_bfloat16* o_lat;       // [T][H][512] final results
+  float* o_lat;               // [T][H][512] final results (fp32)
   float* lse;                 // [T][H] (nullable)
   float* o_part;              // [parts][H][512]
   float* lse_part;            // [parts][H]
@@ -421,7 +421,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_qlat, const __grid_constant
         for (int e = sm_tid; e < kHeads * kR; e += 128) {
           const int h = e / kR, d = e % kR;
           if (final_out)
-            p.o_lat[((int64_t)u.item * H + g * kHeads + h) * kR + d] = __float2bfloat16_rn(0.f);
+            p.o_lat[((int64_t)u.item * H + g * kHeads + h) * kR + d] = 0.f;
           else
             p.o_part[((int64_t)u.part * H + g * kHeads + h) * kR + d] = 0.f;
         }
@@ -579,7 +579,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_qlat, const __grid_constant
             const float l = l_s[h];
             const float val = l > 0.f ? o[j] / l : 0.f;
             if (final_out)
-              p.o_lat[(row0 + h) * kR + d] = __float2bfloat16_rn(val);
+              p.o_lat[(row0 + h) * kR + d] = val;
             else
               p.o_part[(row0 + h) * kR + d] = val;
           }

@@ -184,6 +184,37 @@ mla_status launch_proj(const void* A, const void* Bw, void* out, int32_t T, cons
   return launch_check(what);
 }
 
+// The output projection with fp32 o_lat (see gemm::proj_a32_kernel): A boxes of 32 fp32
+// columns x 128 rows with the 128-byte swizzle, weights as for launch_proj.
+template <int KBLK, int N, int STAGES>
+mla_status launch_proj_a32(const void* A, const void* Bw, void* out, int32_t T, const mla_dims& d, cudaStream_t st) {
+  using C = mla::gemm::CfgA32<KBLK, N, STAGES>;
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return fail(MLA_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+  if (reinterpret_cast<uintptr_t>(A) % 16 != 0) return fail(MLA_ERR_INVALID, "o_lat %p is not 16-byte aligned", A);
+  CUtensorMap ta, tb;
+  const cuuint64_t dims[2] = {(cuuint64_t)d.H * d.R, (cuuint64_t)T};
+  const cuuint64_t strides[1] = {(cuuint64_t)d.H * d.R * 4};
+  const cuuint32_t box[2] = {32, 128};
+  const cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(&ta, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<void*>(A), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(MLA_ERR_CUDA, "cuTensorMapEncodeTiled (fp32 A) failed (%d)", (int)r);
+  if (mla_status s = make_map_2d(&tb, Bw, (uint64_t)d.R, (uint64_t)d.H * d.Dv, (uint64_t)d.R * 2, 64)) return s;
+  auto kern = mla::gemm::proj_a32_kernel<KBLK, N, STAGES>;
+  if (mla_status s = ensure_smem_attr((const void*)kern, C::kSmemBytes)) return s;
+  mla::gemm::Params p;
+  p.out = static_cast<__nv_bfloat16*>(out);
+  p.T = T;
+  p.H = d.H;
+  p.n_total = d.Dv;
+  p.timeout_ns = g_timeout_ns.load();
+  const dim3 grid(d.H, (T + mla::gemm::kM - 1) / mla::gemm::kM, d.Dv / N);
+  kern<<<grid, 128, C::kSmemBytes, st>>>(ta, tb, p);
+  return launch_check("out_proj (tcgen05, fp32 o_lat)");
+}
+
 // The SM-pair kernel serves 128 rows per cluster: all heads of one query token for
 // H=128, or the heads of up to two consecutive query tokens of a sequence for H=64
 // (with one query token per sequence the odd CTA's rows are idle).
@@ -328,14 +359,13 @@ mla_status mla_out_proj(const void* o_lat, const void* W_UV, void* out, int32_t 
   if (pol == MLA_POLICY_TCGEN05 && !outproj_tc_ok(d))
     return fail(MLA_ERR_UNSUPPORTED, "tensor-core output projection needs bf16, R=512, Dv=128");
   if (pol != MLA_POLICY_SIMT && outproj_tc_ok(d))
-    return launch_proj<8, 128, false, 6>(o_lat, W_UV, out, T, d, d.R, d.H * d.Dv, d.R, d.Dv, as_stream(stream),
-                                         "out_proj (tcgen05)");
+    return launch_proj_a32<8, 128, 4>(o_lat, W_UV, out, T, d, as_stream(stream));
   const dim3 grid(d.H, (T + mla::simt::kTT - 1) / mla::simt::kTT);
   const size_t smem = sizeof(float) * mla::simt::kTT * d.R;
   if (smem > 48 * 1024) return fail(MLA_ERR_UNSUPPORTED, "R=%d too large", d.R);
   if (d.dtype == MLA_BF16)
     mla::simt::outproj_kernel<__nv_bfloat16><<<grid, 256, smem, as_stream(stream)>>>(
-        static_cast<const __nv_bfloat16*>(o_lat), static_cast<const __nv_bfloat16*>(W_UV),
+        static_cast<const float*>(o_lat), static_cast<const __nv_bfloat16*>(W_UV),
         static_cast<__nv_bfloat16*>(out), T, d.H, d.Dv, d.R);
   else
     mla::simt::outproj_kernel<float><<<grid, 256, smem, as_stream(stream)>>>(
@@ -615,7 +645,7 @@ mla_status mla_decode_attn(const void* q_lat, const void* q_rope, const void* kv
     p.num_pages = num_pages;
     p.H = d.H;
     p.scale_log2 = scale * 1.4426950408889634f;
-    p.o_lat = static_cast<__nv_bfloat16*>(o_lat);
+    p.o_lat = static_cast<float*>(o_lat);
     p.lse = lse;
     p.o_part = o_part;
     p.lse_part = lse_part;
@@ -633,12 +663,12 @@ mla_status mla_decode_attn(const void* q_lat, const void* q_rope, const void* kv
       if (mla_status s = make_map_2d(&tk32, kv_cache, d.R + d.Dr, (uint64_t)num_pages * d.page_size,
                                      (uint64_t)(d.R + d.Dr) * 2, 32, 64))
         return s;
-      // output stores: 32 x 32 blocks of final rows (bf16) and of partial rows (fp32)
-      if (mla_status s = make_store_map_2d(&to, o_lat, false, d.R, (uint64_t)T * d.H, (uint64_t)d.R * 2, 32, 32))
+      // output stores: fp32 blocks of 16 rows x 32 columns, final rows and partial rows
+      if (mla_status s = make_store_map_2d(&to, o_lat, true, d.R, (uint64_t)T * d.H, (uint64_t)d.R * 4, 32, 16))
         return s;
       if (info->num_parts > 0) {
         if (mla_status s = make_store_map_2d(&top, o_part, true, d.R, (uint64_t)info->num_parts * d.H,
-                                             (uint64_t)d.R * 4, 32, 32))
+                                             (uint64_t)d.R * 4, 32, 16))
           return s;
       } else {
         top = to;   // never used: the plan has no partial outputs
@@ -696,22 +726,13 @@ mla_status mla_combine(const int32_t* plan_dev, const mla_plan_info* info, const
     return s;
   if (d.R <= 512 && d.R % 4 == 0) {
     const dim3 gv(info->num_items, (d.H + 3) / 4);
-    if (d.dtype == MLA_BF16)
-      mla::simt::combine_vec_kernel<__nv_bfloat16><<<gv, 128, 0, as_stream(stream)>>>(
-          plan_dev, o_part, lse_part, static_cast<__nv_bfloat16*>(o_lat), lse, d.H, d.R);
-    else
-      mla::simt::combine_vec_kernel<float><<<gv, 128, 0, as_stream(stream)>>>(
-          plan_dev, o_part, lse_part, static_cast<float*>(o_lat), lse, d.H, d.R);
+    mla::simt::combine_vec_kernel<<<gv, 128, 0, as_stream(stream)>>>(plan_dev, o_part, lse_part,
+                                                                      static_cast<float*>(o_lat), lse, d.H, d.R);
     return launch_check("combine");
   }
   const dim3 grid(info->num_items, d.H);
-  if (d.dtype == MLA_BF16)
-    mla::simt::combine_kernel<__nv_bfloat16><<<grid, 128, 0, as_stream(stream)>>>(
-        plan_dev, o_part, lse_part, static_cast<__nv_bfloat16*>(o_lat), lse, d.H, d.R);
-  else
-    mla::simt::combine_kernel<float><<<grid, 128, 0, as_stream(stream)>>>(plan_dev, o_part, lse_part,
-                                                                           static_cast<float*>(o_lat), lse,
-                                                                           d.H, d.R);
+  mla::simt::combine_kernel<<<grid, 128, 0, as_stream(stream)>>>(plan_dev, o_part, lse_part,
+                                                                 static_cast<float*>(o_lat), lse, d.H, d.R);
   return launch_check("combine");
 }
 

@@ -95,13 +95,13 @@ __global__ void absorb_kernel(const T* __restrict__ qn, const T* __restrict__ w,
 // out[t][h][v] = sum_r W_UV[h][v][r] * o_lat[t][h][r]
 // grid (H, ceil(T/kTT)), block 256: the kTT latent rows in shared memory, one warp per v.
 template <typename T>
-__global__ void outproj_kernel(const T* __restrict__ ol, const T* __restrict__ w, T* __restrict__ out,
+__global__ void outproj_kernel(const float* __restrict__ ol, const T* __restrict__ w, T* __restrict__ out,
                                int32_t T_, int32_t H, int32_t Dv, int32_t R) {
   extern __shared__ float so[];  // [kTT][R]
   const int32_t h = blockIdx.x, t0 = blockIdx.y * kTT;
   for (int32_t e = threadIdx.x; e < kTT * R; e += blockDim.x) {
     const int32_t t = t0 + e / R, r = e % R;
-    so[e] = t < T_ ? to_f32(ol[((int64_t)t * H + h) * R + r]) : 0.f;
+    so[e] = t < T_ ? ol[((int64_t)t * H + h) * R + r] : 0.f;
   }
   __syncthreads();
   const int32_t warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nwarp = blockDim.x >> 5;
@@ -132,7 +132,7 @@ struct DecodeSimtArgs {
   const int32_t* seq_lens;
   int32_t max_pages, num_pages, H, R, Dr, page_size;
   float scale;
-  void* o_lat;
+  void* o_lat;        // fp32 [T][H][R]
   float* lse;
   float* o_part;
   float* lse_part;
@@ -197,12 +197,12 @@ __global__ void decode_kernel(const T* __restrict__ q_lat, const T* __restrict__
   const float inv = tot > 0.f ? 1.f / tot : 0.f;
   const float lse_v = tot > 0.f ? M + logf(tot) : -CUDART_INF_F;
   if (u.part < 0) {
-    T* dst = reinterpret_cast<T*>(a.o_lat) + ((int64_t)u.item * a.H + h) * a.R;
+    float* dst = static_cast<float*>(a.o_lat) + ((int64_t)u.item * a.H + h) * a.R;
     for (int32_t e = threadIdx.x; e < a.R; e += blockDim.x) {
       float s = 0.f;
 #pragma unroll
       for (int k = 0; k < 4; ++k) s = fmaf(wgt[k], os[k * a.R + e], s);
-      dst[e] = from_f32<T>(s * inv);
+      dst[e] = s * inv;
     }
     if (threadIdx.x == 0 && a.lse) a.lse[(int64_t)u.item * a.H + h] = lse_v;
   } else {
@@ -219,9 +219,8 @@ __global__ void decode_kernel(const T* __restrict__ q_lat, const T* __restrict__
 
 // ------------------------------------------------------------------ a6: split-KV combine
 // grid (num_items, H), block 128. Items computed by a single unit are skipped.
-template <typename T>
 __global__ void combine_kernel(const int32_t* __restrict__ plan_w, const float* __restrict__ o_part,
-                               const float* __restrict__ lse_part, T* __restrict__ o_lat,
+                               const float* __restrict__ lse_part, float* __restrict__ o_lat,
                                float* __restrict__ lse, int32_t H, int32_t R) {
   const PlanView plan{plan_w};
   const int32_t item = blockIdx.x, h = blockIdx.y;
@@ -242,7 +241,7 @@ __global__ void combine_kernel(const int32_t* __restrict__ plan_w, const float* 
       const float wgt = (M == -CUDART_INF_F) ? 0.f : expf(z - M);
       if (wgt > 0.f) acc = fmaf(wgt, o_part[((int64_t)(first + s) * H + h) * R + e], acc);
     }
-    o_lat[((int64_t)item * H + h) * R + e] = from_f32<T>(acc * inv);
+    o_lat[((int64_t)item * H + h) * R + e] = acc * inv;
   }
   if (threadIdx.x == 0 && lse) lse[(int64_t)item * H + h] = tot > 0.f ? M + logf(tot) : -CUDART_INF_F;
 }
@@ -250,11 +249,10 @@ __global__ void combine_kernel(const int32_t* __restrict__ plan_w, const float* 
 // Same merge, one warp per (item, head), rows of R <= 512 (R % 4 == 0) as float4:
 // grid (num_items, ceil(H / 4)), block 128. Each part's weight is computed once per
 // lane; the parts' rows are accumulated in ascending part order, as above.
-template <typename T>
 __global__ void __launch_bounds__(128) combine_vec_kernel(const int32_t* __restrict__ plan_w,
                                                           const float* __restrict__ o_part,
                                                           const float* __restrict__ lse_part,
-                                                          T* __restrict__ o_lat, float* __restrict__ lse,
+                                                          float* __restrict__ o_lat, float* __restrict__ lse,
                                                           int32_t H, int32_t R) {
   const PlanView plan{plan_w};
   const int32_t item = blockIdx.x;
@@ -301,20 +299,13 @@ __global__ void __launch_bounds__(128) combine_vec_kernel(const int32_t* __restr
     }
   }
   const float inv = tot > 0.f ? 1.f / tot : 0.f;
-  T* dst = o_lat + ((int64_t)item * H + h) * R;
+  float* dst = o_lat + ((int64_t)item * H + h) * R;
 #pragma unroll
   for (int k = 0; k < 4; ++k) {
     const int32_t i = lane + 32 * k;
-    if (i < nv) {
-      const float4 o = make_float4(acc[k].x * inv, acc[k].y * inv, acc[k].z * inv, acc[k].w * inv);
-      if constexpr (sizeof(T) == 2) {
-        __nv_bfloat162 lo = __floats2bfloat162_rn(o.x, o.y), hi = __floats2bfloat162_rn(o.z, o.w);
-        *reinterpret_cast<uint2*>(dst + 4 * i) =
-            make_uint2(*reinterpret_cast<uint32_t*>(&lo), *reinterpret_cast<uint32_t*>(&hi));
-      } else {
-        *reinterpret_cast<float4*>(dst + 4 * i) = o;
-      }
-    }
+    if (i < nv)
+      *reinterpret_cast<float4*>(dst + 4 * i) =
+          make_float4(acc[k].x * inv, acc[k].y * inv, acc[k].z * inv, acc[k].w * inv);
   }
   if (lane == 0 && lse) lse[(int64_t)item * H + h] = tot > 0.f ? M + logf(tot) : -CUDART_INF_F;
 }

@@ -50,7 +50,7 @@ class DecodeStep:
         dt = self.q_nope.dtype
         H, R, Dv = spec.H, spec.R, spec.Dv
         self.q_lat = torch.empty((self.T, H, R), dtype=dt, device=d)
-        self.o_lat = torch.empty((self.T, H, R), dtype=dt, device=d)
+        self.o_lat = torch.empty((self.T, H, R), dtype=torch.float32, device=d)   # fp32 for every dtype
         self.lse = torch.empty((self.T, H), dtype=torch.float32, device=d)
         self.out = torch.empty((self.T, H, Dv), dtype=dt, device=d)
         # the cache append and the query absorption are independent: the append runs on

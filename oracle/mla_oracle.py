@@ -195,15 +195,18 @@ def decode_absorbed(q_nope, q_rope, kv_cache, block_table, seq_lens, W_UK, W_UV,
                     q_len=1, page_size=64, intermediates=None):
     """The absorbed pipeline in float64 (cross-check of the reference semantics).
 
-    intermediates="bf16" rounds the two tensors a bf16 pipeline stores between its
-    steps, the absorbed query ql and the latent output o_lat, to bf16; everything
-    else stays float64. This is the reference for an end-to-end check of such a
-    pipeline on inputs where those two roundings alone move the result by more than
-    a per-step tolerance (queries that see only a few tokens)."""
-    rnd = round_bf16 if intermediates == "bf16" else (lambda a: a)
-    ql = rnd(absorb_q(q_nope, W_UK))
+    intermediates="bf16" rounds the two tensors a bf16 pipeline may store between its
+    steps, the absorbed query ql and the latent output o_lat, to bf16;
+    intermediates="q_lat" rounds only ql (a pipeline that keeps o_lat in fp32);
+    everything else stays float64. This is the reference for an end-to-end check of
+    such a pipeline on inputs where those roundings alone move the result by more
+    than a per-step tolerance (queries that see only a few tokens)."""
+    ident = lambda a: a  # noqa: E731
+    rnd_q = round_bf16 if intermediates in ("bf16", "q_lat") else ident
+    rnd_o = round_bf16 if intermediates == "bf16" else ident
+    ql = rnd_q(absorb_q(q_nope, W_UK))
     a = attend_latent(ql, q_rope, kv_cache, block_table, seq_lens, scale, q_len, page_size)
-    ol = np.where(np.isnan(a["o_lat"]), np.nan, rnd(np.nan_to_num(a["o_lat"])))
+    ol = np.where(np.isnan(a["o_lat"]), np.nan, rnd_o(np.nan_to_num(a["o_lat"])))
     return dict(out=out_proj(ol, W_UV), o_lat=ol, lse=a["lse"])
 
 

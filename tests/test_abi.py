@@ -34,7 +34,7 @@ def test_library_exports_every_declared_symbol():
 
 
 def test_abi_version_and_error_text():
-    assert mla.mla_abi_version() == 2
+    assert mla.mla_abi_version() == 3
     with pytest.raises(mla.MlaError) as e:
         mla.mla_set_policy(7)
     assert e.value.status == mla._binding.MLA_ERR_INVALID

@@ -123,13 +123,20 @@ def test_out_proj_matches_oracle(case, policy):
     w = proj_case(case)
     spec = w["spec"]
     step = dec.DecodeStep(w)
-    ol = wl.latent_outputs(spec, step.T, seed=4)
-    step.o_lat.copy_(dec.to_torch(ol, step.device))
+    ol = wl.latent_outputs(spec, step.T, seed=4, fp32=True)   # o_lat is fp32 for every dtype
+    step.o_lat.copy_(torch.from_numpy(ol).to(step.device))
     run_policy(policy)
     step.project()
     torch.cuda.synchronize()
     ref = orc.out_proj(ol, w["W_UV"])
-    assert_close(host(step.out), ref, spec.dtype == "f32", "out")
+    got = host(step.out)
+    assert_close(got, ref, spec.dtype == "f32", "out")
+    if spec.dtype == "bf16":
+        # o_lat enters in full: only the bf16 store of `out` rounds (half a bf16 ulp, 2^-9
+        # relative); o_lat cut to bf16 first would add ~1e-3 absolute here (512 terms of
+        # |w| ~ 0.04 times |o| ~ 0.1 with 2^-9 relative errors)
+        err = np.abs(got - ref)
+        assert np.all(err <= 2.0 ** -8 * np.abs(ref) + 2e-5), float((err - 2.0 ** -8 * np.abs(ref)).max())
 
 
 # ----------------------------------------------------------------------------- a3-a6: attention (+ combine)
@@ -216,11 +223,11 @@ def test_tcgen05_policy_rejects_unsupported_dims():
 def test_whole_step_matches_oracle(policy, H, q_len, lens, sms):
     """append -> absorb -> attention (policy under test) -> combine -> projection.
 
-    Against the oracle of the same bf16 pipeline (absorbed query and latent output
-    stored in bf16, all else fp64) at the bf16 tolerance everywhere, and against the
-    exact non-absorbed definition on every query that sees at least 64 tokens. (With
-    only a few visible tokens the two bf16 stores alone move `out` by more than the
-    tolerance: the oracle shows it, see test_oracle.py.)"""
+    Against the oracle of the same pipeline (the absorbed query stored in bf16, all else
+    fp64; o_lat stays fp32) at the bf16 tolerance everywhere, and against the exact
+    non-absorbed definition on every query that sees at least 17 tokens. (With only a
+    few visible tokens of comparable weight the bf16 store of the absorbed query alone
+    moves `out` by more than the tolerance.)"""
     spec = small_spec(H=H, q_len=q_len)
     empty = wl.make(spec, seed=21, seq_lens=lens, new_rows_in_cache=False)
     full = wl.make(spec, seed=21, seq_lens=lens)
@@ -237,15 +244,15 @@ def test_whole_step_matches_oracle(policy, H, q_len, lens, sms):
     mla.mla_check_status()
     args = (full["q_nope"], full["q_rope"], full["kv_cache"], full["block_table"], full["seq_lens"],
             full["W_UK"], full["W_UV"], full["scale"])
-    mixed = orc.decode_absorbed(*args, q_len=q_len, page_size=spec.page_size, intermediates="bf16")
+    mixed = orc.decode_absorbed(*args, q_len=q_len, page_size=spec.page_size, intermediates="q_lat")
     out, lse = host(step.out), host(step.lse)
-    assert_close(out, mixed["out"], False, "out vs bf16-pipeline oracle")
-    assert_close(lse, mixed["lse"], False, "lse vs bf16-pipeline oracle")
+    assert_close(out, mixed["out"], False, "out vs bf16-query pipeline oracle")
+    assert_close(lse, mixed["lse"], False, "lse vs bf16-query pipeline oracle")
     exact = orc.decode_nonabsorbed(*args, q_len=q_len, page_size=spec.page_size)
     vis = np.array([max(0, L - q_len + i + 1) for L in lens for i in range(q_len)])
-    long_ctx = vis >= 64
-    assert long_ctx.any()
-    assert_close(out[long_ctx], exact["out"][long_ctx], False, "out vs definition")
+    seen = vis >= 17
+    assert seen.any()
+    assert_close(out[seen], exact["out"][seen], False, "out vs definition")
 
 
 @pytest.mark.parametrize("H", [64, 128])
@@ -325,8 +332,8 @@ def _full_step(name):
 @pytest.mark.parametrize("name", FULL[:3])
 def test_full_size_workload_every_output(name):
     """Every (query, head) of the workload against the fp64 absorbed pipeline with the
-    kernels' two bf16 stores (q_lat, o_lat) rounded the same way: out, lse and o_lat,
-    elementwise at the bf16 bound. That oracle is pinned to the non-absorbed definition
+    absorbed query rounded to bf16 as the kernels store it (o_lat stays fp32): out, lse
+    and o_lat, elementwise at the bf16 bound. That oracle is pinned to the non-absorbed definition
     (tests/test_oracle.py); here the definition itself is checked too, on a sample that
     always holds the longest sequence (for the long-context workload: 131,072 tokens
     with per-token logit noise of std 4)."""
@@ -334,7 +341,7 @@ def test_full_size_workload_every_output(name):
     full, out, lse, o_lat = _full_step(name)
     args = (full["q_nope"], full["q_rope"], full["kv_cache"], full["block_table"], full["seq_lens"],
             full["W_UK"], full["W_UV"], full["scale"])
-    mixed = orc.decode_absorbed(*args, q_len=spec.q_len, page_size=spec.page_size, intermediates="bf16")
+    mixed = orc.decode_absorbed(*args, q_len=spec.q_len, page_size=spec.page_size, intermediates="q_lat")
     assert_close(out, mixed["out"], False, f"{name} out, every query and head")
     assert_close(lse, mixed["lse"], False, f"{name} lse, every query and head")
     assert_close(o_lat, mixed["o_lat"], False, f"{name} o_lat, every query and head")

@@ -440,3 +440,21 @@ def test_bf16_intermediates_variant_stays_near_the_definition():
     d = np.abs(mixed["out"] - ref["out"])
     assert 0 < d.max() < 2e-3 + 1e-2 * np.abs(ref["out"]).max()
     np.testing.assert_array_equal(mixed["o_lat"], orc.round_bf16(mixed["o_lat"]))
+    # only the query rounded: still within the bound at this length, o_lat off the bf16 grid
+    qonly = orc.decode_absorbed(*args, q_len=s.q_len, page_size=s.page_size, intermediates="q_lat")
+    dq = np.abs(qonly["out"] - ref["out"])
+    assert 0 < dq.max() < 2e-3 + 1e-2 * np.abs(ref["out"]).max()
+    assert np.any(qonly["o_lat"] != orc.round_bf16(qonly["o_lat"]))
+
+
+def test_query_only_rounding_is_exact_when_the_query_is_on_the_bf16_grid():
+    """With q_nope = 0 the absorbed query is 0, which bf16 holds exactly: rounding only the
+    query then changes nothing, and the pipeline equals the non-absorbed definition."""
+    w = small_bf16(lens=(70, 5, 129))
+    s = w["spec"]
+    qn = np.zeros_like(w["q_nope"])
+    args = (qn, w["q_rope"], w["kv_cache"], w["block_table"], w["seq_lens"], w["W_UK"], w["W_UV"], w["scale"])
+    exact = orc.decode_nonabsorbed(*args, q_len=s.q_len, page_size=s.page_size)
+    qonly = orc.decode_absorbed(*args, q_len=s.q_len, page_size=s.page_size, intermediates="q_lat")
+    np.testing.assert_allclose(qonly["out"], exact["out"], rtol=0, atol=1e-10)
+    np.testing.assert_allclose(qonly["lse"], exact["lse"], rtol=0, atol=1e-10)

@@ -19,7 +19,7 @@ over the 576 columns), the scale in log2 units, a reference maximum moved only w
 page's maximum exceeds it by more than 24 (log2 units) with O and l rescaled then,
 p = 2^(x - m) in fp32, l summed in fp32 from the unrounded p (two halves of 32 tokens
 per row, added at the end), O accumulated from bf16(p) (+ P_lo on the pages the rule
-picks) in fp32, and o = O / l rounded to bf16. The method's definition (softmax of the
+picks) in fp32, and o = O / l kept in fp32 (the kernel's o_lat). The method's definition (softmax of the
 scaled scores, weighted sum of the latent rows) is the Primer page's "Under the hood"
 absorbed form, which the oracle pins to the non-absorbed definition.
 """
@@ -81,7 +81,7 @@ def page_wise_o_lat(q, rows, n, scale, p_lo, stats=None):
         O = f32(O * al[:, None] + P @ R[:, :512])
         m = mu
     l = f32(l2[:, 0].astype(np.float64) + l2[:, 1])
-    return bf16_rn(O / np.maximum(l, 1e-30)[:, None]).astype(np.float64)
+    return f32(O / np.maximum(l, 1e-30)[:, None]).astype(np.float64)
 
 
 def worst_ratio(H, q_len, lens, noise, p_lo, seed=11, stats=None):
