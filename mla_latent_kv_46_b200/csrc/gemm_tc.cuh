@@ -41,6 +41,7 @@ struct Cfg {
   static constexpr int kOffBar = STAGES * kStageBytes;
   static constexpr int kSmemBytes = kOffBar + 256 + 1024;      // barriers + alignment slack
   static constexpr int kNInstr = N > 256 ? 256 : N;            // N per MMA
+  static_assert(N % 64 == 0, "the epilogue writes 64-column groups");
   static constexpr int kNHalves = N / kNInstr;
   static constexpr uint32_t kCols = N <= 32 ? 32 : (N <= 64 ? 64 : (N <= 128 ? 128 : (N <= 256 ? 256 : 512)));
   static constexpr uint32_t kIdesc = ptx::idesc_bf16_f32(kM, kNInstr, 0, B_MN ? 1 : 0);
@@ -156,22 +157,26 @@ proj_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
   ptx::tc_fence_after();
   const int row = m0 + 32 * warp + lane;
   if (done) {
+    // four 16-column TMEM loads in flight per wait, then 128 contiguous bytes of the row
 #pragma unroll 1
-    for (int c = 0; c < N; c += 16) {
-      float v[16];
-      ptx::tmem_ld_32x32b_x16(tbase + ((32u * warp) << 16) + c, v);
+    for (int c0 = 0; c0 < N; c0 += 64) {
+      float v[4][16];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) ptx::tmem_ld_32x32b_x16(tbase + ((32u * warp) << 16) + c0 + 16 * q, v[q]);
       ptx::tmem_wait_ld();
       if (row < p.T) {
-        uint4 pk[2];
+        uint4 pk[8];
         uint32_t* w = reinterpret_cast<uint32_t*>(pk);
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          __nv_bfloat162 b2 = __floats2bfloat162_rn(v[2 * j], v[2 * j + 1]);
-          w[j] = *reinterpret_cast<uint32_t*>(&b2);
-        }
-        uint4* dst = reinterpret_cast<uint4*>(p.out + ((int64_t)row * p.H + h) * p.n_total + n0 + c);
-        dst[0] = pk[0];
-        dst[1] = pk[1];
+        for (int q = 0; q < 4; ++q)
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            __nv_bfloat162 b2 = __floats2bfloat162_rn(v[q][2 * j], v[q][2 * j + 1]);
+            w[8 * q + j] = *reinterpret_cast<uint32_t*>(&b2);
+          }
+        uint4* dst = reinterpret_cast<uint4*>(p.out + ((int64_t)row * p.H + h) * p.n_total + n0 + c0);
+#pragma unroll
+        for (int k = 0; k < 8; ++k) dst[k] = pk[k];
       }
     }
   }
@@ -189,9 +194,11 @@ proj_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
 // hi = bf16(x) and lo = bf16(x - hi) (together ~16 significant bits) and the MMA runs
 // twice per K step, hi and lo against the same weight tile. Per stage TMA brings the
 // 128 x 64 fp32 block of A (two 32-column boxes, 128-byte swizzle: 128-byte rows) and
-// the N x 64 weight block; warps 2 and 3 turn each A row, in place, into its hi row
-// (where the first box's row was) and its lo row (the second box's), in the K-major
-// 128-byte-swizzled layout the MMA reads; warp 1 issues the MMAs; warp 0 the loads.
+// the N x 64 weight block; warps 2-5 turn each A row (one per thread), in place, into its
+// hi row (where the first box's row was) and its lo row (the second box's), in the K-major
+// 128-byte-swizzled layout the MMA reads; warp 1 issues the MMAs; warp 0 the loads;
+// warps 0-3 read the accumulators back (warp w reaches TMEM lanes 32w..32w+31).
+constexpr int kA32Threads = 192;
 template <int KBLK, int N, int STAGES>
 struct CfgA32 {
   static constexpr int kABytes = kM * kKB * 4;                 // 32 KiB fp32, then hi | lo bf16
@@ -205,7 +212,7 @@ struct CfgA32 {
 };
 
 template <int KBLK, int N, int STAGES>
-__global__ void __launch_bounds__(128, 1)
+__global__ void __launch_bounds__(kA32Threads, 1)
 proj_a32_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, const Params p) {
   using C = CfgA32<KBLK, N, STAGES>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -222,7 +229,7 @@ proj_a32_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
     *abort_flag = 0;
     for (int s = 0; s < STAGES; ++s) {
       ptx::mbar_init(bar(s), 1);
-      ptx::mbar_init(bar(STAGES + s), 2);
+      ptx::mbar_init(bar(STAGES + s), 4);
       ptx::mbar_init(bar(2 * STAGES + s), 1);
     }
     ptx::mbar_init(bar(3 * STAGES), 1);
@@ -268,16 +275,14 @@ proj_a32_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
     // copies still in flight land in this CTA's shared memory: wait (bounded) for them
     for (int kb = (KBLK > STAGES ? KBLK - STAGES : 0); kb < KBLK; ++kb)
       wait_all(bar(kb % STAGES), (kb / STAGES) & 1);
-  } else if (warp == 2 || warp == 3) {
+  } else if (warp >= 2 && warp < 6) {
     // ---------------------------------------------------------------- fp32 -> bf16 hi, lo
-    const int t = 32 * (warp - 2) + lane;   // rows t and t + 64
+    const int r = 32 * (warp - 2) + lane;   // this thread's row of A
     for (int kb = 0; kb < KBLK; ++kb) {
       const int s = kb % STAGES, use = kb / STAGES;
       if (!wait_all(bar(s), use & 1)) { give_up(); ok = false; break; }
       const uint32_t sa = sbase + s * C::kStageBytes;
-#pragma unroll 1
-      for (int rr = 0; rr < 2; ++rr) {
-        const int r = t + 64 * rr;
+      {
         const uint32_t row0 = sa + (uint32_t)r * 128u, row1 = row0 + C::kABytes / 2;
         float x[64];
 #pragma unroll
@@ -342,28 +347,32 @@ proj_a32_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
     }
   }
 
-  // ---------------------------------------------------------------- epilogue (all warps)
-  const bool done = ok && wait_all(bar(3 * STAGES), 0);
-  if (!done) give_up();
+  // ---------------------------------------------------------------- epilogue (warps 0-3)
+  const bool done = warp < 4 && ok && wait_all(bar(3 * STAGES), 0);
+  if (warp < 4 && !done) give_up();
   ptx::tc_fence_after();
   const int row = m0 + 32 * warp + lane;
   if (done) {
+    // four 16-column TMEM loads in flight per wait, then 128 contiguous bytes of the row
 #pragma unroll 1
-    for (int c = 0; c < N; c += 16) {
-      float v[16];
-      ptx::tmem_ld_32x32b_x16(tbase + ((32u * warp) << 16) + c, v);
+    for (int c0 = 0; c0 < N; c0 += 64) {
+      float v[4][16];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) ptx::tmem_ld_32x32b_x16(tbase + ((32u * warp) << 16) + c0 + 16 * q, v[q]);
       ptx::tmem_wait_ld();
       if (row < p.T) {
-        uint4 pk[2];
+        uint4 pk[8];
         uint32_t* w = reinterpret_cast<uint32_t*>(pk);
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          __nv_bfloat162 b2 = __floats2bfloat162_rn(v[2 * j], v[2 * j + 1]);
-          w[j] = *reinterpret_cast<uint32_t*>(&b2);
-        }
-        uint4* dst = reinterpret_cast<uint4*>(p.out + ((int64_t)row * p.H + h) * p.n_total + n0 + c);
-        dst[0] = pk[0];
-        dst[1] = pk[1];
+        for (int q = 0; q < 4; ++q)
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            __nv_bfloat162 b2 = __floats2bfloat162_rn(v[q][2 * j], v[q][2 * j + 1]);
+            w[8 * q + j] = *reinterpret_cast<uint32_t*>(&b2);
+          }
+        uint4* dst = reinterpret_cast<uint4*>(p.out + ((int64_t)row * p.H + h) * p.n_total + n0 + c0);
+#pragma unroll
+        for (int k = 0; k < 8; ++k) dst[k] = pk[k];
       }
     }
   }

@@ -211,7 +211,7 @@ mla_status launch_proj_a32(const void* A, const void* Bw, void* out, int32_t T, 
   p.n_total = d.Dv;
   p.timeout_ns = g_timeout_ns.load();
   const dim3 grid(d.H, (T + mla::gemm::kM - 1) / mla::gemm::kM, d.Dv / N);
-  kern<<<grid, 128, C::kSmemBytes, st>>>(ta, tb, p);
+  kern<<<grid, mla::gemm::kA32Threads, C::kSmemBytes, st>>>(ta, tb, p);
   return launch_check("out_proj (tcgen05, fp32 o_lat)");
 }
 
@@ -332,7 +332,7 @@ mla_status mla_absorb_q(const void* q_nope, const void* W_UK, void* q_lat, int32
   if (pol == MLA_POLICY_TCGEN05 && !absorb_tc_ok(d))
     return fail(MLA_ERR_UNSUPPORTED, "tensor-core absorb needs bf16, Dn=128, R=512");
   if (pol != MLA_POLICY_SIMT && absorb_tc_ok(d))
-    return launch_proj<2, 128, true, 2>(q_nope, W_UK, q_lat, T, d, d.Dn, d.H * d.Dn, d.R, d.R, as_stream(stream),
+    return launch_proj<2, 256, true, 2>(q_nope, W_UK, q_lat, T, d, d.Dn, d.H * d.Dn, d.R, d.R, as_stream(stream),
                                         "absorb_q (tcgen05)");
   const dim3 grid((d.R + 127) / 128, d.H, (T + mla::simt::kTT - 1) / mla::simt::kTT);
   const size_t smem = sizeof(float) * mla::simt::kTT * d.Dn;

@@ -247,8 +247,10 @@ __global__ void combine_kernel(const int32_t* __restrict__ plan_w, const float* 
 }
 
 // Same merge, one warp per (item, head), rows of R <= 512 (R % 4 == 0) as float4:
-// grid (num_items, ceil(H / 4)), block 128. Each part's weight is computed once per
-// lane; the parts' rows are accumulated in ascending part order, as above.
+// grid (num_items, ceil(H / 4)), block 128. One pass over the parts, two at a time, each
+// part's lse loaded together with its row (a single round trip to memory per pair):
+// the running maximum M and the sums are rescaled when a part raises M, as an online
+// softmax does, so the result equals the max-first merge up to fp32 rounding.
 __global__ void __launch_bounds__(128) combine_vec_kernel(const int32_t* __restrict__ plan_w,
                                                           const float* __restrict__ o_part,
                                                           const float* __restrict__ lse_part,
@@ -261,24 +263,19 @@ __global__ void __launch_bounds__(128) combine_vec_kernel(const int32_t* __restr
   if (h >= H) return;
   const int32_t first = plan.item_parts()[2 * item], np = plan.item_parts()[2 * item + 1];
   if (np == 0) return;
-  float M = -CUDART_INF_F;
-  for (int32_t s = 0; s < np; ++s) M = fmaxf(M, lse_part[(int64_t)(first + s) * H + h]);
   const int32_t nv = R / 4;
   float4 acc[4];
 #pragma unroll
   for (int k = 0; k < 4; ++k) acc[k] = make_float4(0.f, 0.f, 0.f, 0.f);
-  float tot = 0.f;
-  // parts two at a time, so that each lane has eight 16-byte loads in flight (a part with
-  // no visible token holds zeros and weighs 0)
+  float M = -CUDART_INF_F, tot = 0.f;
   for (int32_t s = 0; s < np; s += 2) {
     const bool two = s + 1 < np;
-    float wgt[2];
+    float z[2];
     float4 v[2][4];
 #pragma unroll
     for (int q = 0; q < 2; ++q) {
       const int32_t ps = first + s + (q && two ? 1 : 0);
-      const float z = lse_part[(int64_t)ps * H + h];
-      wgt[q] = (q && !two) || M == -CUDART_INF_F ? 0.f : expf(z - M);
+      z[q] = (q && !two) ? -CUDART_INF_F : lse_part[(int64_t)ps * H + h];
       const float4* src = reinterpret_cast<const float4*>(o_part + ((int64_t)ps * H + h) * R);
 #pragma unroll
       for (int k = 0; k < 4; ++k) {
@@ -286,17 +283,19 @@ __global__ void __launch_bounds__(128) combine_vec_kernel(const int32_t* __restr
         v[q][k] = i < nv ? __ldcs(src + i) : make_float4(0.f, 0.f, 0.f, 0.f);
       }
     }
+    const float Mn = fmaxf(M, fmaxf(z[0], z[1]));
+    if (Mn == -CUDART_INF_F) continue;   // no part so far saw a token
+    const float r = expf(M - Mn);        // 0 while M is -inf
+    const float w0 = expf(z[0] - Mn), w1 = expf(z[1] - Mn);
+    tot = tot * r + (w0 + w1);
 #pragma unroll
-    for (int q = 0; q < 2; ++q) {
-      tot += wgt[q];
-#pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        acc[k].x = fmaf(wgt[q], v[q][k].x, acc[k].x);
-        acc[k].y = fmaf(wgt[q], v[q][k].y, acc[k].y);
-        acc[k].z = fmaf(wgt[q], v[q][k].z, acc[k].z);
-        acc[k].w = fmaf(wgt[q], v[q][k].w, acc[k].w);
-      }
+    for (int k = 0; k < 4; ++k) {
+      acc[k].x = fmaf(w1, v[1][k].x, fmaf(w0, v[0][k].x, acc[k].x * r));
+      acc[k].y = fmaf(w1, v[1][k].y, fmaf(w0, v[0][k].y, acc[k].y * r));
+      acc[k].z = fmaf(w1, v[1][k].z, fmaf(w0, v[0][k].z, acc[k].z * r));
+      acc[k].w = fmaf(w1, v[1][k].w, fmaf(w0, v[0][k].w, acc[k].w * r));
     }
+    M = Mn;
   }
   const float inv = tot > 0.f ? 1.f / tot : 0.f;
   float* dst = o_lat + ((int64_t)item * H + h) * R;
