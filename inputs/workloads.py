@@ -77,6 +77,11 @@ WORKLOADS: Dict[str, WorkloadSpec] = {
         name="longctx_h64_b4_l131072", B=4, H=64, R=512, Dr=64, Dn=128, Dv=128, q_len=1,
         dtype="bf16", seq_len=131072, w_std=1.0 / math.sqrt(512), logit_noise_std=4.0,
         description="long-context split-KV decode, 4 x 131072 tokens, logit noise std 4"),
+    "mtp2_h128_b64_ragged": WorkloadSpec(
+        name="mtp2_h128_b64_ragged", B=64, H=128, R=512, Dr=64, Dn=128, Dv=128, q_len=2,
+        dtype="bf16", seq_len=None, ragged=(512, 16384), w_std=1.0 / math.sqrt(512),
+        description="two new tokens per sequence (multi-token decode), H=128, 64 sequences, "
+                    "lengths uniform in [512,16384]"),
     "causal_chunk_h64_b8_2048p256": WorkloadSpec(
         name="causal_chunk_h64_b8_2048p256", B=8, H=64, R=512, Dr=64, Dn=128, Dv=128, q_len=256,
         dtype="bf16", seq_len=2048 + 256, w_std=1.0 / math.sqrt(512), all_query_positions=True,

@@ -456,51 +456,86 @@ mla_status mla_plan_splits(const int32_t* seq_lens_host, int32_t B, int32_t q_le
     // (a group is cut where a slot fills up); C is the smallest capacity whose fill
     // needs at most S slots, found by bisection, so the heaviest slot is as light as
     // this contiguous layout allows.
-    auto fill = [&](double C, bool emit) -> int64_t {
+    // A layout is a sequence of groups (b, k) laid out in order over the slots
+    // [slot0, slot0 + ns).
+    struct Grp { int32_t b, k; };
+    auto fill = [&](const std::vector<Grp>& order, int64_t slot0, double C, bool emit) -> int64_t {
       int64_t slot = 0;
       double acc = 0.0;
       bool used = false;
-      for (int32_t b = 0; b < B; ++b) {
-        for (int32_t k = 0; k < groups_per_seq; ++k) {
-          const int32_t it = b * q_len + k * ipu;
-          const int32_t n = std::min(ipu, q_len - k * ipu);
-          int32_t left = group_pages(b, k), pb = 0;
-          if (left == 0) {
-            if (emit) units.push_back({it, b, 0, 0, (int32_t)slot, n});
+      for (const Grp& g : order) {
+        const int32_t b = g.b, k = g.k;
+        const int32_t it = b * q_len + k * ipu;
+        const int32_t n = std::min(ipu, q_len - k * ipu);
+        int32_t left = group_pages(b, k), pb = 0;
+        if (left == 0) {
+          if (emit) units.push_back({it, b, 0, 0, (int32_t)(slot0 + slot), n});
+          continue;
+        }
+        while (left > 0) {
+          const double room = C - acc - cost;
+          if (used && room < 1.0) {   // not even one more page fits: the next slot
+            ++slot;
+            acc = 0.0;
+            used = false;
             continue;
           }
-          while (left > 0) {
-            const double room = C - acc - cost;
-            if (used && room < 1.0) {   // not even one more page fits: the next slot
-              ++slot;
-              acc = 0.0;
-              used = false;
-              continue;
-            }
-            const int32_t take = (int32_t)std::min<double>(left, std::max(1.0, std::floor(room)));
-            if (emit) units.push_back({it, b, pb, pb + take, (int32_t)slot, n});
-            used = true;
-            pb += take;
-            left -= take;
-            acc += cost + take;
-          }
+          const int32_t take = (int32_t)std::min<double>(left, std::max(1.0, std::floor(room)));
+          if (emit) units.push_back({it, b, pb, pb + take, (int32_t)(slot0 + slot), n});
+          used = true;
+          pb += take;
+          left -= take;
+          acc += cost + take;
         }
       }
       return slot + 1;
     };
-    int64_t groups = 0;
-    for (int32_t b = 0; b < B; ++b)
-      for (int32_t k = 0; k < groups_per_seq; ++k) groups += group_pages(b, k) > 0;
-    // below lo the pages and one cost per group do not fit in S slots; hi fits in one
-    double lo = ((double)total + cost * (double)groups) / (double)S - 1.0;
-    double hi = (double)total + cost * (double)(groups + S) + 1.0;
-    lo = std::max(lo, cost);
-    for (int it = 0; it < 48 && hi - lo > 0.25; ++it) {
-      const double mid = 0.5 * (lo + hi);
-      if (fill(mid, false) <= S) hi = mid;
-      else lo = mid;
+    // the smallest capacity whose fill of `order` needs at most ns slots (bisection)
+    auto layout = [&](const std::vector<Grp>& order, int64_t slot0, int64_t ns) {
+      int64_t pages = 0, groups = 0;
+      for (const Grp& g : order) {
+        const int32_t pg = group_pages(g.b, g.k);
+        pages += pg;
+        groups += pg > 0;
+      }
+      // below lo the pages and one cost per group do not fit in ns slots; hi fits in one
+      double lo = std::max(cost, ((double)pages + cost * (double)groups) / (double)ns - 1.0);
+      double hi = (double)pages + cost * (double)(groups + ns) + 1.0;
+      for (int it = 0; it < 48 && hi - lo > 0.25; ++it) {
+        const double mid = 0.5 * (lo + hi);
+        if (fill(order, slot0, mid, false) <= ns) hi = mid;
+        else lo = mid;
+      }
+      fill(order, slot0, hi, true);
+    };
+    if (ipu == 1 && q_len >= 2 && S >= 2 * q_len) {
+      // Several query tokens per sequence, one per unit (128 heads fill the pair's rows):
+      // the last token's pages (it sees the most) are laid out on a block of S / q_len
+      // slots, and every token gets a copy of that layout on a block of its own (the
+      // kernel clips each unit to the pages its token sees). The tokens of a sequence
+      // then stream the same pages on slot j of every block at about the same time:
+      // each page is read from DRAM once and served to the other tokens' slots by L2.
+      const int64_t ns = S / q_len;
+      std::vector<Grp> order;
+      order.reserve(B);
+      for (int32_t b = 0; b < B; ++b) order.push_back({b, q_len - 1});
+      const size_t u0 = units.size();
+      layout(order, 0, ns);
+      const std::vector<U> base(units.begin() + (std::ptrdiff_t)u0, units.end());
+      units.resize(u0);
+      for (int32_t k = 0; k < q_len; ++k)
+        for (U u : base) {
+          u.item = u.b * q_len + k;
+          u.slot += (int32_t)(k * ns);
+          units.push_back(u);
+        }
+    } else {
+      std::vector<Grp> order;
+      order.reserve((size_t)B * groups_per_seq);
+      for (int32_t b = 0; b < B; ++b)
+        for (int32_t k = 0; k < groups_per_seq; ++k) order.push_back({b, k});
+      layout(order, 0, S);
     }
-    fill(hi, true);
   }
   const int32_t num_slots = units.empty() ? 0 : units.back().slot + 1;
   // parts: items with more than one unit (every token of a split group is split)

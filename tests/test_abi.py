@@ -137,6 +137,32 @@ def test_plan_balances_pages_and_units_over_pair_slots(lens):
     assert work.max() <= share + UNIT_COST + 1, (work.max(), share)
 
 
+@pytest.mark.parametrize("q_len", [2, 4])
+def test_plan_puts_each_token_of_128_heads_on_its_own_aligned_slot_block(q_len):
+    """128 heads, q_len tokens per sequence (one token per SM-pair unit): the last token's
+    pages are laid out on 74 // q_len slots and every token gets the same layout on a
+    block of its own, so a sequence's tokens read the same pages on slot j of every block
+    (and each token's units, clipped to its pages by the kernel, cover them in order)."""
+    lens = np.random.default_rng(1).integers(512, 16385, 64).astype(np.int32)
+    max_pages = int((lens.max() + 63) // 64)
+    plan, info = mla.mla_plan_splits(lens, len(lens), q_len, max_pages, dims(H=128), 148)
+    p = parse_plan(plan)
+    ns = 74 // q_len
+    assert info.num_slots == q_len * ns
+    blocks = [[] for _ in range(q_len)]
+    for u in p["units"]:
+        k = u[0] % q_len
+        assert k * ns <= u[5] < (k + 1) * ns
+        blocks[k].append((u[1], u[2], u[3], u[5] - k * ns))
+    for k in range(1, q_len):
+        assert blocks[k] == blocks[0]
+    last = (lens + 63) // 64
+    for b in range(len(lens)):
+        segs = sorted((pb, pe) for bb, pb, pe, _ in blocks[0] if bb == b)
+        assert segs[0][0] == 0 and segs[-1][1] == last[b]
+        assert all(segs[i][1] == segs[i + 1][0] for i in range(len(segs) - 1))
+
+
 def test_plan_balances_pages_for_the_single_cta_kernel():
     """Other head counts (one CTA per 64 heads) are planned on pages alone: slots differ
     by at most one page."""

@@ -185,6 +185,18 @@ def test_paired_token_attention_matches_oracle(q_len, sms):
         assert step.info.num_parts > 0
 
 
+@pytest.mark.parametrize("sms", [148, 20])
+@pytest.mark.parametrize("q_len", [2, 4])
+def test_multi_token_128_heads_attention_matches_oracle(q_len, sms):
+    """128 heads, several new tokens per sequence: each token's units sit on a slot block
+    of their own with the same page ranges as the other tokens' (the kernel clips a
+    unit to the pages its token sees), so some units of the earlier tokens are empty."""
+    step = attention_case("tcgen05", 128, q_len, [300, 65, q_len, 1000, 130, 129], sms)
+    assert step.info.head_groups == 2
+    if sms == 20:
+        assert step.info.num_parts > 0
+
+
 @pytest.mark.parametrize("policy", ["simt", "tcgen05"])
 def test_attention_with_large_logit_offsets(policy):
     """Per-token logit noise of std 4 (the long-context workload's stress): the
@@ -311,7 +323,7 @@ def test_incremental_gpu_decode_equals_full_causal_tiny():
 # ----------------------------------------------------------------------------- full-size workloads, every output
 
 FULL = ["kimi_h64_b64_l4096", "deepseek_h128_b128_ragged", "longctx_h64_b4_l131072",
-        "causal_chunk_h64_b8_2048p256"]
+        "causal_chunk_h64_b8_2048p256", "mtp2_h128_b64_ragged"]
 
 
 def _full_step(name):
@@ -329,7 +341,7 @@ def _full_step(name):
     return wl.make(spec, seed=0), out, lse, o_lat
 
 
-@pytest.mark.parametrize("name", FULL[:3])
+@pytest.mark.parametrize("name", FULL[:3] + FULL[4:])
 def test_full_size_workload_every_output(name):
     """Every (query, head) of the workload against the fp64 absorbed pipeline with the
     absorbed query rounded to bf16 as the kernels store it (o_lat stays fp32): out, lse
