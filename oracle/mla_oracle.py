@@ -251,3 +251,49 @@ def cache_append(kv_cache, block_table, seq_lens, new_ckr, q_len, page_size=64):
                 continue
             out[int(block_table[b][pos // page_size]), pos % page_size] = new_ckr[b * q_len + i]
     return out
+
+
+# ----------------------------------------------------------------------------- cache-write prologue
+
+def token_positions(seq_lens, q_len):
+    """Absolute position of every new token, [B * q_len]: token i of sequence b (L_b
+    cached tokens, its q_len new ones included) sits at L_b - q_len + i."""
+    return np.array([int(L) - q_len + i for L in seq_lens for i in range(q_len)], dtype=np.int64)
+
+
+def rope(x, pos, base=10000.0):
+    """Rotary position embedding of the last axis (width d, even) at positions `pos`
+    (broadcast over the leading axes): dims i and i + d/2 (i < d/2) form a plane turned
+    by the angle pos * base^(-2i/d). The pages fix only that the shared key carries the
+    position (modeldna primer, "Under the hood"); the frequencies (base 10000, exponent
+    -2i/d) and this pairing are the usual reading, stated as such in the design notes."""
+    x = np.asarray(x, dtype=np.float64)
+    d = x.shape[-1]
+    half = d // 2
+    theta = base ** (-2.0 * np.arange(half, dtype=np.float64) / d)
+    ang = np.asarray(pos, dtype=np.float64)[..., None] * theta
+    c, s = np.cos(ang), np.sin(ang)
+    x1, x2 = x[..., :half], x[..., half:]
+    return np.concatenate([x1 * c - x2 * s, x1 * s + x2 * c], axis=-1)
+
+
+def rms_norm(x, gain, eps):
+    """RMSNorm of the last axis: x / sqrt(mean(x^2) + eps) * gain (the GatedMLA docs'
+    kv_rmsnorm on the compressed KV feature, "Projection geometry and stored weights")."""
+    x = np.asarray(x, dtype=np.float64)
+    return x / np.sqrt(np.mean(x * x, axis=-1, keepdims=True) + eps) * to_f64(gain)
+
+
+def cache_write_rows(hidden, W_DKV, kv_gain, positions, R, eps=1e-6, rope_base=10000.0):
+    """The rows a decode step appends to the cache, [T, R + Dr], float64.
+
+    The down projection W_DKV maps each token's hidden state (width M) to the compressed
+    KV feature (R) and the shared key (Dr) in one matrix, M -> R_kv + D_s (GatedMLA docs,
+    "Projection geometry and stored weights"; W_DKV stored out x in as nn.Linear). The
+    feature is normalised by kv_rmsnorm; the shared key is rotated by its token's
+    position (rope above): [c ; k] is the cached row.
+      hidden [T, M], W_DKV [R + Dr, M], kv_gain [R], positions [T]"""
+    f = to_f64(hidden) @ to_f64(W_DKV).T
+    c = rms_norm(f[:, :R], kv_gain, eps)
+    k = rope(f[:, R:], positions, rope_base)
+    return np.concatenate([c, k], axis=1)

@@ -458,3 +458,76 @@ def test_query_only_rounding_is_exact_when_the_query_is_on_the_bf16_grid():
     qonly = orc.decode_absorbed(*args, q_len=s.q_len, page_size=s.page_size, intermediates="q_lat")
     np.testing.assert_allclose(qonly["out"], exact["out"], rtol=0, atol=1e-10)
     np.testing.assert_allclose(qonly["lse"], exact["lse"], rtol=0, atol=1e-10)
+
+
+# ----------------------------------------------------------------------------- cache-write prologue
+
+def test_rope_equals_a_complex_rotation():
+    """Rotate-half RoPE is multiplication of z_i = x_i + i x_{i+d/2} by exp(i pos theta_i),
+    theta_i = base^(-2i/d): checked through numpy's complex arithmetic (another route to
+    the same numbers); for d = 2 the plane turns by exactly pos radians."""
+    rng = np.random.default_rng(3)
+    x = rng.standard_normal((5, 64))
+    pos = np.array([0, 1, 7, 4096, 131071])
+    theta = 10000.0 ** (-2.0 * np.arange(32) / 64)
+    z = (x[:, :32] + 1j * x[:, 32:]) * np.exp(1j * pos[:, None] * theta)
+    np.testing.assert_allclose(orc.rope(x, pos), np.concatenate([z.real, z.imag], 1), rtol=0, atol=1e-12)
+    v = np.array([[0.6, -0.8]])
+    for p in (1, 2, 3.5):
+        np.testing.assert_allclose(orc.rope(v, np.array([p]))[0],
+                                   [0.6 * np.cos(p) + 0.8 * np.sin(p), 0.6 * np.sin(p) - 0.8 * np.cos(p)],
+                                   rtol=0, atol=1e-15)
+
+
+def test_rope_scores_depend_only_on_the_position_difference():
+    """The decoupled key's purpose: rope(q, m) . rope(k, n) is a function of m - n."""
+    rng = np.random.default_rng(4)
+    q, k = rng.standard_normal(64), rng.standard_normal(64)
+    for m, n in [(5, 2), (100, 0), (70000, 65000)]:
+        ref = orc.rope(q, np.array(m)) @ orc.rope(k, np.array(n))
+        for s in (1, 17, 1000):
+            got = orc.rope(q, np.array(m + s)) @ orc.rope(k, np.array(n + s))
+            assert abs(got - ref) < 1e-9 * (1 + abs(ref))
+
+
+def test_rope_composes_keeps_norms_and_is_the_identity_at_zero():
+    rng = np.random.default_rng(5)
+    x = rng.standard_normal((4, 64))
+    a, b = np.array([3, 10, 512, 9000]), np.array([1, 6, 100, 31])
+    np.testing.assert_allclose(orc.rope(orc.rope(x, a), b), orc.rope(x, a + b), rtol=0, atol=1e-10)
+    np.testing.assert_allclose(np.linalg.norm(orc.rope(x, a), axis=1), np.linalg.norm(x, axis=1), rtol=1e-14)
+    np.testing.assert_array_equal(orc.rope(x, np.zeros(4)), x)
+
+
+def test_rms_norm_matches_torch_and_has_unit_rms():
+    rng = np.random.default_rng(6)
+    x = rng.standard_normal((6, 512)) * np.array([[1e-3], [1.0], [30.0], [2.0], [0.5], [7.0]])
+    gain = rng.standard_normal(512)
+    ref = torch.nn.functional.rms_norm(torch.from_numpy(x), (512,), weight=torch.from_numpy(gain), eps=1e-6)
+    np.testing.assert_allclose(orc.rms_norm(x, gain, 1e-6), ref.numpy(), rtol=1e-12, atol=1e-12)
+    unit = orc.rms_norm(x[1:], np.ones(512), 0.0)
+    np.testing.assert_allclose(np.sqrt(np.mean(unit ** 2, axis=1)), 1.0, rtol=1e-12)
+
+
+def test_cache_write_rows_against_scalar_loops():
+    """Brute force on a tiny case: the projection, the norm of the latent part and the
+    rotation of the shared key written out one element at a time."""
+    rng = np.random.default_rng(7)
+    T, M, R, Dr = 3, 8, 6, 4
+    hidden, W = rng.standard_normal((T, M)), rng.standard_normal((R + Dr, M))
+    gain, pos, eps = rng.standard_normal(R), np.array([0, 3, 11]), 1e-6
+    got = orc.cache_write_rows(hidden, W, gain, pos, R, eps=eps, rope_base=10000.0)
+    for t in range(T):
+        f = [sum(hidden[t][m] * W[j][m] for m in range(M)) for j in range(R + Dr)]
+        ms = sum(f[j] * f[j] for j in range(R)) / R
+        for j in range(R):
+            assert abs(got[t][j] - f[j] / math.sqrt(ms + eps) * gain[j]) < 1e-12
+        for i in range(Dr // 2):
+            th = 10000.0 ** (-2.0 * i / Dr) * pos[t]
+            a, b = f[R + i], f[R + Dr // 2 + i]
+            assert abs(got[t][R + i] - (a * math.cos(th) - b * math.sin(th))) < 1e-12
+            assert abs(got[t][R + Dr // 2 + i] - (a * math.sin(th) + b * math.cos(th))) < 1e-12
+
+
+def test_token_positions_follow_the_append_convention():
+    np.testing.assert_array_equal(orc.token_positions([5, 2, 9], 2), [3, 4, 0, 1, 7, 8])
