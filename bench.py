@@ -236,6 +236,49 @@ def wl_cache_bytes(spec, lens):
     return int(np.sum(lens, dtype=np.int64)) * (spec.R + spec.Dr) * elem
 
 
+def time_cache_write(step, spec, stream, M=7168, reps=20):
+    """The cache-write prologue (mla_cache_write: down projection of the step's new tokens'
+    hidden states, width M = 7168 as in DeepSeek-scale models, kv_rmsnorm, rotary shared
+    key, append; the query's rope part turned in place) timed on its own, outside the
+    step: CUDA events around each call on the launching stream. It rewrites the rows the
+    step's append wrote. None where the dims have no prologue kernel."""
+    import torch
+    import mla_latent_kv_46_b200 as mla
+    from mla_latent_kv_46_b200 import decoder as dec
+    from inputs import workloads as wl
+    if spec.dtype != "bf16" or spec.R != 512 or spec.Dr != 64 or spec.page_size != 64:
+        return None
+    pin = wl.prologue_inputs(spec, step.T, M, seed=3)
+    hidden, W, gain = (dec.to_torch(pin[k], step.device) for k in ("hidden", "W_DKV", "kv_gain"))
+
+    ws_bytes = mla.mla_cache_write_workspace_size(step.T, M)
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=step.device)
+
+    def call():
+        mla.mla_cache_write(hidden, W, gain, M, step.kv, step.block_table, step.seq_lens, step.B, step.q_len,
+                            step.max_pages, step.num_pages, step.q_rope, 1e-6, 10000.0, ws, ws_bytes, step.dims,
+                            stream)
+    for _ in range(3):
+        call()
+    torch.cuda.synchronize()
+    ts = []
+    for _ in range(reps):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        call()
+        e1.record(stream)
+        e1.synchronize()
+        ts.append(e0.elapsed_time(e1))
+    mla.mla_check_status()
+    ms = statistics.median(ts)
+    wbytes = (spec.R + spec.Dr) * M * 2
+    abytes = step.T * M * 2
+    return {"ms": ms, "hidden_width": M, "tokens": step.T, "weight_bytes": wbytes,
+            "gb_per_s": (wbytes + abytes) / (ms / 1e3) / 1e9, "launches": 2,
+            "kernels": "cache_write_gemm_kernel (split-K down projection), cache_write_finish_kernel (norm, "
+                       "rotations, append)"}
+
+
 def needs_flush(cache_bytes):
     """Inputs larger than twice the L2 evict it on their own: every step streams the whole
     cache through L2, so nothing a step reads is still resident at the next one. Smaller
@@ -432,6 +475,8 @@ def run_gpu(args):
            "h2d_bytes_per_step": hostin.h2d_bytes(step), "d2h_bytes_per_step": hostin.d2h_bytes(),
            "ms_per_step": e2e_ms / e2e_steps, "mode": e2e_mode}
 
+    prologue = time_cache_write(step, spec, stream)
+
     line = None
     if rank == 0:
         cpu = None
@@ -448,7 +493,7 @@ def run_gpu(args):
                 "config": workload_config(spec, w, argparse.Namespace(gpus=world, seqs=args.seqs), job_tokens),
                 "tflops": job_flops * args.steps / (total_ms_max / 1e3) / 1e12,
                 "per_kernel_ms": {n: per_kernel[n] / args.steps for n in names},
-                "roofline": roof, "cpu_baseline": cpu, "e2e": e2e,
+                "roofline": roof, "cpu_baseline": cpu, "e2e": e2e, "cache_write": prologue,
                 "gpu_launches": step.launches_per_step() * args.steps,
                 "clocks": clk.summary()}
         print(json.dumps(line), flush=True)

@@ -137,6 +137,32 @@ mla_status mla_cache_append(void* kv_cache, const int32_t* block_table, const in
                             const void* new_ckr, int32_t B, int32_t q_len, int32_t max_pages,
                             int32_t num_pages, mla_dims d, void* stream);
 
+/* ---------------------------------------------------------------- cache-write prologue
+ * The rows a step appends, computed from the new tokens' hidden states, then appended
+ * as mla_cache_append does (survey row f1). For every new token t (token i of sequence
+ * b, position pos = seq_lens[b] - q_len + i):
+ *   f = W_DKV h_t                       (kimi-k3 docs "GatedMLA", "Projection geometry and
+ *                                        stored weights": one down projection M -> R_kv + D_s
+ *                                        to the compressed KV feature and the shared key)
+ *   c = f[:R] / sqrt(mean(f[:R]^2) + eps) * kv_gain       (kv_rmsnorm on the feature)
+ *   k = rope(f[R:], pos): dims i and i + Dr/2 turned by pos * rope_base^(-2i/Dr)
+ *       (the shared key carries the position: modeldna "learn/mla", "Under the hood";
+ *       the frequencies and the pairing are the usual reading, the pages fix neither)
+ * and [c ; k] (bf16) is written to the token's row of its page. If q_rope is not NULL
+ * its rows [B*q_len][H][Dr] (bf16) are turned in place by the same rule at the query
+ * token's position. fp32 accumulation and normalisation; angles in double precision.
+ *   hidden [B*q_len][M] bf16, W_DKV [R+Dr][M] bf16 (out x in), kv_gain [R] bf16; M a
+ *   multiple of 64; dims bf16, R=512, Dr=64, page_size=64 (else MLA_ERR_UNSUPPORTED, as
+ *   under the SIMT policy: the prologue has only a tensor-core kernel). Tokens with pos <
+ *   0 are skipped; a page id outside the pool is skipped and reported by mla_check_status.
+ *   workspace: >= mla_cache_write_workspace_size(B*q_len, M) bytes, 16-byte aligned: the
+ *   down projection is split over K (fp32 partial sums there, added by the last kernel). */
+size_t mla_cache_write_workspace_size(int32_t T, int32_t M);
+mla_status mla_cache_write(const void* hidden, const void* W_DKV, const void* kv_gain, int32_t M,
+                           void* kv_cache, const int32_t* block_table, const int32_t* seq_lens, int32_t B,
+                           int32_t q_len, int32_t max_pages, int32_t num_pages, void* q_rope, float eps,
+                           float rope_base, void* workspace, size_t workspace_bytes, mla_dims d, void* stream);
+
 /* ---------------------------------------------------------------- a1: absorb the query
  * q_lat[t][h][:] = q_nope[t][h][:] @ W_UK[h]  (modeldna "learn/mla", "Under the
  * hood": the key up-projection folds into the query; W_UK[h] is head h's slice

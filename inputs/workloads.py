@@ -254,6 +254,17 @@ def latent_queries(spec: WorkloadSpec, T: int, seed: int = 0) -> np.ndarray:
     return _store(spec, g.standard_normal((T, spec.H, spec.R), dtype=np.float32) * np.float32(0.5))
 
 
+def prologue_inputs(spec: WorkloadSpec, T: int, M: int, seed: int = 0) -> dict:
+    """Seeded inputs of the cache-write prologue in the workload's storage dtype: hidden
+    states [T, M] ~ N(0, 1), the down projection W_DKV [R + Dr, M] ~ N(0, 1/M) (unit-scale
+    outputs) and the latent norm's gain [R] ~ 1 + N(0, 0.1^2)."""
+    g = _rng(seed, 8)
+    hidden = g.standard_normal((T, M), dtype=np.float32)
+    w = g.standard_normal((spec.R + spec.Dr, M), dtype=np.float32) * np.float32(1.0 / math.sqrt(M))
+    gain = np.float32(1.0) + g.standard_normal(spec.R, dtype=np.float32) * np.float32(0.1)
+    return dict(hidden=_store(spec, hidden), W_DKV=_store(spec, w), kv_gain=_store(spec, gain))
+
+
 def latent_outputs(spec: WorkloadSpec, T: int, seed: int = 0, fp32: bool = False) -> np.ndarray:
     """Seeded stand-in for a latent attention output, [T, H, R]: entries N(0, 0.1^2),
     in the workload's storage dtype, or as float32 values when `fp32`."""

@@ -25,7 +25,7 @@ STATUS_NAMES = {0: "MLA_OK", -1: "MLA_ERR_INVALID", -2: "MLA_ERR_UNSUPPORTED", -
 
 # Every symbol include/mla.h declares.
 EXPORTS = ("mla_abi_version", "mla_last_error", "mla_set_policy", "mla_set_wait_timeout_ns",
-           "mla_check_status", "mla_cache_append", "mla_absorb_q", "mla_plan_capacity", "mla_plan_splits",
+           "mla_check_status", "mla_cache_append", "mla_cache_write", "mla_cache_write_workspace_size", "mla_absorb_q", "mla_plan_capacity", "mla_plan_splits",
            "mla_workspace_size", "mla_decode_attn", "mla_combine", "mla_out_proj", "mla_decode_attn_noalloc",
            "mla_debug_drop_page_load")
 
@@ -65,6 +65,8 @@ def _load():
         "mla_debug_drop_page_load": (I32, [I32]),
         "mla_check_status": (I32, [P]),
         "mla_cache_append": (I32, [P, P, P, P, I32, I32, I32, I32, D, P]),
+        "mla_cache_write": (I32, [P, P, P, I32, P, P, P, I32, I32, I32, I32, P, F, F, P, SZ, D, P]),
+        "mla_cache_write_workspace_size": (SZ, [I32, I32]),
         "mla_absorb_q": (I32, [P, P, P, I32, D, P]),
         "mla_plan_capacity": (SZ, [I32, I32, I32]),
         "mla_plan_splits": (I32, [P, I32, I32, I32, D, I32, P, SZ, INFO]),
@@ -135,6 +137,17 @@ def mla_check_status(stream=None) -> None:
 def mla_cache_append(kv_cache, block_table, seq_lens, new_ckr, B, q_len, max_pages, num_pages, dims, stream=None):
     _check(_lib.mla_cache_append(_ptr(kv_cache), _ptr(block_table), _ptr(seq_lens), _ptr(new_ckr), B, q_len,
                                  max_pages, num_pages, dims, _stream(stream)), "mla_cache_append")
+
+
+def mla_cache_write_workspace_size(T, M) -> int:
+    return _lib.mla_cache_write_workspace_size(T, M)
+
+
+def mla_cache_write(hidden, W_DKV, kv_gain, M, kv_cache, block_table, seq_lens, B, q_len, max_pages, num_pages,
+                    q_rope, eps, rope_base, workspace, workspace_bytes, dims, stream=None):
+    _check(_lib.mla_cache_write(_ptr(hidden), _ptr(W_DKV), _ptr(kv_gain), M, _ptr(kv_cache), _ptr(block_table),
+                                _ptr(seq_lens), B, q_len, max_pages, num_pages, _ptr(q_rope), eps, rope_base,
+                                _ptr(workspace), workspace_bytes, dims, _stream(stream)), "mla_cache_write")
 
 
 def mla_absorb_q(q_nope, W_UK, q_lat, T, dims, stream=None):

@@ -22,6 +22,7 @@
 #include "decode_tc.cuh"
 #include "gemm_tc.cuh"
 #include "decode_2sm.cuh"
+#include "cache_write.cuh"
 
 namespace {
 
@@ -319,6 +320,64 @@ mla_status mla_cache_append(void* kv_cache, const int32_t* block_table, const in
         static_cast<float*>(kv_cache), block_table, seq_lens, static_cast<const float*>(new_ckr), q_len,
         max_pages, num_pages, row, d.page_size);
   return launch_check("cache_append");
+}
+
+// ------------------------------------------------------------------------------- cache-write prologue
+size_t mla_cache_write_workspace_size(int32_t T, int32_t M) {
+  if (T <= 0 || M <= 0 || M % mla::cw::kKB != 0) return 0;
+  return (size_t)mla::cw::slices_for(M) * (size_t)T * mla::cw::kRow * sizeof(float);
+}
+
+mla_status mla_cache_write(const void* hidden, const void* W_DKV, const void* kv_gain, int32_t M,
+                           void* kv_cache, const int32_t* block_table, const int32_t* seq_lens, int32_t B,
+                           int32_t q_len, int32_t max_pages, int32_t num_pages, void* q_rope, float eps,
+                           float rope_base, void* workspace, size_t workspace_bytes, mla_dims d, void* stream) {
+  if (mla_status s = check_dims(d)) return s;
+  if (B < 0 || q_len <= 0 || max_pages <= 0 || num_pages <= 0 || M <= 0)
+    return fail(MLA_ERR_INVALID, "bad sizes B=%d q_len=%d max_pages=%d num_pages=%d M=%d", B, q_len, max_pages,
+                num_pages, M);
+  if (!(eps >= 0.f) || !std::isfinite(eps)) return fail(MLA_ERR_INVALID, "eps must be finite and >= 0");
+  if (!(rope_base > 1.f) || !std::isfinite(rope_base)) return fail(MLA_ERR_INVALID, "rope_base must be > 1");
+  if (d.dtype != MLA_BF16 || d.R != mla::cw::kR || d.Dr != mla::cw::kDr || d.page_size != mla::cw::kPage ||
+      M % mla::cw::kKB != 0)
+    return fail(MLA_ERR_UNSUPPORTED, "the cache-write prologue needs bf16, R=512, Dr=64, page_size=64, M %% 64 == 0");
+  if (g_policy.load() == MLA_POLICY_SIMT)
+    return fail(MLA_ERR_UNSUPPORTED, "the cache-write prologue has only a tensor-core kernel");
+  if (B == 0) return ok();
+  if (!hidden || !W_DKV || !kv_gain || !kv_cache || !block_table || !seq_lens)
+    return fail(MLA_ERR_INVALID, "null pointer");
+  const int32_t T = B * q_len;
+  const size_t need = mla_cache_write_workspace_size(T, M);
+  if (!workspace || workspace_bytes < need)
+    return fail(MLA_ERR_WORKSPACE, "workspace %zu bytes < %zu needed", workspace_bytes, need);
+  if (reinterpret_cast<uintptr_t>(workspace) % 16 != 0) return fail(MLA_ERR_INVALID, "workspace not 16-byte aligned");
+  CUtensorMap ta, tb;
+  if (mla_status s = make_map_2d(&ta, hidden, (uint64_t)M, (uint64_t)T, (uint64_t)M * 2, 128)) return s;
+  if (mla_status s = make_map_2d(&tb, W_DKV, (uint64_t)M, (uint64_t)(d.R + d.Dr), (uint64_t)M * 2, 64)) return s;
+  mla::cw::Params p;
+  p.kv = static_cast<__nv_bfloat16*>(kv_cache);
+  p.block_table = block_table;
+  p.seq_lens = seq_lens;
+  p.gain = static_cast<const __nv_bfloat16*>(kv_gain);
+  p.part = static_cast<float*>(workspace);
+  p.T = T;
+  p.q_len = q_len;
+  p.max_pages = max_pages;
+  p.num_pages = num_pages;
+  p.kblk = M / mla::cw::kKB;
+  p.slices = mla::cw::slices_for(M);
+  p.eps = eps;
+  p.rope_base = rope_base;
+  p.timeout_ns = g_timeout_ns.load();
+  cudaStream_t st = as_stream(stream);
+  if (mla_status s = ensure_smem_attr((const void*)mla::cw::cache_write_gemm_kernel, mla::cw::Cfg::kSmemBytes))
+    return s;
+  const dim3 grid((T + mla::cw::kM - 1) / mla::cw::kM, mla::cw::kColBlocks, p.slices);
+  mla::cw::cache_write_gemm_kernel<<<grid, 128, mla::cw::Cfg::kSmemBytes, st>>>(ta, tb, p);
+  if (mla_status s = launch_check("cache_write (down projection)")) return s;
+  mla::cw::cache_write_finish_kernel<<<T, mla::cw::kFinishThreads, 0, st>>>(
+      p, static_cast<__nv_bfloat16*>(q_rope), d.H);
+  return launch_check("cache_write (norm, rotation, append)");
 }
 
 // ------------------------------------------------------------------------------- absorb

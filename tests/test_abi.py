@@ -163,6 +163,36 @@ def test_plan_puts_each_token_of_128_heads_on_its_own_aligned_slot_block(q_len):
         assert all(segs[i][1] == segs[i + 1][0] for i in range(len(segs) - 1))
 
 
+@pytest.mark.parametrize("case", ["null", "dims", "eps", "base", "M", "workspace"])
+def test_cache_write_rejects_bad_arguments_before_launch(case):
+    d = dims(H=128)
+    args = dict(hidden=16, W_DKV=16, kv_gain=16, M=1024, kv_cache=16, block_table=16, seq_lens=16, B=2, q_len=1,
+                max_pages=4, num_pages=8, q_rope=None, eps=1e-6, rope_base=10000.0, workspace=16,
+                workspace_bytes=1 << 30, dims=d)
+    if case == "null":
+        args["hidden"] = None
+    elif case == "dims":
+        args["dims"] = dims(H=128, R=256)
+    elif case == "eps":
+        args["eps"] = float("nan")
+    elif case == "base":
+        args["rope_base"] = 1.0
+    elif case == "M":
+        args["M"] = 100
+    else:
+        args["workspace_bytes"] = mla.mla_cache_write_workspace_size(2, 1024) - 1
+    with pytest.raises(mla.MlaError) as e:
+        mla.mla_cache_write(**args, stream=0)
+    assert e.value.status in (mla._binding.MLA_ERR_INVALID, mla._binding.MLA_ERR_UNSUPPORTED,
+                              mla._binding.MLA_ERR_WORKSPACE)
+
+
+def test_cache_write_workspace_holds_one_fp32_row_per_token_and_k_slice():
+    assert mla.mla_cache_write_workspace_size(128, 7168) == 16 * 128 * 576 * 4
+    assert mla.mla_cache_write_workspace_size(5, 1024) == 8 * 5 * 576 * 4
+    assert mla.mla_cache_write_workspace_size(5, 100) == 0
+
+
 def test_plan_balances_pages_for_the_single_cta_kernel():
     """Other head counts (one CTA per 64 heads) are planned on pages alone: slots differ
     by at most one page."""

@@ -466,3 +466,54 @@ def test_decode_is_deterministic(name):
         outs.append((step.out.clone(), step.lse.clone()))
     mla.mla_check_status()
     assert torch.equal(outs[0][0], outs[1][0]) and torch.equal(outs[0][1], outs[1][1])
+
+
+# ----------------------------------------------------------------------------- cache-write prologue
+
+def _cache_write_case(lens, q_len, M, seed=31, with_q=True):
+    spec = small_spec(H=128, q_len=q_len)
+    w = wl.make(spec, seed=seed, seq_lens=lens, new_rows_in_cache=False)
+    step = dec.DecodeStep(w)
+    T = step.T
+    pin = wl.prologue_inputs(spec, T, M, seed=seed)
+    hidden, W, gain = (dec.to_torch(pin[k], step.device) for k in ("hidden", "W_DKV", "kv_gain"))
+    before = step.kv.view(torch.int16).cpu().numpy()      # bit patterns
+    q0 = host(step.q_rope)
+    ws_bytes = mla.mla_cache_write_workspace_size(T, M)
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=step.device)
+    mla.mla_cache_write(hidden, W, gain, M, step.kv, step.block_table, step.seq_lens, step.B, q_len, step.max_pages,
+                        step.num_pages, step.q_rope if with_q else None, 1e-6, 10000.0, ws, ws_bytes, step.dims)
+    torch.cuda.synchronize()
+    mla.mla_check_status()
+    pos = orc.token_positions(lens, q_len)
+    rows = orc.cache_write_rows(pin["hidden"], pin["W_DKV"], pin["kv_gain"], pos, spec.R, eps=1e-6)
+    after = step.kv.view(torch.int16).cpu().numpy()
+    bt = np.asarray(w["block_table"])
+    written = np.zeros(after.shape[:2], bool)
+    for t, p in enumerate(pos):
+        if p < 0:
+            continue
+        b = t // q_len
+        pg, r = int(bt[b][p // 64]), p % 64
+        written[pg, r] = True
+        got = orc.to_f64(after[pg, r].view(np.uint16))
+        assert_close(got, rows[t], False, f"cache row of token {t} (position {p})")
+    np.testing.assert_array_equal(after[~written], before[~written])   # nothing else touched
+    if with_q:
+        qr = orc.rope(q0, pos[:, None])
+        assert_close(host(step.q_rope), qr, False, "q_rope turned in place")
+    return rows
+
+
+@pytest.mark.parametrize("q_len,lens", [(1, [70, 5, 129, 1]), (2, [70, 2, 129]), (4, [300, 4, 65])])
+def test_cache_write_matches_oracle(q_len, lens):
+    """Down projection, kv_rmsnorm of the latent, rotary shared key, append: the rows the
+    prologue writes against the oracle's, at the bf16 bound, and every other cache row
+    unchanged; the query's rope part turned in place."""
+    _cache_write_case(lens, q_len, M=1024)
+
+
+def test_cache_write_at_model_width_and_long_positions():
+    """Hidden width 7168 (112 K blocks) and positions up to 131071, where the lowest
+    frequency's angle is large: every written row against the oracle."""
+    _cache_write_case([131072, 4096, 70000, 1], 1, M=7168)
