@@ -12,6 +12,8 @@ Sources (page title, then the section used):
               then compute causal attention", "Output projection and optional gate".
   [Primer]    modeldna.ai, "learn/mla": "Under the hood" and its cache-size table.
   [Ticket]    "MLA + KV cache (Tier 3 #5)": "Description", "Acceptance criteria".
+  [Softved]   softved.com.np, "Introduction to MLA vs. KV Cache in Large Language
+              Models": "Practical Implementation Tips for MLA in LLM Serving".
   [Tutorial]  "ARCH-MLA. Multihead Latent Attention | MLA 与紧凑 KV 表示":
               "Step 4：实现 KV 表示账本" (the KV-state ledger and its tests).
 
@@ -20,6 +22,7 @@ Modules:
               the split-KV log-sum-exp merge, cache append, full causal forward.
   loops       a scalar pure-Python restatement for tiny brute-force cases.
   ledger      the per-token KV-state byte ledger.
+  fp8         the 8-bit (E4M3) cache: rounding, codes, per-token power-of-two scales.
 
 Every function here is pinned by a ``-m "not gpu"`` test in tests/test_oracle.py
 against something other than itself (closed forms, a library routine, brute force,
