@@ -231,7 +231,11 @@ def reduce_over_ranks(world, device, sums=(), maxes=()):
     return out[0], out[1]
 
 
-def wl_cache_bytes(spec, lens):
+def wl_cache_bytes(spec, lens, fp8=False):
+    """Algorithmic cache bytes of one pass: every valid row once; the 8-bit cache reads
+    R + Dr codes and one scale byte per token."""
+    if fp8:
+        return int(np.sum(lens, dtype=np.int64)) * (spec.R + spec.Dr + 1)
     elem = 2 if spec.dtype == "bf16" else 4
     return int(np.sum(lens, dtype=np.int64)) * (spec.R + spec.Dr) * elem
 
@@ -303,12 +307,15 @@ def workload_config(spec, w, args, job_tokens=None):
            "seq_lens": (f"uniform in [{spec.ragged[0]},{spec.ragged[1]}], {seed}" if spec.ragged
                         else f"{spec.seq_len} each"),
            "cached_tokens": int(np.sum(lens, dtype=np.int64)),
-           "l2": l2_method(wl_cache_bytes(spec, lens)),
+           "l2": l2_method(wl_cache_bytes(spec, lens, getattr(args, "cache", "bf16") == "fp8")),
            "parallelism": f"replicas x{args.gpus} (independent sequences per GPU)"}
     if args.gpus > 1:
         cfg["global_batch"] = int(len(lens)) * args.gpus
         if job_tokens is not None:
             cfg["cached_tokens_all_ranks"] = int(job_tokens)
+    if getattr(args, "cache", "bf16") == "fp8":
+        cfg["cache"] = ("E4M3 codes (576 per token) + one power-of-two scale byte per token, 577 bytes per "
+                        "token; the bf16 rows of the workload quantised once on the device before timing")
     if getattr(args, "seqs", 0):
         cfg["subset"] = f"first {args.seqs} sequences only (profiling run, not a bench line)"
     return cfg
@@ -341,7 +348,8 @@ def run_gpu(args):
         w = wl.make(spec, seed=rank, seq_lens=wl.seq_lens_of(spec, rank)[:args.seqs])
     else:
         w = wl.make(spec, seed=rank)
-    step = dec.DecodeStep(w, device=dev)
+    fp8 = args.cache == "fp8"
+    step = dec.DecodeStep(w, device=dev, cache=args.cache)
     mla.mla_set_policy(mla.MLA_POLICY_AUTO)
     stream = torch.cuda.current_stream()
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
@@ -360,7 +368,7 @@ def run_gpu(args):
     mla.mla_check_status()
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(len(names) + 1)] for _ in range(args.steps)]
     barrier()
-    flush_each = needs_flush(wl.cache_bytes(spec, w["seq_lens"]))
+    flush_each = needs_flush(wl_cache_bytes(spec, w["seq_lens"], fp8))
     with ClockSampler(dev.index) as clk:
         for k in range(args.steps):
             if flush_each:
@@ -387,7 +395,7 @@ def run_gpu(args):
         step_ms.append(e[0].elapsed_time(e[-1]))
     # this rank's batch; the job's work is the sum over ranks (each rank decodes its own
     # ragged batch) and its time the slowest rank's
-    cache_bytes = wl.cache_bytes(spec, w["seq_lens"])
+    cache_bytes = wl_cache_bytes(spec, w["seq_lens"], fp8)
     flops = wl.attention_flops(spec, w["seq_lens"])
     tokens = int(np.sum(w["seq_lens"], dtype=np.int64))
     (job_bytes, job_flops, job_tokens), (total_ms_max,) = reduce_over_ranks(
@@ -399,9 +407,11 @@ def run_gpu(args):
     peaks, peak_src = load_peaks()
     attn_ms = per_kernel["attend"] / args.steps
     t_hbm = cache_bytes / (peaks["hbm_gbs"] * 1e9)
+    # (the 8-bit cache too: its query enters the score MMAs as two E4M3 pieces, two 8-bit
+    # MMAs per K step at twice the rate, the tensor time of one bf16 MMA)
     t_tc = flops / (peaks["bf16_tflops"] * 1e12)
     bound = "hbm" if t_hbm >= t_tc else "tensor"
-    traffic, sha = traffic_record(spec.name, spec.H, spec.q_len)
+    traffic, sha = traffic_record(spec.name + ("_fp8" if fp8 else ""), spec.H, spec.q_len)
     if args.seqs:
         traffic = None   # the committed figure is for the whole workload
     if bound == "hbm":
@@ -475,7 +485,7 @@ def run_gpu(args):
            "h2d_bytes_per_step": hostin.h2d_bytes(step), "d2h_bytes_per_step": hostin.d2h_bytes(),
            "ms_per_step": e2e_ms / e2e_steps, "mode": e2e_mode}
 
-    prologue = time_cache_write(step, spec, stream)
+    prologue = None if fp8 else time_cache_write(step, spec, stream)
 
     line = None
     if rank == 0:
@@ -489,8 +499,9 @@ def run_gpu(args):
             cpu["absorbed_form"] = {"value": b2 / t2 / 1e9, "unit": "GB/s", "sample": desc2, "seconds": t2}
         line = {"metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
                 "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
-                "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-                "config": workload_config(spec, w, argparse.Namespace(gpus=world, seqs=args.seqs), job_tokens),
+                "vs_baseline": None, "dtype": "e4m3 cache, bf16 queries" if fp8 else "bf16", "data": "synthetic",
+                "config": workload_config(spec, w, argparse.Namespace(gpus=world, seqs=args.seqs, cache=args.cache),
+                                          job_tokens),
                 "tflops": job_flops * args.steps / (total_ms_max / 1e3) / 1e12,
                 "per_kernel_ms": {n: per_kernel[n] / args.steps for n in names},
                 "roofline": roof, "cpu_baseline": cpu, "e2e": e2e, "cache_write": prologue,
@@ -510,6 +521,8 @@ def main():
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--cache", default="bf16", choices=["bf16", "fp8"],
+                    help="cache format: bf16 rows, or E4M3 codes with per-token scales")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")

@@ -54,7 +54,7 @@
 extern "C" {
 #endif
 
-#define MLA_ABI_VERSION 3
+#define MLA_ABI_VERSION 4
 
 typedef enum {
   MLA_OK = 0,
@@ -236,6 +236,53 @@ mla_status mla_combine(const int32_t* plan_dev, const mla_plan_info* info, const
  * per K step, so o_lat keeps ~16 significant bits; fp32 accumulation)              */
 mla_status mla_out_proj(const void* o_lat, const void* W_UV, void* out, int32_t T, mla_dims d,
                         void* stream);
+
+/* ---------------------------------------------------------------- 8-bit (E4M3) latent cache
+ * The softved page "Introduction to MLA vs. KV Cache in Large Language Models" ("Practical
+ * Implementation Tips for MLA in LLM Serving") advises quantising the latent cache to cut
+ * its memory further; it fixes no format. This library's reading (survey row f2):
+ *  - every element of a cached row [c ; k_rope] is one byte, an E4M3 code of the OCP 8-bit
+ *    floating-point format (sign, 4 exponent bits with bias 7, 3 mantissa bits, subnormals,
+ *    no infinities, 0x7F/0xFF NaN, largest finite 448): kv_codes [num_pages][64][576] uint8;
+ *  - every row has one power-of-two scale 2^k shared by c and k_rope, stored as the byte
+ *    k + 127: kv_scales [num_pages][64] uint8. k is the smallest integer in [-126, 7] with
+ *    max_i |x_i| <= 448 * 2^k (a row beyond 448 * 2^7 keeps k = 7 and saturates);
+ *  - code_i = x_i * 2^-k rounded to nearest, ties to even, saturating at +-448; the row
+ *    stands for code_i * 2^k exactly. 577 bytes per token instead of 1,152.
+ * Decoding attends over those exact values: mla_decode_attn_fp8 computes what
+ * mla_decode_attn computes for a bf16 cache holding code * 2^k (which bf16 represents
+ * exactly). Queries, o_lat, lse, plans, mla_combine and mla_out_proj are unchanged.
+ * Geometry: bf16 rows, R=512, Dr=64, page_size=64 (else MLA_ERR_UNSUPPORTED).
+ *
+ * Quantises n dense bf16 rows [n][576] into codes [n][576] and scale bytes [n]
+ * (rows 16-byte aligned, codes 8-byte aligned). Converts an existing bf16 pool. */
+mla_status mla_quantize_rows_fp8(const void* rows, void* codes, void* scales, int64_t n, mla_dims d,
+                                 void* stream);
+
+/* mla_cache_append for the 8-bit cache: new_ckr[b*q_len + i] (bf16 [576], 16-byte
+ * aligned) is quantised into position seq_lens[b] - q_len + i of sequence b (codes and
+ * scale byte). Positions < 0 are skipped; a page id outside the pool is skipped and
+ * reported by mla_check_status. */
+mla_status mla_cache_append_fp8(void* kv_codes, void* kv_scales, const int32_t* block_table,
+                                const int32_t* seq_lens, const void* new_ckr, int32_t B, int32_t q_len,
+                                int32_t max_pages, int32_t num_pages, mla_dims d, void* stream);
+
+/* Workspace of mla_decode_attn_fp8: the split partials exactly as mla_workspace_size lays
+ * them out (so mla_combine takes the same buffer), then the query split into two E4M3
+ * pieces per element ([2][T*H][576] bytes) and its per-row scales ([T*H] fp32). */
+size_t mla_workspace_size_fp8(const mla_plan_info* info, mla_dims d);
+
+/* a3-a5 over the 8-bit cache, for a plan made by mla_plan_splits with the same dims, q_len
+ * and max_pages. Arguments as for mla_decode_attn, plus kv_scales (16-byte aligned); the workspace is
+ * required (>= mla_workspace_size_fp8, 256-byte aligned). Two launches: the query split
+ * (q_lat, q_rope -> workspace), then the SM-pair decode kernel, which scores against the
+ * codes on the 8-bit tensor cores, applies each token's scale to its score column, and
+ * widens the codes times the scale to bf16 for the value sum. H must be 64 or 128. */
+mla_status mla_decode_attn_fp8(const void* q_lat, const void* q_rope, const void* kv_codes, const void* kv_scales,
+                               const int32_t* block_table, const int32_t* seq_lens, int32_t B, int32_t q_len,
+                               int32_t max_pages, int32_t num_pages, float scale, const int32_t* plan_dev,
+                               const mla_plan_info* info, void* o_lat, float* lse, void* workspace,
+                               size_t workspace_bytes, mla_dims d, void* stream);
 
 /* ---------------------------------------------------------------- allocation-free decode
  * The pages describe no counterpart of this call; it exists for callers that cannot

@@ -27,7 +27,8 @@ STATUS_NAMES = {0: "MLA_OK", -1: "MLA_ERR_INVALID", -2: "MLA_ERR_UNSUPPORTED", -
 EXPORTS = ("mla_abi_version", "mla_last_error", "mla_set_policy", "mla_set_wait_timeout_ns",
            "mla_check_status", "mla_cache_append", "mla_cache_write", "mla_cache_write_workspace_size", "mla_absorb_q", "mla_plan_capacity", "mla_plan_splits",
            "mla_workspace_size", "mla_decode_attn", "mla_combine", "mla_out_proj", "mla_decode_attn_noalloc",
-           "mla_debug_drop_page_load")
+           "mla_debug_drop_page_load", "mla_quantize_rows_fp8", "mla_cache_append_fp8", "mla_workspace_size_fp8",
+           "mla_decode_attn_fp8")
 
 
 class MlaError(RuntimeError):
@@ -56,6 +57,7 @@ def _load():
         raise ImportError(f"{LIB_PATH} is not built; run `python mla_latent_kv_46_b200/build.py`")
     lib = ctypes.CDLL(LIB_PATH)
     P, I32, U64, SZ, F = ctypes.c_void_p, ctypes.c_int32, ctypes.c_uint64, ctypes.c_size_t, ctypes.c_float
+    I64 = ctypes.c_int64
     D, INFO = Dims, ctypes.POINTER(PlanInfo)
     sig = {
         "mla_abi_version": (I32, []),
@@ -75,6 +77,10 @@ def _load():
         "mla_combine": (I32, [P, INFO, P, SZ, P, P, D, P]),
         "mla_out_proj": (I32, [P, P, P, I32, D, P]),
         "mla_decode_attn_noalloc": (I32, [P, P, P, P, P, I32, I32, I32, I32, F, P, INFO, P, P, D, P]),
+        "mla_quantize_rows_fp8": (I32, [P, P, P, I64, D, P]),
+        "mla_cache_append_fp8": (I32, [P, P, P, P, P, I32, I32, I32, I32, D, P]),
+        "mla_workspace_size_fp8": (SZ, [INFO, D]),
+        "mla_decode_attn_fp8": (I32, [P, P, P, P, P, P, I32, I32, I32, I32, F, P, INFO, P, P, P, SZ, D, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -202,3 +208,27 @@ def dims_of(spec) -> Dims:
     """Dims from an inputs.workloads.WorkloadSpec."""
     return Dims(spec.H, spec.Dn, spec.Dr, spec.Dv, spec.R, spec.page_size,
                 MLA_BF16 if spec.dtype == "bf16" else MLA_F32)
+
+
+def mla_quantize_rows_fp8(rows, codes, scales, n, dims, stream=None):
+    _check(_lib.mla_quantize_rows_fp8(_ptr(rows), _ptr(codes), _ptr(scales), n, dims, _stream(stream)),
+           "mla_quantize_rows_fp8")
+
+
+def mla_cache_append_fp8(kv_codes, kv_scales, block_table, seq_lens, new_ckr, B, q_len, max_pages, num_pages, dims,
+                         stream=None):
+    _check(_lib.mla_cache_append_fp8(_ptr(kv_codes), _ptr(kv_scales), _ptr(block_table), _ptr(seq_lens),
+                                     _ptr(new_ckr), B, q_len, max_pages, num_pages, dims, _stream(stream)),
+           "mla_cache_append_fp8")
+
+
+def mla_workspace_size_fp8(info, dims) -> int:
+    return _lib.mla_workspace_size_fp8(ctypes.byref(info), dims)
+
+
+def mla_decode_attn_fp8(q_lat, q_rope, kv_codes, kv_scales, block_table, seq_lens, B, q_len, max_pages, num_pages,
+                        scale, plan_dev, info, o_lat, lse, workspace, workspace_bytes, dims, stream=None):
+    _check(_lib.mla_decode_attn_fp8(_ptr(q_lat), _ptr(q_rope), _ptr(kv_codes), _ptr(kv_scales), _ptr(block_table),
+                                    _ptr(seq_lens), B, q_len, max_pages, num_pages, scale, _ptr(plan_dev),
+                                    ctypes.byref(info), _ptr(o_lat), _ptr(lse), _ptr(workspace), workspace_bytes,
+                                    dims, _stream(stream)), "mla_decode_attn_fp8")

@@ -61,6 +61,19 @@
 // travel the same way to a barrier of the receiving CTA. MMA completion is committed
 // to both CTAs. Every wait is bounded; a CTA that gives up raises the device status
 // word and sets both CTAs' abort flags.
+//
+// 8-bit cache (template F8 = true; codes and per-token power-of-two scales, see
+// fp8_kernels.cuh). The query arrives split into two E4M3 pieces per element (hi, lo)
+// times 2^e per row. Scores: one tcgen05.mma.cta_group::2.kind::f8f6f4 with M = 256 per
+// K step of 32 codes: each CTA's 128 A rows are its 64 rows' hi pieces (TMEM lanes 0-63)
+// and lo pieces (lanes 64-127), so lane m holds hi . codes and lane 64 + m lo . codes of
+// row m for all 64 tokens; the two softmax warps of those lanes swap one half of the
+// columns through shared memory and add. The softmax scales column t by the token's 2^k
+// and the row by 2^-e. Values: four more warps (one warpgroup) widen the page's codes of
+// the CTA's 256 latent columns, times 2^k, to bf16 in the value slot (exact), so the value
+// MMA and P are those of the bf16 cache. Warp 2 loads those codes and the page's 64
+// scale bytes into a local ring; the converter publishes the page's scales to the softmax
+// before it waits for a free value slot.
 #pragma once
 
 #include "common.cuh"
@@ -76,35 +89,63 @@ constexpr int kPage = 64, kR = 512, kDr = 64, kRow = kR + kDr;
 constexpr int kChunks = kRow / 64;     // 64-column chunks of a row (8 latent + rope)
 constexpr int kQTmemChunks = 7;        // query chunks held in TMEM (latent 0-447)
 constexpr int kQSmemChunks = kChunks - kQTmemChunks;   // latent 448-511 and rope
-constexpr int kBox32 = 32 * 128;       // 32 rows x 64 bf16, 128-byte swizzle
-constexpr int kBox64 = 64 * 128;       // 64 rows x 64 bf16
-constexpr int kQBytes = kQSmemChunks * kBox64;     // 16,384
-constexpr int kQKSlotBytes = kChunks * kBox32;     // 36,864
-constexpr int kPVSlotBytes = 8 * kBox32;           // 32,768
-constexpr int kQKSlots = 3, kPVSlots = 2;
+constexpr int kBox32 = 32 * 128;       // 32 rows x 128 bytes, 128-byte swizzle
+constexpr int kBox64 = 64 * 128;       // 64 rows x 128 bytes
 constexpr int kPBytes = kCtaRows * kPage * 2;      // 8,192
 constexpr int kSoftWarps = 4;
 constexpr int kFirstSoftWarp = 4;
-constexpr int kThreads = 32 * (kFirstSoftWarp + kSoftWarps);
+constexpr int kFirstConvWarp = 8;      // (8-bit cache) the warpgroup that widens value operands
+constexpr int kConvWarps = 4;
+// 8-bit cache: a row is 576 one-byte codes; TMA boxes are 128 codes wide, the fifth (at
+// column 512) holds the 64 rope codes and 64 columns of zero fill
+constexpr int kF8Boxes = 5;
+constexpr int kF8Steps = kRow / 32;    // K steps of 32 codes per row (18)
+constexpr int kF8QTmemSteps = 14;      // of which the query holds 0-13 (columns 0-447) in TMEM
 
-constexpr int kOffQ = 0;
-constexpr int kOffQK = kOffQ + kQBytes;
-constexpr int kOffPV = kOffQK + kQKSlots * kQKSlotBytes;
-constexpr int kOffP = kOffPV + kPVSlots * kPVSlotBytes;   // two buffers of P_hi then P_lo
-constexpr int kMaxBars = 32;
-constexpr int kOffBar = kOffP + 4 * kPBytes;              // kMaxBars mbarriers
-constexpr int kOffXmax = kOffBar + kMaxBars * 8;          // float[2][128]: row maxima of the lane halves
-constexpr int kOffXl = kOffXmax + 2 * 128 * 4;            // float[128]: row sums of the lane halves
-constexpr int kOffFlag = kOffXl + 128 * 4;                // uint32[4][8] (even CTA): P_lo wanted, per tile % 4
-                                                          // and softmax warp (0-3 even CTA, 4-7 odd CTA)
-constexpr int kOffXal = kOffFlag + 4 * 8 * 4;             // float[2][128]: the pair's rescale factors, per row
-constexpr int kOffXflg = kOffXal + 2 * 128 * 4;           // uint32[2][4]: a moved reference among 32 rows
-constexpr int kOffXinv = kOffXflg + 2 * 4 * 4;            // float[128]: the pair's 1 / l, per row
-constexpr int kOffTmem = kOffXinv + 128 * 4;
-constexpr int kOffAbort = kOffTmem + 8;
-constexpr int kSmemUsed = kOffAbort + 8;
-constexpr int kSmemBytes = kSmemUsed + 1024;
-static_assert(kSmemBytes <= 232448, "shared memory of one CTA");
+// Shared-memory layout: F8 = false for the bf16 cache, true for the 8-bit cache.
+template <bool F8>
+struct Lay {
+  static constexpr int kThreads = 32 * (F8 ? kFirstConvWarp + kConvWarps : kFirstSoftWarp + kSoftWarps);
+  // the query's shared-memory part: bf16 latent 448-511 and rope (two 64-row boxes), or
+  // (F8) the high and low E4M3 pieces of columns 448-575 (one 64-row box each)
+  static constexpr int kQBytes = kQSmemChunks * kBox64;                  // 16,384
+  static constexpr int kQKSlotBytes = (F8 ? kF8Boxes : kChunks) * kBox32;   // 20,480 / 36,864
+  static constexpr int kQKSlots = 3;
+  static constexpr int kPV8SlotBytes = 2 * kBox64;   // (F8) 64 tokens x the CTA's two 128-code latent blocks
+  static constexpr int kPV8Slots = F8 ? 2 : 0;
+  static constexpr int kPVSlotBytes = 8 * kBox32;    // 32,768
+  static constexpr int kPVSlots = 2;
+  static constexpr int kOffQ = 0;
+  static constexpr int kOffQK = kOffQ + kQBytes;
+  static constexpr int kOffPV8 = kOffQK + kQKSlots * kQKSlotBytes;
+  static constexpr int kOffPV = kOffPV8 + kPV8Slots * kPV8SlotBytes;
+  static constexpr int kOffP = kOffPV + kPVSlots * kPVSlotBytes;   // two buffers of P_hi then P_lo
+  static constexpr int kOffXch = kOffP + 4 * kPBytes;               // (F8) float[128][32]: score halves exchanged
+  static constexpr int kOffXs8 = kOffXch + (F8 ? 128 * 32 * 4 : 0);   // (F8) uint8[slot][64]: scale bytes per code slot
+  static constexpr int kOffXsc = kOffXs8 + (F8 ? kPV8Slots * 64 : 0);  // (F8) float[4][64]: token scales
+  static constexpr int kMaxBars = F8 ? 40 : 32;
+  static constexpr int kOffBar = kOffXsc + (F8 ? 4 * 64 * 4 : 0);  // kMaxBars mbarriers
+  static constexpr int kOffXmax = kOffBar + kMaxBars * 8;   // float[2][128]: row maxima of the lane halves
+  static constexpr int kOffXl = kOffXmax + 2 * 128 * 4;     // float[128]: row sums of the lane halves
+  static constexpr int kOffFlag = kOffXl + 128 * 4;         // uint32[4][8] (even CTA): P_lo wanted, per tile % 4
+                                                            // and softmax warp (0-3 even CTA, 4-7 odd CTA)
+  static constexpr int kOffXal = kOffFlag + 4 * 8 * 4;      // float[2][128]: the pair's rescale factors, per row
+  static constexpr int kOffXflg = kOffXal + 2 * 128 * 4;    // uint32[2][4]: a moved reference among 32 rows
+  static constexpr int kOffXinv = kOffXflg + 2 * 4 * 4;     // float[128]: the pair's 1 / l, per row
+  static constexpr int kOffTmem = kOffXinv + 128 * 4;
+  static constexpr int kOffAbort = kOffTmem + 8;
+  static constexpr int kSmemUsed = kOffAbort + 8;
+  static constexpr int kSmemBytes = kSmemUsed + 1024;
+  static_assert(kSmemBytes <= 232448, "shared memory of one CTA");
+  static_assert(kOffQK % 1024 == 0 && kOffPV8 % 1024 == 0 && kOffPV % 1024 == 0 && kOffP % 1024 == 0 &&
+                    kOffXs8 % 16 == 0 &&
+                    kQKSlotBytes % 1024 == 0,
+                "swizzled buffers on 1 KiB boundaries");
+};
+constexpr int kThreads = Lay<false>::kThreads;
+constexpr int kSmemBytes = Lay<false>::kSmemBytes;
+constexpr int kThreadsF8 = Lay<true>::kThreads;
+constexpr int kSmemBytesF8 = Lay<true>::kSmemBytes;
 
 enum {
   B_QK_FULL = 0,                   // +slot (even CTA): score operands of both CTAs landed
@@ -125,16 +166,23 @@ enum {
   B_LX_FULL = B_AL_FULL + 2,       // both CTAs' 1 / l of a unit (likewise)
   B_ALL4,                          // the four softmax warps (epilogue staging)
   B_DRAIN,
-  kNumBars
+  B_PV8_FULL,                      // +slot (F8): this CTA's value codes landed
+  B_PV8_EMPTY = B_PV8_FULL + 3,    // +slot (F8): this CTA's converter warps read them
+  B_CV_FULL = B_PV8_EMPTY + 3,     // +page % 4 (F8): this CTA's token scales of the page written
+  kNumBars = B_CV_FULL + 4
 };
-static_assert(kNumBars <= kMaxBars, "barrier area");
-static_assert(kQKSlots <= 3 && kPVSlots <= 2, "barrier slots");
+static_assert(kNumBars <= Lay<true>::kMaxBars && B_PV8_FULL <= Lay<false>::kMaxBars, "barrier area");
+static_assert(Lay<true>::kQKSlots <= 3 && Lay<true>::kPVSlots <= 2 && Lay<true>::kPV8Slots <= 3, "barrier slots");
 
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColO = 0, kColS = 256, kColQ = 288;
 static_assert(kColQ + 32 * kQTmemChunks <= kTmemCols, "TMEM columns");
+// (F8) scores of an M = 256 MMA: 64 columns; the query piece of each lane: 112 columns
+constexpr uint32_t kColQ8 = kColS + 64;
+static_assert(kColQ8 + 4 * kF8QTmemSteps * 2 <= kTmemCols, "TMEM columns (8-bit cache)");
 constexpr uint32_t kIdescS = ptx::idesc_bf16_f32(128, 64, 0, 0);    // Q (K-major) x KV^T (K-major)
 constexpr uint32_t kIdescV = ptx::idesc_bf16_f32(256, 128, 1, 0);   // C^T (M-major) x P^T (K-major)
+constexpr uint32_t kIdescS8 = ptx::idesc_e4m3_f32(256, 64, 0, 0);   // (F8) query pieces x codes, both K-major
 // log2 units: p stays below 2^24, far inside the range of the bf16 P and of the fp32
 // sums (at most 2^24 x 2^17 tokens x |c|), so the reference moves (and O is rescaled)
 // only when a row's maximum jumps by that much, which almost never happens
@@ -235,19 +283,27 @@ __device__ __forceinline__ int32_t page_id(const Params& p, const Unit2& u, int3
   return page;
 }
 
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
+// F8 = false: bf16 cache; tm_kv: the cache in 32-row boxes, tm_q / tm_qr: q_lat / q_rope
+// in 64-row boxes. F8 = true: 8-bit cache (codes and per-token scales, p.kv_scale);
+// tm_kv: the codes in 32-row boxes of 128 codes, tm_q: the split query (p.q8) in 64-row
+// boxes (high pieces), tm_ql: the same for the low pieces, tm_qr: the codes in 64-row
+// boxes. tm_o / tm_op: fp32 output stores (final rows, partial rows).
+template <bool F8>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Lay<F8>::kThreads, 1)
 decode_2sm_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_constant__ CUtensorMap tm_q,
                   const __grid_constant__ CUtensorMap tm_qr, const __grid_constant__ CUtensorMap tm_o,
-                  const __grid_constant__ CUtensorMap tm_op, const Params p) {
+                  const __grid_constant__ CUtensorMap tm_op, const __grid_constant__ CUtensorMap tm_ql,
+                  const Params p) {
+  using L = Lay<F8>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sbase = ptx::smem_u32(smem);
   const uint32_t rank = ptx::cluster_rank();
   const bool even = rank == 0;
-  auto bar = [&](int i) { return sbase + kOffBar + 8u * i; };
+  auto bar = [&](int i) { return sbase + L::kOffBar + 8u * i; };
   auto lead = [&](uint32_t local) { return ptx::map_peer(local, 0); };   // the even CTA's copy
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kOffAbort);
-  volatile uint32_t* lo_flag = reinterpret_cast<volatile uint32_t*>(smem + kOffFlag);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kOffAbort);
+  volatile uint32_t* lo_flag = reinterpret_cast<volatile uint32_t*>(smem + L::kOffFlag);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const PlanView plan{p.plan};
@@ -259,13 +315,21 @@ decode_2sm_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_consta
   if (threadIdx.x == 0) {
     *abort_flag = 0;
     for (int i = 0; i < 32; ++i) lo_flag[i] = 0u;
-    for (int s = 0; s < kQKSlots; ++s) {
+    for (int s = 0; s < L::kQKSlots; ++s) {
       ptx::mbar_init(bar(B_QK_FULL + s), 1);
       ptx::mbar_init(bar(B_QK_EMPTY + s), 1);
     }
-    for (int s = 0; s < kPVSlots; ++s) {
-      ptx::mbar_init(bar(B_PV_FULL + s), 1);
+    for (int s = 0; s < L::kPVSlots; ++s) {
+      // bf16: the TMA bytes; F8: every converter warp of both CTAs
+      ptx::mbar_init(bar(B_PV_FULL + s), F8 ? 2 * kConvWarps : 1);
       ptx::mbar_init(bar(B_PV_EMPTY + s), 1);
+    }
+    if constexpr (F8) {
+      for (int s = 0; s < L::kPV8Slots; ++s) {
+        ptx::mbar_init(bar(B_PV8_FULL + s), 1);
+        ptx::mbar_init(bar(B_PV8_EMPTY + s), kConvWarps);
+      }
+      for (int i = 0; i < 4; ++i) ptx::mbar_init(bar(B_CV_FULL + i), kConvWarps / 2);   // warps of block 0
     }
     ptx::mbar_init(bar(B_S_FULL), 1);
     ptx::mbar_init(bar(B_S_EMPTY), 2 * kSoftWarps);
@@ -285,7 +349,7 @@ decode_2sm_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_consta
     ptx::fence_mbar_init();
   }
   if (warp == 1) {
-    ptx::tmem_alloc_pair(sbase + kOffTmem, kTmemCols);
+    ptx::tmem_alloc_pair(sbase + L::kOffTmem, kTmemCols);
     ptx::tmem_relinquish_pair();
   }
   if (warp == 0 && lane == 0) {
@@ -294,12 +358,13 @@ decode_2sm_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_consta
     ptx::prefetch_tmap(&tm_qr);
     ptx::prefetch_tmap(&tm_o);
     ptx::prefetch_tmap(&tm_op);
+    if (F8) ptx::prefetch_tmap(&tm_ql);
   }
   ptx::tc_fence_before();
   __syncthreads();
   ptx::cluster_sync();   // both CTAs' barriers exist before anyone arrives, loads or issues
   ptx::tc_fence_after();
-  const uint32_t tbase = *reinterpret_cast<volatile uint32_t*>(smem + kOffTmem);
+  const uint32_t tbase = *reinterpret_cast<volatile uint32_t*>(smem + L::kOffTmem);
 #ifdef MLA_TRACE
   if (threadIdx.x == 0 && p.trace) {
     uint32_t smid;
@@ -314,7 +379,7 @@ decode_2sm_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_consta
   auto fail = [&]() {
     raise_status(kStatusTimeout);
     *abort_flag = 1;
-    ptx::st_cluster_u32(ptx::map_peer(sbase + kOffAbort, rank ^ 1u), 1u);
+    ptx::st_cluster_u32(ptx::map_peer(sbase + L::kOffAbort, rank ^ 1u), 1u);
   };
   auto wait_all = [&](uint32_t b, uint32_t parity) -> bool {
     return __all_sync(0xffffffffu, ptx::mbar_wait_cluster_bounded(b, parity, abort_flag, p.timeout_ns));
@@ -326,13 +391,16 @@ decode_2sm_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_consta
     // operand (64 tokens x own 256 latent)
     const bool leader = ptx::elect_one();
     const bool qk = warp == 0;
-    const int nslots = qk ? kQKSlots : kPVSlots;
+    // F8: warp 2 loads this CTA's value codes for its own converters (local barriers)
+    const int nslots = qk ? L::kQKSlots : (F8 ? L::kPV8Slots : L::kPVSlots);
+    const int empty_bar = qk ? B_QK_EMPTY : (F8 ? B_PV8_EMPTY : B_PV_EMPTY);
+    const int full_bar = qk ? B_QK_FULL : (F8 ? B_PV8_FULL : B_PV_FULL);
     Cursor c = first_page(p, plan, u_begin, u_end);
     uint32_t g = 0;
     bool ok = true;
     while (c.valid && ok) {
       const uint32_t s = g % nslots, ph = (g / nslots) & 1;
-      if (!wait_all(bar((qk ? B_QK_EMPTY : B_PV_EMPTY) + s), ph ^ 1)) { if (leader) fail(); ok = false; break; }
+      if (!wait_all(bar(empty_bar + s), ph ^ 1)) { if (leader) fail(); ok = false; break; }
       const int32_t page = page_id(p, c.u, c.k, leader && qk);
       // (the testing hook leaves the page's barrier without the even CTA's load: the waits
       // on it run out and the kernel reports a timeout)
@@ -342,18 +410,32 @@ decode_2sm_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_consta
           // all nine boxes of the page at once (issued together, the page's rows are read
           // from DRAM together)
           DUO_TRACE(0, g);
-          if (even) ptx::mbar_arrive_expect_tx(bar(B_QK_FULL + s), 2 * kQKSlotBytes);
+          if (even) ptx::mbar_arrive_expect_tx(bar(B_QK_FULL + s), 2 * L::kQKSlotBytes);
           if (!drop) {
-            const uint32_t dst = sbase + kOffQK + s * kQKSlotBytes;
+            const uint32_t dst = sbase + L::kOffQK + s * L::kQKSlotBytes;
+            constexpr int nbox = F8 ? kF8Boxes : kChunks, wbox = F8 ? 128 : 64;
 #pragma unroll 1
-            for (int ch = 0; ch < kChunks; ++ch)
-              ptx::tma_load_2d_pair(dst + ch * kBox32, &tm_kv, lead(bar(B_QK_FULL + s)), 64 * ch,
+            for (int ch = 0; ch < nbox; ++ch)
+              ptx::tma_load_2d_pair(dst + ch * kBox32, &tm_kv, lead(bar(B_QK_FULL + s)), wbox * ch,
                                     page * kPage + 32 * (int32_t)rank);
           }
+        } else if constexpr (F8) {
+          // the CTA's latent blocks 2hh + rank (128 codes each) of all 64 tokens, and the
+          // page's 64 scale bytes (those of page 0 stand in for a page id outside the pool:
+          // its codes read as zeros)
+          DUO_TRACE(1, g);
+          ptx::mbar_arrive_expect_tx(bar(B_PV8_FULL + s), L::kPV8SlotBytes + 64);
+          const uint32_t dst = sbase + L::kOffPV8 + s * L::kPV8SlotBytes;
+#pragma unroll
+          for (int hh = 0; hh < 2; ++hh)
+            ptx::tma_load_2d(dst + hh * kBox64, &tm_qr, bar(B_PV8_FULL + s), 128 * (2 * hh + (int)rank),
+                             page * kPage);
+          ptx::bulk_load_g2s(sbase + L::kOffXs8 + s * 64,
+                             p.kv_scale + (int64_t)(page < p.num_pages ? page : 0) * kPage, 64, bar(B_PV8_FULL + s));
         } else {
           DUO_TRACE(1, g);
-          if (even) ptx::mbar_arrive_expect_tx(bar(B_PV_FULL + s), 2 * kPVSlotBytes);
-          const uint32_t dst = sbase + kOffPV + s * kPVSlotBytes;
+          if (even) ptx::mbar_arrive_expect_tx(bar(B_PV_FULL + s), 2 * L::kPVSlotBytes);
+          const uint32_t dst = sbase + L::kOffPV + s * L::kPVSlotBytes;
           // box (hh, th, b) at ((hh * 2 + th) * 2 + b): latent block 4hh + 2r + b, tokens 32th..
 #pragma unroll 1
           for (int i = 0; i < 8; ++i) {
@@ -370,10 +452,10 @@ decode_2sm_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_consta
     // phases armed last, so no copy is still landing in either CTA. These waits ignore the
     // abort flag (copies in flight land within microseconds) and stop at the wait bound;
     // after one runs out (a phase that cannot complete) the rest are skipped.
-    if (even) {
+    if (even || (F8 && !qk)) {   // (F8: each CTA's value codes count on its own barriers)
       bool landed = true;
       for (uint32_t k = (g >= (uint32_t)nslots ? g - nslots : 0); k < g && landed; ++k)
-        landed = __all_sync(0xffffffffu, ptx::mbar_wait_cluster_timed(bar((qk ? B_QK_FULL : B_PV_FULL) + k % nslots),
+        landed = __all_sync(0xffffffffu, ptx::mbar_wait_cluster_timed(bar(full_bar + k % nslots),
                                                                       (k / nslots) & 1, p.timeout_ns));
     }
   } else if (warp == 3) {
@@ -393,18 +475,31 @@ decode_2sm_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_consta
       if (even && leader && more) {
         const int64_t qrow = (int64_t)nu.item * H;
         const int64_t rows = min((int64_t)kRows, TH - qrow);
-        if (rows > 0) ptx::prefetch_l2_bulk(p.q_lat + qrow * kR, (uint32_t)(rows * kR * 2));
+        if (rows > 0) {
+          if constexpr (F8) {
+            ptx::prefetch_l2_bulk(p.q8 + qrow * kRow, (uint32_t)(rows * kRow));
+            ptx::prefetch_l2_bulk(p.q8 + (TH + qrow) * kRow, (uint32_t)(rows * kRow));
+          } else {
+            ptx::prefetch_l2_bulk(p.q_lat + qrow * kR, (uint32_t)(rows * kR * 2));
+          }
+        }
       }
       if (!wait_all(bar(B_Q_EMPTY), (nq & 1) ^ 1)) { if (leader) fail(); break; }
       if (leader) {
-        if (even) ptx::mbar_arrive_expect_tx(bar(B_Q_FULL), 2 * kQBytes);
+        if (even) ptx::mbar_arrive_expect_tx(bar(B_Q_FULL), 2 * L::kQBytes);
         const int32_t qrow = u.item * H + kCtaRows * (int32_t)rank;   // rows past the tensor read zeros
+        if constexpr (F8) {
+          // columns 448-575 of the high and the low pieces
+          ptx::tma_load_2d_pair(sbase + L::kOffQ, &tm_q, lead(bar(B_Q_FULL)), 32 * kF8QTmemSteps, qrow);
+          ptx::tma_load_2d_pair(sbase + L::kOffQ + kBox64, &tm_ql, lead(bar(B_Q_FULL)), 32 * kF8QTmemSteps, qrow);
+        } else {
 #pragma unroll 1
-        for (int ch = 0; ch < kQSmemChunks - 1; ++ch)
-          ptx::tma_load_2d_pair(sbase + kOffQ + ch * kBox64, &tm_q, lead(bar(B_Q_FULL)),
-                                64 * (kQTmemChunks + ch), qrow);
-        ptx::tma_load_2d_pair(sbase + kOffQ + (kQSmemChunks - 1) * kBox64, &tm_qr, lead(bar(B_Q_FULL)), 0,
-                              qrow);
+          for (int ch = 0; ch < kQSmemChunks - 1; ++ch)
+            ptx::tma_load_2d_pair(sbase + L::kOffQ + ch * kBox64, &tm_q, lead(bar(B_Q_FULL)),
+                                  64 * (kQTmemChunks + ch), qrow);
+          ptx::tma_load_2d_pair(sbase + L::kOffQ + (kQSmemChunks - 1) * kBox64, &tm_qr, lead(bar(B_Q_FULL)), 0,
+                                qrow);
+        }
       }
       ++nq;
       ui = ni;
@@ -423,15 +518,32 @@ decode_2sm_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_consta
       auto issue_s = [&]() -> bool {
         if (qc.k == 0 && !wait_all(bar(B_Q_FULL), qc.n & 1)) return false;
         if (qc.k == 0 && leader) DUO_TRACE(12, qc.n);
-        const uint32_t s = gq % kQKSlots, ph = (gq / kQKSlots) & 1;
+        const uint32_t s = gq % L::kQKSlots, ph = (gq / L::kQKSlots) & 1;
         if (!wait_all(bar(B_QK_FULL + s), ph)) return false;
         if (leader) DUO_TRACE(2, gq);
         if (!wait_all(bar(B_S_EMPTY), (gq & 1) ^ 1)) return false;   // both CTAs read S(gq - 1)
         ptx::tc_fence_after();
-        const uint32_t kvs = sbase + kOffQK + s * kQKSlotBytes;
+        const uint32_t kvs = sbase + L::kOffQK + s * L::kQKSlotBytes;
         const uint32_t d_s = tbase + kColS;
         if (leader) {
           DUO_TRACE(3, gq);
+          if constexpr (F8) {
+            // M = 256: each CTA's 128 A rows are its 64 query rows' high pieces (lanes
+            // 0-63) and low pieces (lanes 64-127), so each SM runs a full 128-row MMA. K
+            // steps of 32 codes: step j reads box j / 4 of the page at byte 32 (j % 4); the
+            // query's steps 0-13 are in TMEM (column 8j), steps 14-17 in shared memory (the
+            // high box's 64 rows, then the low box's)
+#pragma unroll 1
+            for (int j = 0; j < kF8Steps; ++j) {
+              const uint64_t dk = ptx::sdesc_sw128(kvs + (j >> 2) * kBox32, 16, 1024) + (uint64_t)(2 * (j & 3));
+              if (j < kF8QTmemSteps)
+                ptx::umma_pair_ts_f8(d_s, tbase + kColQ8 + 8u * j, dk, kIdescS8, j ? 1u : 0u);
+              else
+                ptx::umma_pair_ss_f8(d_s, ptx::sdesc_sw128(sbase + L::kOffQ, 16, 1024) +
+                                              (uint64_t)(2 * (j - kF8QTmemSteps)),
+                                     dk, kIdescS8, 1u);
+            }
+          } else {
 #pragma unroll 1
           for (int ch = 0; ch < kChunks; ++ch) {
             const uint64_t dk = ptx::sdesc_sw128(kvs + ch * kBox32, 16, 1024);
@@ -441,11 +553,12 @@ decode_2sm_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_consta
                 ptx::umma_pair_ts(d_s, tbase + kColQ + 32u * ch + 8u * kk, dk + (uint64_t)(2 * kk), kIdescS,
                                   (ch | kk) ? 1u : 0u);
             } else {
-              const uint64_t dq = ptx::sdesc_sw128(sbase + kOffQ + (ch - kQTmemChunks) * kBox64, 16, 1024);
+              const uint64_t dq = ptx::sdesc_sw128(sbase + L::kOffQ + (ch - kQTmemChunks) * kBox64, 16, 1024);
 #pragma unroll
               for (int kk = 0; kk < 4; ++kk)
                 ptx::umma_pair_ss(d_s, dq + (uint64_t)(2 * kk), dk + (uint64_t)(2 * kk), kIdescS, 1u);
             }
+          }
           }
           ptx::umma_commit_pair(bar(B_QK_EMPTY + s), 3);
           ptx::umma_commit_pair(bar(B_S_FULL), 3);
@@ -461,19 +574,19 @@ decode_2sm_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_consta
         if (leader) DUO_TRACE(4, gv);
         if (vc.k == 0 && vc.n > 0 && !wait_all(bar(B_O_FREE), (vc.n - 1) & 1)) return false;
         if (vc.k == 0 && leader) DUO_TRACE(13, vc.n);
-        const uint32_t s = gv % kPVSlots, ph = (gv / kPVSlots) & 1;
+        const uint32_t s = gv % L::kPVSlots, ph = (gv / L::kPVSlots) & 1;
         if (!wait_all(bar(B_PV_FULL + s), ph)) return false;
         if (leader) DUO_TRACE(8, gv);
         uint32_t want_lo = 0;
 #pragma unroll
         for (int w = 0; w < 2 * kSoftWarps; ++w) want_lo |= lo_flag[8 * (gv & 3) + w];
         ptx::tc_fence_after();
-        const uint32_t pvs = sbase + kOffPV + s * kPVSlotBytes;
+        const uint32_t pvs = sbase + L::kOffPV + s * L::kPVSlotBytes;
         if (leader) {
           DUO_TRACE(5, gv);
 #pragma unroll 1
           for (int part = 0; part < (want_lo ? 2 : 1); ++part) {
-            const uint64_t dp = ptx::sdesc_sw128(sbase + kOffP + (2 * (gv & 1) + part) * kPBytes, 16, 1024);
+            const uint64_t dp = ptx::sdesc_sw128(sbase + L::kOffP + (2 * (gv & 1) + part) * kPBytes, 16, 1024);
 #pragma unroll
             for (int lh = 0; lh < 2; ++lh) {
 #pragma unroll
@@ -505,6 +618,80 @@ decode_2sm_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_consta
       __syncwarp();
       wait_all(bar(B_DRAIN), 0);
     }
+  } else if (F8 && warp >= kFirstConvWarp) {
+    // ================================================================ (F8) value operands to bf16
+    // Thread (t, hh) widens token t's 128 codes of latent block 2hh + rank into the bf16
+    // value slot (the layout the bf16 cache's loads produce) times the token's scale 2^k:
+    // a code's bits placed under a bf16 exponent field give the code's value times
+    // 2^-120 (subnormal codes included), and one bf16 product by 2^(120+k) is exact. Rows
+    // past the unit's visible tokens are written as zeros (P is zero there, and stale
+    // codes must not turn into NaN). Thread t of the first block also publishes the
+    // token's scale for the softmax warps (which apply it to the score column) as soon
+    // as the page's codes and scale bytes land, before it waits for a free value slot.
+    const int ct = (int)threadIdx.x - 32 * kFirstConvWarp;
+    const int t = ct & 63, hh = ct >> 6;
+    const int th = t >> 5, rr = t & 31;
+    volatile float* xsc = reinterpret_cast<volatile float*>(smem + L::kOffXsc);
+    Cursor c = first_page(p, plan, u_begin, u_end);
+    uint32_t g = 0;
+    while (c.valid) {
+      constexpr uint32_t n8 = F8 ? L::kPV8Slots : 1;   // (the bf16 kernel has no such warps)
+      const uint32_t s8 = g % n8, ph8 = (g / n8) & 1;
+      const uint32_t sb = g & 1, phb = (g >> 1) & 1;
+      const int32_t pos = (c.u.pb + c.k) * kPage + t;
+      const bool valid = pos < max(c.u.ntok[0], c.u.ntok[1]);
+      if (!wait_all(bar(B_PV8_FULL + s8), ph8)) { if (lane == 0) fail(); break; }
+      uint32_t e = valid ? (uint32_t)smem[L::kOffXs8 + s8 * 64 + t] : 127u;
+      e = min(max(e, 1u), 134u);   // 2^(120+k) must be a finite bf16
+      // the page's token scales for the softmax warps first (ring of four: slot g % 4 was
+      // read by the softmax of page g - 4, whose P the value MMAs of page g - 4 consumed
+      // before this warp could convert page g - 2)
+      if (hh == 0) {
+        xsc[64 * (g & 3) + t] = valid ? __uint_as_float(e << 23) : 0.f;
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive(bar(B_CV_FULL + (g & 3)));
+      }
+      if (!wait_all(bar(B_PV_EMPTY + sb), phb ^ 1)) { if (lane == 0) fail(); break; }
+      const uint32_t src = sbase + L::kOffPV8 + s8 * L::kPV8SlotBytes + hh * kBox64 + t * 128;
+      const uint32_t dst = sbase + L::kOffPV + sb * L::kPVSlotBytes + ((hh * 2 + th) * 2) * kBox32 + rr * 128;
+      const uint32_t mul = ((e + 120u) << 7) * 0x00010001u;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {   // codes 16j..16j+15 of the block
+        uint32_t w[4];
+        asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                     : "=r"(w[0]), "=r"(w[1]), "=r"(w[2]), "=r"(w[3])
+                     : "r"(src + (uint32_t)((j ^ (t & 7)) << 4)));
+        uint32_t o[8];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+#pragma unroll
+          for (int h2 = 0; h2 < 2; ++h2) {
+            // codes 4q + 2h2, 4q + 2h2 + 1 into the high bytes of the two 16-bit lanes
+            const uint32_t x = __byte_perm(w[q], 0u, h2 ? 0x3424u : 0x1404u);
+            const uint32_t y = ((x >> 4) & 0x07F007F0u) | (x & 0x80008000u);
+            o[2 * q + h2] = valid ? ptx::mul_bf16x2(y, mul) : 0u;
+          }
+        }
+        // bf16 elements 16j.. are 64-column block j / 4, 16-byte chunks 2 (j % 4) and 2 (j % 4) + 1
+        const uint32_t row = dst + (uint32_t)((j >> 2) * kBox32);
+        const int c0 = 2 * (j & 3);
+        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(row + (uint32_t)((c0 ^ (rr & 7)) << 4)),
+                     "r"(o[0]), "r"(o[1]), "r"(o[2]), "r"(o[3])
+                     : "memory");
+        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(row + (uint32_t)(((c0 + 1) ^ (rr & 7)) << 4)),
+                     "r"(o[4]), "r"(o[5]), "r"(o[6]), "r"(o[7])
+                     : "memory");
+      }
+      ptx::fence_proxy_async_smem();   // the value MMAs read the slot through the async proxy
+      __syncwarp();
+      if (lane == 0) {
+        ptx::mbar_arrive(bar(B_PV8_EMPTY + s8));
+        if (even) ptx::mbar_arrive(bar(B_PV_FULL + sb));
+        else ptx::mbar_arrive_remote(lead(bar(B_PV_FULL + sb)));
+      }
+      advance(p, plan, u_end, c);
+      ++g;
+    }
   } else if (warp >= kFirstSoftWarp) {
     // ================================================================ query staging, softmax, epilogue
     const int sw = warp - kFirstSoftWarp;         // softmax warp 0-3
@@ -516,11 +703,11 @@ decode_2sm_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_consta
     const int prow = kCtaRows * (int)rank + m;    // this thread's score row among the pair's 128
     const uint32_t lane_addr = (32u * q) << 16;
     const int tok = H == kRows ? 0 : (int)rank;   // the unit's query token this CTA's rows belong to
-    volatile float* xmax = reinterpret_cast<volatile float*>(smem + kOffXmax);
-    volatile float* xl = reinterpret_cast<volatile float*>(smem + kOffXl);
-    volatile float* xal = reinterpret_cast<volatile float*>(smem + kOffXal);
-    volatile uint32_t* xflg = reinterpret_cast<volatile uint32_t*>(smem + kOffXflg);
-    volatile float* xinv = reinterpret_cast<volatile float*>(smem + kOffXinv);
+    volatile float* xmax = reinterpret_cast<volatile float*>(smem + L::kOffXmax);
+    volatile float* xl = reinterpret_cast<volatile float*>(smem + L::kOffXl);
+    volatile float* xal = reinterpret_cast<volatile float*>(smem + L::kOffXal);
+    volatile uint32_t* xflg = reinterpret_cast<volatile uint32_t*>(smem + L::kOffXflg);
+    volatile float* xinv = reinterpret_cast<volatile float*>(smem + L::kOffXinv);
     auto peer = [&](uint32_t local) { return ptx::map_peer(local, rank ^ 1u); };
     uint32_t n_pair = 0, n_lx = 0, n_all4 = 0;
     bool ok = true;
@@ -572,13 +759,38 @@ decode_2sm_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_consta
       }
     }
 
-    // The TMEM part of a unit's query (latent 0-383 of this thread's score row, both lane
+    // (F8) the staged query row's scale 2^-e (the split query holds the row times 2^e)
+    float q_scale_next = 1.f;
+    // The TMEM part of a unit's query (latent 0-447 of this thread's score row, both lane
     // halves hold it), once the previous unit's last score MMA is done.
     auto stage_q = [&](const Unit2& u, uint32_t n) -> bool {
       if (!wait_all(bar(B_Q_EMPTY), (n & 1) ^ 1)) return false;
       ptx::tc_fence_after();
       const int64_t row = qrow_of(u.item, prow);
       const bool inside = row < TH;   // rows past the query tensor (an absent token) stay zero
+      if constexpr (F8) {
+        // lane L holds piece L / 64 (high, low) of its row: codes 0-447 in columns 0-111
+        q_scale_next = inside ? p.q_scale[row] : 0.f;
+        const uint8_t* src8 = p.q8 + ((int64_t)half * TH + row) * kRow;
+        uint32_t w[112];
+#pragma unroll
+        for (int i = 0; i < 14; ++i) {
+          uint32_t* d = &w[8 * i];
+          if (inside) {
+            asm volatile("ld.global.nc.v8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+                         : "=r"(d[0]), "=r"(d[1]), "=r"(d[2]), "=r"(d[3]), "=r"(d[4]), "=r"(d[5]), "=r"(d[6]),
+                           "=r"(d[7])
+                         : "l"(src8 + 32 * i));
+          } else {
+#pragma unroll
+            for (int k = 0; k < 8; ++k) d[k] = 0u;
+          }
+        }
+#pragma unroll
+        for (int c = 0; c < 3; ++c)
+          ptx::tmem_st_32x32b_x32(tbase + lane_addr + kColQ8 + 32u * c, *reinterpret_cast<uint32_t(*)[32]>(&w[32 * c]));
+        ptx::tmem_st_32x32b_x16u(tbase + lane_addr + kColQ8 + 96u, *reinterpret_cast<uint32_t(*)[16]>(&w[96]));
+      } else {
       const __nv_bfloat16* src = p.q_lat + row * kR;
 #pragma unroll 1
       for (int ch = 0; ch < kQTmemChunks; ch += 2) {
@@ -601,6 +813,7 @@ decode_2sm_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_consta
         }
         ptx::tmem_st_32x32b_x32(tbase + lane_addr + kColQ + 32u * ch, w[0]);
         if (ch + 1 < kQTmemChunks) ptx::tmem_st_32x32b_x32(tbase + lane_addr + kColQ + 32u * (ch + 1), w[1]);
+      }
       }
       ptx::tmem_wait_st();
       ptx::tc_fence_before();
@@ -632,7 +845,7 @@ decode_2sm_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_consta
         const float l = pend.l + xl[L ^ 64];   // half 0 + half 1
         const float inv_l = l > 0.f ? 1.f / l : 0.f;
         xinv[prow] = inv_l;
-        const uint32_t xa = sbase + kOffXinv + 4u * prow;
+        const uint32_t xa = sbase + L::kOffXinv + 4u * prow;
         ptx::st_async_u32(peer(xa), __float_as_uint(inv_l), peer(bar(B_LX_FULL)));
         if (tok < pend.n) {
           const int64_t row = qrow_of(pend.item, prow);
@@ -656,7 +869,7 @@ decode_2sm_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_consta
       // in the warp's two tiles in the idle P buffers, and hand each to a TMA store (final
       // rows to o_lat, partial rows to the workspace). The stores run in the background; a
       // tile is restaged once the store two blocks back has read it.
-      const uint32_t tiles = sbase + kOffP + (uint32_t)sw * kPBytes;   // 2 x 4 KiB
+      const uint32_t tiles = sbase + L::kOffP + (uint32_t)sw * kPBytes;   // 2 x 4 KiB
       uint32_t nst = 0;
 #pragma unroll 1
       for (int c = 0; c < 8; ++c) {
@@ -671,7 +884,7 @@ decode_2sm_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_consta
         for (int k = 0; k < 8; ++k)
           asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
                        : "=f"(inv[4 * k]), "=f"(inv[4 * k + 1]), "=f"(inv[4 * k + 2]), "=f"(inv[4 * k + 3])
-                       : "r"(sbase + kOffXinv + 4u * (n0 + 4 * k)));
+                       : "r"(sbase + L::kOffXinv + 4u * (n0 + 4 * k)));
         ptx::tmem_wait_ld();
         const int x = 256 * lh + 128 * (int)rank + 32 * q;   // this warp's latent columns
         const int64_t row0 = qrow_of(pend.item, n0);
@@ -713,12 +926,14 @@ decode_2sm_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_consta
     if (cur.valid && !stage_q(cur.u, 0)) { fail(); ok = false; }
     uint32_t g = 0;
     float m_ref = -CUDART_INF_F, l_part = 0.f;
+    float sl2 = p.scale_log2;   // the row's logit scale (log2 units)
     while (cur.valid && ok) {
       const Unit2& u = cur.u;
       if (cur.k == 0) {
         if (pend.on && !epilogue(g - 1)) { fail(); ok = false; break; }
         m_ref = -CUDART_INF_F;
         l_part = 0.f;
+        if (F8) sl2 = p.scale_log2 * q_scale_next;
       }
       const int32_t ntok = tok < u.n ? max(u.ntok[tok], 0) : 0;
       // ------------------------------------------------ this thread's 32 scores
@@ -726,7 +941,29 @@ decode_2sm_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_consta
       ptx::tc_fence_after();
       if (sw == 0 && lane == 0) DUO_TRACE(6, g);
       float v[32];
-      {
+      if constexpr (F8) {
+        // lane L holds piece L / 64 of row m for all 64 tokens: keep tokens 32 half.. and
+        // hand the other 32 to the partner lane L ^ 64 (the other piece of the same row)
+        // through shared memory (16-byte chunks swizzled by the row), then add its half
+        {
+          uint32_t r[32];
+          ptx::tmem_ld_32x32b_x32(tbase + lane_addr + kColS + 32u * (uint32_t)(half ^ 1), r);
+          ptx::tmem_wait_ld();
+          const uint32_t xr = sbase + L::kOffXch + 128u * (uint32_t)L;
+#pragma unroll
+          for (int k = 0; k < 8; ++k)
+            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(xr + (uint32_t)((k ^ (L & 7)) << 4)),
+                         "r"(r[4 * k]), "r"(r[4 * k + 1]), "r"(r[4 * k + 2]), "r"(r[4 * k + 3])
+                         : "memory");
+        }
+        {
+          uint32_t r[32];
+          ptx::tmem_ld_32x32b_x32(tbase + lane_addr + kColS + 32u * (uint32_t)half, r);
+          ptx::tmem_wait_ld();
+#pragma unroll
+          for (int t = 0; t < 32; ++t) v[t] = __uint_as_float(r[t]);
+        }
+      } else {
         uint32_t r[32];
         ptx::tmem_ld_32x32b_x32(tbase + lane_addr + kColS, r);
         ptx::tmem_wait_ld();
@@ -736,11 +973,42 @@ decode_2sm_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_consta
       ptx::tc_fence_before();
       __syncwarp();
       if (lane == 0) arrive_read(B_S_EMPTY);
+      if constexpr (F8) {
+        if (!pair_sync()) { fail(); ok = false; break; }
+        const uint32_t xr = sbase + L::kOffXch + 128u * (uint32_t)(L ^ 64);
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          float x0, x1, x2, x3;
+          asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
+                       : "=f"(x0), "=f"(x1), "=f"(x2), "=f"(x3)
+                       : "r"(xr + (uint32_t)((k ^ (L & 7)) << 4)));
+          v[4 * k] += x0;
+          v[4 * k + 1] += x1;
+          v[4 * k + 2] += x2;
+          v[4 * k + 3] += x3;
+        }
+      }
       // the unit's last score MMA is done: stage the next unit's query
       if (cur.k == u.npg - 1) {
         int32_t ui = cur.ui;
         Unit2 nu;
         if (next_unit(p, plan, ui, u_end, nu) && !stage_q(nu, cur.n + 1)) { fail(); ok = false; break; }
+      }
+      if constexpr (F8) {
+        // score column t times the token's scale (the MMA summed the raw codes)
+        if (!wait_all(bar(B_CV_FULL + (g & 3)), (g >> 2) & 1)) { fail(); ok = false; break; }
+        const uint32_t xs = sbase + L::kOffXsc + 256u * (g & 3) + 128u * (uint32_t)half;
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          float w0, w1, w2, w3;
+          asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
+                       : "=f"(w0), "=f"(w1), "=f"(w2), "=f"(w3)
+                       : "r"(xs + 16u * k));
+          v[4 * k] *= w0;
+          v[4 * k + 1] *= w1;
+          v[4 * k + 2] *= w2;
+          v[4 * k + 3] *= w3;
+        }
       }
       const int32_t tok0 = (u.pb + cur.k) * kPage + 32 * half;
       if (tok0 + 32 > ntok) {
@@ -759,7 +1027,7 @@ decode_2sm_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_consta
       // ------------------------------------------------ the row's maximum over both lane halves
       xmax[128 * (g & 1) + L] = mx;
       if (!pair_sync()) { fail(); ok = false; break; }
-      const float mrow = fmaxf(mx, xmax[128 * (g & 1) + (L ^ 64)]) * p.scale_log2;
+      const float mrow = fmaxf(mx, xmax[128 * (g & 1) + (L ^ 64)]) * sl2;
       const bool need = mrow > m_ref + kRescaleThreshold;
       const float mu = need ? mrow : m_ref;
       const float al = need ? ptx::ex2(m_ref - mu) : 1.f;
@@ -768,14 +1036,14 @@ decode_2sm_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_consta
       // (each CTA's O^T holds every row of the pair); one thread per row sends its factor
       const uint32_t ab = g & 1;
       if (half == 0) {
-        const uint32_t xa = sbase + kOffXal + 4u * (128 * ab + prow);
+        const uint32_t xa = sbase + L::kOffXal + 4u * (128 * ab + prow);
         xal[128 * ab + prow] = al;
         ptx::st_async_u32(peer(xa), __float_as_uint(al), peer(bar(B_AL_FULL + ab)));
         const uint32_t moved = __any_sync(0xffffffffu, need && cur.k > 0) ? 1u : 0u;
         if (lane == 0) {
           const uint32_t fi = 4 * ab + 2 * rank + (q & 1);
           xflg[fi] = moved;
-          ptx::st_async_u32(peer(sbase + kOffXflg + 4u * fi), moved, peer(bar(B_AL_FULL + ab)));
+          ptx::st_async_u32(peer(sbase + L::kOffXflg + 4u * fi), moved, peer(bar(B_AL_FULL + ab)));
         }
         __syncwarp();
         if (lane == 0) {
@@ -788,8 +1056,8 @@ decode_2sm_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_consta
       float sum4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int i = 0; i < 16; ++i) {
-        const float a0 = ptx::ex2(fmaf(v[2 * i], p.scale_log2, nz));
-        const float a1 = ptx::ex2(fmaf(v[2 * i + 1], p.scale_log2, nz));
+        const float a0 = ptx::ex2(fmaf(v[2 * i], sl2, nz));
+        const float a1 = ptx::ex2(fmaf(v[2 * i + 1], sl2, nz));
         sum4[i & 3] += a0 + a1;
         __nv_bfloat162 h2 = __floats2bfloat162_rn(a0, a1);
         ph[i] = *reinterpret_cast<uint32_t*>(&h2);
@@ -799,7 +1067,7 @@ decode_2sm_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_consta
       }
       l_part = l_part * al + ((sum4[0] + sum4[1]) + (sum4[2] + sum4[3]));
       m_ref = mu;
-      const float pmax = ptx::ex2(fmaf(mx, p.scale_log2, nz));
+      const float pmax = ptx::ex2(fmaf(mx, sl2, nz));
       const bool want_lo = pmax * kLoShare > l_part;
       // ------------------------------------------------ P to shared memory once the previous value MMAs are done
       // P buffer g % 2 was last read by the value MMAs of page g - 2
@@ -827,7 +1095,7 @@ decode_2sm_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_consta
       }
       {
         // row m, tokens 32h..32h+31 = 16-byte chunks 4h..4h+3 of the 128-byte row (128-byte swizzle)
-        const uint32_t prow_s = sbase + kOffP + 2u * kPBytes * (g & 1) + (uint32_t)m * 128u;
+        const uint32_t prow_s = sbase + L::kOffP + 2u * kPBytes * (g & 1) + (uint32_t)m * 128u;
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
           const uint32_t off = (uint32_t)(((4 * half + i) ^ (m & 7)) << 4);
@@ -845,7 +1113,7 @@ decode_2sm_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_consta
       __syncwarp();   // every lane's P stores before lane 0's release
       if (sw == 0 && lane == 0) DUO_TRACE(7, g);
       if (lane == 0) {
-        const uint32_t fa = sbase + kOffFlag + 4u * (8 * (g & 3) + 4 * rank + sw);
+        const uint32_t fa = sbase + L::kOffFlag + 4u * (8 * (g & 3) + 4 * rank + sw);
         if (even) {
           lo_flag[8 * (g & 3) + sw] = any_lo;
           if (sw == 0) ptx::mbar_arrive_expect_tx(bar(B_P_FULL), 4u * kSoftWarps);   // the odd CTA's words

@@ -110,6 +110,10 @@ struct Params {
   uint64_t timeout_ns;
   unsigned long long* trace;  // per-CTA event clocks, only in builds with MLA_TRACE
   int32_t drop_load;          // testing hook: CTA 0 skips the load of its page with this ordinal (-1: none)
+  // 8-bit cache (SM-pair kernel only)
+  const uint8_t* kv_scale = nullptr;   // [num_pages][64] biased exponents of the rows' scales
+  const uint8_t* q8 = nullptr;         // [2][T*H][576] the query rows split into E4M3 high and low pieces
+  const float* q_scale = nullptr;      // [T*H] 2^-e of each split row
 };
 
 // Optional event trace (build with -DMLA_TRACE): per CTA 1024 clock64 values;

@@ -23,6 +23,7 @@
 #include "gemm_tc.cuh"
 #include "decode_2sm.cuh"
 #include "cache_write.cuh"
+#include "fp8_kernels.cuh"
 
 namespace {
 
@@ -124,6 +125,25 @@ mla_status make_map_2d(CUtensorMap* m, const void* base, uint64_t cols, uint64_t
                   box_cols == 64 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return fail(MLA_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+  return MLA_OK;
+}
+
+// 2-D tensor map of one-byte elements (E4M3 codes): boxes of 128 x box_rows with the
+// 128-byte swizzle. Columns of a box past `cols` read as zero.
+mla_status make_map_u8_2d(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows, uint64_t pitch_bytes,
+                          uint32_t box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return fail(MLA_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+  if (reinterpret_cast<uintptr_t>(base) % 16 != 0)
+    return fail(MLA_ERR_INVALID, "tensor base %p is not 16-byte aligned", base);
+  const cuuint64_t dims[2] = {cols, rows};
+  const cuuint64_t strides[1] = {pitch_bytes};
+  const cuuint32_t box[2] = {128, box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(MLA_ERR_CUDA, "cuTensorMapEncodeTiled (codes) failed (%d)", (int)r);
   return MLA_OK;
 }
 
@@ -767,10 +787,10 @@ mla_status mla_decode_attn(const void* q_lat, const void* q_rope, const void* kv
       } else {
         top = to;   // never used: the plan has no partial outputs
       }
-      if (mla_status s = ensure_smem_attr((const void*)mla::duo::decode_2sm_kernel, mla::duo::kSmemBytes))
+      if (mla_status s = ensure_smem_attr((const void*)mla::duo::decode_2sm_kernel<false>, mla::duo::kSmemBytes))
         return s;
-      mla::duo::decode_2sm_kernel<<<grid, mla::duo::kThreads, mla::duo::kSmemBytes, st>>>(tk32, tq, tr, to, top,
-                                                                                          p);
+      mla::duo::decode_2sm_kernel<false><<<grid, mla::duo::kThreads, mla::duo::kSmemBytes, st>>>(
+          tk32, tq, tr, to, top, tq, p);
       return launch_check("decode_attn (tcgen05, SM pair)");
     }
     mla::tc::decode_kernel<<<grid, 256, mla::tc::kSmemBytes, st>>>(tq, tr, tk, p);
@@ -809,6 +829,133 @@ mla_status mla_decode_attn(const void* q_lat, const void* q_rope, const void* kv
 }
 
 // ------------------------------------------------------------------------------- combine
+// ------------------------------------------------------------------------------- 8-bit cache
+static bool fp8_dims_ok(const mla_dims& d) {
+  return d.dtype == MLA_BF16 && d.R == 512 && d.Dr == 64 && d.page_size == 64;
+}
+
+mla_status mla_quantize_rows_fp8(const void* rows, void* codes, void* scales, int64_t n, mla_dims d,
+                                 void* stream) {
+  if (mla_status s = check_dims(d)) return s;
+  if (!fp8_dims_ok(d)) return fail(MLA_ERR_UNSUPPORTED, "the 8-bit cache needs bf16 rows with R=512, Dr=64");
+  if (n < 0) return fail(MLA_ERR_INVALID, "bad row count %lld", (long long)n);
+  if (n == 0) return ok();
+  if (!rows || !codes || !scales) return fail(MLA_ERR_INVALID, "null pointer");
+  if (reinterpret_cast<uintptr_t>(rows) % 16 != 0 || reinterpret_cast<uintptr_t>(codes) % 8 != 0)
+    return fail(MLA_ERR_INVALID, "rows must be 16-byte and codes 8-byte aligned");
+  mla::f8::quantise_rows_kernel<<<(unsigned)((n + 7) / 8), 256, 0, as_stream(stream)>>>(
+      static_cast<const __nv_bfloat16*>(rows), static_cast<uint8_t*>(codes), static_cast<uint8_t*>(scales), n,
+      nullptr, nullptr, 1, 1, 1, d.page_size);
+  return launch_check("quantize_rows_fp8");
+}
+
+mla_status mla_cache_append_fp8(void* kv_codes, void* kv_scales, const int32_t* block_table,
+                                const int32_t* seq_lens, const void* new_ckr, int32_t B, int32_t q_len,
+                                int32_t max_pages, int32_t num_pages, mla_dims d, void* stream) {
+  if (mla_status s = check_dims(d)) return s;
+  if (!fp8_dims_ok(d)) return fail(MLA_ERR_UNSUPPORTED, "the 8-bit cache needs bf16 rows with R=512, Dr=64, page 64");
+  if (B < 0 || q_len <= 0 || max_pages <= 0 || num_pages <= 0)
+    return fail(MLA_ERR_INVALID, "bad sizes B=%d q_len=%d max_pages=%d num_pages=%d", B, q_len, max_pages,
+                num_pages);
+  if (B == 0) return ok();
+  if (!kv_codes || !kv_scales || !block_table || !seq_lens || !new_ckr) return fail(MLA_ERR_INVALID, "null pointer");
+  if (reinterpret_cast<uintptr_t>(new_ckr) % 16 != 0 || reinterpret_cast<uintptr_t>(kv_codes) % 8 != 0)
+    return fail(MLA_ERR_INVALID, "new_ckr must be 16-byte and kv_codes 8-byte aligned");
+  const int64_t n = (int64_t)B * q_len;
+  mla::f8::quantise_rows_kernel<<<(unsigned)((n + 7) / 8), 256, 0, as_stream(stream)>>>(
+      static_cast<const __nv_bfloat16*>(new_ckr), static_cast<uint8_t*>(kv_codes), static_cast<uint8_t*>(kv_scales),
+      n, block_table, seq_lens, q_len, max_pages, num_pages, d.page_size);
+  return launch_check("cache_append_fp8");
+}
+
+// The 8-bit decode's workspace: the split partials (as mla_workspace_size), then the
+// split query [2][T*H][576] codes and its row scales [T*H] fp32.
+static size_t fp8_query_offset(const mla_plan_info* info, const mla_dims& d) {
+  return (mla_workspace_size(info, d) + 255) / 256 * 256;
+}
+
+size_t mla_workspace_size_fp8(const mla_plan_info* info, mla_dims d) {
+  if (!info || check_dims(d) != MLA_OK) return 0;
+  const size_t rows = (size_t)std::max(0, info->num_items) * d.H;
+  return fp8_query_offset(info, d) + (2 * rows * 576 + 255) / 256 * 256 + rows * sizeof(float);
+}
+
+mla_status mla_decode_attn_fp8(const void* q_lat, const void* q_rope, const void* kv_codes, const void* kv_scales,
+                               const int32_t* block_table, const int32_t* seq_lens, int32_t B, int32_t q_len,
+                               int32_t max_pages, int32_t num_pages, float scale, const int32_t* plan_dev,
+                               const mla_plan_info* info, void* o_lat, float* lse, void* workspace,
+                               size_t workspace_bytes, mla_dims d, void* stream) {
+  if (mla_status s = check_dims(d)) return s;
+  if (B < 0 || q_len <= 0 || max_pages <= 0 || num_pages <= 0)
+    return fail(MLA_ERR_INVALID, "bad sizes B=%d q_len=%d max_pages=%d num_pages=%d", B, q_len, max_pages,
+                num_pages);
+  if (!(scale > 0.f) || !std::isfinite(scale)) return fail(MLA_ERR_INVALID, "scale must be positive");
+  if (!fp8_dims_ok(d) || !pair_decode(d, q_len))
+    return fail(MLA_ERR_UNSUPPORTED,
+                "the 8-bit cache decode runs on the SM-pair tensor-core kernel: bf16 queries, R=512, Dr=64, "
+                "page_size=64, H=64 or 128, and a policy other than SIMT");
+  if (mla_status s = check_info(info, B, q_len, max_pages, d)) return s;
+  if (B == 0 || info->num_units == 0) return ok();
+  if (!q_lat || !q_rope || !kv_codes || !kv_scales || !block_table || !seq_lens || !plan_dev || !o_lat)
+    return fail(MLA_ERR_INVALID, "null pointer");
+  if (reinterpret_cast<uintptr_t>(kv_scales) % 16 != 0)
+    return fail(MLA_ERR_INVALID, "kv_scales must be 16-byte aligned (each page's 64 bytes are bulk-copied)");
+  const size_t need = mla_workspace_size_fp8(info, d);
+  if (!workspace || workspace_bytes < need)
+    return fail(MLA_ERR_WORKSPACE, "workspace %zu bytes < %zu needed", workspace_bytes, need);
+  if (reinterpret_cast<uintptr_t>(workspace) % 256 != 0) return fail(MLA_ERR_INVALID, "workspace not 256-byte aligned");
+  float *o_part, *lse_part;
+  if (mla_status s = split_workspace(info, d, workspace, workspace_bytes, &o_part, &lse_part)) return s;
+  const int64_t T = (int64_t)B * q_len, rows = T * d.H;
+  uint8_t* q8 = static_cast<uint8_t*>(workspace) + fp8_query_offset(info, d);
+  float* q_scale = reinterpret_cast<float*>(q8 + (2 * (size_t)rows * 576 + 255) / 256 * 256);
+  cudaStream_t st = as_stream(stream);
+  CUtensorMap tk32, tk64, tqh, tql, to, top;
+  const uint64_t cache_rows = (uint64_t)num_pages * d.page_size;
+  if (mla_status s = make_map_u8_2d(&tk32, kv_codes, 576, cache_rows, 576, 32)) return s;
+  if (mla_status s = make_map_u8_2d(&tk64, kv_codes, 576, cache_rows, 576, 64)) return s;
+  if (mla_status s = make_map_u8_2d(&tqh, q8, 576, (uint64_t)rows, 576, 64)) return s;
+  if (mla_status s = make_map_u8_2d(&tql, q8 + (size_t)rows * 576, 576, (uint64_t)rows, 576, 64)) return s;
+  if (mla_status s = make_store_map_2d(&to, o_lat, true, d.R, (uint64_t)rows, (uint64_t)d.R * 4, 32, 16)) return s;
+  if (info->num_parts > 0) {
+    if (mla_status s = make_store_map_2d(&top, o_part, true, d.R, (uint64_t)info->num_parts * d.H,
+                                         (uint64_t)d.R * 4, 32, 16))
+      return s;
+  } else {
+    top = to;   // never used: the plan has no partial outputs
+  }
+  mla::f8::split_query_kernel<<<(unsigned)((rows + 7) / 8), 256, 0, st>>>(
+      static_cast<const __nv_bfloat16*>(q_lat), static_cast<const __nv_bfloat16*>(q_rope), q8, q_scale, rows);
+  if (mla_status s = launch_check("decode_attn_fp8 (split query)")) return s;
+  mla::tc::Params p;
+  p.plan = plan_dev;
+  p.block_table = block_table;
+  p.seq_lens = seq_lens;
+  p.max_pages = max_pages;
+  p.num_pages = num_pages;
+  p.H = d.H;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.o_lat = static_cast<float*>(o_lat);
+  p.lse = lse;
+  p.o_part = o_part;
+  p.lse_part = lse_part;
+  p.kv = nullptr;
+  p.q_lat = static_cast<const __nv_bfloat16*>(q_lat);
+  p.q_rope = static_cast<const __nv_bfloat16*>(q_rope);
+  p.timeout_ns = g_timeout_ns.load();
+  p.trace = g_trace;
+  p.drop_load = g_drop_load.load();
+  p.kv_scale = static_cast<const uint8_t*>(kv_scales);
+  p.q8 = q8;
+  p.q_scale = q_scale;
+  if (mla_status s = ensure_smem_attr((const void*)mla::duo::decode_2sm_kernel<true>, mla::duo::kSmemBytesF8))
+    return s;
+  const dim3 grid(info->num_slots * info->head_groups);
+  mla::duo::decode_2sm_kernel<true><<<grid, mla::duo::kThreadsF8, mla::duo::kSmemBytesF8, st>>>(tk32, tqh, tk64, to,
+                                                                                               top, tql, p);
+  return launch_check("decode_attn_fp8 (tcgen05, SM pair)");
+}
+
 mla_status mla_combine(const int32_t* plan_dev, const mla_plan_info* info, const void* workspace,
                        size_t workspace_bytes, void* o_lat, float* lse, mla_dims d, void* stream) {
   if (mla_status s = check_dims(d)) return s;

@@ -25,9 +25,14 @@ def num_sms(device=None) -> int:
 
 
 class DecodeStep:
-    def __init__(self, w: dict, device="cuda:0", sms: int | None = None):
+    """cache="fp8": the cache is held as E4M3 codes and per-token scale bytes (the 8-bit
+    cache calls); the codes come from w["kv_codes"] / w["kv_scales"] when given, else
+    the workload's bf16 rows are quantised on the device by mla_quantize_rows_fp8."""
+
+    def __init__(self, w: dict, device="cuda:0", sms: int | None = None, cache: str = "bf16"):
         spec = w["spec"]
         self.spec = spec
+        self.fp8 = cache == "fp8"
         self.device = torch.device(device)
         self.dims = mla.dims_of(spec)
         self.B = int(len(w["seq_lens"]))
@@ -39,7 +44,21 @@ class DecodeStep:
         self.sms = sms or num_sms(self.device)
         self.seq_lens_host = np.ascontiguousarray(w["seq_lens"], dtype=np.int32)
         d = self.device
-        self.kv = to_torch(w["kv_cache"], d)
+        if self.fp8:
+            P, ps = self.num_pages, spec.page_size
+            if "kv_codes" in w:
+                self.kv_codes = to_torch(w["kv_codes"], d)
+                self.kv_scales = to_torch(w["kv_scales"], d)
+            else:
+                rows = to_torch(w["kv_cache"], d)
+                self.kv_codes = torch.empty((P, ps, spec.row), dtype=torch.uint8, device=d)
+                self.kv_scales = torch.empty((P, ps), dtype=torch.uint8, device=d)
+                mla.mla_quantize_rows_fp8(rows, self.kv_codes, self.kv_scales, P * ps, self.dims)
+                torch.cuda.synchronize(d)
+                del rows
+            self.kv = None
+        else:
+            self.kv = to_torch(w["kv_cache"], d)
         self.block_table = to_torch(w["block_table"], d)
         self.seq_lens = to_torch(self.seq_lens_host, d)
         self.q_nope = to_torch(w["q_nope"], d)
@@ -65,11 +84,15 @@ class DecodeStep:
         cap = mla.mla_plan_capacity(self.B, self.q_len, self.sms)
         self.plan = torch.zeros(cap, dtype=torch.int32, device=self.device)
         self.plan[:info.plan_words].copy_(torch.from_numpy(plan))
-        self.ws_bytes = mla.mla_workspace_size(info, self.dims)
+        self.ws_bytes = (mla.mla_workspace_size_fp8 if self.fp8 else mla.mla_workspace_size)(info, self.dims)
         self.workspace = torch.empty(max(self.ws_bytes, 256), dtype=torch.uint8, device=self.device)
 
     # ---------------------------------------------------------------- individual calls
     def append(self, stream=None):
+        if self.fp8:
+            mla.mla_cache_append_fp8(self.kv_codes, self.kv_scales, self.block_table, self.seq_lens, self.new_ckr,
+                                     self.B, self.q_len, self.max_pages, self.num_pages, self.dims, stream)
+            return
         mla.mla_cache_append(self.kv, self.block_table, self.seq_lens, self.new_ckr, self.B, self.q_len,
                              self.max_pages, self.num_pages, self.dims, stream)
 
@@ -77,6 +100,12 @@ class DecodeStep:
         mla.mla_absorb_q(self.q_nope, self.W_UK, self.q_lat, self.T, self.dims, stream)
 
     def attend(self, stream=None):
+        if self.fp8:
+            mla.mla_decode_attn_fp8(self.q_lat, self.q_rope, self.kv_codes, self.kv_scales, self.block_table,
+                                    self.seq_lens, self.B, self.q_len, self.max_pages, self.num_pages, self.scale,
+                                    self.plan, self.info, self.o_lat, self.lse, self.workspace, self.ws_bytes,
+                                    self.dims, stream)
+            return
         mla.mla_decode_attn(self.q_lat, self.q_rope, self.kv, self.block_table, self.seq_lens, self.B, self.q_len,
                             self.max_pages, self.num_pages, self.scale, self.plan, self.info, self.o_lat, self.lse,
                             self.workspace, self.ws_bytes, self.dims, stream)
@@ -118,7 +147,8 @@ class DecodeStep:
         return t
 
     def launches_per_step(self, append=True) -> int:
-        return int(append) + 3 + int(self.info.num_parts > 0)
+        # (the 8-bit cache's decode is two launches: the query split, then attention)
+        return int(append) + 3 + int(self.info.num_parts > 0) + int(self.fp8)
 
 
 class HostInputs:

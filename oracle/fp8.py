@@ -97,6 +97,8 @@ def quantise_rows(rows):
 
 
 def dequantise_rows(codes, scale_bytes) -> np.ndarray:
-    """The float64 rows the codes stand for: code * 2^(e - 127), exact."""
+    """The float64 rows the codes stand for: code * 2^(e - 127), exact (the code's value
+    read from the table of all 256 decoded codes)."""
     k = np.asarray(scale_bytes, dtype=np.int64) - SCALE_BIAS
-    return np.ldexp(e4m3_decode(codes), k[..., None])
+    table = e4m3_decode(np.arange(256, dtype=np.uint8))
+    return np.ldexp(table[np.asarray(codes, dtype=np.uint8)], k[..., None])

@@ -34,7 +34,7 @@ def test_library_exports_every_declared_symbol():
 
 
 def test_abi_version_and_error_text():
-    assert mla.mla_abi_version() == 3
+    assert mla.mla_abi_version() == 4
     with pytest.raises(mla.MlaError) as e:
         mla.mla_set_policy(7)
     assert e.value.status == mla._binding.MLA_ERR_INVALID
@@ -287,3 +287,56 @@ def test_plan_records_max_pages_and_decode_rejects_another():
         with pytest.raises(mla.MlaError) as e:
             mla.mla_decode_attn_noalloc(16, 16, 16, 16, 16, 3, 1, mp, 100, 0.1, 16, info, 16, None, d, stream=0)
         assert "max_pages" in mla.mla_last_error()
+
+
+@pytest.mark.parametrize("case", ["null", "dims_R", "dims_f32", "H", "workspace", "align"])
+def test_fp8_decode_rejects_bad_arguments_before_launch(case):
+    d = dims(H=128)
+    lens = np.array([100, 7], np.int32)
+    plan, info = mla.mla_plan_splits(lens, 2, 1, 4, d, 148)
+    args = dict(q_lat=256, q_rope=256, kv_codes=256, kv_scales=256, block_table=256, seq_lens=256, B=2, q_len=1,
+                max_pages=4, num_pages=8, scale=0.07, plan_dev=256, info=info, o_lat=256, lse=None, workspace=256,
+                workspace_bytes=1 << 30, dims=d)
+    if case == "null":
+        args["kv_scales"] = None
+    elif case == "dims_R":
+        args["dims"] = dims(H=128, R=256)
+    elif case == "dims_f32":
+        args["dims"] = dims(H=128, dtype=mla.MLA_F32)
+    elif case == "H":
+        args["dims"] = dims(H=192)
+    elif case == "workspace":
+        args["workspace_bytes"] = mla.mla_workspace_size_fp8(info, d) - 1
+    else:
+        args["workspace"] = 256 + 16
+    with pytest.raises(mla.MlaError) as e:
+        mla.mla_decode_attn_fp8(**args, stream=0)
+    assert e.value.status in (mla._binding.MLA_ERR_INVALID, mla._binding.MLA_ERR_UNSUPPORTED,
+                              mla._binding.MLA_ERR_WORKSPACE)
+
+
+def test_fp8_workspace_is_the_partials_then_the_split_query():
+    d = dims(H=128)
+    info = mla.PlanInfo(num_items=4, num_units=6, num_slots=3, num_parts=5, head_groups=2, plan_words=0)
+    parts = mla.mla_workspace_size(info, d)
+    rows = 4 * 128
+    up = lambda x: (x + 255) // 256 * 256
+    assert mla.mla_workspace_size_fp8(info, d) == up(parts) + up(2 * rows * 576) + rows * 4
+    info0 = mla.PlanInfo(num_items=4, num_units=4, num_slots=4, num_parts=0, head_groups=2, plan_words=0)
+    assert mla.mla_workspace_size_fp8(info0, d) == up(2 * rows * 576) + rows * 4
+
+
+@pytest.mark.parametrize("case", ["null", "dims", "count", "align"])
+def test_fp8_quantize_and_append_reject_bad_arguments(case):
+    d = dims(H=128)
+    if case == "null":
+        call = lambda: mla.mla_quantize_rows_fp8(None, 256, 256, 4, d, stream=0)
+    elif case == "dims":
+        call = lambda: mla.mla_cache_append_fp8(256, 256, 256, 256, 256, 2, 1, 4, 8, dims(H=128, Dr=32), stream=0)
+    elif case == "count":
+        call = lambda: mla.mla_quantize_rows_fp8(256, 256, 256, -1, d, stream=0)
+    else:
+        call = lambda: mla.mla_cache_append_fp8(256, 256, 256, 256, 256 + 8, 2, 1, 4, 8, d, stream=0)
+    with pytest.raises(mla.MlaError) as e:
+        call()
+    assert e.value.status in (mla._binding.MLA_ERR_INVALID, mla._binding.MLA_ERR_UNSUPPORTED)
