@@ -120,11 +120,14 @@ def decode_nonabsorbed(q_nope, q_rope, kv_cache, block_table, seq_lens, W_UK, W_
     return dict(out=out, o_lat=o_lat, lse=lse)
 
 
-def full_causal(C, kr, qn_all, qr_all, W_UK, W_UV, scale, heads=None):
+def full_causal(C, kr, qn_all, qr_all, W_UK, W_UV, scale, heads=None, intermediates=None):
     """Full causal forward over one sequence, every position a query (the GatedMLA
     shape: per-head K = [K_c ; shared k], V, causal SDPA with scale over D + D_s).
 
     C [L,R], kr [L,Dr] (float64), qn_all [L,H,Dn], qr_all [L,H,Dr] (stored values).
+    intermediates="kv_bf16" rounds the per-head content keys K_c = C W_UK^T and the
+    values V = C W_UV^T to bf16, as a pipeline that stores its up-projections in bf16
+    before the attention does; everything else stays float64.
     Returns out [L, H, Dv]."""
     qn, qr = to_f64(qn_all), to_f64(qr_all)
     wuk, wuv = to_f64(W_UK), to_f64(W_UV)
@@ -132,6 +135,9 @@ def full_causal(C, kr, qn_all, qr_all, W_UK, W_UV, scale, heads=None):
     out = np.full((L, H, wuv.shape[1]), np.nan)
     for h in (range(H) if heads is None else heads):
         K, V = reconstruct_kv(C, kr, wuk[h], wuv[h])
+        if intermediates == "kv_bf16":
+            K = np.concatenate([round_bf16(K[:, :wuk.shape[1]]), K[:, wuk.shape[1]:]], axis=1)
+            V = round_bf16(V)
         Q = np.concatenate([qn[:, h], qr[:, h]], axis=1)
         S = scale * (Q @ K.T)
         S[np.triu_indices(L, k=1)] = -np.inf

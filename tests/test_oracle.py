@@ -531,3 +531,28 @@ def test_cache_write_rows_against_scalar_loops():
 
 def test_token_positions_follow_the_append_convention():
     np.testing.assert_array_equal(orc.token_positions([5, 2, 9], 2), [3, 4, 0, 1, 7, 8])
+
+
+def test_stored_up_projection_variant_is_exact_on_the_bf16_grid_and_close_otherwise():
+    """full_causal(intermediates="kv_bf16") rounds only K_c = C W_UK^T and V = C W_UV^T.
+    With weights that pick single latent columns times powers of two, K_c and V are bf16
+    values already and the variant equals the definition; with the workload's weights it
+    stays within the bf16 rounding of those two products."""
+    g = np.random.default_rng(31)
+    L, H, R, Dr, Dn, Dv = 37, 3, 32, 8, 8, 8
+    C = orc.to_f64(wl.f32_to_bf16_bits(g.standard_normal((L, R)).astype(np.float32)))
+    kr = orc.to_f64(wl.f32_to_bf16_bits(g.standard_normal((L, Dr)).astype(np.float32)))
+    qn = wl.f32_to_bf16_bits(g.standard_normal((L, H, Dn)).astype(np.float32))
+    qr = wl.f32_to_bf16_bits(g.standard_normal((L, H, Dr)).astype(np.float32))
+    pick = np.zeros((H, Dn, R))
+    for h in range(H):
+        for d in range(Dn):
+            pick[h, d, g.integers(R)] = 2.0 ** int(g.integers(-3, 3))
+    exact = orc.full_causal(C, kr, qn, qr, pick, pick, 0.25)
+    var = orc.full_causal(C, kr, qn, qr, pick, pick, 0.25, intermediates="kv_bf16")
+    np.testing.assert_array_equal(var, exact)
+    W = g.standard_normal((H, Dn, R)) / np.sqrt(R)
+    exact = orc.full_causal(C, kr, qn, qr, W, W, 0.25)
+    var = orc.full_causal(C, kr, qn, qr, W, W, 0.25, intermediates="kv_bf16")
+    assert not np.array_equal(var, exact)
+    assert np.max(np.abs(var - exact)) < 0.05 * np.max(np.abs(exact))
