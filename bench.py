@@ -515,6 +515,150 @@ def run_gpu(args):
     return 0
 
 
+# ----------------------------------------------------------------------------- prefill workloads
+
+PREFILL_METRIC = "MLA prefill (non-absorbed, causal): TFLOP/s and fraction of the B200 bf16 tensor roofline"
+
+
+def prefill_oracle_sample(spec, pin, budget_s):
+    """The oracle's full causal forward on whole (sequence, head) pairs in order, until
+    about budget_s of CPU work. Returns (flops, seconds, desc)."""
+    from oracle import mla_oracle as orc
+    cu = pin["cu_seqlens"]
+    flops, spent, n = 0, 0.0, 0
+    for b in range(len(pin["seq_lens"])):
+        a, e = int(cu[b]), int(cu[b + 1])
+        rows = orc.to_f64(pin["ckr"][a:e])
+        for h in range(spec.H):
+            t0 = time.perf_counter()
+            orc.full_causal(rows[:, :spec.R], rows[:, spec.R:], pin["q_nope"][a:e], pin["q_rope"][a:e],
+                            pin["W_UK"], pin["W_UV"], spec.scale, heads=[h])
+            spent += time.perf_counter() - t0
+            L = e - a
+            flops += 2 * spec.R * (spec.Dn + spec.Dv) * L + L * (L + 1) // 2 * 2 * (spec.Dn + spec.Dr + spec.Dv)
+            n += 1
+            if spent >= budget_s:
+                return flops, spent, f"oracle (fp64 numpy full causal forward) on {n} (sequence, head) pairs"
+    return flops, spent, f"oracle (fp64 numpy full causal forward) on {n} (sequence, head) pairs"
+
+
+def run_prefill(args):
+    """A step is one mla_prefill_attn call over the workload's packed sequences: the two
+    up-projection GEMMs and the causal attention, inputs resident in HBM."""
+    import torch
+    import __graft_entry__
+    __graft_entry__.build()
+    import mla_latent_kv_46_b200 as mla
+    from mla_latent_kv_46_b200 import decoder as dec
+    from inputs import workloads as wl
+
+    torch.cuda.set_device(0)
+    dev = torch.device("cuda", 0)
+    spec = wl.WORKLOADS[args.workload]
+    pin = wl.prefill_inputs(spec, seed=0)
+    d = mla.dims_of(spec)
+    N, B = int(pin["cu_seqlens"][-1]), len(pin["seq_lens"])
+    t = {k: dec.to_torch(pin[k], dev) for k in ("ckr", "q_nope", "q_rope", "W_UK", "W_UV", "cu_seqlens")}
+    out = torch.empty((N, spec.H, spec.Dv), dtype=torch.bfloat16, device=dev)
+    ws_bytes = mla.mla_prefill_workspace_size(N, d)
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def call(q_nope=t["q_nope"], q_rope=t["q_rope"], ckr=t["ckr"]):
+        mla.mla_prefill_attn(ckr, q_nope, q_rope, t["W_UK"], t["W_UV"], t["cu_seqlens"], pin["cu_seqlens"], B,
+                             spec.scale, out, ws, ws_bytes, d, stream)
+
+    for _ in range(args.warmup):
+        call()
+    torch.cuda.synchronize()
+    mla.mla_check_status()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    with ClockSampler(dev.index) as clk:
+        for e0, e1 in ev:
+            e0.record(stream)
+            call()
+            e1.record(stream)
+        torch.cuda.synchronize()
+    mla.mla_check_status()
+    ms = [a.elapsed_time(b) for a, b in ev]
+    ms_per_step = float(np.mean(ms))
+    fl = wl.prefill_flops(spec, pin["seq_lens"])
+    total = fl["up"] + fl["attention"]
+    peaks, peak_src = load_peaks()
+    achieved = total / (ms_per_step / 1e3) / 1e12
+    roof = {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+            "frac": achieved / peaks["bf16_tflops"], "traffic": None,
+            "peak_source": f"{peak_src} (MEASURED_PEAKS.json)" if peak_src == "measured" else "fallback",
+            "kernel": "mla_prefill_attn (tcgen05 up-projection GEMMs + causal attention), the whole call",
+            "algorithmic_flops_per_launch": total, "flops_up_projection": fl["up"],
+            "flops_attention": fl["attention"], "roofline_ms": 1e3 * total / (peaks["bf16_tflops"] * 1e12),
+            "frac_vs_spec": total / (ms_per_step / 1e3) / 1e12 / SPEC_PEAKS["bf16_tflops"]}
+    # end to end: the step's queries and rows from pinned host memory, the output back
+    host_in = {k: torch.from_numpy(np.ascontiguousarray(pin[k]).view(np.int16)).pin_memory()
+               for k in ("ckr", "q_nope", "q_rope")}
+    host_out = torch.empty((N, spec.H, spec.Dv), dtype=torch.int16).pin_memory()
+    e2e_ms = 0.0
+    for k in range(args.steps + 3):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for name in ("ckr", "q_nope", "q_rope"):
+            t[name].view(torch.int16).copy_(host_in[name], non_blocking=True)
+        call()
+        host_out.copy_(out.view(torch.int16), non_blocking=True)
+        e1.record(stream)
+        e1.synchronize()
+        if k >= 3:
+            e2e_ms += e0.elapsed_time(e1)
+    e2e_ms /= args.steps
+    h2d = sum(x.numel() * x.element_size() for x in host_in.values())
+    cpu = None
+    if not args.no_cpu_baseline:
+        f, sec, desc = prefill_oracle_sample(spec, pin, args.cpu_budget)
+        cpu = {"value": f / sec / 1e12, "unit": "TFLOP/s", "cores": cpu_threads(), "kind": "oracle", "sample": desc,
+               "seconds": sec}
+    lens = pin["seq_lens"]
+    line = {"metric": PREFILL_METRIC, "value": achieved, "unit": "TFLOP/s", "n_gpus": 1, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": spec.name, "B": B, "H": spec.H, "kv_lora_rank": spec.R, "rope_dim": spec.Dr,
+                       "D_nope": spec.Dn, "D_v": spec.Dv, "seq_lens": f"{int(lens[0])} each" if len(set(lens)) == 1
+                       else "ragged", "tokens": N,
+                       "l2": "inputs larger than L2 (the queries alone are "
+                             f"{N * spec.H * (spec.Dn + spec.Dr) * 2 / 1e6:.0f} MB); no flush"},
+            "roofline": roof, "cpu_baseline": cpu,
+            "e2e": {"value": total / (e2e_ms / 1e3) / 1e12, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": host_out.numel() * 2, "ms_per_step": e2e_ms,
+                    "mode": "one step at a time: rows and queries in, output out"},
+            "gpu_launches": 3 * args.steps, "clocks": clk.summary()}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_prefill_reference(args):
+    if int(os.environ.get("RANK", "0")) != 0:
+        return 0
+    from inputs import workloads as wl
+    spec = wl.WORKLOADS[args.workload]
+    pin = wl.prefill_inputs(spec, seed=0)
+    for _ in range(args.warmup):
+        prefill_oracle_sample(spec, pin, 1.0)
+    tot_f, tot_t, desc = 0, 0.0, ""
+    for _ in range(args.steps):
+        f, sec, desc = prefill_oracle_sample(spec, pin, 4.0)
+        tot_f += f
+        tot_t += sec
+    value = tot_f / tot_t / 1e12
+    line = {"metric": PREFILL_METRIC, "value": value, "unit": "TFLOP/s", "impl": "reference", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * tot_t / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": spec.name, "B": spec.B, "H": spec.H},
+            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cpu_threads(), "kind": "oracle",
+                             "sample": f"per step: {desc}"},
+            "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -533,9 +677,10 @@ def main():
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
+    prefill = args.workload.startswith("prefill")
     if args.impl == "reference":
-        return run_reference(args)
-    return run_gpu(args)
+        return run_prefill_reference(args) if prefill else run_reference(args)
+    return run_prefill(args) if prefill else run_gpu(args)
 
 
 if __name__ == "__main__":

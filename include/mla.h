@@ -54,7 +54,7 @@
 extern "C" {
 #endif
 
-#define MLA_ABI_VERSION 4
+#define MLA_ABI_VERSION 5
 
 typedef enum {
   MLA_OK = 0,
@@ -283,6 +283,35 @@ mla_status mla_decode_attn_fp8(const void* q_lat, const void* q_rope, const void
                                int32_t max_pages, int32_t num_pages, float scale, const int32_t* plan_dev,
                                const mla_plan_info* info, void* o_lat, float* lse, void* workspace,
                                size_t workspace_bytes, mla_dims d, void* stream);
+
+/* ---------------------------------------------------------------- f4: non-absorbed prefill
+ * The GatedMLA forward over whole sequences (kimi-k3 docs "GatedMLA": "Build per-head Q,
+ * K and V" and "Observe logits, then compute causal attention"): every position of a
+ * sequence is a query. For head h, K_h = [C W_UK[h]^T ; k_rope] (the shared rope key
+ * broadcast to every head), V_h = C W_UV[h]^T, and
+ *   out[t][h] = sum_{t' <= t} softmax_t'(scale * [q_nope ; q_rope][t][h] . K_h[t']) V_h[t'],
+ * scale = 1/sqrt(Dn + Dr) as for the decode. The non-absorbed form is the cheaper one when
+ * every position is a query: 2 (Dn + Dr + Dv) FLOP per head and (query, key) pair against
+ * the absorbed form's 2 (R + Dr + R). The output gate and Wo that follow in GatedMLA are
+ * plain projections outside this library.
+ *   ckr        [N][R+Dr] bf16: the packed sequences' rows [c ; k_rope] (k_rope rotated)
+ *   q_nope     [N][H][Dn], q_rope [N][H][Dr] bf16 (q_rope rotated)
+ *   W_UK [H][Dn][R], W_UV [H][Dv][R] bf16
+ *   cu_seqlens [B+1] int32 on the DEVICE and cu_seqlens_host the same on the HOST:
+ *              sequence b is rows cu_seqlens[b] .. cu_seqlens[b+1]-1, cu_seqlens[0] = 0
+ *   out        [N][H][Dv] bf16
+ *   workspace  >= mla_prefill_workspace_size(N, d) bytes, 256-byte aligned: the per-head
+ *              K_c and V in bf16 ([N][H][128] each), written by the first two launches
+ * Three launches: two tensor-core GEMMs (the up-projections of every token for all heads),
+ * then causal attention (tensor cores; 128 queries x one head per CTA). Dims: bf16, R=512,
+ * Dr=64, Dn=Dv=128, even H (else MLA_ERR_UNSUPPORTED; no SIMT kernel). Precision: K_c, V
+ * and P enter the MMAs in bf16 (P with its bf16 remainder where one key can dominate a
+ * row), fp32 accumulation and softmax.                                                */
+size_t mla_prefill_workspace_size(int32_t N, mla_dims d);
+mla_status mla_prefill_attn(const void* ckr, const void* q_nope, const void* q_rope, const void* W_UK,
+                            const void* W_UV, const int32_t* cu_seqlens, const int32_t* cu_seqlens_host, int32_t B,
+                            float scale, void* out, void* workspace, size_t workspace_bytes, mla_dims d,
+                            void* stream);
 
 /* ---------------------------------------------------------------- allocation-free decode
  * The pages describe no counterpart of this call; it exists for callers that cannot

@@ -82,6 +82,10 @@ WORKLOADS: Dict[str, WorkloadSpec] = {
         dtype="bf16", seq_len=None, ragged=(512, 16384), w_std=1.0 / math.sqrt(512),
         description="two new tokens per sequence (multi-token decode), H=128, 64 sequences, "
                     "lengths uniform in [512,16384]"),
+    "prefill_h64_b4_l4096": WorkloadSpec(
+        name="prefill_h64_b4_l4096", B=4, H=64, R=512, Dr=64, Dn=128, Dv=128, q_len=4096,
+        dtype="bf16", seq_len=4096, w_std=1.0 / math.sqrt(512), all_query_positions=True,
+        description="non-absorbed prefill (every position a query, causal), H=64, 4 sequences x 4096"),
     "causal_chunk_h64_b8_2048p256": WorkloadSpec(
         name="causal_chunk_h64_b8_2048p256", B=8, H=64, R=512, Dr=64, Dn=128, Dv=128, q_len=256,
         dtype="bf16", seq_len=2048 + 256, w_std=1.0 / math.sqrt(512), all_query_positions=True,
@@ -271,3 +275,36 @@ def latent_outputs(spec: WorkloadSpec, T: int, seed: int = 0, fp32: bool = False
     g = _rng(seed, 7)
     x = g.standard_normal((T, spec.H, spec.R), dtype=np.float32) * np.float32(0.1)
     return x if fp32 else _store(spec, x)
+
+
+def prefill_inputs(spec: WorkloadSpec, seq_lens: Optional[Sequence[int]] = None, seed: int = 0) -> dict:
+    """Packed inputs of a prefill over whole sequences (every position a query): the rows
+    [c ; k_rope] of all sequences back to back [N, R+Dr], their queries [N, H, Dn] and
+    [N, H, Dr], cu_seqlens [B+1] and the weights, in storage dtype. The same per-sequence
+    streams as the decode workloads' rows and queries."""
+    lens = [int(x) for x in (seq_lens if seq_lens is not None else seq_lens_of(spec, seed))]
+    s_all = dataclasses.replace(spec, all_query_positions=True)
+    rows, qns, qrs = [], [], []
+    for b, L in enumerate(lens):
+        rows.append(sequence_rows(s_all, b, L, seed))
+        qn, qr = queries_of(s_all, b, L, seed)
+        qns.append(qn)
+        qrs.append(qr)
+    sdt = np.uint16 if spec.dtype == "bf16" else np.float32
+    cat = lambda xs, shape: np.concatenate(xs) if xs else np.zeros(shape, sdt)  # noqa: E731
+    cu = np.zeros(len(lens) + 1, np.int32)
+    cu[1:] = np.cumsum(lens)
+    wuk, wuv = weights_of(spec, seed)
+    return dict(spec=spec, seq_lens=np.asarray(lens, np.int32), cu_seqlens=cu,
+                ckr=cat(rows, (0, spec.row)), q_nope=cat(qns, (0, spec.H, spec.Dn)),
+                q_rope=cat(qrs, (0, spec.H, spec.Dr)), W_UK=wuk, W_UV=wuv, scale=spec.scale)
+
+
+def prefill_flops(spec: WorkloadSpec, seq_lens) -> dict:
+    """FLOPs of a non-absorbed prefill: the up-projections (2 R H (Dn + Dv) per token) and
+    the causal attention (2 H (Dn + Dr + Dv) per (query, key) pair, key <= query)."""
+    lens = np.asarray(seq_lens, dtype=np.int64)
+    pairs = int(np.sum(lens * (lens + 1) // 2))
+    up = int(lens.sum()) * 2 * spec.R * spec.H * (spec.Dn + spec.Dv)
+    attn = pairs * 2 * spec.H * (spec.Dn + spec.Dr + spec.Dv)
+    return dict(pairs=pairs, up=up, attention=attn)

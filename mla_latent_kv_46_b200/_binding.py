@@ -28,7 +28,7 @@ EXPORTS = ("mla_abi_version", "mla_last_error", "mla_set_policy", "mla_set_wait_
            "mla_check_status", "mla_cache_append", "mla_cache_write", "mla_cache_write_workspace_size", "mla_absorb_q", "mla_plan_capacity", "mla_plan_splits",
            "mla_workspace_size", "mla_decode_attn", "mla_combine", "mla_out_proj", "mla_decode_attn_noalloc",
            "mla_debug_drop_page_load", "mla_quantize_rows_fp8", "mla_cache_append_fp8", "mla_workspace_size_fp8",
-           "mla_decode_attn_fp8")
+           "mla_decode_attn_fp8", "mla_prefill_workspace_size", "mla_prefill_attn")
 
 
 class MlaError(RuntimeError):
@@ -81,6 +81,8 @@ def _load():
         "mla_cache_append_fp8": (I32, [P, P, P, P, P, I32, I32, I32, I32, D, P]),
         "mla_workspace_size_fp8": (SZ, [INFO, D]),
         "mla_decode_attn_fp8": (I32, [P, P, P, P, P, P, I32, I32, I32, I32, F, P, INFO, P, P, P, SZ, D, P]),
+        "mla_prefill_workspace_size": (SZ, [I32, D]),
+        "mla_prefill_attn": (I32, [P, P, P, P, P, P, P, I32, F, P, P, SZ, D, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -232,3 +234,16 @@ def mla_decode_attn_fp8(q_lat, q_rope, kv_codes, kv_scales, block_table, seq_len
                                     _ptr(seq_lens), B, q_len, max_pages, num_pages, scale, _ptr(plan_dev),
                                     ctypes.byref(info), _ptr(o_lat), _ptr(lse), _ptr(workspace), workspace_bytes,
                                     dims, _stream(stream)), "mla_decode_attn_fp8")
+
+
+def mla_prefill_workspace_size(N, dims) -> int:
+    return _lib.mla_prefill_workspace_size(N, dims)
+
+
+def mla_prefill_attn(ckr, q_nope, q_rope, W_UK, W_UV, cu_seqlens, cu_seqlens_host, B, scale, out, workspace,
+                     workspace_bytes, dims, stream=None):
+    """cu_seqlens: device int32 [B+1]; cu_seqlens_host: the same as a host numpy int32 array."""
+    host = np.ascontiguousarray(cu_seqlens_host, dtype=np.int32)
+    _check(_lib.mla_prefill_attn(_ptr(ckr), _ptr(q_nope), _ptr(q_rope), _ptr(W_UK), _ptr(W_UV), _ptr(cu_seqlens),
+                                 host.ctypes.data, B, scale, _ptr(out), _ptr(workspace), workspace_bytes, dims,
+                                 _stream(stream)), "mla_prefill_attn")

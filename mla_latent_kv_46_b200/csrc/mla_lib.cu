@@ -24,6 +24,7 @@
 #include "decode_2sm.cuh"
 #include "cache_write.cuh"
 #include "fp8_kernels.cuh"
+#include "prefill.cuh"
 
 namespace {
 
@@ -954,6 +955,93 @@ mla_status mla_decode_attn_fp8(const void* q_lat, const void* q_rope, const void
   mla::duo::decode_2sm_kernel<true><<<grid, mla::duo::kThreadsF8, mla::duo::kSmemBytesF8, st>>>(tk32, tqh, tk64, to,
                                                                                                top, tql, p);
   return launch_check("decode_attn_fp8 (tcgen05, SM pair)");
+}
+
+// ------------------------------------------------------------------------------- prefill (non-absorbed)
+static bool prefill_dims_ok(const mla_dims& d) {
+  return d.dtype == MLA_BF16 && d.R == 512 && d.Dr == 64 && d.Dn == 128 && d.Dv == 128 && d.H % 2 == 0;
+}
+
+size_t mla_prefill_workspace_size(int32_t N, mla_dims d) {
+  if (N <= 0 || check_dims(d) != MLA_OK || !prefill_dims_ok(d)) return 0;
+  return 2 * (((size_t)N * d.H * 128 * 2 + 255) / 256 * 256);
+}
+
+mla_status mla_prefill_attn(const void* ckr, const void* q_nope, const void* q_rope, const void* W_UK,
+                            const void* W_UV, const int32_t* cu_seqlens, const int32_t* cu_seqlens_host, int32_t B,
+                            float scale, void* out, void* workspace, size_t workspace_bytes, mla_dims d,
+                            void* stream) {
+  if (mla_status s = check_dims(d)) return s;
+  if (!prefill_dims_ok(d))
+    return fail(MLA_ERR_UNSUPPORTED, "prefill needs bf16, R=512, Dr=64, Dn=Dv=128 and an even head count");
+  if (g_policy.load() == MLA_POLICY_SIMT)
+    return fail(MLA_ERR_UNSUPPORTED, "prefill has only a tensor-core kernel (policy is SIMT)");
+  if (B < 0) return fail(MLA_ERR_INVALID, "bad B=%d", B);
+  if (!(scale > 0.f) || !std::isfinite(scale)) return fail(MLA_ERR_INVALID, "scale must be positive");
+  if (B == 0) return ok();
+  if (!cu_seqlens_host || !cu_seqlens) return fail(MLA_ERR_INVALID, "null cu_seqlens");
+  if (cu_seqlens_host[0] != 0) return fail(MLA_ERR_INVALID, "cu_seqlens[0] must be 0");
+  int32_t max_qtiles = 0, tiles = 0;
+  for (int32_t b = 0; b < B; ++b) {
+    const int32_t L = cu_seqlens_host[b + 1] - cu_seqlens_host[b];
+    if (L < 0) return fail(MLA_ERR_INVALID, "cu_seqlens must not decrease (sequence %d)", b);
+    const int32_t t = (L + mla::pf::kM - 1) / mla::pf::kM;
+    max_qtiles = std::max(max_qtiles, t);
+    tiles += t;
+  }
+  const int32_t N = cu_seqlens_host[B];
+  if (N == 0) return ok();
+  if (!ckr || !q_nope || !q_rope || !W_UK || !W_UV || !out) return fail(MLA_ERR_INVALID, "null pointer");
+  const size_t need = mla_prefill_workspace_size(N, d);
+  if (!workspace || workspace_bytes < need) return fail(MLA_ERR_WORKSPACE, "workspace %zu bytes < %zu needed",
+                                                        workspace_bytes, need);
+  if (reinterpret_cast<uintptr_t>(workspace) % 256 != 0) return fail(MLA_ERR_INVALID, "workspace not 256-byte aligned");
+  __nv_bfloat16* kc = static_cast<__nv_bfloat16*>(workspace);
+  __nv_bfloat16* vv = reinterpret_cast<__nv_bfloat16*>(static_cast<char*>(workspace) + need / 2);
+  cudaStream_t st = as_stream(stream);
+  const int32_t HD = d.H * 128;
+  // up-projections: K_c = C W_UK^T and V = C W_UV^T for all heads at once (one GEMM each,
+  // A = the latent columns of the packed rows, B = the weights as [H*128][512], K-major)
+  {
+    using C = mla::gemm::Cfg<8, 256, false, 3>;
+    auto kern = mla::gemm::proj_kernel<8, 256, false, 3>;
+    if (mla_status s = ensure_smem_attr((const void*)kern, C::kSmemBytes)) return s;
+    CUtensorMap ta;
+    if (mla_status s = make_map_2d(&ta, ckr, 512, (uint64_t)N, 576 * 2, 128)) return s;
+    const void* W[2] = {W_UK, W_UV};
+    __nv_bfloat16* O[2] = {kc, vv};
+    for (int i = 0; i < 2; ++i) {
+      CUtensorMap tb;
+      if (mla_status s = make_map_2d(&tb, W[i], 512, (uint64_t)HD, 512 * 2, 64)) return s;
+      mla::gemm::Params gp;
+      gp.out = O[i];
+      gp.T = N;
+      gp.H = 1;
+      gp.n_total = HD;
+      gp.timeout_ns = g_timeout_ns.load();
+      const dim3 grid(1, (N + mla::gemm::kM - 1) / mla::gemm::kM, HD / 256);
+      kern<<<grid, 128, C::kSmemBytes, st>>>(ta, tb, gp);
+      if (mla_status s = launch_check("prefill (up-projection)")) return s;
+    }
+  }
+  CUtensorMap tqn, tqr, tkc, tkr, tv;
+  if (mla_status s = make_map_2d(&tqn, q_nope, HD, (uint64_t)N, (uint64_t)HD * 2, 128)) return s;
+  if (mla_status s = make_map_2d(&tqr, q_rope, (uint64_t)d.H * 64, (uint64_t)N, (uint64_t)d.H * 64 * 2, 128)) return s;
+  if (mla_status s = make_map_2d(&tkc, kc, HD, (uint64_t)N, (uint64_t)HD * 2, 128)) return s;
+  if (mla_status s = make_map_2d(&tkr, ckr, 576, (uint64_t)N, 576 * 2, 128)) return s;
+  if (mla_status s = make_map_2d(&tv, vv, HD, (uint64_t)N, (uint64_t)HD * 2, 128)) return s;
+  if (mla_status s = ensure_smem_attr((const void*)mla::pf::prefill_attn_kernel, mla::pf::kSmemBytes)) return s;
+  mla::pf::Params pp;
+  pp.cu_seqlens = cu_seqlens;
+  pp.B = B;
+  pp.H = d.H;
+  pp.max_qtiles = max_qtiles;
+  pp.scale_log2 = scale * 1.4426950408889634f;
+  pp.out = static_cast<__nv_bfloat16*>(out);
+  pp.timeout_ns = g_timeout_ns.load();
+  const dim3 grid(tiles, d.H);
+  mla::pf::prefill_attn_kernel<<<grid, mla::pf::kThreads, mla::pf::kSmemBytes, st>>>(tqn, tqr, tkc, tkr, tv, pp);
+  return launch_check("prefill (attention)");
 }
 
 mla_status mla_combine(const int32_t* plan_dev, const mla_plan_info* info, const void* workspace,

@@ -34,7 +34,7 @@ def test_library_exports_every_declared_symbol():
 
 
 def test_abi_version_and_error_text():
-    assert mla.mla_abi_version() == 4
+    assert mla.mla_abi_version() == 5
     with pytest.raises(mla.MlaError) as e:
         mla.mla_set_policy(7)
     assert e.value.status == mla._binding.MLA_ERR_INVALID
@@ -340,3 +340,34 @@ def test_fp8_quantize_and_append_reject_bad_arguments(case):
     with pytest.raises(mla.MlaError) as e:
         call()
     assert e.value.status in (mla._binding.MLA_ERR_INVALID, mla._binding.MLA_ERR_UNSUPPORTED)
+
+
+@pytest.mark.parametrize("case", ["dims", "odd_heads", "decreasing", "first", "workspace", "null"])
+def test_prefill_rejects_bad_arguments_before_launch(case):
+    d = dims(H=8)
+    cu = np.array([0, 100, 300], np.int32)
+    args = dict(ckr=256, q_nope=256, q_rope=256, W_UK=256, W_UV=256, cu_seqlens=256, cu_seqlens_host=cu, B=2,
+                scale=0.07, out=256, workspace=256, workspace_bytes=1 << 30, dims=d)
+    if case == "dims":
+        args["dims"] = mla.Dims(8, 128, 64, 64, 512, 64, mla.MLA_BF16)   # Dv = 64
+    elif case == "odd_heads":
+        args["dims"] = dims(H=7)
+    elif case == "decreasing":
+        args["cu_seqlens_host"] = np.array([0, 100, 50], np.int32)
+    elif case == "first":
+        args["cu_seqlens_host"] = np.array([4, 100, 300], np.int32)
+    elif case == "workspace":
+        args["workspace_bytes"] = mla.mla_prefill_workspace_size(300, d) - 1
+    else:
+        args["q_rope"] = None
+    with pytest.raises(mla.MlaError) as e:
+        mla.mla_prefill_attn(**args, stream=0)
+    assert e.value.status in (mla._binding.MLA_ERR_INVALID, mla._binding.MLA_ERR_UNSUPPORTED,
+                              mla._binding.MLA_ERR_WORKSPACE)
+
+
+def test_prefill_workspace_holds_bf16_keys_and_values_of_every_head():
+    d = dims(H=64)
+    assert mla.mla_prefill_workspace_size(16384, d) == 2 * 16384 * 64 * 128 * 2
+    assert mla.mla_prefill_workspace_size(3, dims(H=2)) == 2 * ((3 * 2 * 128 * 2 + 255) // 256 * 256)
+    assert mla.mla_prefill_workspace_size(100, mla.Dims(8, 64, 64, 128, 512, 64, mla.MLA_BF16)) == 0   # Dn = 64
