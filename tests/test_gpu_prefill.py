@@ -57,12 +57,14 @@ def ulp_bf16(x):
     return np.where(a > 0, np.exp2(e - 7), 0.0)
 
 
-def one_ulp_allowance(C, kr, qn, qr, W_UK, W_UV, scale, h):
-    """[L, Dv] first-order effect on out of moving every stored K_c and V element of head h
-    by one bf16 ulp. The kernels round the up-projections from fp32 sums, the oracle from
-    exact products, so the two may pick neighbouring bf16 values where the exact value
-    lies within fp32 error of a rounding boundary: sum_t p_t ulp(V_t) for the values and
-    sum_t p_t |V_t - out| scale sum_c |q_c| ulp(K_c,tc) for the keys."""
+def one_ulp_allowance(C, kr, qn, qr, W_UK, W_UV, scale, h, top=4):
+    """[L, Dv] first-order effect on out of a one-ulp difference in the stored K_c and V
+    elements of the `top` keys that carry the most weight in each row (head h). The
+    kernels round the up-projections from fp32 sums, the oracle from exact products, so
+    the two may pick neighbouring bf16 values where an exact value lies within fp32 error
+    of a rounding boundary (rare: one element in tens of thousands); only a flip in a
+    heavily weighted key moves an output measurably. Values: sum_t p_t ulp(V_t,d); keys:
+    sum_t p_t (|V_t,d| + |out_d|) scale max_c |q_c| ulp(K_t,c)."""
     Kc = orc.round_bf16(C @ orc.to_f64(W_UK)[h].T)
     V = orc.round_bf16(C @ orc.to_f64(W_UV)[h].T)
     q = np.concatenate([orc.to_f64(qn)[:, h], orc.to_f64(qr)[:, h]], axis=1)
@@ -73,13 +75,16 @@ def one_ulp_allowance(C, kr, qn, qr, W_UK, W_UV, scale, h):
     P = np.exp(S - S.max(axis=1, keepdims=True))
     P /= P.sum(axis=1, keepdims=True)
     out = P @ V
-    dS = scale * (np.abs(q[:, :Kc.shape[1]]) @ ulp_bf16(Kc).T)         # [L queries, L keys]
-    tv = P @ ulp_bf16(V)
-    tk = np.einsum("ik,ik,ikd->id", P, dS, np.abs(V[None, :, :] - out[:, None, :]))
+    k = min(top, L)
+    idx = np.argpartition(-P, k - 1, axis=1)[:, :k]                   # [L, k] heaviest keys
+    pk = np.take_along_axis(P, idx, axis=1)[:, :, None]                # [L, k, 1]
+    tv = np.sum(pk * ulp_bf16(V)[idx], axis=1)
+    dq = np.max(np.abs(q[:, None, :Kc.shape[1]]) * ulp_bf16(Kc)[idx], axis=2)[:, :, None]   # [L, k, 1]
+    tk = np.sum(pk * scale * dq * (np.abs(V[idx]) + np.abs(out)[:, None, :]), axis=1)
     return tv + tk
 
 
-def check(pin, got, heads=None, exact_min_keys=129, exact=True):
+def check(pin, got, heads=None, exact_min_keys=129, check_exact=True):
     spec = pin["spec"]
     cu = pin["cu_seqlens"]
     hs = list(range(spec.H)) if heads is None else list(heads)
@@ -101,7 +106,7 @@ def check(pin, got, heads=None, exact_min_keys=129, exact=True):
             bad = err > bound
             assert not np.any(bad), (f"sequence {b} head {h} (stored-intermediates oracle): {bad.sum()} of "
                                      f"{bad.size} outside the bound; worst ratio {(err / bound).max():.2f}")
-        if exact and e - a >= exact_min_keys:
+        if check_exact and e - a >= exact_min_keys:
             exact = orc.full_causal(C, kr, qn, qr, pin["W_UK"], pin["W_UV"], spec.scale, heads=hs)
             lo = exact_min_keys - 1
             assert_close(got[a + lo:e][:, hs], exact[lo:, hs], False, f"sequence {b} rows >= {exact_min_keys} keys")
@@ -121,7 +126,7 @@ def test_prefill_large_logit_offsets_move_the_reference():
     past the absolute bound at any length (up to ~2x): this case is held to the
     stored-intermediates oracle."""
     pin = wl.prefill_inputs(prefill_spec(4, noise=4.0), [700, 333], seed=5)
-    check(pin, run_prefill(pin), exact=False)
+    check(pin, run_prefill(pin), check_exact=False)
 
 
 def test_prefill_long_sequences_sampled_heads():
