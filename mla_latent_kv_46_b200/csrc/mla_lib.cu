@@ -1003,8 +1003,9 @@ mla_status mla_prefill_attn(const void* ckr, const void* q_nope, const void* q_r
   // up-projections: K_c = C W_UK^T and V = C W_UV^T for all heads at once (one GEMM each,
   // A = the latent columns of the packed rows, B = the weights as [H*128][512], K-major)
   {
-    using C = mla::gemm::Cfg<8, 256, false, 3>;
-    auto kern = mla::gemm::proj_kernel<8, 256, false, 3>;
+    // two stages (97 KiB): two CTAs per SM, one's epilogue under the other's main loop
+    using C = mla::gemm::Cfg<8, 256, false, 2>;
+    auto kern = mla::gemm::proj_kernel<8, 256, false, 2>;
     if (mla_status s = ensure_smem_attr((const void*)kern, C::kSmemBytes)) return s;
     CUtensorMap ta;
     if (mla_status s = make_map_2d(&ta, ckr, 512, (uint64_t)N, 576 * 2, 128)) return s;
