@@ -191,3 +191,52 @@ def test_full_size_fp8_every_output(name):
     assert_close(out, ref["out"], False, f"{name} out (8-bit cache)")
     assert_close(lse, ref["lse"], False, f"{name} lse (8-bit cache)")
     assert_close(o_lat, ref["o_lat"], False, f"{name} o_lat (8-bit cache)")
+
+
+@pytest.mark.parametrize("H,q_len", [(128, 1), (64, 2)])
+def test_fp8_bad_page_id_is_reported_not_faulted(H, q_len):
+    """A block-table entry outside the pool: the 8-bit kernel's loads read zeros there (the
+    scale bytes of page 0 stand in), the status word reports it, the next check passes."""
+    spec = small_spec(H=H, q_len=q_len)
+    w = quantised(wl.make(spec, seed=2, seq_lens=[130, 64]))
+    w["block_table"][1, 0] = 10_000
+    step = dec.DecodeStep(w, cache="fp8")
+    step.q_lat.copy_(dec.to_torch(wl.latent_queries(spec, step.T, seed=1), step.device))
+    step.attend()
+    step.combine()
+    torch.cuda.synchronize()
+    with pytest.raises(mla.MlaError) as e:
+        mla.mla_check_status()
+    assert e.value.status == mla._binding.MLA_ERR_INVALID
+    mla.mla_check_status()
+
+
+def test_fp8_dropped_page_load_times_out_and_context_stays_usable():
+    """The testing hook skips one score-operand load of the first CTA: the MMA issuer's
+    wait runs out, every role of both CTAs (converters included) leaves through the abort
+    flag, the status word reports MLA_ERR_TIMEOUT, and the same context then decodes the
+    8-bit cache correctly."""
+    spec = small_spec(H=128)
+    w = quantised(wl.make(spec, seed=4, seq_lens=[700, 300, 129]))
+    step = dec.DecodeStep(w, sms=4, cache="fp8")
+    ql = wl.latent_queries(spec, step.T, seed=9)
+    step.q_lat.copy_(dec.to_torch(ql, step.device))
+    mla.mla_set_wait_timeout_ns(20_000_000)
+    mla.mla_debug_drop_page_load(2)
+    try:
+        step.attend()
+        torch.cuda.synchronize()
+        with pytest.raises(mla.MlaError) as e:
+            mla.mla_check_status()
+        assert e.value.status == mla._binding.MLA_ERR_TIMEOUT
+    finally:
+        mla.mla_debug_drop_page_load(-1)
+        mla.mla_set_wait_timeout_ns(2_000_000_000)
+    mla.mla_check_status()
+    step.attend()
+    step.combine()
+    torch.cuda.synchronize()
+    mla.mla_check_status()
+    ref = orc.attend_latent(ql, w["q_rope"], w["kv_deq"], w["block_table"], w["seq_lens"], w["scale"],
+                            q_len=1, page_size=spec.page_size)
+    assert_close(host(step.o_lat), ref["o_lat"], False, "o_lat (8-bit cache) after the injected timeout")
