@@ -139,7 +139,7 @@ mla_status mla_cache_append(void* kv_cache, const int32_t* block_table, const in
 
 /* ---------------------------------------------------------------- cache-write prologue
  * The rows a step appends, computed from the new tokens' hidden states, then appended
- * as mla_cache_append does (survey row f1). For every new token t (token i of sequence
+ * as mla_cache_append does. For every new token t (token i of sequence
  * b, position pos = seq_lens[b] - q_len + i):
  *   f = W_DKV h_t                       (kimi-k3 docs "GatedMLA", "Projection geometry and
  *                                        stored weights": one down projection M -> R_kv + D_s
@@ -240,7 +240,7 @@ mla_status mla_out_proj(const void* o_lat, const void* W_UV, void* out, int32_t 
 /* ---------------------------------------------------------------- 8-bit (E4M3) latent cache
  * The softved page "Introduction to MLA vs. KV Cache in Large Language Models" ("Practical
  * Implementation Tips for MLA in LLM Serving") advises quantising the latent cache to cut
- * its memory further; it fixes no format. This library's reading (survey row f2):
+ * its memory further; it fixes no format. This library's reading:
  *  - every element of a cached row [c ; k_rope] is one byte, an E4M3 code of the OCP 8-bit
  *    floating-point format (sign, 4 exponent bits with bias 7, 3 mantissa bits, subnormals,
  *    no infinities, 0x7F/0xFF NaN, largest finite 448): kv_codes [num_pages][64][576] uint8;
