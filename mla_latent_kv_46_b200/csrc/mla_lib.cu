@@ -1055,6 +1055,19 @@ mla_status mla_combine(const int32_t* plan_dev, const mla_plan_info* info, const
   if (mla_status s = split_workspace(info, d, const_cast<void*>(workspace), workspace_bytes, &o_part, &lse_part))
     return s;
   if (d.R <= 512 && d.R % 4 == 0) {
+    // parts per query, at least: a few queries cut into many parts spread their parts over
+    // the warps of a block; otherwise one warp per (query, head)
+    const int32_t per_item = info->num_items > 0 ? info->num_parts / info->num_items : 0;
+    if (per_item >= 3) {
+      const dim3 gw(info->num_items, d.H);
+      if (per_item >= 8)
+        mla::simt::combine_wide_kernel<8><<<gw, 256, 0, as_stream(stream)>>>(
+            plan_dev, o_part, lse_part, static_cast<float*>(o_lat), lse, d.H, d.R);
+      else
+        mla::simt::combine_wide_kernel<4><<<gw, 128, 0, as_stream(stream)>>>(
+            plan_dev, o_part, lse_part, static_cast<float*>(o_lat), lse, d.H, d.R);
+      return launch_check("combine");
+    }
     const dim3 gv(info->num_items, (d.H + 3) / 4);
     mla::simt::combine_vec_kernel<<<gv, 128, 0, as_stream(stream)>>>(plan_dev, o_part, lse_part,
                                                                       static_cast<float*>(o_lat), lse, d.H, d.R);

@@ -309,5 +309,94 @@ __global__ void __launch_bounds__(128) combine_vec_kernel(const int32_t* __restr
   if (lane == 0 && lse) lse[(int64_t)item * H + h] = tot > 0.f ? M + logf(tot) : -CUDART_INF_F;
 }
 
+// The same merge with one (item, head)'s parts spread over W warps: grid (num_items, H),
+// block 32 W, rows of R <= 512 (R % 4 == 0). Warp w merges parts w, w + W, w + 2W, ...
+// online, two per round trip, as combine_vec_kernel does, and the W running (maximum,
+// sum, row) triples are then merged through shared memory. For plans that cut a few
+// queries into many parts (long sequences spread over every slot), where one warp's serial
+// pass over all of a query's parts would set the kernel's duration.
+template <int W>
+__global__ void __launch_bounds__(32 * W) combine_wide_kernel(const int32_t* __restrict__ plan_w,
+                                                              const float* __restrict__ o_part,
+                                                              const float* __restrict__ lse_part,
+                                                              float* __restrict__ o_lat, float* __restrict__ lse,
+                                                              int32_t H, int32_t R) {
+  __shared__ float s_m[W], s_t[W];
+  __shared__ float4 s_acc[W][128];
+  const PlanView plan{plan_w};
+  const int32_t item = blockIdx.x, h = blockIdx.y;
+  const int32_t warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int32_t first = plan.item_parts()[2 * item], np = plan.item_parts()[2 * item + 1];
+  if (np == 0) return;   // the same for every thread of the block
+  const int32_t nv = R / 4;
+  float4 acc[4];
+#pragma unroll
+  for (int k = 0; k < 4; ++k) acc[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+  float M = -CUDART_INF_F, tot = 0.f;
+  for (int32_t s = warp; s < np; s += 2 * W) {
+    const bool two = s + W < np;
+    float z[2];
+    float4 v[2][4];
+#pragma unroll
+    for (int q = 0; q < 2; ++q) {
+      const int32_t ps = first + s + (q && two ? W : 0);
+      z[q] = (q && !two) ? -CUDART_INF_F : lse_part[(int64_t)ps * H + h];
+      const float4* src = reinterpret_cast<const float4*>(o_part + ((int64_t)ps * H + h) * R);
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const int32_t i = lane + 32 * k;
+        v[q][k] = i < nv ? __ldcs(src + i) : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+    }
+    const float Mn = fmaxf(M, fmaxf(z[0], z[1]));
+    if (Mn == -CUDART_INF_F) continue;   // no part so far saw a token
+    const float r = expf(M - Mn);        // 0 while M is -inf
+    const float w0 = expf(z[0] - Mn), w1 = expf(z[1] - Mn);
+    tot = tot * r + (w0 + w1);
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      acc[k].x = fmaf(w1, v[1][k].x, fmaf(w0, v[0][k].x, acc[k].x * r));
+      acc[k].y = fmaf(w1, v[1][k].y, fmaf(w0, v[0][k].y, acc[k].y * r));
+      acc[k].z = fmaf(w1, v[1][k].z, fmaf(w0, v[0][k].z, acc[k].z * r));
+      acc[k].w = fmaf(w1, v[1][k].w, fmaf(w0, v[0][k].w, acc[k].w * r));
+    }
+    M = Mn;
+  }
+  // merge the warps' triples: each row rescaled to the common maximum
+  if (lane == 0) {
+    s_m[warp] = M;
+    s_t[warp] = tot;
+  }
+  __syncthreads();
+  float Mx = -CUDART_INF_F;
+#pragma unroll
+  for (int w = 0; w < W; ++w) Mx = fmaxf(Mx, s_m[w]);
+  const float f = M == -CUDART_INF_F ? 0.f : expf(M - Mx);
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const int32_t i = lane + 32 * k;
+    if (i < nv) s_acc[warp][i] = make_float4(acc[k].x * f, acc[k].y * f, acc[k].z * f, acc[k].w * f);
+  }
+  __syncthreads();
+  float T = 0.f;
+#pragma unroll
+  for (int w = 0; w < W; ++w) T += s_m[w] == -CUDART_INF_F ? 0.f : s_t[w] * expf(s_m[w] - Mx);
+  const float inv = T > 0.f ? 1.f / T : 0.f;
+  float* dst = o_lat + ((int64_t)item * H + h) * R;
+  for (int32_t i = threadIdx.x; i < nv; i += 32 * W) {
+    float4 a = s_acc[0][i];
+#pragma unroll
+    for (int w = 1; w < W; ++w) {
+      const float4 b = s_acc[w][i];
+      a.x += b.x;
+      a.y += b.y;
+      a.z += b.z;
+      a.w += b.w;
+    }
+    *reinterpret_cast<float4*>(dst + 4 * i) = make_float4(a.x * inv, a.y * inv, a.z * inv, a.w * inv);
+  }
+  if (threadIdx.x == 0 && lse) lse[(int64_t)item * H + h] = T > 0.f ? Mx + logf(T) : -CUDART_INF_F;
+}
+
 }  // namespace simt
 }  // namespace mla

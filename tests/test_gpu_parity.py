@@ -168,6 +168,21 @@ def test_decode_attention_matches_oracle(policy, H, sms):
         assert step.info.num_parts > 0   # the combine ran
 
 
+@pytest.mark.parametrize("policy,H,lens,sms,warps", [
+    ("tcgen05", 64, [9000, 40], 148, 8),
+    ("tcgen05", 64, [3000, 40], 30, 4),
+    ("tcgen05", 128, [9000, 40, 700], 148, 8),
+    ("simt", 64, [3000, 40, 0], 30, 8),
+])
+def test_many_parts_per_query_combine_matches_oracle(policy, H, lens, sms, warps):
+    """A few long queries cut into many parts: the combine spreads one (query, head)'s
+    parts over 4 or 8 warps (chosen from parts per query) and merges the warps' partial
+    sums; the short queries are single-unit items it skips."""
+    step = attention_case(policy, H, 1, lens, sms)
+    per_item = step.info.num_parts // step.info.num_items
+    assert (8 if per_item >= 8 else 4 if per_item >= 3 else 1) == warps
+
+
 @pytest.mark.parametrize("policy", ["simt", "tcgen05"])
 def test_causal_chunk_attention_matches_oracle(policy):
     attention_case(policy, 64, 5, [70, 5, 129], 6)
