@@ -411,9 +411,15 @@ mla_status mla_absorb_q(const void* q_nope, const void* W_UK, void* q_lat, int32
   const int32_t pol = g_policy.load();
   if (pol == MLA_POLICY_TCGEN05 && !absorb_tc_ok(d))
     return fail(MLA_ERR_UNSUPPORTED, "tensor-core absorb needs bf16, Dn=128, R=512");
-  if (pol != MLA_POLICY_SIMT && absorb_tc_ok(d))
+  if (pol != MLA_POLICY_SIMT && absorb_tc_ok(d)) {
+    // up to 64 rows the weights dominate: four 128-column blocks per head (65 KB of shared
+    // memory, three CTAs per SM) spread them over more SMs than two 256-column blocks do
+    if (T <= 64)
+      return launch_proj<2, 128, true, 2>(q_nope, W_UK, q_lat, T, d, d.Dn, d.H * d.Dn, d.R, d.R,
+                                          as_stream(stream), "absorb_q (tcgen05)");
     return launch_proj<2, 256, true, 2>(q_nope, W_UK, q_lat, T, d, d.Dn, d.H * d.Dn, d.R, d.R, as_stream(stream),
                                         "absorb_q (tcgen05)");
+  }
   const dim3 grid((d.R + 127) / 128, d.H, (T + mla::simt::kTT - 1) / mla::simt::kTT);
   const size_t smem = sizeof(float) * mla::simt::kTT * d.Dn;
   if (smem > 48 * 1024) return fail(MLA_ERR_UNSUPPORTED, "Dn=%d too large", d.Dn);

@@ -19,6 +19,19 @@ __global__ void __launch_bounds__(128) cache_append_vec_kernel(uint4* __restrict
   const int32_t item = blockIdx.x * 4 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
   if (item >= items) return;
   const int32_t b = item / q_len, i = item % q_len;
+  // rows of up to 96 vectors (bf16 576-wide: 72) are read into registers before the
+  // length and page lookups, so the row's load does not wait behind them
+  constexpr int kHeld = 3;
+  const uint4* src = new_ckr + (int64_t)item * row_vec;
+  const bool held = row_vec <= 32 * kHeld;
+  uint4 v[kHeld];
+  if (held) {
+#pragma unroll
+    for (int k = 0; k < kHeld; ++k) {
+      const int32_t e = lane + 32 * k;
+      if (e < row_vec) v[k] = src[e];
+    }
+  }
   const int32_t pos = seq_lens[b] - q_len + i;
   if (pos < 0) return;
   const int32_t pidx = pos / page_size;
@@ -32,7 +45,14 @@ __global__ void __launch_bounds__(128) cache_append_vec_kernel(uint4* __restrict
     return;
   }
   uint4* dst = kv + ((int64_t)page * page_size + pos % page_size) * row_vec;
-  const uint4* src = new_ckr + (int64_t)item * row_vec;
+  if (held) {
+#pragma unroll
+    for (int k = 0; k < kHeld; ++k) {
+      const int32_t e = lane + 32 * k;
+      if (e < row_vec) dst[e] = v[k];
+    }
+    return;
+  }
   for (int32_t e = lane; e < row_vec; e += 32) dst[e] = src[e];
 }
 

@@ -95,15 +95,18 @@ def test_cache_append_bit_exact(dtype):
 
 # ----------------------------------------------------------------------------- a1 / a7
 
+# (tokens: up to 64 rows the tensor-core absorption cuts each head's 512 columns into four
+# blocks, above that into two; 300 rows: three 128-row tiles with a ragged tail)
 PROJ_CASES = [("bf16_h64", "simt"), ("bf16_h64", "tcgen05"), ("bf16_h128", "simt"), ("bf16_h128", "tcgen05"),
-              ("bf16_h64_t300", "tcgen05"), ("f32_tiny", "simt")]
+              ("bf16_h64_t300", "tcgen05"), ("bf16_h64_t64", "tcgen05"), ("bf16_h128_t65", "tcgen05"),
+              ("bf16_h64_t1", "tcgen05"), ("f32_tiny", "simt")]
 
 
 def proj_case(case):
     if case == "f32_tiny":
         return wl.make("tiny_fp32")
-    H = 128 if case == "bf16_h128" else 64
-    n = 300 if case.endswith("t300") else 37     # 300 tokens: three 128-row tiles, ragged tail
+    H = 128 if case.startswith("bf16_h128") else 64
+    n = int(case.rsplit("_t", 1)[1]) if "_t" in case else 37
     return wl.make(small_spec(H=H), seed=3, seq_lens=[5] * n)
 
 
