@@ -361,10 +361,12 @@ def run_gpu(args):
 
     # ---------------------------------------------------------------- device-resident timing
     # The timed steps carry no events between their kernels (an event recorded between two
-    # kernels stalls the stream ~3-4 us): one pair of events around all K steps, or around
-    # each step where an L2 flush runs between steps (outside the events). A second pass
-    # of K steps then brackets each kernel with events for the per-kernel split and the
-    # decode kernel's duration (the roofline); the append runs on a side stream beside the
+    # kernels stalls the stream ~3-4 us): one pair of events around each block of steps,
+    # or around each step where an L2 flush runs between steps (outside the events). Each
+    # timed block is followed by as many untimed steps that bracket every kernel with
+    # events, for the per-kernel split and the decode kernel's duration (the roofline):
+    # the two kinds alternate in four blocks, so both see the same clocks when the power
+    # cap lowers them as the run goes on. The append runs on a side stream beside the
     # absorption (DecodeStep.run), so those two share one interval.
     names = ["append+absorb", "attend", "combine", "project"]
     for _ in range(args.warmup):
@@ -372,39 +374,44 @@ def run_gpu(args):
     torch.cuda.synchronize()
     mla.mla_check_status()
     flush_each = needs_flush(wl_cache_bytes(spec, w["seq_lens"], fp8))
+    nblk = min(4, args.steps)
+    blocks = [args.steps // nblk + (1 if i < args.steps % nblk else 0) for i in range(nblk)]
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(len(names) + 1)] for _ in range(args.steps)]
     bounds = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-              for _ in range(args.steps if flush_each else 1)]
+              for _ in range(args.steps if flush_each else nblk)]
     barrier()
     with ClockSampler(dev.index) as clk:
-        if flush_each:
-            for k, (b0, b1) in enumerate(bounds):
-                flush.fill_(k & 0xFF)      # evict the cache from L2 (outside the timed events)
-                b0.record(stream)
-                step.run(stream=stream)
-                b1.record(stream)
-        else:
-            bounds[0][0].record(stream)
-            for _ in range(args.steps):
-                step.run(stream=stream)
-            bounds[0][1].record(stream)
-        barrier()
-        step_total_ms = float(sum(b0.elapsed_time(b1) for b0, b1 in bounds))
-        # per-kernel split (not part of the timed steps)
-        for k in range(args.steps):
+        k = 0
+        for bi, nb in enumerate(blocks):
             if flush_each:
-                flush.fill_(k & 0xFF)
-            e = ev[k]
-            e[0].record(stream)
-            step.append_and_absorb(stream)
-            e[1].record(stream)
-            step.attend(stream)
-            e[2].record(stream)
-            step.combine(stream)
-            e[3].record(stream)
-            step.project(stream)
-            e[4].record(stream)
+                for j in range(k, k + nb):
+                    b0, b1 = bounds[j]
+                    flush.fill_(j & 0xFF)      # evict the cache from L2 (outside the timed events)
+                    b0.record(stream)
+                    step.run(stream=stream)
+                    b1.record(stream)
+            else:
+                bounds[bi][0].record(stream)
+                for _ in range(nb):
+                    step.run(stream=stream)
+                bounds[bi][1].record(stream)
+            # the same number of steps with every kernel bracketed (not part of the timed steps)
+            for j in range(k, k + nb):
+                if flush_each:
+                    flush.fill_(j & 0xFF)
+                e = ev[j]
+                e[0].record(stream)
+                step.append_and_absorb(stream)
+                e[1].record(stream)
+                step.attend(stream)
+                e[2].record(stream)
+                step.combine(stream)
+                e[3].record(stream)
+                step.project(stream)
+                e[4].record(stream)
+            k += nb
         barrier()
+    step_total_ms = float(sum(b0.elapsed_time(b1) for b0, b1 in bounds))
     mla.mla_check_status()
     per_kernel = {n: 0.0 for n in names}
     attend_ms = []
