@@ -283,6 +283,14 @@ def time_cache_write(step, spec, stream, M=7168, reps=20):
                        "rotations, append)"}
 
 
+def timing_blocks(steps, max_blocks=4):
+    """Sizes of the blocks the timed steps are cut into (each followed by as many steps
+    with every kernel bracketed): at most `max_blocks`, sizes differing by at most one,
+    summing to `steps`."""
+    n = max(1, min(max_blocks, steps))
+    return [steps // n + (1 if i < steps % n else 0) for i in range(n)]
+
+
 def needs_flush(cache_bytes):
     """Inputs larger than twice the L2 evict it on their own: every step streams the whole
     cache through L2, so nothing a step reads is still resident at the next one. Smaller
@@ -374,8 +382,8 @@ def run_gpu(args):
     torch.cuda.synchronize()
     mla.mla_check_status()
     flush_each = needs_flush(wl_cache_bytes(spec, w["seq_lens"], fp8))
-    nblk = min(4, args.steps)
-    blocks = [args.steps // nblk + (1 if i < args.steps % nblk else 0) for i in range(nblk)]
+    blocks = timing_blocks(args.steps)
+    nblk = len(blocks)
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(len(names) + 1)] for _ in range(args.steps)]
     bounds = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
               for _ in range(args.steps if flush_each else nblk)]

@@ -1,6 +1,7 @@
 """The parts of bench.py that run without a GPU: the reference arm (the fp64 oracle on
-the host cores) and the rule that reads a kernel's DRAM traffic from its committed ncu
-summary only while the kernel source is unchanged."""
+the host cores), the rule that reads a kernel's DRAM traffic from its committed ncu
+summary only while the kernel source is unchanged, and the cut of the timed steps into
+blocks."""
 import hashlib
 import json
 import os
@@ -94,3 +95,12 @@ def test_decode_kernel_follows_the_library_dispatch():
     assert bench.decode_kernel_of(64, 2)[0] == "decode_2sm.cuh"
     assert bench.decode_kernel_of(64, 1)[0] == "decode_2sm.cuh"
     assert bench.decode_kernel_of(192, 1)[0] == "decode_tc.cuh"
+
+
+@pytest.mark.parametrize("steps", [1, 2, 3, 4, 5, 7, 50, 200, 201])
+def test_timing_blocks_cover_every_step_once(steps):
+    """The timed steps are cut into at most four blocks of near-equal size (each followed
+    by as many bracketed steps): together exactly `steps`, sizes one apart at most."""
+    b = bench.timing_blocks(steps)
+    assert sum(b) == steps and 1 <= len(b) <= 4 and min(b) >= 1 and max(b) - min(b) <= 1
+
