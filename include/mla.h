@@ -59,7 +59,7 @@ extern "C" {
 typedef enum {
   MLA_OK = 0,
   MLA_ERR_INVALID = -1,      /* bad argument (null pointer, size, layout, plan) */
-  MLA_ERR_UNSUPPORTED = -2,  /* dims or policy this build has no kernel for */
+  MLA_ERR_UNSUPPORTED = -2,  /* dims or policy the library has no kernel for */
   MLA_ERR_WORKSPACE = -3,    /* workspace / plan buffer too small */
   MLA_ERR_CUDA = -4,         /* a CUDA runtime or driver call failed */
   MLA_ERR_TIMEOUT = -5       /* a kernel wait ran out (reported by mla_check_status) */
