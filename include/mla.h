@@ -54,7 +54,7 @@
 extern "C" {
 #endif
 
-#define MLA_ABI_VERSION 5
+#define MLA_ABI_VERSION 6
 
 typedef enum {
   MLA_OK = 0,
@@ -108,6 +108,18 @@ mla_status mla_set_policy(int32_t policy);
 
 /* Bound, in nanoseconds, on every wait inside a kernel (default 2e9). */
 mla_status mla_set_wait_timeout_ns(uint64_t ns);
+
+/* The split planner's estimate of what merging split queries (mla_combine) costs, in
+ * pages of decode work (process-wide; applies to plans for the SM-pair kernel, H=64 and
+ * H=128 on the tensor-core path). Negative (the default): mla_plan_splits cuts queries
+ * wherever a slot fills up, balancing the slots as finely as one page. Zero or more: the
+ * planner also lays every query out whole (no partial results, no merge) and takes that
+ * layout when its heaviest slot is at most the cut layout's plus `pages`: e.g. 64
+ * queries of 64 pages on 74 slots then run one query per slot (64 of the 74 busy)
+ * instead of every query cut in two. The split of work between queries and the token
+ * ranges they see are unchanged; only where the ranges are cut. MLA_ERR_INVALID for NaN.
+ * The split-KV merge it trades against is the log-sum-exp merge of mla_combine. */
+mla_status mla_set_plan_combine_cost(double pages);
 
 /* TEST-ONLY hook for the failure path of the tensor-core decode kernels: while set
  * (ordinal >= 0), the first CTA of each mla_decode_attn launch skips the shared-memory

@@ -24,7 +24,7 @@ STATUS_NAMES = {0: "MLA_OK", -1: "MLA_ERR_INVALID", -2: "MLA_ERR_UNSUPPORTED", -
                 -4: "MLA_ERR_CUDA", -5: "MLA_ERR_TIMEOUT"}
 
 # Every symbol include/mla.h declares.
-EXPORTS = ("mla_abi_version", "mla_last_error", "mla_set_policy", "mla_set_wait_timeout_ns",
+EXPORTS = ("mla_abi_version", "mla_last_error", "mla_set_policy", "mla_set_wait_timeout_ns", "mla_set_plan_combine_cost",
            "mla_check_status", "mla_cache_append", "mla_cache_write", "mla_cache_write_workspace_size", "mla_absorb_q", "mla_plan_capacity", "mla_plan_splits",
            "mla_workspace_size", "mla_decode_attn", "mla_combine", "mla_out_proj", "mla_decode_attn_noalloc",
            "mla_debug_drop_page_load", "mla_quantize_rows_fp8", "mla_cache_append_fp8", "mla_workspace_size_fp8",
@@ -64,6 +64,7 @@ def _load():
         "mla_last_error": (ctypes.c_char_p, []),
         "mla_set_policy": (I32, [I32]),
         "mla_set_wait_timeout_ns": (I32, [U64]),
+        "mla_set_plan_combine_cost": (I32, [ctypes.c_double]),
         "mla_debug_drop_page_load": (I32, [I32]),
         "mla_check_status": (I32, [P]),
         "mla_cache_append": (I32, [P, P, P, P, I32, I32, I32, I32, D, P]),
@@ -132,6 +133,10 @@ def mla_set_policy(policy: int) -> None:
 
 def mla_set_wait_timeout_ns(ns: int) -> None:
     _check(_lib.mla_set_wait_timeout_ns(ns), "mla_set_wait_timeout_ns")
+
+
+def mla_set_plan_combine_cost(pages: float) -> None:
+    _check(_lib.mla_set_plan_combine_cost(float(pages)), "mla_set_plan_combine_cost")
 
 
 def mla_debug_drop_page_load(ordinal: int) -> None:

@@ -31,6 +31,9 @@ namespace {
 thread_local std::string g_last_error;
 std::atomic<int32_t> g_policy{MLA_POLICY_AUTO};
 std::atomic<uint64_t> g_timeout_ns{2000000000ull};
+// The planner's estimate of what merging split queries costs, in pages of decode work
+// (mla_set_plan_combine_cost); negative: plans always cut queries where slots fill up.
+std::atomic<double> g_combine_cost_pages{-1.0};
 unsigned long long* g_trace = nullptr;  // event trace buffer (MLA_TRACE builds only)
 std::atomic<int32_t> g_drop_load{-1};   // testing hook, see mla_debug_drop_page_load
 
@@ -283,6 +286,12 @@ mla_status mla_set_policy(int32_t policy) {
   if (policy < MLA_POLICY_AUTO || policy > MLA_POLICY_TCGEN05)
     return fail(MLA_ERR_INVALID, "unknown policy %d", policy);
   g_policy.store(policy);
+  return ok();
+}
+
+mla_status mla_set_plan_combine_cost(double pages) {
+  if (!(pages == pages)) return fail(MLA_ERR_INVALID, "combine cost is NaN");
+  g_combine_cost_pages.store(pages);
   return ok();
 }
 
@@ -576,23 +585,83 @@ mla_status mla_plan_splits(const int32_t* seq_lens_host, int32_t B, int32_t q_le
       }
       return slot + 1;
     };
+    // The same layout with every group whole: a group that does not fit in what is left
+    // of a slot's capacity C starts the next slot (a group larger than C fills one alone).
+    auto fill_whole = [&](const std::vector<Grp>& order, int64_t slot0, double C, bool emit) -> int64_t {
+      int64_t slot = 0;
+      double acc = 0.0;
+      bool used = false;
+      for (const Grp& g : order) {
+        const int32_t it = g.b * q_len + g.k * ipu;
+        const int32_t n = std::min(ipu, q_len - g.k * ipu);
+        const int32_t pg = group_pages(g.b, g.k);
+        if (pg > 0 && used && acc + cost + pg > C) {
+          ++slot;
+          acc = 0.0;
+          used = false;
+        }
+        if (emit) units.push_back({it, g.b, 0, pg, (int32_t)(slot0 + slot), n});
+        if (pg > 0) {
+          used = true;
+          acc += cost + pg;
+        }
+      }
+      return slot + 1;
+    };
+    // the heaviest slot of the units emitted from index u0 on, and whether a group was cut
+    auto heaviest = [&](size_t u0, bool* cut) {
+      std::vector<double> load;
+      *cut = false;
+      for (size_t k = u0; k < units.size(); ++k) {
+        const U& u = units[k];
+        if ((size_t)u.slot >= load.size()) load.resize(u.slot + 1, 0.0);
+        if (u.pe > u.pb) load[u.slot] += cost + (u.pe - u.pb);
+        if (u.pb > 0) *cut = true;
+      }
+      double m = 0.0;
+      for (double x : load) m = std::max(m, x);
+      return m;
+    };
     // the smallest capacity whose fill of `order` needs at most ns slots (bisection)
+    auto bisect = [&](const std::vector<Grp>& order, int64_t slot0, int64_t ns, double lo, double hi, bool whole) {
+      for (int it = 0; it < 48 && hi - lo > 0.25; ++it) {
+        const double mid = 0.5 * (lo + hi);
+        if ((whole ? fill_whole(order, slot0, mid, false) : fill(order, slot0, mid, false)) <= ns) hi = mid;
+        else lo = mid;
+      }
+      return hi;
+    };
+    const double combine_cost = g_combine_cost_pages.load();
     auto layout = [&](const std::vector<Grp>& order, int64_t slot0, int64_t ns) {
       int64_t pages = 0, groups = 0;
+      int32_t largest = 0;
       for (const Grp& g : order) {
         const int32_t pg = group_pages(g.b, g.k);
         pages += pg;
         groups += pg > 0;
+        largest = std::max(largest, pg);
       }
       // below lo the pages and one cost per group do not fit in ns slots; hi fits in one
-      double lo = std::max(cost, ((double)pages + cost * (double)groups) / (double)ns - 1.0);
-      double hi = (double)pages + cost * (double)(groups + ns) + 1.0;
-      for (int it = 0; it < 48 && hi - lo > 0.25; ++it) {
-        const double mid = 0.5 * (lo + hi);
-        if (fill(order, slot0, mid, false) <= ns) hi = mid;
-        else lo = mid;
-      }
-      fill(order, slot0, hi, true);
+      const double lo = std::max(cost, ((double)pages + cost * (double)groups) / (double)ns - 1.0);
+      const double hi = (double)pages + cost * (double)(groups + ns) + 1.0;
+      const size_t u0 = units.size();
+      fill(order, slot0, bisect(order, slot0, ns, lo, hi, false), true);
+      if (combine_cost < 0.0) return;
+      // With a combine cost set: the layout that keeps every group whole is taken instead
+      // when its heaviest slot is no heavier than the cut layout's plus the merge of the
+      // cut queries' parts (which only the cut layout needs).
+      bool cut = false;
+      const double cut_load = heaviest(u0, &cut);
+      if (!cut) return;
+      const double lo_w = std::max(lo, cost + (double)largest - 1.0);
+      const size_t u1 = units.size();
+      fill_whole(order, slot0, bisect(order, slot0, ns, lo_w, std::max(hi, lo_w + 1.0), true), true);
+      bool cut_w = false;
+      const double whole_load = heaviest(u1, &cut_w);
+      if (units.back().slot - slot0 < ns && whole_load <= cut_load + combine_cost)
+        units.erase(units.begin() + (std::ptrdiff_t)u0, units.begin() + (std::ptrdiff_t)u1);
+      else
+        units.resize(u1);
     };
     if (ipu == 1 && q_len >= 2 && S >= 2 * q_len) {
       // Several query tokens per sequence, one per unit (128 heads fill the pair's rows):

@@ -34,7 +34,7 @@ def test_library_exports_every_declared_symbol():
 
 
 def test_abi_version_and_error_text():
-    assert mla.mla_abi_version() == 5
+    assert mla.mla_abi_version() == 6
     with pytest.raises(mla.MlaError) as e:
         mla.mla_set_policy(7)
     assert e.value.status == mla._binding.MLA_ERR_INVALID
@@ -58,6 +58,28 @@ def dims(H=64, R=512, Dr=64, ps=64, dtype=mla.MLA_BF16):
 @pytest.mark.parametrize("sms", [1, 7, 148])
 @pytest.mark.parametrize("H", [64, 128, 16])
 def test_plan_covers_every_visible_page_once(q_len, sms, H):
+    check_plan_covers(q_len, sms, H)
+
+
+@pytest.fixture
+def combine_cost():
+    """Sets the planner's combine cost for one test and restores the default (off)."""
+    def set_cost(pages):
+        mla.mla_set_plan_combine_cost(pages)
+    yield set_cost
+    mla.mla_set_plan_combine_cost(-1.0)
+
+
+@pytest.mark.parametrize("cost", [0.0, 6.5, 1e9])
+@pytest.mark.parametrize("q_len", [1, 3])
+@pytest.mark.parametrize("sms", [7, 148])
+@pytest.mark.parametrize("H", [64, 128])
+def test_plan_with_a_combine_cost_still_covers_every_visible_page_once(H, sms, q_len, cost, combine_cost):
+    combine_cost(cost)
+    check_plan_covers(q_len, sms, H)
+
+
+def check_plan_covers(q_len, sms, H):
     rng = np.random.default_rng(q_len * 1000 + sms + H)
     lens = rng.integers(0, 700, size=9).astype(np.int32)
     lens[0] = 0
@@ -135,6 +157,75 @@ def test_plan_balances_pages_and_units_over_pair_slots(lens):
     share = (total + UNIT_COST * (groups + 74 - 1)) / 74
     work = pages + UNIT_COST * units
     assert work.max() <= share + UNIT_COST + 1, (work.max(), share)
+
+
+def heaviest_slot(plan, info):
+    pages, units = slot_loads(plan, info)
+    return float((pages + UNIT_COST * units).max())
+
+
+def test_combine_cost_keeps_equal_queries_whole_when_the_merge_costs_more_than_it_saves(combine_cost):
+    """64 queries of 64 pages on 74 pair slots: cut, every query is split in two (slots
+    of ~68.3 pages of work, 128 partial results to merge); whole, one query per slot (71.5:
+    its 64 pages plus one unit's cost) on 64 slots. The whole layout is taken exactly when
+    its heaviest slot is at most the cut one's plus the combine cost."""
+    lens = np.full(64, 4096, np.int32)
+    d = dims(H=64)
+    plan_cut, info_cut = mla.mla_plan_splits(lens, 64, 1, 64, d, 148)
+    assert info_cut.num_parts == 128
+    cut = heaviest_slot(plan_cut, info_cut)
+    whole = 64 + UNIT_COST
+    assert cut < whole
+    combine_cost(whole - cut - 0.01)
+    plan, info = mla.mla_plan_splits(lens, 64, 1, 64, d, 148)
+    assert np.array_equal(plan, plan_cut)
+    combine_cost(whole - cut + 0.01)
+    plan, info = mla.mla_plan_splits(lens, 64, 1, 64, d, 148)
+    assert info.num_parts == 0 and info.num_slots == 64 and info.num_units == 64
+    p = parse_plan(plan)
+    for s_, u in enumerate(p["units"]):
+        assert (u[0], u[2], u[3], u[4], u[5]) == (s_, 0, 64, -1, s_)
+    assert np.all(p["item_parts"] == [-1, 0])
+    assert heaviest_slot(plan, info) == whole
+
+
+def test_combine_cost_keeps_cutting_where_whole_queries_load_a_slot_far_more(combine_cost):
+    """128 ragged queries (512..16384 tokens) on 74 slots: keeping them whole leaves a
+    slot with a 256-page query and more; the cut layout stays, byte for byte."""
+    lens = np.random.default_rng(0).integers(512, 16385, 128).astype(np.int32)
+    d = dims(H=128)
+    plan0, info0 = mla.mla_plan_splits(lens, 128, 1, 256, d, 148)
+    combine_cost(12.0)
+    plan, info = mla.mla_plan_splits(lens, 128, 1, 256, d, 148)
+    assert info0.num_parts > 0 and np.array_equal(plan, plan0)
+
+
+@pytest.mark.parametrize("q_len", [2, 4])
+def test_combine_cost_whole_queries_keep_the_token_blocks_of_128_heads(q_len, combine_cost):
+    """With the merge priced out, every token of the 128-head multi-token layout still
+    gets the same layout on its own slot block, now one whole sequence per unit."""
+    combine_cost(1e9)
+    lens = np.random.default_rng(1).integers(512, 16385, 64).astype(np.int32)
+    max_pages = int((lens.max() + 63) // 64)
+    plan, info = mla.mla_plan_splits(lens, len(lens), q_len, max_pages, dims(H=128), 148)
+    p = parse_plan(plan)
+    ns = 74 // q_len
+    assert info.num_parts == 0 and info.num_units == q_len * len(lens)
+    blocks = [[] for _ in range(q_len)]
+    for u in p["units"]:
+        k = u[0] % q_len
+        assert k * ns <= u[5] < (k + 1) * ns and u[2] == 0 and u[3] == (lens[u[1]] + 63) // 64
+        blocks[k].append((u[1], u[5] - k * ns))
+    for k in range(1, q_len):
+        assert blocks[k] == blocks[0]
+
+
+def test_combine_cost_rejects_nan_and_is_off_by_default(combine_cost):
+    with pytest.raises(mla.MlaError):
+        mla.mla_set_plan_combine_cost(float("nan"))
+    lens = np.full(64, 4096, np.int32)
+    plan, info = mla.mla_plan_splits(lens, 64, 1, 64, dims(H=64), 148)
+    assert info.num_parts == 128
 
 
 @pytest.mark.parametrize("q_len", [2, 4])
